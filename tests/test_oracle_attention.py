@@ -1,0 +1,187 @@
+"""Pins for the oracle's attention forward.
+
+The expected values come from sources other than the oracle:
+
+* torch.nn.functional.scaled_dot_product_attention in fp64 on the CPU.
+  This is the library special case where the mask is boolean and there is
+  no score_mod.
+* torch.logsumexp.
+* Closed forms: the ALiBi geometric weights and the tanh(1) soft-cap
+  worked case.
+* Invariants: rows sum to 1, constant V gives a constant output, GQA equals
+  explicitly repeated kv heads, and a row with every key masked gives 0 and
+  -inf.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import attention as oa
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(shape, generator=g, dtype=torch.float64)
+
+
+def test_noop_equals_sdpa():
+    q, k, v = _rand((2, 3, 37, 16), 1), _rand((2, 3, 45, 16), 2), _rand((2, 3, 45, 16), 3)
+    out, lse = oa.flex_attention(q, k, v, None, (), scale=0.3)
+    ref = F.scaled_dot_product_attention(q, k, v, scale=float(np.float32(0.3)))
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+    s = float(np.float32(0.3)) * (q @ k.transpose(-1, -2))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_default_scale_is_rsqrt_d():
+    q, k, v = _rand((1, 1, 8, 64), 4), _rand((1, 1, 8, 64), 5), _rand((1, 1, 8, 64), 6)
+    out, _ = oa.flex_attention(q, k, v, None, ())
+    ref = F.scaled_dot_product_attention(q, k, v, scale=float(np.float32(1 / 8)))
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_causal_equals_sdpa_is_causal():
+    q, k, v = _rand((1, 2, 64, 32), 7), _rand((1, 2, 64, 32), 8), _rand((1, 2, 64, 32), 9)
+    out, lse = oa.flex_attention(q, k, v, ("causal",), (), scale=0.25)
+    ref = F.scaled_dot_product_attention(q, k, v, is_causal=True, scale=0.25)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+    s = 0.25 * (q @ k.transpose(-1, -2))
+    s = s.masked_fill(~torch.ones(64, 64, dtype=torch.bool).tril(), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_band_mask_equals_sdpa_bool_mask():
+    n, W = 80, 9
+    q, k, v = _rand((1, 1, n, 8), 10), _rand((1, 1, n, 8), 11), _rand((1, 1, n, 8), 12)
+    out, _ = oa.flex_attention(q, k, v, ("and", ("causal",), ("window", W)), (), scale=0.5)
+    band = torch.ones(n, n, dtype=torch.bool).tril() & torch.ones(n, n, dtype=torch.bool).triu(-(W - 1))
+    ref = F.scaled_dot_product_attention(q, k, v, attn_mask=band, scale=0.5)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_gqa_equals_sdpa_enable_gqa():
+    q, k, v = _rand((1, 8, 20, 16), 13), _rand((1, 2, 24, 16), 14), _rand((1, 2, 24, 16), 15)
+    out, _ = oa.flex_attention(q, k, v, None, (), scale=0.2, enable_gqa=True)
+    ref = F.scaled_dot_product_attention(q, k, v, scale=float(np.float32(0.2)), enable_gqa=True)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+    # explicit repeat of each kv head over its 4 query heads
+    rep, _ = oa.flex_attention(q, k.repeat_interleave(4, 1), v.repeat_interleave(4, 1), None, (),
+                               scale=0.2)
+    np.testing.assert_allclose(out, rep, rtol=0, atol=0)
+    with pytest.raises(ValueError):
+        oa.flex_attention(q, k, v, None, (), enable_gqa=False)
+
+
+def test_rows_sum_to_one_and_constant_v():
+    n = 24
+    q, k = _rand((1, 1, n, 8), 16), _rand((1, 1, n, 8), 17)
+    eye = torch.eye(n, dtype=torch.float64)[None, None]        # V = I -> out = P
+    tree = ("and", ("causal",), ("or", ("sink", 2), ("window", 5)))
+    P, _ = oa.flex_attention(q, k, eye, tree, (), scale=1.0)
+    np.testing.assert_allclose(P.sum(-1), 1.0, rtol=0, atol=1e-13)
+    const = torch.full((1, 1, n, 8), 2.5, dtype=torch.float64)
+    out, _ = oa.flex_attention(q, k, const, tree, (("softcap", 5.0),), scale=1.0)
+    np.testing.assert_allclose(out, 2.5, rtol=0, atol=1e-13)
+
+
+def test_fully_masked_rows_are_zero_and_minus_inf():
+    q, k, v = _rand((1, 1, 10, 4), 18), _rand((1, 1, 10, 4), 19), _rand((1, 1, 10, 4), 20)
+    # kv < 0 allows nothing; rows with q_idx < 3 of the OR below are masked too
+    out, lse = oa.flex_attention(q, k, v, ("sink", 0), ())
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+    out, lse = oa.flex_attention(q, k, v, ("and", ("causal",), ("window", 0)), ())
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+def test_alibi_closed_form_geometric_weights():
+    # ALiBi m_h * (j - i) (transformerlab page, "alibi" row). With K = 0 every
+    # score is 0, so the weights of causal row i are proportional to
+    # exp(m (j - i)) for j <= i. One-hot values read the weights back.
+    n, H = 12, 2
+    q = _rand((1, H, n, n), 21)
+    k = torch.zeros((1, H, n, n), dtype=torch.float64)
+    v = torch.eye(n, dtype=torch.float64)[None, None].repeat(1, H, 1, 1)
+    slopes = np.array([0.5, 0.125], np.float32)
+    out, lse = oa.flex_attention(q, k, v, ("causal",), (("alibi", slopes),), scale=1.0)
+    for h, m in enumerate(slopes.astype(np.float64)):
+        r = math.exp(m)
+        for i in range(n):
+            denom = (r ** (i + 1) - 1) / (r - 1)
+            for j in range(n):
+                w = r ** j / denom if j <= i else 0.0
+                assert out[0, h, i, j] == pytest.approx(w, rel=1e-12, abs=1e-15)
+            # lse = log sum_{j<=i} exp(m (j - i)) = log((1 - e^{-m(i+1)}) / (1 - e^{-m}))
+            assert lse[0, h, i] == pytest.approx(
+                math.log((1 - math.exp(-m * (i + 1))) / (1 - math.exp(-m))), rel=1e-12)
+
+
+def test_alibi_default_slopes_and_zero_slopes():
+    np.testing.assert_allclose(oa.default_alibi_slopes(16)[[0, 1, 15]],
+                               [2 ** -0.5, 2 ** -1.0, 2 ** -8.0], rtol=1e-15)
+    q, k, v = _rand((1, 2, 16, 8), 22), _rand((1, 2, 16, 8), 23), _rand((1, 2, 16, 8), 24)
+    a, _ = oa.flex_attention(q, k, v, ("causal",), (("alibi", np.zeros(2, np.float32)),))
+    b, _ = oa.flex_attention(q, k, v, ("causal",), ())
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-15)
+
+
+def test_softcap_golden_tanh1():
+    vals = {}
+    with open(os.path.join(GOLDEN, "softcap_tanh1.txt")) as fh:
+        for line in fh:
+            if line.strip() and not line.startswith("#"):
+                key, val = line.split()
+                vals[key] = float(val)
+    q = torch.tensor([[[[30.0]]]], dtype=torch.float64)
+    k = torch.tensor([[[[1.0], [0.0]]]], dtype=torch.float64)
+    v = torch.tensor([[[[1.0], [0.0]]]], dtype=torch.float64)
+    out, lse = oa.flex_attention(q, k, v, None, (("softcap", vals["cap"]),), scale=1.0)
+    assert out[0, 0, 0, 0] == pytest.approx(vals["out"], rel=1e-14)
+    assert lse[0, 0, 0] == pytest.approx(vals["lse"], rel=1e-14)
+
+
+def test_softcap_huge_cap_is_identity():
+    q, k, v = _rand((1, 1, 16, 8), 25), _rand((1, 1, 16, 8), 26), _rand((1, 1, 16, 8), 27)
+    a, la = oa.flex_attention(q, k, v, ("causal",), (("softcap", 1e30),))
+    b, lb = oa.flex_attention(q, k, v, ("causal",), ())
+    np.testing.assert_allclose(a, b, rtol=1e-12)
+    np.testing.assert_allclose(la, lb, rtol=1e-12)
+
+
+def test_score_mod_order():
+    # softcap then alibi differs from alibi then softcap; order follows the list
+    q, k, v = _rand((1, 1, 16, 8), 28), _rand((1, 1, 16, 8), 29), _rand((1, 1, 16, 8), 30)
+    s = np.array([0.7], np.float32)
+    a, _ = oa.flex_attention(q, k, v, ("causal",), (("softcap", 2.0), ("alibi", s)), scale=1.0)
+    b, _ = oa.flex_attention(q, k, v, ("causal",), (("alibi", s), ("softcap", 2.0)), scale=1.0)
+    assert not np.allclose(a, b)
+
+
+def test_document_mask_equals_sdpa_block_diag():
+    lengths = [5, 11, 4]
+    ids = np.repeat(np.arange(3), lengths).astype(np.int32)
+    n = ids.size
+    q, k, v = _rand((1, 1, n, 8), 31), _rand((1, 1, n, 8), 32), _rand((1, 1, n, 8), 33)
+    out, _ = oa.flex_attention(q, k, v, ("and", ("document", ids[None], ids[None]), ("causal",)), (),
+                               scale=0.4)
+    blocks = [torch.ones(L, L, dtype=torch.bool).tril() for L in lengths]
+    ref = F.scaled_dot_product_attention(q, k, v, attn_mask=torch.block_diag(*blocks),
+                                         scale=float(np.float32(0.4)))
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_sampled_matches_full():
+    q, k, v = _rand((2, 4, 40, 8), 34), _rand((2, 2, 50, 8), 35), _rand((2, 2, 50, 8), 36)
+    tree = ("and", ("causal",), ("window", 7))
+    mods = (("alibi", None),)
+    out, lse = oa.flex_attention(q, k, v, tree, mods, enable_gqa=True)
+    samples = [(0, 0, 0), (1, 3, 39), (0, 2, 17), (1, 1, 5)]
+    so, sl = oa.flex_attention_sampled(q, k, v, samples, tree, mods, enable_gqa=True)
+    for i, (b, h, r) in enumerate(samples):
+        np.testing.assert_allclose(so[i], out[b, h, r], rtol=1e-13, atol=1e-14)
+        assert sl[i] == pytest.approx(lse[b, h, r], rel=1e-13)
