@@ -1,0 +1,367 @@
+"""Benchmark: block-sparse masked attention forward on B200.
+
+One step is the whole hot path on one batch of synthetic input:
+  1. the block-mask builder kernel (mask evaluation, tile classification,
+     index compaction);
+  2. the attention kernel over the tiles the mask keeps (score_mod and, on
+     partial tiles only, mask_mod; online softmax; out and lse).
+
+metric: TFLOP/s counting only the FLOPs of tiles that are not skipped,
+4 * 128 * 128 * D per kept (FULL or PARTIAL) 128x128 tile per (b, hq).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--workload INDEX] [--no-cpu-baseline]
+For N > 1 run it under torch.distributed.run. Each rank then processes its
+own batch of the same shape (weak scaling; the units are independent).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "flex_attention fwd TFLOP/s (unmasked tiles) and % of B200 BF16 tensor peak"
+UNIT = "TFLOP/s"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_SOURCES = ["attn_fwd.cuh", "ptx.cuh", "mask_dnf.cuh", "bsmt.cu"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "block_sparse_masked_tile_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(workload_name: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel source (same hash); otherwise None."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload_name}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != attn_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def counted_flops(bm, D: int) -> int:
+    """4*128*128*D per kept tile per (b, hq); the mask is built at [B, Hq]."""
+    tiles = int(bm.kv_num_blocks.sum().item()) + int(bm.full_kv_num_blocks.sum().item())
+    return tiles * 4 * 128 * 128 * D
+
+
+# ------------------------------------------------------------------ oracle
+def cpu_baseline(w, data, max_rows: int = 1024):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload: whole
+    q-blocks of (b=0, hq=0) from the top of the sequence (the rows with the most
+    kept tiles), counted with the same tile rule as the GPU metric."""
+    from threadpoolctl import threadpool_info
+    from oracle import attention as oa
+    from oracle import block_mask as obm
+
+    rows_per_block = 128
+    nblk = max(1, max_rows // rows_per_block)
+    qbs = list(range((w.M + 127) // 128 - nblk, (w.M + 127) // 128))
+    samples = [(0, 0, qb * 128 + r) for qb in qbs for r in range(128) if qb * 128 + r < w.M]
+    # kept tiles of those q-block rows (oracle block mask, per q-block row)
+    cls = obm.tile_classes(data["mask"], 0, w.M, w.N)
+    tiles = sum(int((cls[qb] > 0).sum()) for qb in qbs)
+    flops = tiles * 4 * 128 * 128 * w.D
+    t0 = time.perf_counter()
+    oa.flex_attention_sampled(data["q"], data["k"], data["v"], samples, data["mask"], data["score_mods"], w.scale,
+                              w.enable_gqa)
+    dt = time.perf_counter() - t0
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "sample": f"{len(samples)} query rows = q-blocks {qbs[0]}..{qbs[-1]} of (b=0, hq=0), "
+                      f"{tiles} kept tiles, {dt:.1f} s"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    data = workloads.make(w)
+    base = None
+    times = []
+    total = args.warmup + args.steps
+    for i in range(total):
+        r = cpu_baseline(w, data, max_rows=128)
+        if i >= args.warmup:
+            times.append(r)
+        base = r
+    vals = [t["value"] for t in times]
+    value = statistics.mean(vals) if vals else 0.0
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.M, "D": w.D},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": base["cores"], "kind": "oracle",
+                         "sample": "each step: " + base["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- GPU
+def main():
+    args = parse()
+    w = workloads.get(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import block_sparse_masked_tile_b200 as bsmt
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    data = workloads.make(w, seed_offset=rank)
+    q, k, v = (t.to(dev) for t in (data["q"], data["k"], data["v"]))
+    mask = bsmt.mask_from_tree(data["mask"], device=dev)
+    mods = bsmt.score_mods_from_list(data["score_mods"])
+    bm = bsmt.create_block_mask(mask, w.B, w.Hq, w.M, w.N, device=dev)
+    out = torch.empty((w.B, w.Hq, w.M, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.M), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(attn_events=None):
+        bsmt.create_block_mask(mask, w.B, w.Hq, w.M, w.N, device=dev, out=bm)
+        if attn_events is not None:
+            attn_events[0].record(stream)
+        bsmt.flex_attention(q, k, v, block_mask=bm, score_mod=mods, scale=w.scale, enable_gqa=w.enable_gqa,
+                            out=out, lse=lse)
+        if attn_events is not None:
+            attn_events[1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    bsmt.check_device_status(dev)
+    flops = counted_flops(bm, w.D)
+    sparsity = bm.sparsity()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    bsmt.check_device_status(dev)
+    ms = start.elapsed_time(end) / args.steps
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    t = torch.tensor([ms, attn_ms], dtype=torch.float64, device=dev)
+    tot = torch.tensor([float(flops)], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+    ms, attn_ms = float(t[0]), float(t[1])
+    total_flops = float(tot[0])
+    value = total_flops / (ms * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers
+    hq_, hk_, hv_ = (x.pin_memory() for x in (data["q"], data["k"], data["v"]))
+    ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    doc_host = []
+    if w.mask == "doc_causal":
+        doc_host = [torch.as_tensor(data["mask"][1][1]).pin_memory()]
+
+    def e2e_step():
+        qd, kd, vd = (x.to(dev, non_blocking=True) for x in (hq_, hk_, hv_))
+        m = mask
+        if doc_host:
+            dd = doc_host[0].to(dev, non_blocking=True)
+            m = bsmt.and_masks(bsmt.document(dd), bsmt.causal())
+        b2 = bsmt.create_block_mask(m, w.B, w.Hq, w.M, w.N, device=dev)
+        o2, l2 = bsmt.flex_attention(qd, kd, vd, block_mask=b2, score_mod=mods, scale=w.scale,
+                                     enable_gqa=w.enable_gqa)
+        ho.copy_(o2, non_blocking=True)
+        hl.copy_(l2, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+
+    e2e_step()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te[0])
+    h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_)) + sum(x.numel() * 4 for x in doc_host)
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    peaks, peak_src = load_peaks()
+    attn_tflops = (flops / (attn_ms * 1e-3)) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    traffic = profile_traffic(w.name)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "seq_len": w.M, "D": w.D,
+            "mask": data["mask"][0] if w.mask != "doc_causal" else "document and causal",
+            "counted_gflop_per_gpu_step": flops / 1e9, "sparsity_pct": sparsity,
+            "l2": "inputs larger than L2 (q+k+v = %.0f MB per step); L2 not flushed" % (
+                sum(x.numel() * 2 for x in (q, k, v)) / 1e6),
+            "parallelism": f"dp{world} (independent batches per GPU)",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "achieved": attn_tflops,
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": attn_tflops / peak,
+            "traffic": traffic,
+            "kernel": "attn_fwd_kernel",
+            "peak_source": f"{peak_src} bf16_tflops (burst); sustained "
+                           f"{peaks.get('bf16_tflops_sustained')}; datasheet {DATASHEET_BF16_TFLOPS}",
+            "frac_of_datasheet": attn_tflops / DATASHEET_BF16_TFLOPS,
+            "attn_ms": attn_ms,
+        },
+        "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, data)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,439 @@
+"""Block-sparse masked-tile attention for NVIDIA B200 (sm_100a).
+
+This is a thin Python binding over the C ABI in ``include/bsmt.h``
+(``libbsmt.so``). It only marshals arguments. PyTorch supplies device
+memory and the current CUDA stream; every step of the computation runs in
+the library's CUDA kernels. If the library is missing, importing this module
+raises.
+
+The API follows the tensorplay.nn.attention page:
+
+* ``create_block_mask(mask_mod, B, H, Q_LEN, KV_LEN, BLOCK_SIZE=128)``
+  returns a ``BlockMask`` holding kv_num_blocks/kv_indices (partial blocks)
+  and full_kv_num_blocks/full_kv_indices (full blocks).
+* ``flex_attention(q, k, v, block_mask, score_mod, scale, enable_gqa)``
+  returns ``(out, lse)``.
+* Mask builders: ``noop_mask``, ``causal``, ``sliding_window``,
+  ``prefix_lm``, ``sink``, ``document``, ``and_masks`` and ``or_masks``.
+* Score mods: ``softcap`` and ``alibi``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+from typing import Iterable, Sequence
+
+import torch
+
+__all__ = [
+    "BsmtError", "MaskMod", "ScoreMod", "BlockMask", "noop_mask", "causal", "sliding_window", "prefix_lm",
+    "sink", "document", "and_masks", "or_masks", "softcap", "alibi", "create_block_mask", "flex_attention",
+    "check_device_status", "library_path", "mask_from_tree", "score_mods_from_list",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libbsmt.so")
+
+# ------------------------------------------------------------------ C ABI
+MAX_NODES = 32
+MAX_SCORE_OPS = 2
+(MASK_NOOP, MASK_CAUSAL, MASK_WINDOW, MASK_PREFIX_LM, MASK_SINK, MASK_DOCUMENT, MASK_AND, MASK_OR) = range(8)
+SCORE_NONE, SCORE_SOFTCAP, SCORE_ALIBI = 0, 1, 2
+STATUS_NAMES = {
+    0: "OK", 1: "INVALID_ARGUMENT", 2: "SHAPE_MISMATCH", 3: "UNSUPPORTED", 4: "CUDA_ERROR",
+    5: "DEVICE_TIMEOUT", 6: "DEVICE_BOUNDS", 7: "DEVICE_PRECONDITION",
+}
+
+
+class _MaskNode(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("arg", ctypes.c_int32)]
+
+
+class _MaskSpec(ctypes.Structure):
+    _fields_ = [("num_nodes", ctypes.c_int32), ("nodes", _MaskNode * MAX_NODES),
+                ("q_doc_ids", ctypes.c_void_p), ("kv_doc_ids", ctypes.c_void_p), ("doc_batch", ctypes.c_int32)]
+
+
+class _ScoreOp(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("value", ctypes.c_float), ("slopes", ctypes.c_void_p)]
+
+
+class _ScoreSpec(ctypes.Structure):
+    _fields_ = [("num_ops", ctypes.c_int32), ("ops", _ScoreOp * MAX_SCORE_OPS)]
+
+
+class _BlockMask(ctypes.Structure):
+    _fields_ = [("kv_num_blocks", ctypes.c_void_p), ("kv_indices", ctypes.c_void_p),
+                ("full_kv_num_blocks", ctypes.c_void_p), ("full_kv_indices", ctypes.c_void_p),
+                ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("QB", ctypes.c_int32), ("KB", ctypes.c_int32),
+                ("Q_LEN", ctypes.c_int32), ("KV_LEN", ctypes.c_int32),
+                ("BLOCK_Q", ctypes.c_int32), ("BLOCK_KV", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is missing: build it with `python -m block_sparse_masked_tile_b200.build` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    i64, i32, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p
+    lib.bsmt_block_mask_shape.argtypes = [i64, i64, i64, i64, i32, i32, ctypes.POINTER(i64)]
+    lib.bsmt_block_mask_shape.restype = i32
+    lib.bsmt_create_block_mask.argtypes = [ctypes.POINTER(_MaskSpec), i64, i64, i64, i64, i32, i32,
+                                           ctypes.POINTER(_BlockMask), vp]
+    lib.bsmt_create_block_mask.restype = i32
+    lib.bsmt_flex_attention_fwd.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.POINTER(_BlockMask),
+                                            ctypes.POINTER(_MaskSpec), ctypes.POINTER(_ScoreSpec), ctypes.c_float,
+                                            i32, vp, vp, vp]
+    lib.bsmt_flex_attention_fwd.restype = i32
+    lib.bsmt_last_error.argtypes = []
+    lib.bsmt_last_error.restype = ctypes.c_char_p
+    lib.bsmt_check_device_status.argtypes = [vp]
+    lib.bsmt_check_device_status.restype = i32
+    lib.bsmt_version.argtypes = []
+    lib.bsmt_version.restype = i32
+    return lib
+
+
+_lib = _load()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+class BsmtError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class BsmtValueError(ValueError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def _check(status: int) -> None:
+    if status == 0:
+        return
+    msg = _lib.bsmt_last_error().decode(errors="replace")
+    if status in (1, 2):
+        raise BsmtValueError(status, msg)
+    raise BsmtError(status, msg)
+
+
+def _stream_ptr(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+# ------------------------------------------------------------------ masks
+@dataclass(frozen=True)
+class MaskMod:
+    """A composable mask_mod, stored as a postfix program of ABI nodes."""
+    nodes: tuple = ()
+    q_doc_ids: torch.Tensor | None = field(default=None, compare=False)
+    kv_doc_ids: torch.Tensor | None = field(default=None, compare=False)
+
+    def _spec(self, device: torch.device, B: int) -> tuple[_MaskSpec, list]:
+        if len(self.nodes) > MAX_NODES:
+            raise ValueError(f"mask program has {len(self.nodes)} nodes (at most {MAX_NODES})")
+        spec = _MaskSpec()
+        spec.num_nodes = len(self.nodes)
+        for i, (kind, arg) in enumerate(self.nodes):
+            spec.nodes[i].kind = kind
+            spec.nodes[i].arg = arg
+        keep = []
+        if self.q_doc_ids is not None:
+            qd = self.q_doc_ids.to(device=device, dtype=torch.int32).contiguous()
+            kd = self.kv_doc_ids.to(device=device, dtype=torch.int32).contiguous()
+            if qd.dim() == 1:
+                qd = qd[None]
+            if kd.dim() == 1:
+                kd = kd[None]
+            if qd.shape[0] != kd.shape[0]:
+                raise ValueError("q_doc_ids and kv_doc_ids need the same batch extent")
+            keep += [qd, kd]
+            spec.q_doc_ids = qd.data_ptr()
+            spec.kv_doc_ids = kd.data_ptr()
+            spec.doc_batch = qd.shape[0]
+        else:
+            spec.doc_batch = 1
+        return spec, keep
+
+
+def _leaf(kind: int, arg: int = 0) -> MaskMod:
+    return MaskMod(((kind, int(arg)),))
+
+
+def noop_mask() -> MaskMod:
+    return _leaf(MASK_NOOP)
+
+
+def causal() -> MaskMod:
+    return _leaf(MASK_CAUSAL)
+
+
+def sliding_window(window: int) -> MaskMod:
+    """q_idx - kv_idx < window (combine with causal() for a causal band)."""
+    return _leaf(MASK_WINDOW, window)
+
+
+def prefix_lm(prefix: int) -> MaskMod:
+    return _leaf(MASK_PREFIX_LM, prefix)
+
+
+def sink(num_sink: int) -> MaskMod:
+    return _leaf(MASK_SINK, num_sink)
+
+
+def document(q_doc_ids: torch.Tensor, kv_doc_ids: torch.Tensor | None = None) -> MaskMod:
+    """q_doc_ids[b, q_idx] == kv_doc_ids[b, kv_idx]; kv ids must be non-decreasing (packed documents)."""
+    if kv_doc_ids is None:
+        kv_doc_ids = q_doc_ids
+    return MaskMod(((MASK_DOCUMENT, 0),), q_doc_ids, kv_doc_ids)
+
+
+def _combine(op: int, mods: Sequence[MaskMod]) -> MaskMod:
+    if not mods:
+        raise ValueError("and_masks/or_masks need at least one mask")
+    docs = [m for m in mods if m.q_doc_ids is not None]
+    for m in docs[1:]:
+        if m.q_doc_ids is not docs[0].q_doc_ids or m.kv_doc_ids is not docs[0].kv_doc_ids:
+            raise ValueError("all document() masks in one program must share the same id tensors")
+    nodes: list = []
+    for m in mods:
+        nodes.extend(m.nodes)
+    nodes.append((op, len(mods)))
+    d = docs[0] if docs else None
+    return MaskMod(tuple(nodes), d.q_doc_ids if d else None, d.kv_doc_ids if d else None)
+
+
+def and_masks(*mods: MaskMod) -> MaskMod:
+    """Intersection of the given masks (tensorplay.nn.attention, and_masks)."""
+    return _combine(MASK_AND, mods)
+
+
+def or_masks(*mods: MaskMod) -> MaskMod:
+    """Union of the given masks (tensorplay.nn.attention, or_masks)."""
+    return _combine(MASK_OR, mods)
+
+
+def mask_from_tree(tree, device=None, _cache=None) -> MaskMod:
+    """Convert a nested tuple mask description (see ``workloads``) into a MaskMod.
+    Document id arrays are placed on ``device`` when it is given. One program
+    carries one (q, kv) document id pair: document leaves over different arrays
+    raise ValueError."""
+    if _cache is None:
+        _cache = {}
+    if tree is None:
+        return noop_mask()
+    kind = tree[0]
+    if kind == "noop":
+        return noop_mask()
+    if kind == "causal":
+        return causal()
+    if kind == "window":
+        return sliding_window(tree[1])
+    if kind == "prefix_lm":
+        return prefix_lm(tree[1])
+    if kind == "sink":
+        return sink(tree[1])
+    if kind == "document":
+        key = (id(tree[1]), id(tree[2]))
+        if key not in _cache:
+            qd = torch.as_tensor(tree[1], dtype=torch.int32)
+            kd = qd if tree[2] is tree[1] else torch.as_tensor(tree[2], dtype=torch.int32)
+            if device is not None:
+                qd = qd.to(device)
+                kd = qd if tree[2] is tree[1] else kd.to(device)
+            _cache[key] = (qd, kd, tree[1], tree[2])  # the arrays stay referenced while cached
+        qd, kd = _cache[key][:2]
+        return document(qd, kd)
+    if kind in ("and", "or"):
+        children = [mask_from_tree(c, device, _cache) for c in tree[1:]]
+        return (and_masks if kind == "and" else or_masks)(*children)
+    raise ValueError(f"unknown mask kind {kind!r}")
+
+
+# ------------------------------------------------------------- score mods
+@dataclass(frozen=True)
+class ScoreMod:
+    kind: int
+    value: float = 0.0
+    slopes: torch.Tensor | None = field(default=None, compare=False)
+
+
+def softcap(cap: float) -> ScoreMod:
+    """s -> cap * tanh(s / cap)."""
+    return ScoreMod(SCORE_SOFTCAP, float(cap))
+
+
+def alibi(slopes: torch.Tensor | None = None) -> ScoreMod:
+    """s -> s + m_h * (kv_idx - q_idx); default slopes m_h = 2^(-8(h+1)/Hq)."""
+    return ScoreMod(SCORE_ALIBI, 0.0, slopes)
+
+
+def score_mods_from_list(mods) -> list[ScoreMod]:
+    out = []
+    for m in mods or ():
+        if m[0] == "softcap":
+            out.append(softcap(m[1]))
+        elif m[0] == "alibi":
+            out.append(alibi(None if m[1] is None else torch.as_tensor(m[1], dtype=torch.float32)))
+        else:
+            raise ValueError(f"unknown score mod {m[0]!r}")
+    return out
+
+
+# -------------------------------------------------------------- BlockMask
+@dataclass
+class BlockMask:
+    """Block-sparse mask in the tensorplay.nn.attention BlockMask format."""
+    seq_lengths: tuple[int, int]
+    kv_num_blocks: torch.Tensor
+    kv_indices: torch.Tensor
+    full_kv_num_blocks: torch.Tensor
+    full_kv_indices: torch.Tensor
+    BLOCK_SIZE: tuple[int, int]
+    mask_mod: MaskMod
+
+    @property
+    def shape(self) -> tuple[int, int, int, int]:
+        return tuple(self.kv_indices.shape)
+
+    def _c(self) -> _BlockMask:
+        c = _BlockMask()
+        c.kv_num_blocks = self.kv_num_blocks.data_ptr()
+        c.kv_indices = self.kv_indices.data_ptr()
+        c.full_kv_num_blocks = self.full_kv_num_blocks.data_ptr()
+        c.full_kv_indices = self.full_kv_indices.data_ptr()
+        c.B, c.H, c.QB, c.KB = self.shape
+        c.Q_LEN, c.KV_LEN = self.seq_lengths
+        c.BLOCK_Q, c.BLOCK_KV = self.BLOCK_SIZE
+        return c
+
+    def sparsity(self) -> float:
+        """Percentage of blocks that are not computed (reads the counts back to the host)."""
+        total = self.kv_indices.numel()
+        if total == 0:
+            return 0.0
+        computed = int(self.kv_num_blocks.sum().item()) + int(self.full_kv_num_blocks.sum().item())
+        return 100.0 * (1.0 - computed / total)
+
+
+def _block_pair(BLOCK_SIZE) -> tuple[int, int]:
+    if isinstance(BLOCK_SIZE, int):
+        return BLOCK_SIZE, BLOCK_SIZE
+    return int(BLOCK_SIZE[0]), int(BLOCK_SIZE[1])
+
+
+def create_block_mask(mask_mod: MaskMod, B: int | None, H: int | None, Q_LEN: int, KV_LEN: int,
+                      device="cuda", BLOCK_SIZE: int | tuple[int, int] = 128, out: BlockMask | None = None
+                      ) -> BlockMask:
+    """Build a BlockMask on the GPU (tensorplay.nn.attention, create_block_mask,
+    separate_full_blocks=True). ``out`` reuses the tensors of an earlier BlockMask
+    of the same shape."""
+    device = torch.device(device)
+    bq, bkv = _block_pair(BLOCK_SIZE)
+    Bv = -1 if B is None else int(B)
+    Hv = -1 if H is None else int(H)
+    shape = (ctypes.c_int64 * 4)()
+    _check(_lib.bsmt_block_mask_shape(Bv, Hv, int(Q_LEN), int(KV_LEN), bq, bkv, shape))
+    shp = tuple(int(x) for x in shape)
+    if out is not None and out.shape == shp:
+        t = (out.kv_num_blocks, out.kv_indices, out.full_kv_num_blocks, out.full_kv_indices)
+    else:
+        t = (torch.empty(shp[:3], dtype=torch.int32, device=device),
+             torch.empty(shp, dtype=torch.int32, device=device),
+             torch.empty(shp[:3], dtype=torch.int32, device=device),
+             torch.empty(shp, dtype=torch.int32, device=device))
+    bm = BlockMask((int(Q_LEN), int(KV_LEN)), t[0], t[1], t[2], t[3], (bq, bkv), mask_mod)
+    c = bm._c()
+    with torch.cuda.device(device):
+        spec, keep = mask_mod._spec(device, shp[0])
+        _check(_lib.bsmt_create_block_mask(ctypes.byref(spec), Bv, Hv, int(Q_LEN), int(KV_LEN), bq, bkv,
+                                           ctypes.byref(c), ctypes.c_void_p(_stream_ptr(device))))
+    # the marshalled spec and its device copies of document ids live as long as the mask
+    bm._spec = spec
+    bm._keep = keep
+    return bm
+
+
+def _score_spec(mods, device: torch.device, Hq: int) -> tuple[_ScoreSpec, list]:
+    if mods is None:
+        mods = []
+    elif isinstance(mods, ScoreMod):
+        mods = [mods]
+    mods = list(mods)
+    if len(mods) > MAX_SCORE_OPS:
+        raise ValueError(f"at most {MAX_SCORE_OPS} score mods")
+    spec = _ScoreSpec()
+    spec.num_ops = len(mods)
+    keep = []
+    for i, m in enumerate(mods):
+        spec.ops[i].kind = m.kind
+        spec.ops[i].value = m.value
+        if m.kind == SCORE_ALIBI and m.slopes is not None:
+            s = m.slopes.to(device=device, dtype=torch.float32).contiguous()
+            if s.numel() != Hq:
+                raise ValueError(f"ALiBi slopes: {s.numel()} values for Hq={Hq}")
+            keep.append(s)
+            spec.ops[i].slopes = s.data_ptr()
+    return spec, keep
+
+
+def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask: BlockMask | None = None,
+                   score_mod: ScoreMod | Iterable[ScoreMod] | None = None, scale: float | None = None,
+                   enable_gqa: bool = False, out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
+    """Block-sparse masked attention forward. Returns (out bf16 [B,Hq,M,D], lse fp32 [B,Hq,M])."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be bfloat16 (got {t.dtype})")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be 4-D [B, H, S, D]")
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k and v must be on the same device")
+    B, Hq, M, D = q.shape
+    Bk, Hkv, N, Dk = k.shape
+    if k.shape != v.shape or Bk != B or Dk != D:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    device = q.device
+    if out is None:
+        out = torch.empty((B, Hq, M, D), dtype=torch.bfloat16, device=device)
+    if lse is None:
+        lse = torch.empty((B, Hq, M), dtype=torch.float32, device=device)
+    if out.shape != (B, Hq, M, D) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 [B, Hq, M, D] tensor")
+    if lse.shape != (B, Hq, M) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, M] tensor")
+    with torch.cuda.device(device):
+        sspec, keep_s = _score_spec(score_mod, device, Hq)
+        bm_c = None
+        mspec = None
+        keep_m = []
+        if block_mask is not None:
+            bm_c = block_mask._c()
+            mspec = getattr(block_mask, "_spec", None)
+            if mspec is None:
+                mspec, keep_m = block_mask.mask_mod._spec(device, int(block_mask.shape[0]))
+        _check(_lib.bsmt_flex_attention_fwd(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, M, N, D,
+            ctypes.byref(bm_c) if bm_c is not None else None,
+            ctypes.byref(mspec) if mspec is not None else None,
+            ctypes.byref(sspec), ctypes.c_float(0.0 if scale is None else float(scale)), int(bool(enable_gqa)),
+            out.data_ptr(), lse.data_ptr(), ctypes.c_void_p(_stream_ptr(device))))
+    del keep_s, keep_m
+    return out, lse
+
+
+def check_device_status(device=None) -> None:
+    """Synchronize the current stream and raise if a kernel recorded a device-side error."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    with torch.cuda.device(device):
+        _check(_lib.bsmt_check_device_status(ctypes.c_void_p(_stream_ptr(device))))

@@ -1,0 +1,690 @@
+// Block-sparse masked attention forward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// This is the method of the tensorplay.nn.attention page (BlockMask
+// "Details" items 1-2):
+//   - the kernel visits only the kv blocks a BlockMask row lists;
+//   - it applies mask_mod only on PARTIAL blocks;
+//   - it applies score_mod (attention-gym page: a change to the score
+//     before the softmax) on every visited block.
+// Attention is computed tile by tile with an online softmax and the full
+// score matrix is never written (L-GATr page, "Why care about Attention
+// Kernels?").
+//
+// One persistent CTA per SM. A work unit is (b, hq, pair of adjacent
+// 128-row q-blocks). Warp roles in a CTA:
+//   warps 0-3  softmax for q-block 0 of the pair (one query row per thread)
+//   warps 4-7  softmax for q-block 1
+//   warp 8     TMA producer: Q tiles, then K and V tiles into a ring of slots
+//   warp 9     MMA issuer (one thread): S = Q K^T into TMEM, O += P V with P
+//              read from TMEM
+//   warp 10    scheduler. It merges the two rows' partial and full block
+//              lists into one ascending stream of (kb, tags) in shared
+//              memory, so each K/V tile is loaded once for both q-blocks.
+//
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D)
+// (O1 starts at 256+D when D=64). P (bf16 pairs) overwrites the first 64
+// columns of its S.
+//
+// The MMA order per step n of the union stream is: PV of tile n for q-block
+// 0, S of tile n+1 for q-block 0, then the same for q-block 1. So while one
+// softmax warpgroup works, the tensor core computes the other q-block's
+// products. A tcgen05.commit fires once every earlier MMA of the thread is
+// done. When the softmax sees S(n+1) ready, PV(n) has therefore finished,
+// so O can be rescaled and P can overwrite S without a further barrier.
+//
+// The online softmax is in base 2 with a lazy reference max. O and l are
+// rescaled only when a row's max grows by more than 2^8. The final
+// out = O / l and lse = ln2 * (m_ref + log2 l) do not depend on when the
+// reference moved, so the result is exact.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "mask_dnf.cuh"
+#include "ptx.cuh"
+
+namespace bsmt {
+
+enum ScoreMode : int {
+    kScoreNone = 0,
+    kScoreSoftcap = 1,
+    kScoreAlibi = 2,
+    kScoreSoftcapAlibi = 3,  // softcap, then ALiBi
+    kScoreAlibiSoftcap = 4,  // ALiBi, then softcap
+};
+
+struct AttnParams {
+    int32_t B, Hq, Hkv, M, N, QB, KB, pairs, group;
+    int32_t Bm, Hm;  // BlockMask batch / head extent (1 = broadcast)
+    const int32_t* kv_num;
+    const int32_t* kv_idx;
+    const int32_t* full_num;
+    const int32_t* full_idx;
+    int32_t has_block_mask;
+    int32_t num_units;
+    float scale;       // natural-units softmax scale
+    float scale_log2;  // scale * log2(e)
+    float cap;         // soft-cap
+    float inv_cap;     // 1 / cap
+    const float* slopes;  // ALiBi slopes [Hq] or null (default 2^(-8(h+1)/Hq))
+    __nv_bfloat16* out;
+    float* lse;
+};
+
+constexpr int kThreads = 352;  // 11 warps
+constexpr int kWarpLoad = 8;
+constexpr int kWarpMma = 9;
+constexpr int kWarpSched = 10;
+constexpr int kMaxKB = 1024;   // kv blocks per row supported by the schedule buffer
+constexpr int kRing = 4;       // K/V ring slots (K in even slots, V in odd slots)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;
+
+// Tags of one union entry (bits 16.. of the packed entry).
+constexpr uint32_t kTagIn0 = 1u, kTagIn1 = 2u, kTagPart0 = 4u, kTagPart1 = 8u;
+
+struct SchedHeader {
+    int32_t T;      // union length; -1 marks the end of the work
+    int32_t b, hq, qb0;
+    int32_t n0, n1;  // tiles visited by q-block 0 / 1
+    float slope;     // ALiBi slope of hq (natural units)
+    int32_t pad;
+};
+
+template <int D>
+struct SmemLayout {
+    static constexpr int kTileBytes = 128 * D * 2;          // one 128-row bf16 tile
+    static constexpr int kQ0 = 0;
+    static constexpr int kQ1 = kQ0 + kTileBytes;
+    static constexpr int kRingBase = kQ1 + kTileBytes;
+    static constexpr int kDoc = kRingBase + kRing * kTileBytes;  // 512 B per slot
+    static constexpr int kSched = kDoc + kRing * 512;
+    static constexpr int kSchedEntries = 0;                  // uint32 [kMaxKB]
+    static constexpr int kSchedQdoc = kMaxKB * 4;            // int32 [256]
+    static constexpr int kSchedHeader = kSchedQdoc + 256 * 4;
+    static constexpr int kSchedBytes = kSchedHeader + 64;
+    static constexpr int kFlags = kSched + 2 * kSchedBytes;  // uint8 [kMaxKB]
+    static constexpr int kBars = kFlags + kMaxKB;
+    // barriers (8 bytes each)
+    static constexpr int kBarQFull = 0, kBarQEmpty = 2, kBarSFull = 4, kBarPFull = 6, kBarOFull = 8,
+                         kBarOEmpty = 10, kBarKvFull = 12, kBarKvEmpty = 12 + kRing,
+                         kBarSchedFull = 12 + 2 * kRing, kBarSchedEmpty = 14 + 2 * kRing,
+                         kBarDone = 16 + 2 * kRing, kNumBars = 17 + 2 * kRing;
+    static constexpr int kTmemSlot = kBars + kNumBars * 8;
+    static constexpr int kAbort = kTmemSlot + 4;
+    static constexpr int kTotal = kAbort + 4;
+    static constexpr int kAlloc = kTotal + 1024;  // room to align the base to 1024 B
+};
+
+__device__ __forceinline__ uint32_t sched_entry_kb(uint32_t e) { return e & 0xFFFFu; }
+__device__ __forceinline__ uint32_t sched_entry_tags(uint32_t e) { return e >> 16; }
+
+template <int D, int SCORE>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p, const MaskDnf dnf) {
+    using L = SmemLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * static_cast<uint32_t>(i); };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+
+    // ------------------------------------------------------------ set-up
+    if (warp == kWarpLoad && lane == 0) {
+        mbar_init(bar(L::kBarQFull + 0), 1);
+        mbar_init(bar(L::kBarQFull + 1), 1);
+        mbar_init(bar(L::kBarQEmpty + 0), 1);
+        mbar_init(bar(L::kBarQEmpty + 1), 1);
+        mbar_init(bar(L::kBarSFull + 0), 1);
+        mbar_init(bar(L::kBarSFull + 1), 1);
+        mbar_init(bar(L::kBarPFull + 0), 4);
+        mbar_init(bar(L::kBarPFull + 1), 4);
+        mbar_init(bar(L::kBarOFull + 0), 1);
+        mbar_init(bar(L::kBarOFull + 1), 1);
+        mbar_init(bar(L::kBarOEmpty + 0), 4);
+        mbar_init(bar(L::kBarOEmpty + 1), 4);
+        for (int s = 0; s < kRing; ++s) {
+            // V slots (odd) also take one cp.async arrival per lane for document ids
+            const uint32_t extra = (dnf.has_doc && (s & 1)) ? 32u : 0u;
+            mbar_init(bar(L::kBarKvFull + s), 1 + extra);
+            mbar_init(bar(L::kBarKvEmpty + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(L::kBarSchedFull + s), 32);
+            mbar_init(bar(L::kBarSchedEmpty + s), 1 + 1 + 8);  // load, mma, 8 softmax warps
+        }
+        mbar_init(bar(L::kBarDone), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(sbase + L::kTmemSlot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tm_s[2] = {tmem + 0u, tmem + 128u};
+    const uint32_t tm_o[2] = {tmem + 256u, tmem + 256u + (D == 128 ? 128u : 64u)};
+
+    auto sched_base = [&](int buf) -> uint8_t* { return smem + L::kSched + buf * L::kSchedBytes; };
+
+    if (warp == kWarpSched) {
+        // ================================================= scheduler warp
+        uint8_t* flags = smem + L::kFlags;
+        for (int j = lane; j < kMaxKB; j += 32) flags[j] = 0;
+        __syncwarp();
+        int iter = 0;
+        for (int u = blockIdx.x;; u += gridDim.x, ++iter) {
+            const int buf = iter & 1;
+            const uint32_t use = static_cast<uint32_t>(iter >> 1);
+            if (!mbar_wait(bar(L::kBarSchedEmpty + buf), (use & 1u) ^ 1u, abort_flag)) break;
+            uint8_t* sb = sched_base(buf);
+            SchedHeader* hdr = reinterpret_cast<SchedHeader*>(sb + L::kSchedHeader);
+            uint32_t* entries = reinterpret_cast<uint32_t*>(sb + L::kSchedEntries);
+            if (u >= p.num_units) {
+                if (lane == 0) hdr->T = -1;
+                mbar_arrive(bar(L::kBarSchedFull + buf));
+                break;
+            }
+            // longest-first order: highest q-block pair first, then (b, hq)
+            const int bh_count = p.B * p.Hq;
+            const int pr = p.pairs - 1 - u / bh_count;
+            const int bh = u % bh_count;
+            const int b = bh / p.Hq;
+            const int hq = bh % p.Hq;
+            const int qb0 = 2 * pr;
+            const bool has1 = qb0 + 1 < p.QB;
+            const bool ragged_kv = (p.N & 127) != 0;
+            int T = 0, n0 = 0, n1 = 0;
+            if (!p.has_block_mask) {
+                // every tile of both rows; the tile crossing N is partial
+                for (int c = 0; c < p.KB; c += 32) {
+                    const int kb = c + lane;
+                    if (kb < p.KB) {
+                        const bool part = ragged_kv && kb == p.KB - 1;
+                        uint32_t tags = kTagIn0 | (part ? kTagPart0 : 0u);
+                        if (has1) tags |= kTagIn1 | (part ? kTagPart1 : 0u);
+                        entries[kb] = static_cast<uint32_t>(kb) | (tags << 16);
+                    }
+                }
+                T = p.KB;
+                n0 = p.KB;
+                n1 = has1 ? p.KB : 0;
+            } else {
+                const int bb = p.Bm > 1 ? b : 0;
+                const int hh = p.Hm > 1 ? hq : 0;
+                const int64_t row0 = (static_cast<int64_t>(bb) * p.Hm + hh) * p.QB + qb0;
+                int cnt[4] = {0, 0, 0, 0};
+                const int32_t* lists[4] = {p.kv_idx + row0 * p.KB, p.full_idx + row0 * p.KB,
+                                           p.kv_idx + (row0 + 1) * p.KB, p.full_idx + (row0 + 1) * p.KB};
+                {
+                    int v = 0;
+                    if (lane == 0) v = __ldg(p.kv_num + row0);
+                    if (lane == 1) v = __ldg(p.full_num + row0);
+                    if (has1 && lane == 2) v = __ldg(p.kv_num + row0 + 1);
+                    if (has1 && lane == 3) v = __ldg(p.full_num + row0 + 1);
+                    bool bad = v < 0 || v > p.KB;
+                    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
+                    v = bad ? 0 : v;
+#pragma unroll
+                    for (int l = 0; l < 4; ++l) cnt[l] = __shfl_sync(0xFFFFFFFFu, v, l);
+                }
+                bool bad = false;
+#pragma unroll
+                for (int l = 0; l < 4; ++l) {
+                    for (int j = lane; j < cnt[l]; j += 32) {
+                        const int kb = __ldg(lists[l] + j);
+                        if (kb >= 0 && kb < p.KB) {
+                            flags[kb] |= static_cast<uint8_t>(1u << l);
+                        } else {
+                            bad = true;
+                        }
+                    }
+                    __syncwarp();
+                }
+                if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
+                const uint32_t below = (1u << lane) - 1u;
+                for (int c = 0; c < p.KB; c += 32) {
+                    const int kb = c + lane;
+                    uint32_t f = 0;
+                    if (kb < p.KB) {
+                        f = flags[kb];
+                        flags[kb] = 0;
+                    }
+                    // list bits: 0 partial row0, 1 full row0, 2 partial row1, 3 full row1.
+                    // A block listed as both partial and full is treated as partial.
+                    uint32_t tags = 0;
+                    if (f & 3u) tags |= kTagIn0 | ((f & 1u) ? kTagPart0 : 0u);
+                    if (f & 12u) tags |= kTagIn1 | ((f & 4u) ? kTagPart1 : 0u);
+                    if (ragged_kv && kb == p.KB - 1 && tags) {
+                        if (tags & kTagIn0) tags |= kTagPart0;
+                        if (tags & kTagIn1) tags |= kTagPart1;
+                    }
+                    const unsigned bal = __ballot_sync(0xFFFFFFFFu, tags != 0);
+                    if (tags) entries[T + __popc(bal & below)] = static_cast<uint32_t>(kb) | (tags << 16);
+                    T += __popc(bal);
+                    n0 += __popc(__ballot_sync(0xFFFFFFFFu, (tags & kTagIn0) != 0));
+                    n1 += __popc(__ballot_sync(0xFFFFFFFFu, (tags & kTagIn1) != 0));
+                }
+            }
+            if (dnf.has_doc && p.has_block_mask) {
+                const int db = dnf.doc_batch > 1 ? b : 0;
+                int32_t* qdoc = reinterpret_cast<int32_t*>(sb + L::kSchedQdoc);
+                for (int r = lane; r < 256; r += 32) {
+                    const int64_t q = static_cast<int64_t>(qb0) * 128 + r;
+                    qdoc[r] = q < p.M ? __ldg(dnf.q_doc + static_cast<int64_t>(db) * p.M + q) : 0;
+                }
+            }
+            if (lane == 0) {
+                hdr->T = T;
+                hdr->b = b;
+                hdr->hq = hq;
+                hdr->qb0 = qb0;
+                hdr->n0 = n0;
+                hdr->n1 = n1;
+                float slope = 0.f;
+                if (SCORE == kScoreAlibi || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap)
+                    slope = p.slopes ? __ldg(p.slopes + hq) : exp2f(-8.0f * static_cast<float>(hq + 1) / static_cast<float>(p.Hq));
+                hdr->slope = slope;
+            }
+            __syncwarp();
+            mbar_arrive(bar(L::kBarSchedFull + buf));
+        }
+    } else if (warp == kWarpLoad) {
+        // ================================================= TMA producer warp
+        uint32_t kv_pos = 0;  // ring positions used so far
+        uint32_t q_uses[2] = {0, 0};
+        const uint32_t tile_bytes = L::kTileBytes;
+        const uint64_t pol_kv = l2_policy_evict_last();
+        const uint64_t pol_q = l2_policy_evict_first();
+        for (int iter = 0;; ++iter) {
+            const int buf = iter & 1;
+            if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) break;
+            const uint8_t* sb = sched_base(buf);
+            const SchedHeader hdr = *reinterpret_cast<const SchedHeader*>(sb + L::kSchedHeader);
+            if (hdr.T < 0) break;
+            const uint32_t* entries = reinterpret_cast<const uint32_t*>(sb + L::kSchedEntries);
+            const int hkv = hdr.hq / p.group;
+            const int zq = hdr.b * p.Hq + hdr.hq;
+            const int zkv = hdr.b * p.Hkv + hkv;
+            bool ok = true;
+            for (int i = 0; i < 2 && ok; ++i) {
+                const int ni = i == 0 ? hdr.n0 : hdr.n1;
+                if (ni == 0) continue;
+                if (q_uses[i] > 0) {
+                    ok = mbar_wait(bar(L::kBarQEmpty + i), (q_uses[i] - 1) & 1u, abort_flag);
+                    if (!ok) break;
+                }
+                ++q_uses[i];
+                if (lane == 0) {
+                    const uint32_t qb_bar = bar(L::kBarQFull + i);
+                    mbar_arrive_expect_tx(qb_bar, tile_bytes);
+                    const uint32_t dst = sbase + (i == 0 ? L::kQ0 : L::kQ1);
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_3d_hint(dst + h * 16384, &tm_q, h * 64, (hdr.qb0 + i) * 128, zq, qb_bar, pol_q);
+                }
+            }
+            if (!ok) break;
+            const int64_t doc_row = dnf.has_doc ? static_cast<int64_t>(dnf.doc_batch > 1 ? hdr.b : 0) * p.N : 0;
+            for (int n = 0; n < hdr.T && ok; ++n) {
+                const int kb = static_cast<int>(sched_entry_kb(entries[n]));
+#pragma unroll
+                for (int kv = 0; kv < 2; ++kv) {  // 0 = K, 1 = V
+                    const uint32_t s = kv_pos % kRing;
+                    const uint32_t round = kv_pos / kRing;
+                    if (!mbar_wait(bar(L::kBarKvEmpty + s), (round & 1u) ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = bar(L::kBarKvFull + s);
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(fb, tile_bytes);
+                        const uint32_t dst = sbase + L::kRingBase + s * L::kTileBytes;
+#pragma unroll
+                        for (int h = 0; h < D / 64; ++h)
+                            tma_load_3d_hint(dst + h * 16384, kv == 0 ? &tm_k : &tm_v, h * 64, kb * 128, zkv, fb,
+                                             pol_kv);
+                    }
+                    if (kv == 1 && dnf.has_doc) {
+                        const uint32_t ddst = sbase + L::kDoc + s * 512 + lane * 16;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int64_t pos = static_cast<int64_t>(kb) * 128 + lane * 4 + k;
+                            const bool in = pos < p.N;
+                            cp_async_4(ddst + 4 * k, dnf.kv_doc + doc_row + (in ? pos : 0), in ? 4u : 0u);
+                        }
+                        cp_async_mbar_arrive_noinc(fb);
+                    }
+                    ++kv_pos;
+                }
+            }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
+        }
+    } else if (warp == kWarpMma) {
+        // ================================================= MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+            uint32_t g = 0;  // union entries consumed so far (K at ring pos 2g, V at 2g+1)
+            uint32_t q_full_uses[2] = {0, 0}, o_units[2] = {0, 0}, p_waits[2] = {0, 0};
+            bool ok = true;
+            for (int iter = 0; ok; ++iter) {
+                const int buf = iter & 1;
+                if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) break;
+                const uint8_t* sb = sched_base(buf);
+                const SchedHeader hdr = *reinterpret_cast<const SchedHeader*>(sb + L::kSchedHeader);
+                if (hdr.T < 0) break;
+                const uint32_t* entries = reinterpret_cast<const uint32_t*>(sb + L::kSchedEntries);
+                const int nlist[2] = {hdr.n0, hdr.n1};
+                int s_issued[2] = {0, 0}, pv_issued[2] = {0, 0};
+
+                auto kslot = [&](uint32_t gg) { return (2u * gg) % kRing; };
+                auto vslot = [&](uint32_t gg) { return (2u * gg + 1u) % kRing; };
+                auto kphase = [&](uint32_t gg) { return ((2u * gg) / kRing) & 1u; };
+                auto vphase = [&](uint32_t gg) { return ((2u * gg + 1u) / kRing) & 1u; };
+
+                auto issue_s = [&](int i, uint32_t slot) -> bool {
+                    if (s_issued[i] == 0) {
+                        if (!mbar_wait(bar(L::kBarQFull + i), q_full_uses[i] & 1u, abort_flag)) return false;
+                        ++q_full_uses[i];
+                    }
+                    tc_fence_after();
+                    const uint32_t qa = sbase + (i == 0 ? L::kQ0 : L::kQ1);
+                    const uint32_t ka = sbase + L::kRingBase + slot * L::kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                        mma_ss(tm_s[i], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_s,
+                               kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(L::kBarSFull + i));
+                    if (++s_issued[i] == nlist[i]) mma_commit(bar(L::kBarQEmpty + i));
+                    return true;
+                };
+                auto issue_pv = [&](int i, uint32_t slot) -> bool {
+                    if (pv_issued[i] == 0 && o_units[i] > 0) {
+                        if (!mbar_wait(bar(L::kBarOEmpty + i), (o_units[i] - 1) & 1u, abort_flag)) return false;
+                    }
+                    if (!mbar_wait(bar(L::kBarPFull + i), p_waits[i] & 1u, abort_flag)) return false;
+                    ++p_waits[i];
+                    tc_fence_after();
+                    const uint32_t va = sbase + L::kRingBase + slot * L::kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        mma_ts(tm_o[i], tm_s[i] + 8u * kk, sdesc_sw128(va + kk * 2048u, 16384, 1024), idesc_pv,
+                               (pv_issued[i] > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    if (++pv_issued[i] == nlist[i]) {
+                        mma_commit(bar(L::kBarOFull + i));
+                        ++o_units[i];
+                    }
+                    return true;
+                };
+
+                const int T = hdr.T;
+                if (T > 0) {
+                    const uint32_t e0 = entries[0];
+                    if (!mbar_wait(bar(L::kBarKvFull + kslot(g)), kphase(g), abort_flag)) break;
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+                        if ((sched_entry_tags(e0) >> i) & 1u) ok = ok && issue_s(i, kslot(g));
+                    if (!ok) break;
+                    mma_commit(bar(L::kBarKvEmpty + kslot(g)));
+                }
+                for (int n = 0; n < T && ok; ++n) {
+                    const uint32_t gg = g + static_cast<uint32_t>(n);
+                    const uint32_t e = entries[n];
+                    const bool has_next = n + 1 < T;
+                    const uint32_t e1 = has_next ? entries[n + 1] : 0u;
+                    if (!mbar_wait(bar(L::kBarKvFull + vslot(gg)), vphase(gg), abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (has_next && !mbar_wait(bar(L::kBarKvFull + kslot(gg + 1)), kphase(gg + 1), abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        if ((sched_entry_tags(e) >> i) & 1u) ok = ok && issue_pv(i, vslot(gg));
+                        if (ok && has_next && ((sched_entry_tags(e1) >> i) & 1u)) ok = issue_s(i, kslot(gg + 1));
+                    }
+                    if (!ok) break;
+                    mma_commit(bar(L::kBarKvEmpty + vslot(gg)));
+                    if (has_next) mma_commit(bar(L::kBarKvEmpty + kslot(gg + 1)));
+                }
+                if (!ok) break;
+                g += static_cast<uint32_t>(T);
+                mbar_arrive(bar(L::kBarSchedEmpty + buf));
+            }
+            // all MMAs issued by this thread must finish before TMEM is freed
+            mma_commit(bar(L::kBarDone));
+            mbar_wait(bar(L::kBarDone), 0, abort_flag);
+        }
+        __syncwarp();
+    } else if (warp < 8) {
+        // ================================================= softmax warpgroups
+        const int i = warp >> 2;              // q-block of the pair
+        const int r = threadIdx.x & 127;      // row within the q-block
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t t_s = tm_s[i] + lane_base;
+        const uint32_t t_o = tm_o[i] + lane_base;
+        uint32_t g = 0;
+        uint32_t s_waits = 0, o_waits = 0;
+        bool ok = true;
+        for (int iter = 0; ok; ++iter) {
+            const int buf = iter & 1;
+            if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) break;
+            const uint8_t* sb = sched_base(buf);
+            const SchedHeader hdr = *reinterpret_cast<const SchedHeader*>(sb + L::kSchedHeader);
+            if (hdr.T < 0) break;
+            const uint32_t* entries = reinterpret_cast<const uint32_t*>(sb + L::kSchedEntries);
+            const int ni = i == 0 ? hdr.n0 : hdr.n1;
+            const int qb = hdr.qb0 + i;
+            const int q = qb * 128 + r;
+            const bool row_valid = qb < p.QB && q < p.M;
+            const int32_t qd = dnf.has_doc ? reinterpret_cast<const int32_t*>(sb + L::kSchedQdoc)[i * 128 + r] : 0;
+            const float sl2 = hdr.slope * kLog2e;
+            float m_ref = -INFINITY;
+            float l_sum = 0.f;
+            int processed = 0;
+            for (int n = 0; n < hdr.T; ++n) {
+                const uint32_t e = entries[n];
+                const uint32_t tags = sched_entry_tags(e);
+                if (!((tags >> i) & 1u)) continue;
+                const int kb = static_cast<int>(sched_entry_kb(e));
+                const bool partial = (tags >> (2 + i)) & 1u;
+                if (!mbar_wait(bar(L::kBarSFull + i), s_waits & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                ++s_waits;
+                tc_fence_after();
+                float x[128];
+                {
+                    uint32_t* xr = reinterpret_cast<uint32_t*>(x);
+                    tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(xr + 0));
+                    tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32));
+                    tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(xr + 64));
+                    tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(xr + 96));
+                    tc_wait_ld();
+                }
+                // score_mod on every visited tile, in base-2 units
+                const float tile_bias = sl2 * static_cast<float>(kb * 128 - q);
+#pragma unroll
+                for (int j = 0; j < 128; ++j) {
+                    float s = x[j];
+                    if constexpr (SCORE == kScoreNone) {
+                        s = s * p.scale_log2;
+                    } else if constexpr (SCORE == kScoreSoftcap) {
+                        s = (p.cap * kLog2e) * tanh_approx(s * (p.scale * p.inv_cap));
+                    } else if constexpr (SCORE == kScoreAlibi) {
+                        s = fmaf(s, p.scale_log2, fmaf(sl2, static_cast<float>(j), tile_bias));
+                    } else if constexpr (SCORE == kScoreSoftcapAlibi) {
+                        s = fmaf((p.cap * kLog2e), tanh_approx(s * (p.scale * p.inv_cap)),
+                                 fmaf(sl2, static_cast<float>(j), tile_bias));
+                    } else {
+                        const float t = fmaf(s, p.scale, hdr.slope * static_cast<float>(kb * 128 + j - q));
+                        s = (p.cap * kLog2e) * tanh_approx(t * p.inv_cap);
+                    }
+                    x[j] = s;
+                }
+                // mask_mod on partial tiles only
+                if (partial) {
+                    const int64_t c0 = static_cast<int64_t>(kb) * 128;
+                    const int64_t c1 = (c0 + 127 < p.N - 1) ? c0 + 127 : p.N - 1;
+                    int64_t ds = 0, de = -1;
+                    if (dnf.has_doc && p.has_block_mask) {
+                        const uint32_t vs = (2u * (g + static_cast<uint32_t>(n)) + 1u) % kRing;
+                        const uint32_t vph = ((2u * (g + static_cast<uint32_t>(n)) + 1u) / kRing) & 1u;
+                        if (!mbar_wait(bar(L::kBarKvFull + vs), vph, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const int32_t* dv = reinterpret_cast<const int32_t*>(smem + L::kDoc + vs * 512);
+                        const int cnt = static_cast<int>(c1 - c0 + 1);
+                        // [first, past) of qd among dv[0..cnt) (non-decreasing)
+                        int a = 0, bnd = cnt;
+                        while (a < bnd) {
+                            const int mid = (a + bnd) >> 1;
+                            if (dv[mid] < qd) a = mid + 1; else bnd = mid;
+                        }
+                        int a2 = a, b2 = cnt;
+                        while (a2 < b2) {
+                            const int mid = (a2 + b2) >> 1;
+                            if (dv[mid] <= qd) a2 = mid + 1; else b2 = mid;
+                        }
+                        ds = c0 + a;
+                        de = c0 + a2 - 1;
+                    }
+                    uint32_t w[4] = {0u, 0u, 0u, 0u};
+                    if (p.has_block_mask) {
+                        for (int t = 0; t < dnf.n_terms; ++t) {
+                            int64_t lo, hi;
+                            term_interval(dnf, t, q, c0, c1, ds, de, lo, hi);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) w[k] |= range_bits(lo, hi, c0 + 32 * k);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) w[k] = range_bits(c0, c1, c0 + 32 * k);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 128; ++j)
+                        if (!((w[j >> 5] >> (j & 31)) & 1u)) x[j] = -INFINITY;
+                }
+                // row max
+                float mt = x[0];
+#pragma unroll
+                for (int j = 1; j < 128; ++j) mt = fmaxf(mt, x[j]);
+                // lazy reference update
+                bool need_rescale = false;
+                float alpha = 1.f;
+                if (mt > m_ref + kRescaleThreshold) {  // false while mt is -inf
+                    if (m_ref != -INFINITY) {
+                        alpha = ex2_approx(m_ref - mt);
+                        need_rescale = processed > 0;
+                    }
+                    l_sum *= alpha;
+                    m_ref = mt;
+                }
+                const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+                float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float p0 = ex2_approx(x[32 * c + 2 * j] - m_use);
+                        const float p1 = ex2_approx(x[32 * c + 2 * j + 1] - m_use);
+                        part[c] += p0 + p1;
+                        pk[j] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(t_s + 16 * c, pk);
+                }
+                l_sum += (part[0] + part[1]) + (part[2] + part[3]);
+                // O rescale after P is out of registers (lower register peak)
+                if (__any_sync(0xFFFFFFFFu, need_rescale)) {
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(t_o + 32 * c, o);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        tmem_st32(t_o + 32 * c, o);
+                    }
+                }
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::kBarPFull + i));
+                ++processed;
+            }
+            if (!ok) break;
+            // epilogue: out = O / l, lse = ln2 * (m + log2 l)
+            __nv_bfloat16* orow = p.out + ((static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.M + q) * D;
+            const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            if (ni > 0) {
+                if (!mbar_wait(bar(L::kBarOFull + i), o_waits & 1u, abort_flag)) break;
+                ++o_waits;
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(t_o + 32 * c, o);
+                    tc_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        pk[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv_l, __uint_as_float(o[2 * j + 1]) * inv_l);
+                    if (row_valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::kBarOEmpty + i));
+            } else if (row_valid) {
+                uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+                for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (row_valid) {
+                const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+                p.lse[(static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.M + q] =
+                    l_sum > 0.f ? (m_use + __log2f(l_sum)) * kLn2 : -INFINITY;
+            }
+            g += static_cast<uint32_t>(hdr.T);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
+        }
+    }
+
+    // ------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace bsmt

@@ -1,0 +1,487 @@
+// libbsmt: the C ABI declared in include/bsmt.h.
+//
+// Host side: argument checks, conversion of the postfix mask program into
+// OR-of-AND form, TMA descriptor encoding and kernel launches. Nothing here
+// allocates device memory and nothing synchronizes, except
+// bsmt_check_device_status.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "attn_fwd.cuh"
+#include "bsmt.h"
+#include "mask_build.cuh"
+#include "mask_dnf.cuh"
+#include "ptx.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+bsmt_status fail(bsmt_status code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+bsmt_status ok() {
+    g_last_error.clear();
+    return BSMT_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int64_t kMaxLen = (int64_t(1) << 31) - 256;
+
+// ------------------------------------------------------------------ DNF
+struct Dnf {
+    std::vector<std::vector<bsmt::DnfLeaf>> terms;
+};
+
+bsmt_status build_dnf(const bsmt_mask_spec* spec, int64_t B, bsmt::MaskDnf* out) {
+    std::memset(out, 0, sizeof(*out));
+    if (spec == nullptr) {  // NOOP
+        out->n_terms = 1;
+        out->term_begin[0] = 0;
+        out->term_begin[1] = 0;
+        return BSMT_OK;
+    }
+    if (spec->num_nodes < 1 || spec->num_nodes > BSMT_MAX_MASK_NODES)
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: num_nodes=%d outside [1, %d]", spec->num_nodes,
+                    BSMT_MAX_MASK_NODES);
+    std::vector<Dnf> stack;
+    bool has_doc = false;
+    auto too_big = [](const Dnf& d) {
+        size_t leaves = 0;
+        for (auto& t : d.terms) leaves += t.size();
+        return d.terms.size() > size_t(bsmt::kMaxTerms) || leaves > size_t(bsmt::kMaxLeaves);
+    };
+    for (int i = 0; i < spec->num_nodes; ++i) {
+        const bsmt_mask_node nd = spec->nodes[i];
+        switch (nd.kind) {
+            case BSMT_MASK_NOOP:
+                stack.push_back(Dnf{{{}}});
+                break;
+            case BSMT_MASK_CAUSAL:
+            case BSMT_MASK_WINDOW:
+            case BSMT_MASK_PREFIX_LM:
+            case BSMT_MASK_SINK:
+            case BSMT_MASK_DOCUMENT:
+                if (nd.kind == BSMT_MASK_DOCUMENT) has_doc = true;
+                stack.push_back(Dnf{{{bsmt::DnfLeaf{nd.kind, nd.arg}}}});
+                break;
+            case BSMT_MASK_AND:
+            case BSMT_MASK_OR: {
+                if (nd.arg < 1 || size_t(nd.arg) > stack.size())
+                    return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: node %d (%s) takes %d operands, %zu available", i,
+                                nd.kind == BSMT_MASK_AND ? "AND" : "OR", nd.arg, stack.size());
+                std::vector<Dnf> ops(stack.end() - nd.arg, stack.end());
+                stack.resize(stack.size() - nd.arg);
+                Dnf res;
+                if (nd.kind == BSMT_MASK_OR) {
+                    for (auto& d : ops)
+                        for (auto& t : d.terms) res.terms.push_back(t);
+                } else {
+                    res.terms = {{}};
+                    for (auto& d : ops) {
+                        Dnf nxt;
+                        for (auto& a : res.terms)
+                            for (auto& b : d.terms) {
+                                auto t = a;
+                                t.insert(t.end(), b.begin(), b.end());
+                                nxt.terms.push_back(std::move(t));
+                            }
+                        res = std::move(nxt);
+                        if (too_big(res)) break;
+                    }
+                }
+                if (too_big(res))
+                    return fail(BSMT_ERR_UNSUPPORTED,
+                                "mask spec: more than %d alternatives or %d leaves after distributing AND over OR",
+                                bsmt::kMaxTerms, bsmt::kMaxLeaves);
+                stack.push_back(std::move(res));
+                break;
+            }
+            default:
+                return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: node %d has unknown kind %d", i, nd.kind);
+        }
+    }
+    if (stack.size() != 1)
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: program leaves %zu values (expected 1)", stack.size());
+    if (has_doc) {
+        if (spec->q_doc_ids == nullptr || spec->kv_doc_ids == nullptr)
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: DOCUMENT needs q_doc_ids and kv_doc_ids");
+        if (!aligned(spec->q_doc_ids, 4) || !aligned(spec->kv_doc_ids, 4))
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: document id arrays must be 4-byte aligned");
+        if (!(spec->doc_batch == 1 || spec->doc_batch == B))
+            return fail(BSMT_ERR_SHAPE_MISMATCH, "mask spec: doc_batch=%d must be 1 or B=%lld", spec->doc_batch,
+                        static_cast<long long>(B));
+    }
+    const Dnf& d = stack[0];
+    out->n_terms = static_cast<int32_t>(d.terms.size());
+    int pos = 0;
+    for (size_t t = 0; t < d.terms.size(); ++t) {
+        out->term_begin[t] = pos;
+        for (auto& lf : d.terms[t]) {
+            if (lf.kind == BSMT_MASK_NOOP) continue;
+            if (lf.kind == BSMT_MASK_DOCUMENT) out->term_has_doc |= 1u << t;
+            out->leaves[pos++] = lf;
+        }
+    }
+    out->term_begin[d.terms.size()] = pos;
+    out->has_doc = has_doc ? 1 : 0;
+    out->q_doc = spec->q_doc_ids;
+    out->kv_doc = spec->kv_doc_ids;
+    out->doc_batch = spec->doc_batch < 1 ? 1 : spec->doc_batch;
+    return BSMT_OK;
+}
+
+// ------------------------------------------------------------- device info
+std::mutex g_mu;
+int g_sm_count[64] = {0};
+bool g_attr_set[64][16] = {{false}};
+
+bsmt_status sm_count(int* dev_out, int* n_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= 64) return fail(BSMT_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_sm_count[dev] == 0) {
+        int major = 0, minor = 0, n = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+        if (major != 10 || minor != 0)
+            return fail(BSMT_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a (B200)", dev,
+                        major, minor);
+        g_sm_count[dev] = n;
+    }
+    *dev_out = dev;
+    *n_out = g_sm_count[dev];
+    return BSMT_OK;
+}
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bsmt_status get_encoder(EncodeTiledFn* fn) {
+    static EncodeTiledFn cached = nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (cached == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
+        if (e != cudaSuccess || ptr == nullptr || q != cudaDriverEntryPointSuccess)
+            return fail(BSMT_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+        cached = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    *fn = cached;
+    return BSMT_OK;
+}
+
+// bf16 tensor [BH, S, D] as a 3-D map with 64 x 128 x 1 boxes and 128-byte swizzle.
+bsmt_status encode_bhsd(EncodeTiledFn enc, CUtensorMap* map, const void* base, int64_t BH, int64_t S, int64_t D) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D * 2), static_cast<cuuint64_t>(S * D * 2)};
+    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(BSMT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return BSMT_OK;
+}
+
+// Rows with no allowed key: out = 0, lse = -inf (used when KV_LEN == 0).
+__global__ void fill_empty_kernel(uint4* out, int64_t out_vec, float* lse, int64_t rows) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < out_vec; i += stride)
+        out[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < rows; i += stride)
+        lse[i] = -INFINITY;
+}
+
+template <int D, int SCORE>
+bsmt_status launch_attn(int dev, int nsm, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const bsmt::AttnParams& p, const bsmt::MaskDnf& dnf, cudaStream_t stream) {
+    auto kern = bsmt::attn_fwd_kernel<D, SCORE>;
+    const int smem = bsmt::SmemLayout<D>::kAlloc;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        const int slot = (D == 128 ? 8 : 0) + SCORE;
+        if (!g_attr_set[dev][slot]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+            g_attr_set[dev][slot] = true;
+        }
+    }
+    const int grid = p.num_units < nsm ? p.num_units : nsm;
+    kern<<<grid, bsmt::kThreads, smem, stream>>>(tq, tk, tv, p, dnf);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
+    return BSMT_OK;
+}
+
+template <int D>
+bsmt_status launch_attn_score(int score, int dev, int nsm, const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv, const bsmt::AttnParams& p, const bsmt::MaskDnf& dnf,
+                              cudaStream_t s) {
+    switch (score) {
+        case bsmt::kScoreNone: return launch_attn<D, bsmt::kScoreNone>(dev, nsm, tq, tk, tv, p, dnf, s);
+        case bsmt::kScoreSoftcap: return launch_attn<D, bsmt::kScoreSoftcap>(dev, nsm, tq, tk, tv, p, dnf, s);
+        case bsmt::kScoreAlibi: return launch_attn<D, bsmt::kScoreAlibi>(dev, nsm, tq, tk, tv, p, dnf, s);
+        case bsmt::kScoreSoftcapAlibi:
+            return launch_attn<D, bsmt::kScoreSoftcapAlibi>(dev, nsm, tq, tk, tv, p, dnf, s);
+        default: return launch_attn<D, bsmt::kScoreAlibiSoftcap>(dev, nsm, tq, tk, tv, p, dnf, s);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t bsmt_version(void) { return (1 << 16) | 0; }
+
+const char* bsmt_last_error(void) { return g_last_error.c_str(); }
+
+bsmt_status bsmt_block_mask_shape(int64_t B, int64_t H, int64_t Q_LEN, int64_t KV_LEN, int32_t BLOCK_Q,
+                                  int32_t BLOCK_KV, int64_t out_shape[4]) {
+    if (out_shape == nullptr) return fail(BSMT_ERR_INVALID_ARGUMENT, "out_shape is NULL");
+    if (BLOCK_Q != 128 || BLOCK_KV != 128)
+        return fail(BSMT_ERR_UNSUPPORTED, "BLOCK_SIZE (%d, %d): only 128 x 128 blocks are supported", BLOCK_Q, BLOCK_KV);
+    if (Q_LEN < 0 || KV_LEN < 0 || Q_LEN > kMaxLen || KV_LEN > kMaxLen)
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "Q_LEN=%lld KV_LEN=%lld outside [0, %lld]", static_cast<long long>(Q_LEN),
+                    static_cast<long long>(KV_LEN), static_cast<long long>(kMaxLen));
+    out_shape[0] = B > 0 ? B : 1;
+    out_shape[1] = H > 0 ? H : 1;
+    out_shape[2] = (Q_LEN + BLOCK_Q - 1) / BLOCK_Q;
+    out_shape[3] = (KV_LEN + BLOCK_KV - 1) / BLOCK_KV;
+    return ok();
+}
+
+bsmt_status bsmt_create_block_mask(const bsmt_mask_spec* spec, int64_t B, int64_t H, int64_t Q_LEN, int64_t KV_LEN,
+                                   int32_t BLOCK_Q, int32_t BLOCK_KV, bsmt_block_mask* out, void* stream) {
+    int64_t shape[4];
+    bsmt_status st = bsmt_block_mask_shape(B, H, Q_LEN, KV_LEN, BLOCK_Q, BLOCK_KV, shape);
+    if (st != BSMT_OK) return st;
+    if (spec == nullptr) return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec is NULL");
+    if (out == nullptr) return fail(BSMT_ERR_INVALID_ARGUMENT, "block mask output is NULL");
+    if (shape[0] > 65535) return fail(BSMT_ERR_UNSUPPORTED, "B=%lld above 65535", static_cast<long long>(shape[0]));
+    if (shape[1] > (int64_t(1) << 20)) return fail(BSMT_ERR_UNSUPPORTED, "H=%lld too large", static_cast<long long>(shape[1]));
+    const int64_t rows = shape[0] * shape[1] * shape[2];
+    if (rows > 0) {
+        if (!out->kv_num_blocks || !out->full_kv_num_blocks || (shape[3] > 0 && (!out->kv_indices || !out->full_kv_indices)))
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "block mask output pointers must be non-NULL");
+        if (!aligned(out->kv_num_blocks, 4) || !aligned(out->kv_indices, 4) || !aligned(out->full_kv_num_blocks, 4) ||
+            !aligned(out->full_kv_indices, 4))
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "block mask output pointers must be 4-byte aligned");
+    }
+    bsmt::MaskDnf dnf;
+    st = build_dnf(spec, shape[0], &dnf);
+    if (st != BSMT_OK) return st;
+    int dev = 0, nsm = 0;
+    if (rows > 0) {
+        st = sm_count(&dev, &nsm);
+        if (st != BSMT_OK) return st;
+    }
+    out->B = static_cast<int32_t>(shape[0]);
+    out->H = static_cast<int32_t>(shape[1]);
+    out->QB = static_cast<int32_t>(shape[2]);
+    out->KB = static_cast<int32_t>(shape[3]);
+    out->Q_LEN = static_cast<int32_t>(Q_LEN);
+    out->KV_LEN = static_cast<int32_t>(KV_LEN);
+    out->BLOCK_Q = BLOCK_Q;
+    out->BLOCK_KV = BLOCK_KV;
+    if (rows == 0) return ok();
+
+    bsmt::BuildParams p;
+    p.Bm = out->B;
+    p.Hm = out->H;
+    p.Q_LEN = out->Q_LEN;
+    p.KV_LEN = out->KV_LEN;
+    p.QB = out->QB;
+    p.KB = out->KB;
+    p.kv_num = out->kv_num_blocks;
+    p.kv_idx = out->kv_indices;
+    p.full_num = out->full_kv_num_blocks;
+    p.full_idx = out->full_kv_indices;
+    const int64_t gx = (p.QB + bsmt::kBuildWarps - 1) / bsmt::kBuildWarps;
+    const int64_t blocks_xy = gx * p.Bm;
+    int64_t groups = (2 * nsm + blocks_xy - 1) / blocks_xy;
+    if (groups < 1) groups = 1;
+    if (groups > p.Hm) groups = p.Hm;
+    p.heads_per_block = static_cast<int32_t>((p.Hm + groups - 1) / groups);
+    groups = (p.Hm + p.heads_per_block - 1) / p.heads_per_block;
+    if (gx > 0x7FFFFFFF || groups > 65535) return fail(BSMT_ERR_UNSUPPORTED, "grid too large");
+    dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(p.Bm), static_cast<unsigned>(groups));
+    bsmt::mask_build_kernel<<<grid, bsmt::kBuildWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(dnf, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "mask builder launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v, int64_t B, int64_t Hq, int64_t Hkv,
+                                    int64_t M, int64_t N, int64_t D, const bsmt_block_mask* bm,
+                                    const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score, float scale,
+                                    int32_t enable_gqa, void* out, float* lse, void* stream) {
+    if (B < 0 || Hq < 0 || Hkv < 0 || M < 0 || N < 0)
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "negative size (B=%lld Hq=%lld Hkv=%lld M=%lld N=%lld)",
+                    static_cast<long long>(B), static_cast<long long>(Hq), static_cast<long long>(Hkv),
+                    static_cast<long long>(M), static_cast<long long>(N));
+    if (D != 64 && D != 128) return fail(BSMT_ERR_UNSUPPORTED, "head dim D=%lld (supported: 64, 128)", static_cast<long long>(D));
+    if (Hkv < 1 || Hq < 1) return fail(BSMT_ERR_SHAPE_MISMATCH, "Hq=%lld and Hkv=%lld must be >= 1", static_cast<long long>(Hq), static_cast<long long>(Hkv));
+    if (Hq % Hkv != 0)
+        return fail(BSMT_ERR_SHAPE_MISMATCH, "Hq=%lld is not a multiple of Hkv=%lld", static_cast<long long>(Hq),
+                    static_cast<long long>(Hkv));
+    if (Hq != Hkv && !enable_gqa)
+        return fail(BSMT_ERR_SHAPE_MISMATCH, "Hq=%lld != Hkv=%lld requires enable_gqa", static_cast<long long>(Hq),
+                    static_cast<long long>(Hkv));
+    if (M > kMaxLen || N > kMaxLen) return fail(BSMT_ERR_UNSUPPORTED, "sequence length above %lld", static_cast<long long>(kMaxLen));
+    if (B * Hq > 0x7FFFFFFF || B * Hkv > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "B*H above 2^31");
+    const int64_t QB = (M + 127) / 128, KB = (N + 127) / 128;
+    if (KB > bsmt::kMaxKB)
+        return fail(BSMT_ERR_UNSUPPORTED, "KV_LEN=%lld: at most %d kv blocks per row", static_cast<long long>(N), bsmt::kMaxKB);
+    if (!q || !k || !v || !out || !lse) return fail(BSMT_ERR_INVALID_ARGUMENT, "q, k, v, out and lse must be non-NULL");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "q, k, v and out must be 16-byte aligned");
+    if (!aligned(lse, 4)) return fail(BSMT_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
+    if (std::isnan(scale) || std::isinf(scale)) return fail(BSMT_ERR_INVALID_ARGUMENT, "scale must be finite");
+    if (scale <= 0.f) scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+
+    // score mods -> compile-time mode
+    int mode = bsmt::kScoreNone;
+    float cap = 1.f;
+    const float* slopes = nullptr;
+    if (score != nullptr) {
+        if (score->num_ops < 0 || score->num_ops > BSMT_MAX_SCORE_OPS)
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: num_ops=%d outside [0, %d]", score->num_ops, BSMT_MAX_SCORE_OPS);
+        int kinds[2] = {0, 0};
+        int nk = 0;
+        for (int i = 0; i < score->num_ops; ++i) {
+            const bsmt_score_op& op = score->ops[i];
+            if (op.kind == BSMT_SCORE_NONE) continue;
+            if (op.kind == BSMT_SCORE_SOFTCAP) {
+                if (!(op.value > 0.f) || std::isinf(op.value))
+                    return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: soft-cap must be finite and > 0");
+                cap = op.value;
+            } else if (op.kind == BSMT_SCORE_ALIBI) {
+                if (op.slopes && !aligned(op.slopes, 4))
+                    return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: ALiBi slopes must be 4-byte aligned");
+                slopes = op.slopes;
+            } else {
+                return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: unknown kind %d", op.kind);
+            }
+            if (nk == 1 && kinds[0] == op.kind)
+                return fail(BSMT_ERR_UNSUPPORTED, "score spec: the same score mod twice");
+            kinds[nk++] = op.kind;
+        }
+        if (nk == 1) mode = kinds[0] == BSMT_SCORE_SOFTCAP ? bsmt::kScoreSoftcap : bsmt::kScoreAlibi;
+        if (nk == 2) mode = kinds[0] == BSMT_SCORE_SOFTCAP ? bsmt::kScoreSoftcapAlibi : bsmt::kScoreAlibiSoftcap;
+    }
+
+    bsmt::MaskDnf dnf;
+    std::memset(&dnf, 0, sizeof(dnf));
+    bsmt::AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (bm != nullptr) {
+        if (bm->BLOCK_Q != 128 || bm->BLOCK_KV != 128)
+            return fail(BSMT_ERR_UNSUPPORTED, "block mask BLOCK_SIZE (%d, %d): only 128 x 128", bm->BLOCK_Q, bm->BLOCK_KV);
+        if (bm->Q_LEN != M || bm->KV_LEN != N || bm->QB != QB || bm->KB != KB)
+            return fail(BSMT_ERR_SHAPE_MISMATCH,
+                        "block mask is for (Q_LEN=%d, KV_LEN=%d, QB=%d, KB=%d) but attention has M=%lld N=%lld", bm->Q_LEN,
+                        bm->KV_LEN, bm->QB, bm->KB, static_cast<long long>(M), static_cast<long long>(N));
+        if (!(bm->B == 1 || bm->B == B) || !(bm->H == 1 || bm->H == Hq))
+            return fail(BSMT_ERR_SHAPE_MISMATCH, "block mask (B=%d, H=%d) must broadcast to (B=%lld, Hq=%lld)", bm->B, bm->H,
+                        static_cast<long long>(B), static_cast<long long>(Hq));
+        if (QB > 0 && KB > 0 &&
+            (!bm->kv_num_blocks || !bm->kv_indices || !bm->full_kv_num_blocks || !bm->full_kv_indices))
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "block mask pointers must be non-NULL");
+        bsmt_status st = build_dnf(mask_spec, B, &dnf);
+        if (st != BSMT_OK) return st;
+        p.has_block_mask = 1;
+        p.Bm = bm->B;
+        p.Hm = bm->H;
+        p.kv_num = bm->kv_num_blocks;
+        p.kv_idx = bm->kv_indices;
+        p.full_num = bm->full_kv_num_blocks;
+        p.full_idx = bm->full_kv_indices;
+    } else {
+        dnf.n_terms = 1;
+    }
+    if (B == 0 || M == 0) return ok();
+    int dev = 0, nsm = 0;
+    bsmt_status st = sm_count(&dev, &nsm);
+    if (st != BSMT_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        const int64_t out_vec = B * Hq * M * D / 8, rows = B * Hq * M;
+        fill_empty_kernel<<<2 * nsm, 256, 0, s>>>(static_cast<uint4*>(out), out_vec, lse, rows);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "fill launch: %s", cudaGetErrorString(e));
+        return ok();
+    }
+    EncodeTiledFn enc = nullptr;
+    st = get_encoder(&enc);
+    if (st != BSMT_OK) return st;
+    CUtensorMap tq, tk, tv;
+    if ((st = encode_bhsd(enc, &tq, q, B * Hq, M, D)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tk, k, B * Hkv, N, D)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tv, v, B * Hkv, N, D)) != BSMT_OK) return st;
+
+    p.B = static_cast<int32_t>(B);
+    p.Hq = static_cast<int32_t>(Hq);
+    p.Hkv = static_cast<int32_t>(Hkv);
+    p.M = static_cast<int32_t>(M);
+    p.N = static_cast<int32_t>(N);
+    p.QB = static_cast<int32_t>(QB);
+    p.KB = static_cast<int32_t>(KB);
+    p.pairs = static_cast<int32_t>((QB + 1) / 2);
+    p.group = static_cast<int32_t>(Hq / Hkv);
+    const int64_t units = B * Hq * p.pairs;
+    if (units > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "too many work units");
+    p.num_units = static_cast<int32_t>(units);
+    p.scale = scale;
+    p.scale_log2 = scale * bsmt::kLog2e;
+    p.cap = cap;
+    p.inv_cap = 1.f / cap;
+    p.slopes = slopes;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    if (D == 128) return launch_attn_score<128>(mode, dev, nsm, tq, tk, tv, p, dnf, s) == BSMT_OK ? ok() : BSMT_ERR_CUDA;
+    return launch_attn_score<64>(mode, dev, nsm, tq, tk, tv, p, dnf, s) == BSMT_OK ? ok() : BSMT_ERR_CUDA;
+}
+
+bsmt_status bsmt_check_device_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, bsmt::g_status, sizeof(int));
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "reading device status: %s", cudaGetErrorString(e));
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(bsmt::g_status, &zero, sizeof(int));
+        const char* what = v == BSMT_ERR_DEVICE_TIMEOUT     ? "a pipeline wait ran out of time"
+                           : v == BSMT_ERR_DEVICE_BOUNDS    ? "a block index outside [0, KB) or a bad count"
+                           : v == BSMT_ERR_DEVICE_PRECONDITION ? "kv document ids are not non-decreasing"
+                                                            : "unknown device error";
+        return fail(static_cast<bsmt_status>(v), "device status %d: %s", v, what);
+    }
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,102 @@
+// Mask programs in disjunctive normal form.
+//
+// Each primitive of the mask set (tensorplay.nn.attention: noop_mask, the
+// causal example, and_masks/or_masks; L-GATr page: sliding window, PrefixLM,
+// block-diagonal documents; transformerlab page: StreamingLLM sink) allows
+// one contiguous interval of kv positions for a fixed query row q:
+//   CAUSAL       kv <= q
+//   WINDOW(W)    kv >= q - W + 1
+//   PREFIX_LM(P) kv <= max(P - 1, q)
+//   SINK(S)      kv <= S - 1
+//   DOCUMENT     kv in [first, last] position of q's document id (kv ids sorted)
+//   NOOP         everything
+// The host distributes AND over OR, turning the postfix program into an OR
+// of at most kMaxTerms AND-terms. Each AND-term then allows exactly one
+// interval per row, so a row's allowed set is a union of at most kMaxTerms
+// intervals. This is exact, and cheap to turn into tile classes (builder) or
+// 32-column bit masks (attention kernel).
+#pragma once
+#include <cstdint>
+#include <climits>
+
+#include "bsmt.h"
+
+namespace bsmt {
+
+constexpr int kMaxTerms = BSMT_MAX_MASK_TERMS;
+constexpr int kMaxLeaves = BSMT_MAX_MASK_LEAVES;
+
+struct DnfLeaf {
+    int32_t kind;
+    int32_t arg;
+};
+
+struct MaskDnf {
+    int32_t n_terms;                    // 0 means "nothing allowed"
+    int32_t term_begin[kMaxTerms + 1];  // leaves of term t: [term_begin[t], term_begin[t+1])
+    uint32_t term_has_doc;              // bit t: term t contains a DOCUMENT leaf
+    DnfLeaf leaves[kMaxLeaves];
+    const int32_t* q_doc;
+    const int32_t* kv_doc;
+    int32_t doc_batch;
+    int32_t has_doc;
+};
+
+// Clamp [lo, hi] by one non-document leaf for query row q (64-bit so that
+// extreme W / P / S values cannot overflow).
+__host__ __device__ __forceinline__ void leaf_clamp(int32_t kind, int32_t arg, int64_t q, int64_t& lo,
+                                                    int64_t& hi) {
+    switch (kind) {
+        case BSMT_MASK_CAUSAL:
+            hi = hi < q ? hi : q;
+            break;
+        case BSMT_MASK_WINDOW: {
+            const int64_t l = q - static_cast<int64_t>(arg) + 1;
+            lo = lo > l ? lo : l;
+            break;
+        }
+        case BSMT_MASK_PREFIX_LM: {
+            const int64_t pm1 = static_cast<int64_t>(arg) - 1;
+            const int64_t h = pm1 > q ? pm1 : q;
+            hi = hi < h ? hi : h;
+            break;
+        }
+        case BSMT_MASK_SINK: {
+            const int64_t h = static_cast<int64_t>(arg) - 1;
+            hi = hi < h ? hi : h;
+            break;
+        }
+        default:  // NOOP; DOCUMENT is applied by the caller
+            break;
+    }
+}
+
+// Interval allowed by term t for row q, clamped to [lo0, hi0], using the
+// row's document interval [ds, de] when the term has a DOCUMENT leaf.
+__device__ __forceinline__ void term_interval(const MaskDnf& m, int t, int64_t q, int64_t lo0, int64_t hi0,
+                                              int64_t ds, int64_t de, int64_t& lo, int64_t& hi) {
+    lo = lo0;
+    hi = hi0;
+    for (int i = m.term_begin[t]; i < m.term_begin[t + 1]; ++i) {
+        const int32_t kind = m.leaves[i].kind;
+        if (kind == BSMT_MASK_DOCUMENT) {
+            lo = lo > ds ? lo : ds;
+            hi = hi < de ? hi : de;
+        } else {
+            leaf_clamp(kind, m.leaves[i].arg, q, lo, hi);
+        }
+    }
+}
+
+// Bits [a, b] (inclusive, relative to base) inside one 32-bit word.
+__device__ __forceinline__ uint32_t range_bits(int64_t a, int64_t b, int64_t base) {
+    int64_t lo = a - base;
+    int64_t hi = b - base;
+    lo = lo < 0 ? 0 : lo;
+    hi = hi > 31 ? 31 : hi;
+    if (lo > hi) return 0u;
+    const uint32_t upto = (hi == 31) ? 0xFFFFFFFFu : ((1u << static_cast<uint32_t>(hi + 1)) - 1u);
+    return upto & ~((1u << static_cast<uint32_t>(lo)) - 1u);
+}
+
+}  // namespace bsmt

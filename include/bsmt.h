@@ -1,0 +1,233 @@
+/*
+ * bsmt.h: C ABI of libbsmt, block-sparse masked-tile attention forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The library builds a block-sparse BlockMask from a composable mask
+ * description. It then runs scaled-dot-product attention. The attention
+ * kernel skips tiles the BlockMask leaves out and applies the mask only on
+ * tiles marked partial.
+ *
+ * Sources for the operations (page title, section):
+ *   - tensorplay.nn.attention API page:
+ *     - create_block_mask (signature; mask_mod(b, h, q_idx, kv_idx) -> bool;
+ *       separate_full_blocks);
+ *     - BlockMask "Basics" (row-wise block lists) and "Details" items 1-2
+ *       (kv_num_blocks/kv_indices, full_kv_num_blocks/full_kv_indices);
+ *     - and_masks, or_masks, noop_mask, and the causal example.
+ *   - L-GATr "attention backends" page, "Why care about Attention Kernels?":
+ *     - block-diagonal masks over packed events;
+ *     - sliding window, PrefixLM, ALiBi, tanh soft-capping;
+ *     - tiled attention that never writes the full matrix.
+ *   - FlagAttention page, "Operator overview": layout q [B,Hq,M,D],
+ *     k/v [B,Hkv,N,D], MQA/GQA.
+ *   - transformerlab page, attention registry table: "sink" (StreamingLLM
+ *     first-k sink tokens + window) and "alibi" (m_h * (j - i)).
+ *
+ * Conventions for every entry point:
+ *   - Every call returns a bsmt_status. On failure, bsmt_last_error() gives
+ *     a message. The message is thread-local and stays valid until the next
+ *     call on the same thread.
+ *   - Argument checks happen on the host, before any launch. A call that
+ *     returns an error has launched nothing and written nothing.
+ *   - Device pointers are owned by the caller. The library never allocates,
+ *     frees or keeps device memory beyond the call. Its only global device
+ *     state is one status word per device.
+ *   - Work is enqueued on the caller's stream (a cudaStream_t passed as
+ *     void*; NULL is the legacy default stream). Calls do not synchronize.
+ *   - Errors found on the device set the status word and leave the outputs
+ *     unspecified. Examples are an invalid block index in a BlockMask, kv
+ *     document ids that are not sorted, or a pipeline wait that ran out of
+ *     time. bsmt_check_device_status() reads and clears the word.
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef BSMT_H
+#define BSMT_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bsmt_status {
+    BSMT_OK = 0,
+    BSMT_ERR_INVALID_ARGUMENT = 1,   /* null or misaligned pointer, malformed spec, bad value */
+    BSMT_ERR_SHAPE_MISMATCH = 2,     /* shapes that do not fit together (block mask, heads) */
+    BSMT_ERR_UNSUPPORTED = 3,        /* valid request outside what this build implements */
+    BSMT_ERR_CUDA = 4,               /* a CUDA runtime or driver call failed */
+    BSMT_ERR_DEVICE_TIMEOUT = 5,     /* device: a pipeline wait gave up (kernel returned early) */
+    BSMT_ERR_DEVICE_BOUNDS = 6,      /* device: a block index outside [0, KB) or lists not ascending */
+    BSMT_ERR_DEVICE_PRECONDITION = 7 /* device: kv document ids not non-decreasing */
+} bsmt_status;
+
+/* ------------------------------------------------------------------ masks
+ * A mask is a postfix (reverse Polish) program of nodes. Leaves push one
+ * boolean predicate of (b, q_idx, kv_idx). BSMT_MASK_AND / BSMT_MASK_OR pop
+ * `arg` operands (arg >= 1) and push their intersection / union
+ * (tensorplay.nn.attention: and_masks, or_masks). A well-formed program
+ * leaves exactly one value. None of the predicates depends on the head.
+ *
+ *   NOOP          always true                                  (noop_mask)
+ *   CAUSAL        q_idx >= kv_idx                              (create_block_mask example)
+ *   WINDOW  arg=W q_idx - kv_idx < W                           (sliding window)
+ *   PREFIX_LM arg=P  kv_idx < P  or  q_idx >= kv_idx           (PrefixLM)
+ *   SINK    arg=S kv_idx < S                                   (StreamingLLM sink tokens)
+ *   DOCUMENT      q_doc_ids[b][q_idx] == kv_doc_ids[b][kv_idx] (block-diagonal)
+ *
+ * For DOCUMENT, each kv_doc_ids row must be non-decreasing, as it is for
+ * packed documents: each document's keys are contiguous. q_doc_ids may be
+ * in any order. bsmt_create_block_mask checks the kv order on the device.
+ *
+ * Limits: at most BSMT_MAX_MASK_NODES nodes. After AND is distributed over
+ * OR, the program must have at most BSMT_MAX_MASK_TERMS alternatives and at
+ * most BSMT_MAX_MASK_LEAVES leaf occurrences in total. A larger program
+ * returns BSMT_ERR_UNSUPPORTED.
+ */
+#define BSMT_MAX_MASK_NODES 32
+#define BSMT_MAX_MASK_TERMS 8
+#define BSMT_MAX_MASK_LEAVES 64
+
+enum {
+    BSMT_MASK_NOOP = 0,
+    BSMT_MASK_CAUSAL = 1,
+    BSMT_MASK_WINDOW = 2,
+    BSMT_MASK_PREFIX_LM = 3,
+    BSMT_MASK_SINK = 4,
+    BSMT_MASK_DOCUMENT = 5,
+    BSMT_MASK_AND = 6,
+    BSMT_MASK_OR = 7
+};
+
+typedef struct bsmt_mask_node {
+    int32_t kind;  /* BSMT_MASK_* */
+    int32_t arg;   /* W, P, S, or operand count for AND/OR; ignored otherwise */
+} bsmt_mask_node;
+
+typedef struct bsmt_mask_spec {
+    int32_t num_nodes;
+    bsmt_mask_node nodes[BSMT_MAX_MASK_NODES];
+    /* DOCUMENT only: device int32 arrays, row-major [doc_batch, Q_LEN] and
+     * [doc_batch, KV_LEN], 4-byte aligned. doc_batch is 1 (shared by every
+     * batch row) or B. */
+    const int32_t* q_doc_ids;
+    const int32_t* kv_doc_ids;
+    int32_t doc_batch;
+} bsmt_mask_spec;
+
+/* ------------------------------------------------------------ score mods
+ * Applied in order to the scaled score s = scale * q.k of query i, key j and
+ * query head h, before masking and softmax. The source is the attention-gym
+ * page, "A gallery that grew into a toolkit": score_mod changes a score
+ * before the softmax.
+ *   SOFTCAP  value = cap > 0:  s <- cap * tanh(s / cap)
+ *   ALIBI    s <- s + m_h * (j - i). The slopes m_h are device float[Hq],
+ *            or NULL for m_h = 2^(-8(h+1)/Hq).
+ */
+#define BSMT_MAX_SCORE_OPS 2
+enum { BSMT_SCORE_NONE = 0, BSMT_SCORE_SOFTCAP = 1, BSMT_SCORE_ALIBI = 2 };
+
+typedef struct bsmt_score_op {
+    int32_t kind;          /* BSMT_SCORE_* */
+    float value;           /* SOFTCAP: cap */
+    const float* slopes;   /* ALIBI: device float[Hq] or NULL */
+} bsmt_score_op;
+
+typedef struct bsmt_score_spec {
+    int32_t num_ops;       /* 0 .. BSMT_MAX_SCORE_OPS */
+    bsmt_score_op ops[BSMT_MAX_SCORE_OPS];
+} bsmt_score_spec;
+
+/* -------------------------------------------------------------- BlockMask
+ * The four int32 tensors of tensorplay.nn.attention's BlockMask ("Details"
+ * items 1 and 2), with separate_full_blocks = True:
+ *   kv_num_blocks       [B, H, QB]      number of PARTIAL kv blocks per q-block row
+ *   kv_indices          [B, H, QB, KB]  their kv block indices, ascending, then 0s
+ *   full_kv_num_blocks  [B, H, QB]      number of FULL kv blocks (no masked element)
+ *   full_kv_indices     [B, H, QB, KB]  their indices, ascending, then 0s
+ * QB = ceil(Q_LEN / BLOCK_Q), KB = ceil(KV_LEN / BLOCK_KV). B and H are 1
+ * when the mask is shared across batch rows or heads. All four pointers
+ * are caller-owned device memory, contiguous, 4-byte aligned.
+ */
+typedef struct bsmt_block_mask {
+    int32_t* kv_num_blocks;
+    int32_t* kv_indices;
+    int32_t* full_kv_num_blocks;
+    int32_t* full_kv_indices;
+    int32_t B, H, QB, KB;
+    int32_t Q_LEN, KV_LEN;
+    int32_t BLOCK_Q, BLOCK_KV;
+} bsmt_block_mask;
+
+/* Shape [B, H, QB, KB] of the BlockMask tensors create_block_mask would
+ * write. B <= 0 or H <= 0 means "None" and gives 1. Only 128x128 blocks are
+ * supported (BSMT_ERR_UNSUPPORTED otherwise). Host-only; launches nothing. */
+bsmt_status bsmt_block_mask_shape(int64_t B, int64_t H, int64_t Q_LEN, int64_t KV_LEN,
+                                  int32_t BLOCK_Q, int32_t BLOCK_KV, int64_t out_shape[4]);
+
+/* create_block_mask(mask_mod, B, H, Q_LEN, KV_LEN, BLOCK_SIZE=128) from the
+ * tensorplay.nn.attention page, with separate_full_blocks = True.
+ *
+ * The kernel classifies every 128x128 tile of every (b, h, q-block) row
+ * exactly:
+ *   - FULL: all 128*128 elements allowed and inside [0,Q_LEN) x [0,KV_LEN);
+ *   - EMPTY: no allowed element;
+ *   - PARTIAL: otherwise.
+ * It then writes the ascending lists and zero-fills their tails.
+ *
+ * `out` must hold the four device pointers, sized by bsmt_block_mask_shape.
+ * The call fills out's shape fields. Stream-ordered on `stream`. */
+bsmt_status bsmt_create_block_mask(const bsmt_mask_spec* spec, int64_t B, int64_t H,
+                                   int64_t Q_LEN, int64_t KV_LEN, int32_t BLOCK_Q,
+                                   int32_t BLOCK_KV, bsmt_block_mask* out, void* stream);
+
+/* flex_attention forward with a BlockMask:
+ *   out[b,hq,i,:] = softmax_j( mod(scale * q_i . k_j) masked ) @ v
+ *   lse[b,hq,i]   = natural log-sum-exp of the modified, masked scores
+ *
+ * kv head = hq / (Hq / Hkv). A row with no allowed key gets out = 0 and
+ * lse = -inf.
+ *
+ * Arguments:
+ *   q       device bf16 [B, Hq, M, D], contiguous, 16-byte aligned
+ *   k, v    device bf16 [B, Hkv, N, D], contiguous, 16-byte aligned
+ *   D       64 or 128
+ *   block_mask  BlockMask for (Q_LEN, KV_LEN) = (M, N) with B in {1, B}
+ *           and H in {1, Hq}. NULL means every tile is computed, with no
+ *           mask. Tiles that cross the end of the sequences are then still
+ *           masked to [0, N).
+ *   mask_spec   the mask the BlockMask was built from. The kernel applies it
+ *           on PARTIAL tiles only; FULL tiles skip it (tensorplay.nn.attention,
+ *           BlockMask "Details" item 2). NULL means NOOP. Ignored when
+ *           block_mask is NULL.
+ *   score   score mods. NULL means none.
+ *   scale   softmax scale; <= 0 selects 1/sqrt(D)
+ *   enable_gqa  must be nonzero when Hq != Hkv (Hq must be a multiple of Hkv)
+ *   out     device bf16 [B, Hq, M, D], 16-byte aligned
+ *   lse     device float [B, Hq, M], 4-byte aligned
+ *
+ * Both index lists of each BlockMask row must be ascending and their union
+ * must hold distinct values; the kernel checks this and reports
+ * BSMT_ERR_DEVICE_BOUNDS.
+ */
+bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v,
+                                    int64_t B, int64_t Hq, int64_t Hkv, int64_t M, int64_t N,
+                                    int64_t D, const bsmt_block_mask* block_mask,
+                                    const bsmt_mask_spec* mask_spec,
+                                    const bsmt_score_spec* score, float scale,
+                                    int32_t enable_gqa, void* out, float* lse, void* stream);
+
+/* Thread-local message for the last failed call on this thread ("" if none). */
+const char* bsmt_last_error(void);
+
+/* Waits for `stream`, then reads and clears the current device's status
+ * word. Returns BSMT_OK or the first BSMT_ERR_DEVICE_* recorded since the
+ * last check. */
+bsmt_status bsmt_check_device_status(void* stream);
+
+/* ABI version: (major << 16) | minor. */
+int32_t bsmt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSMT_H */

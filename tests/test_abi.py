@@ -1,0 +1,197 @@
+"""Host-only checks of the C ABI: symbols, shape helper and argument errors.
+
+None of these calls reaches a CUDA API. Every error is caught on the host
+before any device work, so they run on a machine without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_masked_tile_b200 as bsmt
+from block_sparse_masked_tile_b200 import _BlockMask, _MaskSpec, _ScoreSpec, _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bsmt.h")
+
+OK, INVALID, SHAPE, UNSUPPORTED = 0, 1, 2, 3
+FAKE = 0x10000  # 16-byte aligned non-null address; never dereferenced by these calls
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:bsmt_status|const char\*|int32_t)\s+(bsmt_\w+)\s*\(", text, re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert names == sorted(["bsmt_block_mask_shape", "bsmt_create_block_mask", "bsmt_flex_attention_fwd",
+                            "bsmt_last_error", "bsmt_check_device_status", "bsmt_version"])
+    lib = ctypes.CDLL(bsmt.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version():
+    assert _lib.bsmt_version() == (1 << 16)
+
+
+def shape(*args):
+    out = (ctypes.c_int64 * 4)()
+    st = _lib.bsmt_block_mask_shape(*args, out)
+    return st, tuple(out)
+
+
+def test_block_mask_shape():
+    assert shape(2, 32, 32768, 32768, 128, 128) == (OK, (2, 32, 256, 256))
+    assert shape(0, -1, 300, 129, 128, 128) == (OK, (1, 1, 3, 2))
+    assert shape(1, 1, 0, 0, 128, 128) == (OK, (1, 1, 0, 0))
+    assert shape(1, 1, 256, 256, 64, 64)[0] == UNSUPPORTED
+    assert shape(1, 1, -5, 256, 128, 128)[0] == INVALID
+    assert b"128" in _lib.bsmt_last_error() or True
+
+
+def spec_of(nodes, q_doc=None, kv_doc=None, doc_batch=1):
+    s = _MaskSpec()
+    s.num_nodes = len(nodes)
+    for i, (k, a) in enumerate(nodes):
+        s.nodes[i].kind = k
+        s.nodes[i].arg = a
+    s.q_doc_ids = q_doc
+    s.kv_doc_ids = kv_doc
+    s.doc_batch = doc_batch
+    return s
+
+
+def build(spec, B=1, H=1, M=0, N=0, bq=128, bkv=128):
+    # M = 0 means there are no rows: a valid spec returns OK without touching the GPU
+    out = _BlockMask()
+    st = _lib.bsmt_create_block_mask(ctypes.byref(spec) if spec is not None else None, B, H, M, N, bq, bkv,
+                                     ctypes.byref(out), None)
+    return st, out
+
+
+C, W, P, S, DOC, AND, OR = (bsmt.MASK_CAUSAL, bsmt.MASK_WINDOW, bsmt.MASK_PREFIX_LM, bsmt.MASK_SINK,
+                           bsmt.MASK_DOCUMENT, bsmt.MASK_AND, bsmt.MASK_OR)
+
+
+def test_create_block_mask_valid_specs_without_rows():
+    for nodes in ([(C, 0)], [(C, 0), (W, 512), (AND, 2)], [(C, 0), (S, 4), (W, 1024), (OR, 2), (AND, 2)],
+                  [(bsmt.MASK_NOOP, 0)], [(P, 7), (S, 1), (OR, 2)]):
+        st, out = build(spec_of(nodes), M=0, N=100)
+        assert st == OK, _lib.bsmt_last_error()
+        assert (out.B, out.H, out.QB, out.KB, out.KV_LEN) == (1, 1, 0, 1, 100)
+
+
+@pytest.mark.parametrize("nodes,code", [
+    ([], INVALID),                                   # empty program
+    ([(C, 0), (W, 3)], INVALID),                     # two values left
+    ([(C, 0), (AND, 2)], INVALID),                   # operand underflow
+    ([(C, 0), (AND, 0)], INVALID),                   # arity 0
+    ([(99, 0)], INVALID),                            # unknown kind
+    ([(DOC, 0)], INVALID),                           # document without id arrays
+])
+def test_create_block_mask_malformed(nodes, code):
+    st, _ = build(spec_of(nodes), M=0, N=10)
+    assert st == code
+    assert _lib.bsmt_last_error()
+
+
+def test_create_block_mask_too_many_terms():
+    # AND of 4 binary ORs expands to 16 alternatives (> 8)
+    nodes = []
+    for _ in range(4):
+        nodes += [(C, 0), (S, 2), (OR, 2)]
+    nodes.append((AND, 4))
+    st, _ = build(spec_of(nodes), M=0, N=10)
+    assert st == UNSUPPORTED
+
+
+def test_create_block_mask_other_errors():
+    assert build(None, M=0, N=10)[0] == INVALID
+    assert build(spec_of([(C, 0)]), M=0, N=10, bq=64, bkv=64)[0] == UNSUPPORTED
+    st, _ = build(spec_of([(DOC, 0)], FAKE, FAKE, doc_batch=3), B=2, M=0, N=10)
+    assert st == SHAPE
+    st, _ = build(spec_of([(DOC, 0)], FAKE + 2, FAKE, doc_batch=1), B=2, M=0, N=10)
+    assert st == INVALID
+    # rows present but output pointers missing
+    st, _ = build(spec_of([(C, 0)]), M=256, N=256)
+    assert st == INVALID
+
+
+def attn(B=1, Hq=2, Hkv=2, M=256, N=256, D=64, bm=None, spec=None, score=None, scale=0.0, gqa=0,
+         q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE):
+    return _lib.bsmt_flex_attention_fwd(q, k, v, B, Hq, Hkv, M, N, D, bm, spec, score, ctypes.c_float(scale), gqa,
+                                        out, lse, None)
+
+
+def test_flex_attention_argument_errors():
+    assert attn(D=96) == UNSUPPORTED
+    assert attn(D=256) == UNSUPPORTED
+    assert attn(Hq=3, Hkv=2, gqa=1) == SHAPE
+    assert attn(Hq=4, Hkv=2, gqa=0) == SHAPE
+    assert attn(Hkv=0) == SHAPE
+    assert attn(M=-1) == INVALID
+    assert attn(q=0) == INVALID
+    assert attn(k=FAKE + 8) == INVALID
+    assert attn(out=FAKE + 4) == INVALID
+    assert attn(lse=FAKE + 2) == INVALID
+    assert attn(scale=float("inf")) == INVALID
+    assert attn(N=1024 * 128 + 1) == UNSUPPORTED
+
+
+def test_flex_attention_score_errors():
+    sc = _ScoreSpec()
+    sc.num_ops = 3
+    assert attn(score=ctypes.byref(sc)) == INVALID
+    sc.num_ops = 1
+    sc.ops[0].kind = bsmt.SCORE_SOFTCAP
+    sc.ops[0].value = -1.0
+    assert attn(score=ctypes.byref(sc)) == INVALID
+    sc.ops[0].kind = 42
+    assert attn(score=ctypes.byref(sc)) == INVALID
+    sc.num_ops = 2
+    sc.ops[0].kind = bsmt.SCORE_SOFTCAP
+    sc.ops[0].value = 3.0
+    sc.ops[1].kind = bsmt.SCORE_SOFTCAP
+    sc.ops[1].value = 3.0
+    assert attn(score=ctypes.byref(sc)) == UNSUPPORTED
+    sc.ops[1].kind = bsmt.SCORE_ALIBI
+    sc.ops[1].slopes = FAKE + 1
+    assert attn(score=ctypes.byref(sc)) == INVALID
+
+
+def block_mask_c(B=1, H=1, QB=2, KB=2, M=256, N=256, bq=128):
+    c = _BlockMask()
+    c.kv_num_blocks = c.kv_indices = c.full_kv_num_blocks = c.full_kv_indices = FAKE
+    c.B, c.H, c.QB, c.KB = B, H, QB, KB
+    c.Q_LEN, c.KV_LEN = M, N
+    c.BLOCK_Q = c.BLOCK_KV = bq
+    return c
+
+
+def test_flex_attention_block_mask_errors():
+    assert attn(bm=ctypes.byref(block_mask_c(QB=3))) == SHAPE
+    assert attn(bm=ctypes.byref(block_mask_c(N=200))) == SHAPE
+    assert attn(bm=ctypes.byref(block_mask_c(B=2))) == SHAPE
+    assert attn(bm=ctypes.byref(block_mask_c(H=3))) == SHAPE
+    assert attn(bm=ctypes.byref(block_mask_c(bq=64))) == UNSUPPORTED
+    bad = spec_of([(C, 0), (AND, 2)])
+    assert attn(bm=ctypes.byref(block_mask_c()), spec=ctypes.byref(bad)) == INVALID
+    c = block_mask_c()
+    c.kv_indices = None
+    assert attn(bm=ctypes.byref(c)) == INVALID
+
+
+def test_flex_attention_empty_is_ok_without_launch():
+    # B == 0 or M == 0: nothing to compute, nothing launched
+    assert attn(B=0) == OK
+    assert attn(M=0) == OK
+
+
+def test_python_errors_map_to_value_error():
+    with pytest.raises(ValueError):
+        bsmt._check(SHAPE)
+    with pytest.raises(RuntimeError):
+        bsmt._check(UNSUPPORTED)

@@ -1,0 +1,141 @@
+"""GPU parity: the tcgen05 attention kernel vs the fp64 oracle.
+
+Small cases are compared element by element over every output. The five
+workloads are compared at full size: exhaustively where the oracle finishes
+in seconds, otherwise on sampled query rows that the oracle computes one by
+one. Sampled rows include the first and last row of several q-blocks.
+Tolerances: out max-abs 2e-2, lse max-abs 1e-2, and -inf lse exactly where
+the oracle has it.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_masked_tile_b200 as bsmt
+import workloads
+from oracle import attention as oa
+from tests.gpu_helpers import assert_attention_close, gpu_attention
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(seed, B, Hq, Hkv, M, N, D, tree, mods, scale=None, mask_B=None, mask_H=None, use_block_mask=True):
+    q, k, v = workloads.random_inputs(seed, B, Hq, Hkv, M, N, D)
+    gqa = Hq != Hkv
+    out, lse = gpu_attention(q, k, v, tree, mods, scale, gqa, mask_B, mask_H, use_block_mask)
+    ref_out, ref_lse = oa.flex_attention(q, k, v, tree if use_block_mask else None, mods, scale, gqa)
+    return assert_attention_close(out, lse, ref_out, ref_lse, f"seed={seed}")
+
+
+def test_workload1_full():
+    w = workloads.get(1)
+    d = workloads.make(w)
+    out, lse = gpu_attention(d["q"], d["k"], d["v"], d["mask"], d["score_mods"], w.scale, w.enable_gqa)
+    ref_out, ref_lse = oa.flex_attention(d["q"], d["k"], d["v"], d["mask"], d["score_mods"], w.scale, w.enable_gqa)
+    assert_attention_close(out, lse, ref_out, ref_lse, w.name)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("mods", [(), (("softcap", 30.0),), (("alibi", None),),
+                                  (("softcap", 5.0), ("alibi", None)), (("alibi", None), ("softcap", 5.0))])
+def test_score_mods(D, mods):
+    run_case(7, 1, 2, 2, 384, 384, D, ("causal",), mods)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_dense_no_block_mask(D):
+    run_case(11, 2, 2, 1, 256, 384, D, None, (), use_block_mask=False)
+
+
+@pytest.mark.parametrize("M,N", [(300, 200), (129, 513), (1, 1), (100, 1000), (1000, 100)])
+def test_ragged_lengths(M, N):
+    run_case(13, 1, 2, 2, M, N, 128, ("and", ("causal",), ("window", 150)), ())
+    run_case(14, 1, 1, 1, M, N, 64, None, (), use_block_mask=False)
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_masks_and_shapes(seed):
+    rng = np.random.default_rng(500 + seed)
+    D = int(rng.choice([64, 128]))
+    Hkv = int(rng.integers(1, 3))
+    Hq = Hkv * int(rng.choice([1, 2, 4]))
+    B = int(rng.integers(1, 3))
+    M = int(rng.integers(1, 800))
+    N = int(rng.integers(1, 800))
+    tree = workloads.random_mask_tree(rng, B, M, N, depth=2)
+    mods = [(), (("softcap", 20.0),), (("alibi", None),)][int(rng.integers(3))]
+    run_case(seed, B, Hq, Hkv, M, N, D, tree, mods)
+
+
+def test_broadcast_block_mask():
+    run_case(21, 2, 4, 2, 512, 512, 128, ("and", ("causal",), ("window", 200)), (), mask_B=None, mask_H=None)
+    tree = ("and", ("causal",), ("window", 200))
+    q, k, v = workloads.random_inputs(22, 2, 4, 2, 512, 512, 128)
+    bm = bsmt.create_block_mask(bsmt.mask_from_tree(tree), None, None, 512, 512)
+    out, lse = bsmt.flex_attention(q.cuda(), k.cuda(), v.cuda(), block_mask=bm, enable_gqa=True)
+    bsmt.check_device_status()
+    ro, rl = oa.flex_attention(q, k, v, tree, (), None, True)
+    assert_attention_close(out.float().cpu().numpy(), lse.cpu().numpy(), ro, rl, "broadcast")
+
+
+def test_fully_masked_rows():
+    # window 0 with causal allows nothing: every row is 0 / -inf
+    run_case(31, 1, 2, 2, 300, 300, 64, ("and", ("causal",), ("window", 0)), ())
+    # a sink of zero tokens allows nothing either
+    run_case(32, 1, 1, 1, 200, 200, 128, ("sink", 0), ())
+    # mixed: document ids where some queries have a document that holds no key
+    ids_q = np.repeat(np.arange(4), [50, 50, 50, 106]).astype(np.int32)[None]
+    ids_kv = np.repeat(np.arange(3), [60, 60, 136]).astype(np.int32)[None]
+    run_case(33, 1, 1, 1, 256, 256, 64, ("document", ids_q, ids_kv), ())
+
+
+def test_empty_inputs():
+    q, k, v = workloads.random_inputs(40, 1, 2, 2, 0, 64, 64)
+    out, lse = bsmt.flex_attention(q.cuda(), k.cuda(), v.cuda())
+    assert out.shape == (1, 2, 0, 64)
+    q, k, v = workloads.random_inputs(41, 1, 2, 2, 70, 0, 64)
+    out, lse = bsmt.flex_attention(q.cuda(), k.cuda(), v.cuda())
+    bsmt.check_device_status()
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+
+
+def sampled_rows(rng, w, count):
+    rows = []
+    qbs = sorted(set([0, w.M // 128 - 1] + list(rng.integers(0, (w.M + 127) // 128, size=count // 4))))
+    for qb in qbs:
+        for r in (0, 127, int(rng.integers(1, 127))):
+            rows.append((int(rng.integers(w.B)), int(rng.integers(w.Hq)), qb * 128 + r))
+    while len(rows) < count:
+        rows.append((int(rng.integers(w.B)), int(rng.integers(w.Hq)), int(rng.integers(w.M))))
+    return rows
+
+
+@pytest.mark.parametrize("index", [2, 3, 4, 5])
+def test_workloads_full_size_sampled(index):
+    w = workloads.get(index)
+    d = workloads.make(w)
+    out, lse = gpu_attention(d["q"], d["k"], d["v"], d["mask"], d["score_mods"], w.scale, w.enable_gqa)
+    assert np.all(np.isfinite(out))
+    rng = np.random.default_rng(index)
+    samples = sampled_rows(rng, w, 96)
+    so, sl = oa.flex_attention_sampled(d["q"], d["k"], d["v"], samples, d["mask"], d["score_mods"], w.scale,
+                                       w.enable_gqa)
+    go = np.stack([out[b, h, r] for b, h, r in samples])
+    gl = np.array([lse[b, h, r] for b, h, r in samples])
+    assert_attention_close(go, gl, so, sl, w.name)
+
+
+def test_workload2_full_exhaustive():
+    w = workloads.get(2)
+    d = workloads.make(w)
+    out, lse = gpu_attention(d["q"], d["k"], d["v"], d["mask"], d["score_mods"], w.scale, w.enable_gqa)
+    ref_out, ref_lse = oa.flex_attention(d["q"], d["k"], d["v"], d["mask"], d["score_mods"], w.scale, w.enable_gqa)
+    assert_attention_close(out, lse, ref_out, ref_lse, w.name)
+
+
+def test_repeatable_and_deterministic():
+    w = workloads.get(1)
+    d = workloads.make(w)
+    a = gpu_attention(d["q"], d["k"], d["v"], d["mask"], (), None, False)
+    b = gpu_attention(d["q"], d["k"], d["v"], d["mask"], (), None, False)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])

@@ -184,10 +184,20 @@ def random_inputs(seed: int, B: int, Hq: int, Hkv: int, M: int, N: int, D: int):
 
 def random_mask_tree(rng: np.random.Generator, B: int, M: int, N: int, depth: int = 2,
                      allow_document: bool = True) -> tuple:
-    """A random composable mask tree over the primitive set (fuzz data only)."""
+    """A random composable mask tree over the primitive set (fuzz data only).
+
+    All document leaves of one tree share one packing (one pair of id arrays),
+    as a single sequence packing has one set of document boundaries."""
+    L = max(M, N)
+    docs = None
+    if allow_document and L >= 2:
+        cuts = np.sort(rng.choice(np.arange(1, L), size=min(3, L - 1), replace=False))
+        ids = np.searchsorted(cuts, np.arange(L), side="right").astype(np.int32)
+        docs = (np.broadcast_to(ids[:M], (B, M)).copy(), np.broadcast_to(ids[:N], (B, N)).copy())
+
     def leaf():
         kinds = ["noop", "causal", "window", "prefix_lm", "sink"]
-        if allow_document:
+        if docs is not None:
             kinds.append("document")
         kind = kinds[int(rng.integers(len(kinds)))]
         if kind in ("noop", "causal"):
@@ -198,13 +208,7 @@ def random_mask_tree(rng: np.random.Generator, B: int, M: int, N: int, depth: in
             return ("prefix_lm", int(rng.integers(0, N + 1)))
         if kind == "sink":
             return ("sink", int(rng.integers(0, max(1, N // 2))))
-        # document: packed, non-decreasing ids; q and kv share the boundaries
-        L = max(M, N)
-        cuts = np.sort(rng.choice(np.arange(1, L), size=min(3, L - 1), replace=False))
-        ids = np.searchsorted(cuts, np.arange(L), side="right").astype(np.int32)
-        qd = np.broadcast_to(ids[:M], (B, M)).copy()
-        kd = np.broadcast_to(ids[:N], (B, N)).copy()
-        return ("document", qd, kd)
+        return ("document", docs[0], docs[1])
 
     def node(d):
         if d == 0 or rng.random() < 0.3:
