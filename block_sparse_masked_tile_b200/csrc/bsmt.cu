@@ -356,7 +356,10 @@ bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v,
     const int64_t QB = (M + 127) / 128, KB = (N + 127) / 128;
     if (KB > bsmt::kMaxKB)
         return fail(BSMT_ERR_UNSUPPORTED, "KV_LEN=%lld: at most %d kv blocks per row", static_cast<long long>(N), bsmt::kMaxKB);
-    if (!q || !k || !v || !out || !lse) return fail(BSMT_ERR_INVALID_ARGUMENT, "q, k, v, out and lse must be non-NULL");
+    // a tensor with no elements may be passed as NULL (its pointer is never used)
+    const bool q_has = B * Hq * M > 0, kv_has = B * Hkv * N > 0;
+    if ((q_has && (!q || !out || !lse)) || (kv_has && (!k || !v)))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "q, k, v, out and lse must be non-NULL when they hold elements");
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
         return fail(BSMT_ERR_INVALID_ARGUMENT, "q, k, v and out must be 16-byte aligned");
     if (!aligned(lse, 4)) return fail(BSMT_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");

@@ -204,6 +204,7 @@ bsmt_status bsmt_create_block_mask(const bsmt_mask_spec* spec, int64_t B, int64_
  *   enable_gqa  must be nonzero when Hq != Hkv (Hq must be a multiple of Hkv)
  *   out     device bf16 [B, Hq, M, D], 16-byte aligned
  *   lse     device float [B, Hq, M], 4-byte aligned
+ *   A tensor with no elements (M == 0, N == 0 or B == 0) may be NULL.
  *
  * Both index lists of each BlockMask row must be ascending and their union
  * must hold distinct values; the kernel checks this and reports
