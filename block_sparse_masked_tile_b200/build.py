@@ -43,11 +43,35 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
         "-I", INCLUDE, "-I", CSRC,
         "-o", LIB + ".tmp",
     ] + [os.path.join(CSRC, f) for f in SOURCES] + ["-lcudart"]
-    if ptxas_verbose:
-        cmd[1:1] = ["-Xptxas", "-v"]
-    subprocess.run(cmd, check=True)
+    cmd[1:1] = ["-Xptxas", "-v"]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if ptxas_verbose or res.returncode != 0:
+        sys.stderr.write(res.stderr)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed")
+    check_attention_registers(res.stderr)
     os.replace(LIB + ".tmp", LIB)
     return LIB
+
+
+# The attention kernel is sized for 168 registers per thread (384 threads, one
+# CTA per SM); a different count means the launch or the layout changed.
+LAUNCH_REGS = 168
+
+
+def check_attention_registers(ptxas_log: str) -> None:
+    current = None
+    seen = 0
+    for line in ptxas_log.splitlines():
+        if "Compiling entry function" in line:
+            current = line
+        elif "Used" in line and "registers" in line and current and "attn_fwd_kernel" in current:
+            regs = int(line.split("Used")[1].split("registers")[0])
+            seen += 1
+            if regs != LAUNCH_REGS:
+                raise RuntimeError(f"attention kernel compiled to {regs} registers, expected {LAUNCH_REGS}")
+    if seen == 0:
+        raise RuntimeError("ptxas report has no attention kernel entries")
 
 
 if __name__ == "__main__":

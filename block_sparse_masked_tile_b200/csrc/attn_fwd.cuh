@@ -71,7 +71,7 @@ struct AttnParams {
     float* lse;
 };
 
-constexpr int kThreads = 352;  // 11 warps
+constexpr int kThreads = 384;  // 12 warps: 3 warpgroups
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpSched = 10;
@@ -119,6 +119,38 @@ struct SmemLayout {
 
 __device__ __forceinline__ uint32_t sched_entry_kb(uint32_t e) { return e & 0xFFFFu; }
 __device__ __forceinline__ uint32_t sched_entry_tags(uint32_t e) { return e >> 16; }
+
+// Columns per 32-column chunk whose exp2 runs on the FMA pipe. At D = 128 the
+// tensor core needs about as many cycles per tile as MUFU needs for all the
+// exponentials; at D = 64 the tensor core needs half as many. Moving part of
+// the exponentials to the FMA pipe lets both finish inside the MMA time.
+template <int D>
+constexpr int kEmuCols = D == 128 ? 12 : 16;
+
+// 2^x on the FMA pipe for a pair: round x to n, 2^f by a degree-3 polynomial
+// for f = x - n in [-1/2, 1/2] (minimax in relative error, max 1.02e-4; the
+// coefficients come from csrc/fit_exp2_poly.py), and n goes straight into the
+// exponent bits. Inputs are clamped at -125 so the exponent field stays
+// positive; 2^-125 is far below what a bf16 P or an fp32 row sum can see.
+constexpr float kExp2C1 = 0.69328314f;
+constexpr float kExp2C2 = 0.24221109f;
+constexpr float kExp2C3 = 0.05500825f;
+
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
+    x0 = fmaxf(x0, -125.f);
+    x1 = fmaxf(x1, -125.f);
+    float t0, t1, n0, n1, f0, f1, q0, q1;
+    add2(t0, t1, x0, x1, kRound, kRound);
+    add2(n0, n1, t0, t1, -kRound, -kRound);
+    fma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);
+    fma2(q0, q1, kExp2C3, kExp2C3, f0, f1, kExp2C2, kExp2C2);
+    fma2(q0, q1, q0, q1, f0, f1, kExp2C1, kExp2C1);
+    fma2(q0, q1, q0, q1, f0, f1, 1.f, 1.f);
+    // the low mantissa bits of t hold n; (bits(t) << 23) adds n to the exponent
+    y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
 
 template <int D, int SCORE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -178,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm_o[2] = {tmem + 256u, tmem + 256u + (D == 128 ? 128u : 64u)};
 
     auto sched_base = [&](int buf) -> uint8_t* { return smem + L::kSched + buf * L::kSchedBytes; };
+
 
     if (warp == kWarpSched) {
         // ================================================= scheduler warp
@@ -523,25 +556,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(xr + 96));
                     tc_wait_ld();
                 }
-                // score_mod on every visited tile, in base-2 units
-                const float tile_bias = sl2 * static_cast<float>(kb * 128 - q);
+                // score_mod on every visited tile. Other modes move to base-2
+                // units here; the plain mode keeps raw scores and folds
+                // scale * log2(e) into the exponent's FFMA below.
+                if constexpr (SCORE != kScoreNone) {
+                    const float tile_bias = sl2 * static_cast<float>(kb * 128 - q);
 #pragma unroll
-                for (int j = 0; j < 128; ++j) {
-                    float s = x[j];
-                    if constexpr (SCORE == kScoreNone) {
-                        s = s * p.scale_log2;
-                    } else if constexpr (SCORE == kScoreSoftcap) {
-                        s = (p.cap * kLog2e) * tanh_approx(s * (p.scale * p.inv_cap));
-                    } else if constexpr (SCORE == kScoreAlibi) {
-                        s = fmaf(s, p.scale_log2, fmaf(sl2, static_cast<float>(j), tile_bias));
-                    } else if constexpr (SCORE == kScoreSoftcapAlibi) {
-                        s = fmaf((p.cap * kLog2e), tanh_approx(s * (p.scale * p.inv_cap)),
-                                 fmaf(sl2, static_cast<float>(j), tile_bias));
-                    } else {
-                        const float t = fmaf(s, p.scale, hdr.slope * static_cast<float>(kb * 128 + j - q));
-                        s = (p.cap * kLog2e) * tanh_approx(t * p.inv_cap);
+                    for (int j = 0; j < 128; ++j) {
+                        float s = x[j];
+                        if constexpr (SCORE == kScoreSoftcap) {
+                            s = (p.cap * kLog2e) * tanh_approx(s * (p.scale * p.inv_cap));
+                        } else if constexpr (SCORE == kScoreAlibi) {
+                            s = fmaf(s, p.scale_log2, fmaf(sl2, static_cast<float>(j), tile_bias));
+                        } else if constexpr (SCORE == kScoreSoftcapAlibi) {
+                            s = fmaf((p.cap * kLog2e), tanh_approx(s * (p.scale * p.inv_cap)),
+                                     fmaf(sl2, static_cast<float>(j), tile_bias));
+                        } else {
+                            const float t = fmaf(s, p.scale, hdr.slope * static_cast<float>(kb * 128 + j - q));
+                            s = (p.cap * kLog2e) * tanh_approx(t * p.inv_cap);
+                        }
+                        x[j] = s;
                     }
-                    x[j] = s;
                 }
                 // mask_mod on partial tiles only
                 if (partial) {
@@ -587,10 +622,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < 128; ++j)
                         if (!((w[j >> 5] >> (j & 31)) & 1u)) x[j] = -INFINITY;
                 }
-                // row max
-                float mt = x[0];
+                // row max: eight independent chains of three-input max
+                float mx[8];
 #pragma unroll
-                for (int j = 1; j < 128; ++j) mt = fmaxf(mt, x[j]);
+                for (int k = 0; k < 8; ++k) {
+                    mx[k] = x[k];
+#pragma unroll
+                    for (int j = 8; j + 16 <= 128; j += 16) mx[k] = fmax3(mx[k], x[j + k], x[j + 8 + k]);
+                    mx[k] = fmaxf(mx[k], x[120 + k]);
+                }
+                constexpr bool kRaw = SCORE == kScoreNone;
+                const float cmul = kRaw ? p.scale_log2 : 1.f;  // scale > 0, so max commutes with it
+                float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+                if constexpr (kRaw) mt *= cmul;
                 // lazy reference update
                 bool need_rescale = false;
                 float alpha = 1.f;
@@ -602,21 +646,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     l_sum *= alpha;
                     m_ref = mt;
                 }
-                const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-                float part[4] = {0.f, 0.f, 0.f, 0.f};
+                const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                // P = 2^(x * cmul - m). The first kEmuCols columns of every
+                // 32-column chunk use the FMA-pipe exp2, the rest MUFU ex2.
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t pk[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float p0 = ex2_approx(x[32 * c + 2 * j] - m_use);
-                        const float p1 = ex2_approx(x[32 * c + 2 * j + 1] - m_use);
-                        part[c] += p0 + p1;
-                        pk[j] = pack_bf16x2(p0, p1);
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int j = 32 * c + 2 * jj;
+                        float a0, a1, p0, p1;
+                        fma2(a0, a1, x[j], x[j + 1], cmul, cmul, neg_m, neg_m);
+                        if (2 * jj < kEmuCols<D>) {
+                            exp2_poly2(p0, p1, a0, a1);
+                        } else {
+                            p0 = ex2_approx(a0);
+                            p1 = ex2_approx(a1);
+                        }
+                        add2(acc[2 * (jj & 3)], acc[2 * (jj & 3) + 1], acc[2 * (jj & 3)], acc[2 * (jj & 3) + 1], p0, p1);
+                        pk[jj] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(t_s + 16 * c, pk);
                 }
-                l_sum += (part[0] + part[1]) + (part[2] + part[3]);
+                // a row whose every element in this tile is masked adds nothing
+                // (the FMA-pipe exp2 returns 2^-125 rather than 0 for -inf)
+                if (mt != -INFINITY)
+                    l_sum += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
                 // O rescale after P is out of registers (lower register peak)
                 if (__any_sync(0xFFFFFFFFu, need_rescale)) {
 #pragma unroll

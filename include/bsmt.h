@@ -84,8 +84,8 @@ typedef enum bsmt_status {
  * returns BSMT_ERR_UNSUPPORTED.
  */
 #define BSMT_MAX_MASK_NODES 32
-#define BSMT_MAX_MASK_TERMS 8
-#define BSMT_MAX_MASK_LEAVES 64
+#define BSMT_MAX_MASK_TERMS 16
+#define BSMT_MAX_MASK_LEAVES 128
 
 enum {
     BSMT_MASK_NOOP = 0,

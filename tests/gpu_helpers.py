@@ -54,3 +54,25 @@ def assert_attention_close(out, lse, ref_out, ref_lse, what=""):
     assert lerr.max(initial=0.0) <= LSE_TOL, f"{what}: lse max-abs {lerr.max():.3e}"
     assert np.all(out[neg_r] == 0.0), f"{what}: fully masked rows must be 0"
     return float(err.max(initial=0.0)), float(lerr.max(initial=0.0))
+
+
+def dnf_size(tree):
+    """(alternatives, leaf occurrences) after distributing AND over OR."""
+    kind = tree[0]
+    if kind in ("and", "or"):
+        parts = [dnf_size(c) for c in tree[1:]]
+        if kind == "or":
+            return sum(t for t, _ in parts), sum(lv for _, lv in parts)
+        terms, leaves = 1, 0
+        for t, lv in parts:
+            leaves = leaves * t + lv * terms
+            terms *= t
+        return terms, leaves
+    return 1, 1
+
+
+def within_dnf_limits(tree) -> bool:
+    if tree is None:
+        return True
+    t, lv = dnf_size(tree)
+    return t <= 16 and lv <= 128

@@ -99,13 +99,16 @@ def test_create_block_mask_malformed(nodes, code):
 
 
 def test_create_block_mask_too_many_terms():
-    # AND of 4 binary ORs expands to 16 alternatives (> 8)
+    # AND of 5 binary ORs expands to 32 alternatives (> 16)
     nodes = []
-    for _ in range(4):
+    for _ in range(5):
         nodes += [(C, 0), (S, 2), (OR, 2)]
-    nodes.append((AND, 4))
+    nodes.append((AND, 5))
     st, _ = build(spec_of(nodes), M=0, N=10)
     assert st == UNSUPPORTED
+    # 16 alternatives are still accepted
+    st, _ = build(spec_of(nodes[:-1 - 3] + [(AND, 4)]), M=0, N=10)
+    assert st == OK, _lib.bsmt_last_error()
 
 
 def test_create_block_mask_other_errors():

@@ -14,7 +14,7 @@ import torch
 import block_sparse_masked_tile_b200 as bsmt
 import workloads
 from oracle import attention as oa
-from tests.gpu_helpers import assert_attention_close, gpu_attention
+from tests.gpu_helpers import assert_attention_close, gpu_attention, within_dnf_limits
 
 pytestmark = pytest.mark.gpu
 
@@ -22,6 +22,10 @@ pytestmark = pytest.mark.gpu
 def run_case(seed, B, Hq, Hkv, M, N, D, tree, mods, scale=None, mask_B=None, mask_H=None, use_block_mask=True):
     q, k, v = workloads.random_inputs(seed, B, Hq, Hkv, M, N, D)
     gqa = Hq != Hkv
+    if use_block_mask and not within_dnf_limits(tree):
+        with pytest.raises(bsmt.BsmtError, match="UNSUPPORTED"):
+            gpu_attention(q, k, v, tree, mods, scale, gqa, mask_B, mask_H, use_block_mask)
+        return None
     out, lse = gpu_attention(q, k, v, tree, mods, scale, gqa, mask_B, mask_H, use_block_mask)
     ref_out, ref_lse = oa.flex_attention(q, k, v, tree if use_block_mask else None, mods, scale, gqa)
     return assert_attention_close(out, lse, ref_out, ref_lse, f"seed={seed}")

@@ -6,7 +6,7 @@ import torch
 import block_sparse_masked_tile_b200 as bsmt
 import workloads
 from oracle import block_mask as obm
-from tests.gpu_helpers import assert_block_mask_equal, block_mask_numpy, gpu_block_mask
+from tests.gpu_helpers import assert_block_mask_equal, block_mask_numpy, gpu_block_mask, within_dnf_limits
 
 pytestmark = pytest.mark.gpu
 
@@ -35,6 +35,10 @@ def test_random_specs_bit_exact(seed):
     M = int(rng.integers(1, 700))
     N = int(rng.integers(1, 700))
     tree = workloads.random_mask_tree(rng, B, M, N, depth=2)
+    if not within_dnf_limits(tree):
+        with pytest.raises(bsmt.BsmtError, match="UNSUPPORTED"):
+            gpu_block_mask(tree, B, H, M, N)
+        return
     bm = gpu_block_mask(tree, B, H, M, N)
     want = obm.create_block_mask(tree, B, H, M, N)
     assert_block_mask_equal(block_mask_numpy(bm), want)
