@@ -15,8 +15,7 @@
 //   warps 0-3  softmax for q-block 0 of the pair (one query row per thread)
 //   warps 4-7  softmax for q-block 1
 //   warp 8     TMA producer: Q tiles, then K and V tiles into a ring of slots
-//   warp 9     MMA issuer (one thread): S = Q K^T into TMEM, O += P V with P
-//              read from TMEM
+//   warp 9     allocates and frees TMEM (no other role)
 //   warp 10    scheduler. It merges the two rows' partial and full block
 //              lists into one ascending stream of (kb, tags) in shared
 //              memory, so each K/V tile is loaded once for both q-blocks.
@@ -25,12 +24,16 @@
 // (O1 starts at 256+D when D=64). P (bf16 pairs) overwrites the first 64
 // columns of its S.
 //
-// The MMA order per step n of the union stream is: PV of tile n for q-block
-// 0, S of tile n+1 for q-block 0, then the same for q-block 1. So while one
-// softmax warpgroup works, the tensor core computes the other q-block's
-// products. A tcgen05.commit fires once every earlier MMA of the thread is
-// done. When the softmax sees S(n+1) ready, PV(n) has therefore finished,
-// so O can be rescaled and P can overwrite S without a further barrier.
+// Each softmax warpgroup issues its own q-block's MMAs from one thread, at
+// the moment its P(n) is stored: PV(n), then S(next) for its next listed
+// tile (S overwrites the TMEM columns that P(n) occupies, and MMAs from one
+// thread run in issue order). While one warpgroup runs its softmax, the
+// tensor core runs the other's products. A tcgen05.commit fires once every
+// earlier MMA of the thread is done, so when a warpgroup sees S(next) ready,
+// its PV(n) has finished: O can be rescaled and P can overwrite S with no
+// further barrier. A K/V ring slot is free once both warpgroups are done
+// with it: the issuing thread commits after the MMA that read the slot, and
+// a warpgroup that skips the entry arrives directly.
 //
 // The online softmax is in base 2 with a lazy reference max. O and l are
 // rescaled only when a row's max grows by more than 2^8. The final
@@ -80,6 +83,7 @@ constexpr int kRing = 4;       // K/V ring slots (K in even slots, V in odd slot
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kRowTerms = 4;   // mask alternatives kept per row in registers
 
 // Tags of one union entry (bits 16.. of the packed entry).
 constexpr uint32_t kTagIn0 = 1u, kTagIn1 = 2u, kTagPart0 = 4u, kTagPart1 = 8u;
@@ -98,11 +102,11 @@ struct SmemLayout {
     static constexpr int kQ0 = 0;
     static constexpr int kQ1 = kQ0 + kTileBytes;
     static constexpr int kRingBase = kQ1 + kTileBytes;
-    static constexpr int kDoc = kRingBase + kRing * kTileBytes;  // 512 B per slot
-    static constexpr int kSched = kDoc + kRing * 512;
+    static constexpr int kSched = kRingBase + kRing * kTileBytes;
     static constexpr int kSchedEntries = 0;                  // uint32 [kMaxKB]
-    static constexpr int kSchedQdoc = kMaxKB * 4;            // int32 [256]
-    static constexpr int kSchedHeader = kSchedQdoc + 256 * 4;
+    static constexpr int kSchedDocLo = kMaxKB * 4;           // int32 [256]: row's document kv interval
+    static constexpr int kSchedDocHi = kSchedDocLo + 256 * 4;
+    static constexpr int kSchedHeader = kSchedDocHi + 256 * 4;
     static constexpr int kSchedBytes = kSchedHeader + 64;
     static constexpr int kFlags = kSched + 2 * kSchedBytes;  // uint8 [kMaxKB]
     static constexpr int kBars = kFlags + kMaxKB;
@@ -110,7 +114,7 @@ struct SmemLayout {
     static constexpr int kBarQFull = 0, kBarQEmpty = 2, kBarSFull = 4, kBarPFull = 6, kBarOFull = 8,
                          kBarOEmpty = 10, kBarKvFull = 12, kBarKvEmpty = 12 + kRing,
                          kBarSchedFull = 12 + 2 * kRing, kBarSchedEmpty = 14 + 2 * kRing,
-                         kBarDone = 16 + 2 * kRing, kNumBars = 17 + 2 * kRing;
+                         kBarDone = 16 + 2 * kRing, kBarTurn = 18 + 2 * kRing, kNumBars = 20 + 2 * kRing;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kTotal = kAbort + 4;
@@ -120,12 +124,12 @@ struct SmemLayout {
 __device__ __forceinline__ uint32_t sched_entry_kb(uint32_t e) { return e & 0xFFFFu; }
 __device__ __forceinline__ uint32_t sched_entry_tags(uint32_t e) { return e >> 16; }
 
-// Columns per 32-column chunk whose exp2 runs on the FMA pipe. At D = 128 the
-// tensor core needs about as many cycles per tile as MUFU needs for all the
-// exponentials; at D = 64 the tensor core needs half as many. Moving part of
-// the exponentials to the FMA pipe lets both finish inside the MMA time.
+// Columns per 32-column chunk whose exp2 runs on the FMA pipe instead of
+// MUFU. The row's exponentials are the softmax's largest cost; a small share
+// on the FMA pipe shortens the MUFU-bound stretch, a larger share costs more
+// issue slots than it saves (measured on B200 for D = 64 and 128).
 template <int D>
-constexpr int kEmuCols = D == 128 ? 12 : 16;
+constexpr int kEmuCols = 8;
 
 // 2^x on the FMA pipe for a pair: round x to n, 2^f by a degree-3 polynomial
 // for f = x - n in [-1/2, 1/2] (minimax in relative error, max 1.02e-4; the
@@ -179,19 +183,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar(L::kBarPFull + 1), 4);
         mbar_init(bar(L::kBarOFull + 0), 1);
         mbar_init(bar(L::kBarOFull + 1), 1);
-        mbar_init(bar(L::kBarOEmpty + 0), 4);
-        mbar_init(bar(L::kBarOEmpty + 1), 4);
         for (int s = 0; s < kRing; ++s) {
-            // V slots (odd) also take one cp.async arrival per lane for document ids
-            const uint32_t extra = (dnf.has_doc && (s & 1)) ? 32u : 0u;
-            mbar_init(bar(L::kBarKvFull + s), 1 + extra);
-            mbar_init(bar(L::kBarKvEmpty + s), 1);
+            mbar_init(bar(L::kBarKvFull + s), 1);
+            mbar_init(bar(L::kBarKvEmpty + s), 2);  // one arrival per softmax warpgroup
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(L::kBarSchedFull + s), 32);
-            mbar_init(bar(L::kBarSchedEmpty + s), 1 + 1 + 8);  // load, mma, 8 softmax warps
+            mbar_init(bar(L::kBarSchedEmpty + s), 1 + 8);  // producer warp, 8 softmax warps
         }
-        mbar_init(bar(L::kBarDone), 1);
+        mbar_init(bar(L::kBarDone + 0), 1);
+        mbar_init(bar(L::kBarDone + 1), 1);
+        mbar_init(bar(L::kBarTurn + 0), 4);
+        mbar_init(bar(L::kBarTurn + 1), 4);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
@@ -212,6 +215,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto sched_base = [&](int buf) -> uint8_t* { return smem + L::kSched + buf * L::kSchedBytes; };
 
 
+    // Register split: the launch gives every thread 168 registers (384
+    // threads, one CTA per SM; build.py checks the count ptxas reports).
+    // Warpgroup 2 (scheduler, producer, MMA issuer, one idle warp) needs
+    // few registers, so it gives them back and the two softmax warpgroups
+    // take them: 128 * 72 + 256 * 216 = 64512 = 384 * 168. Each role sits
+    // inside the branch of its warpgroup's setmaxnreg, so the compiler
+    // allocates each region to its own limit.
+    if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
     if (warp == kWarpSched) {
         // ================================================= scheduler warp
         uint8_t* flags = smem + L::kFlags;
@@ -312,11 +324,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (dnf.has_doc && p.has_block_mask) {
+                // Each row's document interval [first, last] of kv positions with
+                // the row's document id (kv ids are non-decreasing). Rows in a run
+                // usually share one id, so each distinct id is searched once, with
+                // a 33-way warp search over the kv ids.
                 const int db = dnf.doc_batch > 1 ? b : 0;
-                int32_t* qdoc = reinterpret_cast<int32_t*>(sb + L::kSchedQdoc);
-                for (int r = lane; r < 256; r += 32) {
-                    const int64_t q = static_cast<int64_t>(qb0) * 128 + r;
-                    qdoc[r] = q < p.M ? __ldg(dnf.q_doc + static_cast<int64_t>(db) * p.M + q) : 0;
+                const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
+                const int32_t* kd_row = dnf.kv_doc + static_cast<int64_t>(db) * p.N;
+                int32_t* dlo = reinterpret_cast<int32_t*>(sb + L::kSchedDocLo);
+                int32_t* dhi = reinterpret_cast<int32_t*>(sb + L::kSchedDocHi);
+#pragma unroll 1
+                for (int r0 = 0; r0 < 256; r0 += 32) {
+                    const int64_t q = static_cast<int64_t>(qb0) * 128 + r0 + lane;
+                    const bool valid = q < p.M;
+                    const int32_t d = valid ? __ldg(qd_row + q) : 0;
+                    int lo = 0, hi = -1;
+                    bool pending = valid;
+                    unsigned todo;
+                    while ((todo = __ballot_sync(0xFFFFFFFFu, pending)) != 0u) {
+                        const int32_t x = __shfl_sync(0xFFFFFFFFu, d, __ffs(todo) - 1);
+                        const int first = warp_lower_bound(kd_row, p.N, x, lane);
+                        const int past = warp_lower_bound(kd_row, p.N, static_cast<int64_t>(x) + 1, lane);
+                        if (pending && d == x) {
+                            lo = first;
+                            hi = past - 1;
+                            pending = false;
+                        }
+                    }
+                    dlo[r0 + lane] = lo;
+                    dhi[r0 + lane] = hi;
                 }
             }
             if (lane == 0) {
@@ -370,7 +406,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok) break;
-            const int64_t doc_row = dnf.has_doc ? static_cast<int64_t>(dnf.doc_batch > 1 ? hdr.b : 0) * p.N : 0;
             for (int n = 0; n < hdr.T && ok; ++n) {
                 const int kb = static_cast<int>(sched_entry_kb(entries[n]));
 #pragma unroll
@@ -390,16 +425,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_3d_hint(dst + h * 16384, kv == 0 ? &tm_k : &tm_v, h * 64, kb * 128, zkv, fb,
                                              pol_kv);
                     }
-                    if (kv == 1 && dnf.has_doc) {
-                        const uint32_t ddst = sbase + L::kDoc + s * 512 + lane * 16;
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int64_t pos = static_cast<int64_t>(kb) * 128 + lane * 4 + k;
-                            const bool in = pos < p.N;
-                            cp_async_4(ddst + 4 * k, dnf.kv_doc + doc_row + (in ? pos : 0), in ? 4u : 0u);
-                        }
-                        cp_async_mbar_arrive_noinc(fb);
-                    }
                     ++kv_pos;
                 }
             }
@@ -407,109 +432,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
         }
-    } else if (warp == kWarpMma) {
-        // ================================================= MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-            uint32_t g = 0;  // union entries consumed so far (K at ring pos 2g, V at 2g+1)
-            uint32_t q_full_uses[2] = {0, 0}, o_units[2] = {0, 0}, p_waits[2] = {0, 0};
-            bool ok = true;
-            for (int iter = 0; ok; ++iter) {
-                const int buf = iter & 1;
-                if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) break;
-                const uint8_t* sb = sched_base(buf);
-                const SchedHeader hdr = *reinterpret_cast<const SchedHeader*>(sb + L::kSchedHeader);
-                if (hdr.T < 0) break;
-                const uint32_t* entries = reinterpret_cast<const uint32_t*>(sb + L::kSchedEntries);
-                const int nlist[2] = {hdr.n0, hdr.n1};
-                int s_issued[2] = {0, 0}, pv_issued[2] = {0, 0};
-
-                auto kslot = [&](uint32_t gg) { return (2u * gg) % kRing; };
-                auto vslot = [&](uint32_t gg) { return (2u * gg + 1u) % kRing; };
-                auto kphase = [&](uint32_t gg) { return ((2u * gg) / kRing) & 1u; };
-                auto vphase = [&](uint32_t gg) { return ((2u * gg + 1u) / kRing) & 1u; };
-
-                auto issue_s = [&](int i, uint32_t slot) -> bool {
-                    if (s_issued[i] == 0) {
-                        if (!mbar_wait(bar(L::kBarQFull + i), q_full_uses[i] & 1u, abort_flag)) return false;
-                        ++q_full_uses[i];
-                    }
-                    tc_fence_after();
-                    const uint32_t qa = sbase + (i == 0 ? L::kQ0 : L::kQ1);
-                    const uint32_t ka = sbase + L::kRingBase + slot * L::kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                        mma_ss(tm_s[i], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_s,
-                               kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(bar(L::kBarSFull + i));
-                    if (++s_issued[i] == nlist[i]) mma_commit(bar(L::kBarQEmpty + i));
-                    return true;
-                };
-                auto issue_pv = [&](int i, uint32_t slot) -> bool {
-                    if (pv_issued[i] == 0 && o_units[i] > 0) {
-                        if (!mbar_wait(bar(L::kBarOEmpty + i), (o_units[i] - 1) & 1u, abort_flag)) return false;
-                    }
-                    if (!mbar_wait(bar(L::kBarPFull + i), p_waits[i] & 1u, abort_flag)) return false;
-                    ++p_waits[i];
-                    tc_fence_after();
-                    const uint32_t va = sbase + L::kRingBase + slot * L::kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        mma_ts(tm_o[i], tm_s[i] + 8u * kk, sdesc_sw128(va + kk * 2048u, 16384, 1024), idesc_pv,
-                               (pv_issued[i] > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    if (++pv_issued[i] == nlist[i]) {
-                        mma_commit(bar(L::kBarOFull + i));
-                        ++o_units[i];
-                    }
-                    return true;
-                };
-
-                const int T = hdr.T;
-                if (T > 0) {
-                    const uint32_t e0 = entries[0];
-                    if (!mbar_wait(bar(L::kBarKvFull + kslot(g)), kphase(g), abort_flag)) break;
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        if ((sched_entry_tags(e0) >> i) & 1u) ok = ok && issue_s(i, kslot(g));
-                    if (!ok) break;
-                    mma_commit(bar(L::kBarKvEmpty + kslot(g)));
-                }
-                for (int n = 0; n < T && ok; ++n) {
-                    const uint32_t gg = g + static_cast<uint32_t>(n);
-                    const uint32_t e = entries[n];
-                    const bool has_next = n + 1 < T;
-                    const uint32_t e1 = has_next ? entries[n + 1] : 0u;
-                    if (!mbar_wait(bar(L::kBarKvFull + vslot(gg)), vphase(gg), abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    if (has_next && !mbar_wait(bar(L::kBarKvFull + kslot(gg + 1)), kphase(gg + 1), abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        if ((sched_entry_tags(e) >> i) & 1u) ok = ok && issue_pv(i, vslot(gg));
-                        if (ok && has_next && ((sched_entry_tags(e1) >> i) & 1u)) ok = issue_s(i, kslot(gg + 1));
-                    }
-                    if (!ok) break;
-                    mma_commit(bar(L::kBarKvEmpty + vslot(gg)));
-                    if (has_next) mma_commit(bar(L::kBarKvEmpty + kslot(gg + 1)));
-                }
-                if (!ok) break;
-                g += static_cast<uint32_t>(T);
-                mbar_arrive(bar(L::kBarSchedEmpty + buf));
-            }
-            // all MMAs issued by this thread must finish before TMEM is freed
-            mma_commit(bar(L::kBarDone));
-            mbar_wait(bar(L::kBarDone), 0, abort_flag);
-        }
-        __syncwarp();
-    } else if (warp < 8) {
+    }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
         // ================================================= softmax warpgroups
         const int i = warp >> 2;              // q-block of the pair
         const int r = threadIdx.x & 127;      // row within the q-block
@@ -519,6 +444,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t g = 0;
         uint32_t s_waits = 0, o_waits = 0;
         bool ok = true;
+        // The warpgroup's first warp issues this q-block's MMAs: the whole warp
+        // runs the issue logic and one elected lane issues. (A lone lane in a
+        // diverged warp issues several times slower next to busy softmax
+        // warps.) The warp also observes, in order, every K/V slot phase of
+        // the entry stream, including entries this q-block skips: a slot is
+        // released (two arrivals, one per warpgroup) by a commit after the MMA
+        // that read it, or by a plain arrive for a skipped entry.
+        const bool issuer = (warp & 3) == 0;
+        uint32_t q_uses = 0, pf_waits = 0;
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+        const uint64_t q_desc = sdesc_sw128(sbase + (i == 0 ? L::kQ0 : L::kQ1), 16, 1024);
+        auto slot_wait = [&](uint32_t ring_pos) {
+            return mbar_wait(bar(L::kBarKvFull + ring_pos % kRing), (ring_pos / kRing) & 1u, abort_flag);
+        };
+        // The two warpgroups take turns, entry by entry of the stream: a
+        // warpgroup computes entry n only after the other finished entry n-1,
+        // and hands the turn on as soon as its P is stored. Each softmax then
+        // has the SM's issue slots and MUFU to itself while the tensor core
+        // runs the other warpgroup's products. Warpgroup 0 goes first.
+        uint32_t turn_waits = 0;
+        if (i == 1 && lane == 0) mbar_arrive(bar(L::kBarTurn + 0));
+        auto take_turn = [&]() {
+            const bool t_ok = mbar_wait(bar(L::kBarTurn + i), turn_waits & 1u, abort_flag);
+            ++turn_waits;
+            return t_ok;
+        };
+        auto pass_turn = [&]() {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::kBarTurn + (i ^ 1)));
+        };
         for (int iter = 0; ok; ++iter) {
             const int buf = iter & 1;
             if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) break;
@@ -530,22 +486,134 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int qb = hdr.qb0 + i;
             const int q = qb * 128 + r;
             const bool row_valid = qb < p.QB && q < p.M;
-            const int32_t qd = dnf.has_doc ? reinterpret_cast<const int32_t*>(sb + L::kSchedQdoc)[i * 128 + r] : 0;
+            int64_t row_ds = 0, row_de = p.N - 1;
+            if (dnf.has_doc && p.has_block_mask) {
+                row_ds = reinterpret_cast<const int32_t*>(sb + L::kSchedDocLo)[i * 128 + r];
+                row_de = reinterpret_cast<const int32_t*>(sb + L::kSchedDocHi)[i * 128 + r];
+            }
             const float sl2 = hdr.slope * kLog2e;
+            // This row's allowed kv interval per mask alternative (document
+            // leaves included), computed once per unit. Partial tiles then only
+            // turn intervals into bit words. Empty intervals are stored as [1, 0].
+            const bool fast_mask = p.has_block_mask && dnf.n_terms <= kRowTerms;
+            int iv_lo[kRowTerms], iv_hi[kRowTerms];
+#pragma unroll
+            for (int t = 0; t < kRowTerms; ++t) {
+                iv_lo[t] = 1;
+                iv_hi[t] = 0;
+                if (fast_mask && t < dnf.n_terms) {
+                    int64_t lo, hi;
+                    term_interval(dnf, t, q, 0, p.N - 1, row_ds, row_de, lo, hi);
+                    if (hi >= lo) {  // then both lie in [0, N - 1]
+                        iv_lo[t] = static_cast<int>(lo);
+                        iv_hi[t] = static_cast<int>(hi);
+                    }
+                }
+            }
+            // Issuer state for this unit (entries [0, T) sit at global positions g + n).
+            //   ic      next entry whose slots this warpgroup has not observed yet
+            //   pend    entry whose S is issued and whose PV is still to come (-1: none)
+            //   passed  last entry whose turn this warpgroup has handed on
+            // The issuer waits only on loads of entries up to passed + 2. Loads of
+            // later entries may need the other warpgroup to finish entries whose
+            // turn this one has not handed on yet, and waiting on them would
+            // deadlock the two.
+            int ic = 0, pend = -1, passed = -1;
+            bool need_q = ni > 0;
+            int s_issued = 0, pv_issued = 0;
+            // S = Q K^T for entry n
+            auto issue_s = [&](int n) -> bool {
+                const uint32_t gg = g + static_cast<uint32_t>(n);
+                if (!slot_wait(2u * gg)) return false;
+                const uint64_t kd = sdesc_sw128(sbase + L::kRingBase + ((2u * gg) % kRing) * L::kTileBytes, 16, 1024);
+                const bool last = ++s_issued == ni;
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
+                        mma_ss(tm_s[i], q_desc + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(L::kBarSFull + i));
+                    mma_commit(bar(L::kBarKvEmpty + (2u * gg) % kRing));
+                    if (last) mma_commit(bar(L::kBarQEmpty + i));
+                }
+                __syncwarp();
+                return true;
+            };
+            // O (+)= P V for entry n, P read from TMEM
+            auto issue_pv = [&](int n) -> bool {
+                const uint32_t gg = g + static_cast<uint32_t>(n);
+                if (!slot_wait(2u * gg + 1u)) return false;
+                const uint64_t vd = sdesc_sw128(sbase + L::kRingBase + ((2u * gg + 1u) % kRing) * L::kTileBytes, 16384, 1024);
+                const uint32_t acc0 = pv_issued > 0 ? 1u : 0u;
+                const bool last = ++pv_issued == ni;
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tm_o[i], tm_s[i] + 8u * kk, vd + ((kk * 2048u) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+                    mma_commit(bar(L::kBarKvEmpty + (2u * gg + 1u) % kRing));
+                    if (last) mma_commit(bar(L::kBarOFull + i));
+                }
+                __syncwarp();
+                return true;
+            };
+            // observe entries in order as far as allowed: release the slots of
+            // entries this q-block skips, and issue S for its next tile
+            auto advance = [&]() -> bool {
+                while (pend < 0 && ic < hdr.T && ic <= passed + 2) {
+                    if ((sched_entry_tags(entries[ic]) >> i) & 1u) {
+                        if (need_q) {
+                            if (!mbar_wait(bar(L::kBarQFull + i), q_uses & 1u, abort_flag)) return false;
+                            ++q_uses;
+                            need_q = false;
+                        }
+                        if (!issue_s(ic)) return false;
+                        pend = ic;
+                    } else {
+                        const uint32_t gg = g + static_cast<uint32_t>(ic);
+                        if (!slot_wait(2u * gg) || !slot_wait(2u * gg + 1u)) return false;
+                        if (elect_one()) {
+                            mbar_arrive(bar(L::kBarKvEmpty + (2u * gg) % kRing));
+                            mbar_arrive(bar(L::kBarKvEmpty + (2u * gg + 1u) % kRing));
+                        }
+                        __syncwarp();
+                        ++ic;
+                    }
+                }
+                return true;
+            };
+            if (issuer && !advance()) ok = false;
             float m_ref = -INFINITY;
             float l_sum = 0.f;
             int processed = 0;
-            for (int n = 0; n < hdr.T; ++n) {
+            for (int n = 0; n < hdr.T && ok; ++n) {
                 const uint32_t e = entries[n];
                 const uint32_t tags = sched_entry_tags(e);
-                if (!((tags >> i) & 1u)) continue;
+                if (!((tags >> i) & 1u)) {  // not this q-block's tile: hand the turn on
+                    if (!take_turn()) {
+                        ok = false;
+                        break;
+                    }
+                    pass_turn();
+                    if (issuer) {
+                        passed = n;
+                        if (!advance()) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    continue;
+                }
                 const int kb = static_cast<int>(sched_entry_kb(e));
                 const bool partial = (tags >> (2 + i)) & 1u;
-                if (!mbar_wait(bar(L::kBarSFull + i), s_waits & 1u, abort_flag)) {
+                if (!mbar_wait(bar(L::kBarSFull + i), s_waits & 1u, abort_flag) || !take_turn()) {
                     ok = false;
                     break;
                 }
                 ++s_waits;
+                __syncwarp();  // tcgen05.ld/st are warp-collective: reconverge after the waits
                 tc_fence_after();
                 float x[128];
                 {
@@ -582,32 +650,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (partial) {
                     const int64_t c0 = static_cast<int64_t>(kb) * 128;
                     const int64_t c1 = (c0 + 127 < p.N - 1) ? c0 + 127 : p.N - 1;
-                    int64_t ds = 0, de = -1;
-                    if (dnf.has_doc && p.has_block_mask) {
-                        const uint32_t vs = (2u * (g + static_cast<uint32_t>(n)) + 1u) % kRing;
-                        const uint32_t vph = ((2u * (g + static_cast<uint32_t>(n)) + 1u) / kRing) & 1u;
-                        if (!mbar_wait(bar(L::kBarKvFull + vs), vph, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        const int32_t* dv = reinterpret_cast<const int32_t*>(smem + L::kDoc + vs * 512);
-                        const int cnt = static_cast<int>(c1 - c0 + 1);
-                        // [first, past) of qd among dv[0..cnt) (non-decreasing)
-                        int a = 0, bnd = cnt;
-                        while (a < bnd) {
-                            const int mid = (a + bnd) >> 1;
-                            if (dv[mid] < qd) a = mid + 1; else bnd = mid;
-                        }
-                        int a2 = a, b2 = cnt;
-                        while (a2 < b2) {
-                            const int mid = (a2 + b2) >> 1;
-                            if (dv[mid] <= qd) a2 = mid + 1; else b2 = mid;
-                        }
-                        ds = c0 + a;
-                        de = c0 + a2 - 1;
-                    }
+                    const int64_t ds = row_ds, de = row_de;
                     uint32_t w[4] = {0u, 0u, 0u, 0u};
-                    if (p.has_block_mask) {
+                    if (fast_mask) {
+                        const int tc0 = static_cast<int>(c0), tc1 = static_cast<int>(c1);
+#pragma unroll
+                        for (int t = 0; t < kRowTerms; ++t) {
+                            int lo = iv_lo[t], hi = iv_hi[t];
+                            lo = (lo > tc0 ? lo : tc0) - tc0;
+                            hi = (hi < tc1 ? hi : tc1) - tc0;
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) w[k] |= range_bits32(lo - 32 * k, hi - 32 * k);
+                        }
+                    } else if (p.has_block_mask) {
                         for (int t = 0; t < dnf.n_terms; ++t) {
                             int64_t lo, hi;
                             term_interval(dnf, t, q, c0, c1, ds, de, lo, hi);
@@ -687,9 +742,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_wait_st();
                 tc_fence_before();
-                __syncwarp();
+                pass_turn();
                 if (lane == 0) mbar_arrive(bar(L::kBarPFull + i));
                 ++processed;
+                if (issuer) {
+                    // all four warps have stored their rows of P (and rescaled O)
+                    passed = n;
+                    bool iok = mbar_wait(bar(L::kBarPFull + i), pf_waits & 1u, abort_flag);
+                    ++pf_waits;
+                    iok = iok && issue_pv(n);
+                    ic = n + 1;
+                    pend = -1;
+                    iok = iok && advance();
+                    if (!iok) ok = false;
+                }
             }
             if (!ok) break;
             // epilogue: out = O / l, lse = ln2 * (m + log2 l)
@@ -698,6 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ni > 0) {
                 if (!mbar_wait(bar(L::kBarOFull + i), o_waits & 1u, abort_flag)) break;
                 ++o_waits;
+                __syncwarp();
                 tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
@@ -716,8 +783,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(L::kBarOEmpty + i));
             } else if (row_valid) {
                 uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
@@ -731,6 +796,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             g += static_cast<uint32_t>(hdr.T);
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
+        }
+        if (issuer) {  // every MMA this warp issued must finish before TMEM is freed
+            if (elect_one()) mma_commit(bar(L::kBarDone + i));
+            __syncwarp();
+            mbar_wait(bar(L::kBarDone + i), 0, abort_flag);
         }
     }
 

@@ -34,28 +34,6 @@ struct BuildParams {
 constexpr int kBuildWarps = 4;
 constexpr int kWordsPerChunk = 8;  // 256 kv blocks per pass
 
-// First index i in [0, n) with a[i] >= x (n if none). a is non-decreasing
-// and x is uniform over the warp. 33-way split per step (32 probes).
-__device__ __forceinline__ int warp_lower_bound(const int32_t* a, int n, int64_t x, int lane) {
-    int lo = 0, hi = n;
-    while (lo < hi) {
-        const int len = hi - lo;
-        const int p = lo + static_cast<int>((static_cast<int64_t>(lane + 1) * len) / 33);
-        const int64_t v = (p < hi) ? static_cast<int64_t>(__ldg(a + p)) : INT64_MAX;
-        const unsigned ge = __ballot_sync(0xFFFFFFFFu, v >= x);
-        if (ge == 0u) {
-            lo = lo + static_cast<int>((static_cast<int64_t>(32) * len) / 33) + 1;
-        } else {
-            const int f = __ffs(ge) - 1;
-            const int pf = lo + static_cast<int>((static_cast<int64_t>(f + 1) * len) / 33);
-            const int pprev = (f == 0) ? lo - 1 : lo + static_cast<int>((static_cast<int64_t>(f) * len) / 33);
-            hi = pf;
-            lo = pprev + 1;
-        }
-    }
-    return lo;
-}
-
 __global__ void __launch_bounds__(kBuildWarps * 32) mask_build_kernel(const MaskDnf dnf, const BuildParams p) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;

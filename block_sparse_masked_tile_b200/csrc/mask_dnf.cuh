@@ -99,4 +99,34 @@ __device__ __forceinline__ uint32_t range_bits(int64_t a, int64_t b, int64_t bas
     return upto & ~((1u << static_cast<uint32_t>(lo)) - 1u);
 }
 
+// Bits [a, b] of a 32-bit word (positions relative to the word; 32-bit math).
+__device__ __forceinline__ uint32_t range_bits32(int a, int b) {
+    a = a < 0 ? 0 : a;
+    b = b > 31 ? 31 : b;
+    if (a > b) return 0u;
+    return (0xFFFFFFFFu >> (31 - b)) & (0xFFFFFFFFu << a);
+}
+
+// First index i in [0, n) with a[i] >= x (n if none). a is non-decreasing
+// and x is uniform over the warp. 33-way split per step (32 probes).
+__device__ __forceinline__ int warp_lower_bound(const int32_t* a, int n, int64_t x, int lane) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int len = hi - lo;
+        const int p = lo + static_cast<int>((static_cast<int64_t>(lane + 1) * len) / 33);
+        const int64_t v = (p < hi) ? static_cast<int64_t>(__ldg(a + p)) : INT64_MAX;
+        const unsigned ge = __ballot_sync(0xFFFFFFFFu, v >= x);
+        if (ge == 0u) {
+            lo = lo + static_cast<int>((static_cast<int64_t>(32) * len) / 33) + 1;
+        } else {
+            const int f = __ffs(ge) - 1;
+            const int pf = lo + static_cast<int>((static_cast<int64_t>(f + 1) * len) / 33);
+            const int pprev = (f == 0) ? lo - 1 : lo + static_cast<int>((static_cast<int64_t>(f) * len) / 33);
+            hi = pf;
+            lo = pprev + 1;
+        }
+    }
+    return lo;
+}
+
 }  // namespace bsmt
