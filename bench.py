@@ -43,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 ATTN_SOURCES = ["attn_fwd.cuh", "ptx.cuh", "mask_dnf.cuh", "bsmt.cu"]
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -52,7 +52,9 @@ def parse():
     ap.add_argument("--workload", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    return ap.parse_args()
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch size (smaller cases for profiling only)")
+    return ap.parse_args(argv)
 
 
 def load_peaks():
@@ -84,6 +86,19 @@ def profile_traffic(workload_name: str):
     if not m_hash or not m_bytes or m_hash.group(1) != attn_source_hash():
         return None
     return float(m_bytes.group(1))
+
+
+def reduce_over_ranks(dist, device, times_ms, units):
+    """Max over ranks of each time and sum over ranks of the work units.
+
+    Every rank takes the same two all-reduces in the same order and gets the
+    same result. ``dist`` is None for a single process."""
+    t = torch.tensor([float(x) for x in times_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([float(units)], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t], float(u[0])
 
 
 class ClockSampler:
@@ -148,25 +163,29 @@ def counted_flops(bm, D: int) -> int:
 
 
 # ------------------------------------------------------------------ oracle
-def cpu_baseline(w, data, max_rows: int = 1024):
+def cpu_baseline(w, data, max_rows: int = 16384, chunk: int = 1024, cls=None):
     """The fp64 oracle, as it stands, on a bounded sample of the workload: whole
     q-blocks of (b=0, hq=0) from the top of the sequence (the rows with the most
-    kept tiles), counted with the same tile rule as the GPU metric."""
+    kept tiles), in chunks of ``chunk`` rows, counted with the same tile rule as
+    the GPU metric."""
     from threadpoolctl import threadpool_info
     from oracle import attention as oa
     from oracle import block_mask as obm
 
     rows_per_block = 128
-    nblk = max(1, max_rows // rows_per_block)
-    qbs = list(range((w.M + 127) // 128 - nblk, (w.M + 127) // 128))
+    QB = (w.M + 127) // 128
+    nblk = max(1, min(QB, max_rows // rows_per_block))
+    qbs = list(range(QB - nblk, QB))
     samples = [(0, 0, qb * 128 + r) for qb in qbs for r in range(128) if qb * 128 + r < w.M]
     # kept tiles of those q-block rows (oracle block mask, per q-block row)
-    cls = obm.tile_classes(data["mask"], 0, w.M, w.N)
+    if cls is None:
+        cls = obm.tile_classes(data["mask"], 0, w.M, w.N)
     tiles = sum(int((cls[qb] > 0).sum()) for qb in qbs)
     flops = tiles * 4 * 128 * 128 * w.D
     t0 = time.perf_counter()
-    oa.flex_attention_sampled(data["q"], data["k"], data["v"], samples, data["mask"], data["score_mods"], w.scale,
-                              w.enable_gqa)
+    for c0 in range(0, len(samples), chunk):
+        oa.flex_attention_sampled(data["q"], data["k"], data["v"], samples[c0:c0 + chunk], data["mask"],
+                                  data["score_mods"], w.scale, w.enable_gqa)
     dt = time.perf_counter() - t0
     threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": int(threads), "kind": "oracle",
@@ -178,12 +197,14 @@ def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    from oracle import block_mask as obm
     data = workloads.make(w)
+    cls = obm.tile_classes(data["mask"], 0, w.M, w.N)   # counting only, outside the timed oracle calls
     base = None
     times = []
     total = args.warmup + args.steps
     for i in range(total):
-        r = cpu_baseline(w, data, max_rows=128)
+        r = cpu_baseline(w, data, max_rows=1024, cls=cls)
         if i >= args.warmup:
             times.append(r)
         base = r
@@ -205,6 +226,9 @@ def run_reference(args, w):
 def main():
     args = parse()
     w = workloads.get(args.workload)
+    if args.batch:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch)
     if args.impl == "reference":
         run_reference(args, w)
         return
@@ -263,13 +287,7 @@ def main():
     bsmt.check_device_status(dev)
     ms = start.elapsed_time(end) / args.steps
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    t = torch.tensor([ms, attn_ms], dtype=torch.float64, device=dev)
-    tot = torch.tensor([float(flops)], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
-    ms, attn_ms = float(t[0]), float(t[1])
-    total_flops = float(tot[0])
+    (ms, attn_ms), total_flops = reduce_over_ranks(dist, dev, (ms, attn_ms), flops)
     value = total_flops / (ms * 1e-3) / 1e12
 
     # end to end through the public API with host buffers
@@ -304,10 +322,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te[0])
+    (e2e_ms,), _ = reduce_over_ranks(dist, dev, (e2e_ms,), 0)
     h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_)) + sum(x.numel() * 4 for x in doc_host)
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 

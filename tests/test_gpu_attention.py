@@ -143,3 +143,26 @@ def test_repeatable_and_deterministic():
     a = gpu_attention(d["q"], d["k"], d["v"], d["mask"], (), None, False)
     b = gpu_attention(d["q"], d["k"], d["v"], d["mask"], (), None, False)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_invalid_block_mask_is_reported():
+    """Block indices outside [0, KB) and counts above KB are caught before any
+    access: the kernel skips them and sets DEVICE_BOUNDS in the status word."""
+    import dataclasses
+    q, k, v = (t.cuda() for t in workloads.random_inputs(45, 1, 2, 2, 512, 512, 64))
+    bm = bsmt.create_block_mask(bsmt.causal(), 1, 2, 512, 512)
+    KB = bm.shape[-1]
+    bad_index = dataclasses.replace(bm, kv_indices=bm.kv_indices.clone())
+    bad_index.kv_indices[0, 0, 1, 0] = KB           # one past the last block
+    bad_index.kv_indices[0, 1, 2, 0] = -1
+    bad_count = dataclasses.replace(bm, full_kv_num_blocks=bm.full_kv_num_blocks.clone())
+    bad_count.full_kv_num_blocks[0, 1, 3] = KB + 7
+    for bad in (bad_index, bad_count):
+        bsmt.flex_attention(q, k, v, block_mask=bad)
+        with pytest.raises(RuntimeError, match="DEVICE_BOUNDS"):
+            bsmt.check_device_status()
+    # the word was cleared and a valid call afterwards is correct
+    out, lse = bsmt.flex_attention(q, k, v, block_mask=bm)
+    bsmt.check_device_status()
+    ro, rl = oa.flex_attention(q.cpu(), k.cpu(), v.cpu(), ("causal",), (), None, False)
+    assert_attention_close(out.float().cpu().numpy(), lse.cpu().numpy(), ro, rl, "after bounds error")
