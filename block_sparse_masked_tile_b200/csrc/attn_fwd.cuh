@@ -15,7 +15,7 @@
 //   warps 0-3  softmax for q-block 0 of the pair (one query row per thread)
 //   warps 4-7  softmax for q-block 1
 //   warp 8     TMA producer: Q tiles, then K and V tiles into a ring of slots
-//   warp 9     allocates and frees TMEM (no other role)
+//   warp 9     allocates TMEM and issues every MMA (one elected lane)
 //   warp 10    scheduler. It merges the two rows' partial and full block
 //              lists into one ascending stream of (kb, tags) in shared
 //              memory, so each K/V tile is loaded once for both q-blocks.
@@ -24,16 +24,16 @@
 // (O1 starts at 256+D when D=64). P (bf16 pairs) overwrites the first 64
 // columns of its S.
 //
-// Each softmax warpgroup issues its own q-block's MMAs from one thread, at
-// the moment its P(n) is stored: PV(n), then S(next) for its next listed
-// tile (S overwrites the TMEM columns that P(n) occupies, and MMAs from one
-// thread run in issue order). While one warpgroup runs its softmax, the
-// tensor core runs the other's products. A tcgen05.commit fires once every
-// earlier MMA of the thread is done, so when a warpgroup sees S(next) ready,
-// its PV(n) has finished: O can be rescaled and P can overwrite S with no
-// further barrier. A K/V ring slot is free once both warpgroups are done
-// with it: the issuing thread commits after the MMA that read the slot, and
-// a warpgroup that skips the entry arrives directly.
+// The two softmax warpgroups take turns entry by entry. While one runs its
+// softmax, the tensor core runs the other's products. The issuer walks the
+// entry stream in the same order: for each q-block it issues PV(n) as soon
+// as that q-block's P(n) is stored, then S(next). S overwrites the TMEM
+// columns that P(n) occupies, and MMAs from one thread run in issue order.
+// A tcgen05.commit fires once every earlier MMA of the thread is done, so
+// when a warpgroup sees S(next) ready, its PV(n) has finished: O can be
+// rescaled and P can overwrite S with no further barrier. A K/V ring slot is
+// free once both q-blocks are done with it: the issuer commits after the MMA
+// that read the slot, or arrives directly for a q-block that skips it.
 //
 // The online softmax is in base 2 with a lazy reference max. O and l are
 // rescaled only when a row's max grows by more than 2^8. The final
@@ -189,10 +189,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(L::kBarSchedFull + s), 32);
-            mbar_init(bar(L::kBarSchedEmpty + s), 1 + 8);  // producer warp, 8 softmax warps
+            mbar_init(bar(L::kBarSchedEmpty + s), 1 + 8 + 1);  // producer, 8 softmax warps, MMA issuer
         }
         mbar_init(bar(L::kBarDone + 0), 1);
-        mbar_init(bar(L::kBarDone + 1), 1);
         mbar_init(bar(L::kBarTurn + 0), 4);
         mbar_init(bar(L::kBarTurn + 1), 4);
         *abort_flag = 0;
@@ -432,6 +431,100 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
         }
+    } else if (warp == kWarpMma) {
+        // ================================================= MMA issuer warp
+        // Walks the entry stream in order. At entry n, for q-block 0 and then
+        // q-block 1, it finishes entry n-1 (O += P V once that q-block's P
+        // is in TMEM, or a plain release of the V slot if the q-block skips
+        // the entry) and starts entry n (S = Q K^T, or a plain release of
+        // the K slot). This is the order in which the two softmax warpgroups
+        // take their turns, so every wait here ends: P(n-1) of a q-block
+        // needs only products issued before it. The whole warp runs the loop
+        // and an elected lane issues.
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+        const uint64_t q_desc[2] = {sdesc_sw128(sbase + L::kQ0, 16, 1024), sdesc_sw128(sbase + L::kQ1, 16, 1024)};
+        uint32_t g = 0;  // entries of earlier units (entry n uses ring positions 2(g+n), 2(g+n)+1)
+        uint32_t q_uses[2] = {0, 0}, pf_waits[2] = {0, 0};
+        bool ok = true;
+        auto slot_wait = [&](uint32_t pos) {
+            return mbar_wait(bar(L::kBarKvFull + pos % kRing), (pos / kRing) & 1u, abort_flag);
+        };
+        for (int iter = 0; ok; ++iter) {
+            const int buf = iter & 1;
+            if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) break;
+            const uint8_t* sb = sched_base(buf);
+            const SchedHeader hdr = *reinterpret_cast<const SchedHeader*>(sb + L::kSchedHeader);
+            if (hdr.T < 0) break;
+            const uint32_t* entries = reinterpret_cast<const uint32_t*>(sb + L::kSchedEntries);
+            int s_left[2] = {hdr.n0, hdr.n1}, pv_left[2] = {hdr.n0, hdr.n1};
+            uint32_t prev_tags = 0;
+            for (int n = 0; n <= hdr.T && ok; ++n) {
+                const uint32_t tags = n < hdr.T ? sched_entry_tags(entries[n]) : 0u;
+                const uint32_t kpos = 2u * (g + static_cast<uint32_t>(n));
+                const uint32_t vslot = (kpos - 1u) % kRing, kslot = kpos % kRing;
+                const uint64_t vd = sdesc_sw128(sbase + L::kRingBase + vslot * L::kTileBytes, 16384, 1024);
+                const uint64_t kd = sdesc_sw128(sbase + L::kRingBase + kslot * L::kTileBytes, 16, 1024);
+                if (n > 0 && !slot_wait(kpos - 1u)) { ok = false; break; }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    // finish entry n-1 for q-block i (V at ring position kpos - 1)
+                    if (n > 0) {
+                        if ((prev_tags >> i) & 1u) {
+                            if (!mbar_wait(bar(L::kBarPFull + i), pf_waits[i] & 1u, abort_flag)) { ok = false; break; }
+                            ++pf_waits[i];
+                            const uint32_t acc0 = pv_left[i] < (i == 0 ? hdr.n0 : hdr.n1) ? 1u : 0u;
+                            const bool last = --pv_left[i] == 0;
+                            tc_fence_after();
+                            if (elect_one()) {
+#pragma unroll 1
+                                for (int kk = 0; kk < 8; ++kk)
+                                    mma_ts(tm_o[i], tm_s[i] + 8u * kk, vd + ((kk * 2048u) >> 4), idesc_pv,
+                                           kk > 0 ? 1u : acc0);
+                                mma_commit(bar(L::kBarKvEmpty + vslot));
+                                if (last) mma_commit(bar(L::kBarOFull + i));
+                            }
+                        } else if (elect_one()) {
+                            mbar_arrive(bar(L::kBarKvEmpty + vslot));
+                        }
+                        __syncwarp();
+                    }
+                    if (n == hdr.T) continue;
+                    // start entry n for q-block i (K at ring position kpos)
+                    if (i == 0 && !slot_wait(kpos)) { ok = false; break; }
+                    if ((tags >> i) & 1u) {
+                        if (s_left[i] == (i == 0 ? hdr.n0 : hdr.n1)) {  // first tile of this unit: Q
+                            if (!mbar_wait(bar(L::kBarQFull + i), q_uses[i] & 1u, abort_flag)) { ok = false; break; }
+                            ++q_uses[i];
+                        }
+                        const bool last = --s_left[i] == 0;
+                        tc_fence_after();
+                        if (elect_one()) {
+#pragma unroll 1
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t off = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
+                                mma_ss(tm_s[i], q_desc[i] + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+                            }
+                            mma_commit(bar(L::kBarSFull + i));
+                            mma_commit(bar(L::kBarKvEmpty + kslot));
+                            if (last) mma_commit(bar(L::kBarQEmpty + i));
+                        }
+                    } else if (elect_one()) {
+                        mbar_arrive(bar(L::kBarKvEmpty + kslot));
+                    }
+                    __syncwarp();
+                }
+                prev_tags = tags;
+            }
+            if (!ok) break;
+            g += static_cast<uint32_t>(hdr.T);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
+        }
+        // every MMA must finish before TMEM is freed
+        if (elect_one()) mma_commit(bar(L::kBarDone));
+        __syncwarp();
+        mbar_wait(bar(L::kBarDone), 0, abort_flag);
     }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
@@ -441,24 +534,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_s = tm_s[i] + lane_base;
         const uint32_t t_o = tm_o[i] + lane_base;
-        uint32_t g = 0;
         uint32_t s_waits = 0, o_waits = 0;
         bool ok = true;
-        // The warpgroup's first warp issues this q-block's MMAs: the whole warp
-        // runs the issue logic and one elected lane issues. (A lone lane in a
-        // diverged warp issues several times slower next to busy softmax
-        // warps.) The warp also observes, in order, every K/V slot phase of
-        // the entry stream, including entries this q-block skips: a slot is
-        // released (two arrivals, one per warpgroup) by a commit after the MMA
-        // that read it, or by a plain arrive for a skipped entry.
-        const bool issuer = (warp & 3) == 0;
-        uint32_t q_uses = 0, pf_waits = 0;
-        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-        const uint64_t q_desc = sdesc_sw128(sbase + (i == 0 ? L::kQ0 : L::kQ1), 16, 1024);
-        auto slot_wait = [&](uint32_t ring_pos) {
-            return mbar_wait(bar(L::kBarKvFull + ring_pos % kRing), (ring_pos / kRing) & 1u, abort_flag);
-        };
         // The two warpgroups take turns, entry by entry of the stream: a
         // warpgroup computes entry n only after the other finished entry n-1,
         // and hands the turn on as soon as its P is stored. Each softmax then
@@ -510,81 +587,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            // Issuer state for this unit (entries [0, T) sit at global positions g + n).
-            //   ic      next entry whose slots this warpgroup has not observed yet
-            //   pend    entry whose S is issued and whose PV is still to come (-1: none)
-            //   passed  last entry whose turn this warpgroup has handed on
-            // The issuer waits only on loads of entries up to passed + 2. Loads of
-            // later entries may need the other warpgroup to finish entries whose
-            // turn this one has not handed on yet, and waiting on them would
-            // deadlock the two.
-            int ic = 0, pend = -1, passed = -1;
-            bool need_q = ni > 0;
-            int s_issued = 0, pv_issued = 0;
-            // S = Q K^T for entry n
-            auto issue_s = [&](int n) -> bool {
-                const uint32_t gg = g + static_cast<uint32_t>(n);
-                if (!slot_wait(2u * gg)) return false;
-                const uint64_t kd = sdesc_sw128(sbase + L::kRingBase + ((2u * gg) % kRing) * L::kTileBytes, 16, 1024);
-                const bool last = ++s_issued == ni;
-                tc_fence_after();
-                if (elect_one()) {
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
-                        mma_ss(tm_s[i], q_desc + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(bar(L::kBarSFull + i));
-                    mma_commit(bar(L::kBarKvEmpty + (2u * gg) % kRing));
-                    if (last) mma_commit(bar(L::kBarQEmpty + i));
-                }
-                __syncwarp();
-                return true;
-            };
-            // O (+)= P V for entry n, P read from TMEM
-            auto issue_pv = [&](int n) -> bool {
-                const uint32_t gg = g + static_cast<uint32_t>(n);
-                if (!slot_wait(2u * gg + 1u)) return false;
-                const uint64_t vd = sdesc_sw128(sbase + L::kRingBase + ((2u * gg + 1u) % kRing) * L::kTileBytes, 16384, 1024);
-                const uint32_t acc0 = pv_issued > 0 ? 1u : 0u;
-                const bool last = ++pv_issued == ni;
-                tc_fence_after();
-                if (elect_one()) {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tm_o[i], tm_s[i] + 8u * kk, vd + ((kk * 2048u) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
-                    mma_commit(bar(L::kBarKvEmpty + (2u * gg + 1u) % kRing));
-                    if (last) mma_commit(bar(L::kBarOFull + i));
-                }
-                __syncwarp();
-                return true;
-            };
-            // observe entries in order as far as allowed: release the slots of
-            // entries this q-block skips, and issue S for its next tile
-            auto advance = [&]() -> bool {
-                while (pend < 0 && ic < hdr.T && ic <= passed + 2) {
-                    if ((sched_entry_tags(entries[ic]) >> i) & 1u) {
-                        if (need_q) {
-                            if (!mbar_wait(bar(L::kBarQFull + i), q_uses & 1u, abort_flag)) return false;
-                            ++q_uses;
-                            need_q = false;
-                        }
-                        if (!issue_s(ic)) return false;
-                        pend = ic;
-                    } else {
-                        const uint32_t gg = g + static_cast<uint32_t>(ic);
-                        if (!slot_wait(2u * gg) || !slot_wait(2u * gg + 1u)) return false;
-                        if (elect_one()) {
-                            mbar_arrive(bar(L::kBarKvEmpty + (2u * gg) % kRing));
-                            mbar_arrive(bar(L::kBarKvEmpty + (2u * gg + 1u) % kRing));
-                        }
-                        __syncwarp();
-                        ++ic;
-                    }
-                }
-                return true;
-            };
-            if (issuer && !advance()) ok = false;
             float m_ref = -INFINITY;
             float l_sum = 0.f;
             int processed = 0;
@@ -597,13 +599,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     pass_turn();
-                    if (issuer) {
-                        passed = n;
-                        if (!advance()) {
-                            ok = false;
-                            break;
-                        }
-                    }
                     continue;
                 }
                 const int kb = static_cast<int>(sched_entry_kb(e));
@@ -745,17 +740,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pass_turn();
                 if (lane == 0) mbar_arrive(bar(L::kBarPFull + i));
                 ++processed;
-                if (issuer) {
-                    // all four warps have stored their rows of P (and rescaled O)
-                    passed = n;
-                    bool iok = mbar_wait(bar(L::kBarPFull + i), pf_waits & 1u, abort_flag);
-                    ++pf_waits;
-                    iok = iok && issue_pv(n);
-                    ic = n + 1;
-                    pend = -1;
-                    iok = iok && advance();
-                    if (!iok) ok = false;
-                }
             }
             if (!ok) break;
             // epilogue: out = O / l, lse = ln2 * (m + log2 l)
@@ -793,14 +777,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 p.lse[(static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.M + q] =
                     l_sum > 0.f ? (m_use + __log2f(l_sum)) * kLn2 : -INFINITY;
             }
-            g += static_cast<uint32_t>(hdr.T);
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
-        }
-        if (issuer) {  // every MMA this warp issued must finish before TMEM is freed
-            if (elect_one()) mma_commit(bar(L::kBarDone + i));
-            __syncwarp();
-            mbar_wait(bar(L::kBarDone + i), 0, abort_flag);
         }
     }
 
