@@ -24,10 +24,11 @@
 // (O1 starts at 256+D when D=64). P (bf16 pairs) overwrites the first 64
 // columns of its S.
 //
-// The two softmax warpgroups take turns entry by entry. While one runs its
-// softmax, the tensor core runs the other's products. The issuer walks the
-// entry stream in the same order: for each q-block it issues PV(n) as soon
-// as that q-block's P(n) is stored, then S(next). S overwrites the TMEM
+// The two softmax warpgroups work on their own q-blocks and fall into a
+// ping-pong by themselves: while one runs its softmax, the tensor core runs
+// the other's products. The issuer walks the entry stream in order and, for
+// each q-block, issues PV(n) as soon as that q-block's P(n) is stored, then
+// S(next). S overwrites the TMEM
 // columns that P(n) occupies, and MMAs from one thread run in issue order.
 // A tcgen05.commit fires once every earlier MMA of the thread is done, so
 // when a warpgroup sees S(next) ready, its PV(n) has finished: O can be
@@ -114,7 +115,7 @@ struct SmemLayout {
     static constexpr int kBarQFull = 0, kBarQEmpty = 2, kBarSFull = 4, kBarPFull = 6, kBarOFull = 8,
                          kBarOEmpty = 10, kBarKvFull = 12, kBarKvEmpty = 12 + kRing,
                          kBarSchedFull = 12 + 2 * kRing, kBarSchedEmpty = 14 + 2 * kRing,
-                         kBarDone = 16 + 2 * kRing, kBarTurn = 18 + 2 * kRing, kNumBars = 20 + 2 * kRing;
+                         kBarDone = 16 + 2 * kRing, kNumBars = 17 + 2 * kRing;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kTotal = kAbort + 4;
@@ -192,8 +193,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(L::kBarSchedEmpty + s), 1 + 8 + 1);  // producer, 8 softmax warps, MMA issuer
         }
         mbar_init(bar(L::kBarDone + 0), 1);
-        mbar_init(bar(L::kBarTurn + 0), 4);
-        mbar_init(bar(L::kBarTurn + 1), 4);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
@@ -437,10 +436,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // q-block 1, it finishes entry n-1 (O += P V once that q-block's P
         // is in TMEM, or a plain release of the V slot if the q-block skips
         // the entry) and starts entry n (S = Q K^T, or a plain release of
-        // the K slot). This is the order in which the two softmax warpgroups
-        // take their turns, so every wait here ends: P(n-1) of a q-block
-        // needs only products issued before it. The whole warp runs the loop
-        // and an elected lane issues.
+        // the K slot). Every wait here ends: P(n-1) of a q-block needs only
+        // its S(n-1), issued before, and each load it waits for needs only
+        // slot releases made at earlier entries. The whole warp runs the
+        // loop and an elected lane issues.
         constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
         const uint64_t q_desc[2] = {sdesc_sw128(sbase + L::kQ0, 16, 1024), sdesc_sw128(sbase + L::kQ1, 16, 1024)};
@@ -536,22 +535,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_o = tm_o[i] + lane_base;
         uint32_t s_waits = 0, o_waits = 0;
         bool ok = true;
-        // The two warpgroups take turns, entry by entry of the stream: a
-        // warpgroup computes entry n only after the other finished entry n-1,
-        // and hands the turn on as soon as its P is stored. Each softmax then
-        // has the SM's issue slots and MUFU to itself while the tensor core
-        // runs the other warpgroup's products. Warpgroup 0 goes first.
-        uint32_t turn_waits = 0;
-        if (i == 1 && lane == 0) mbar_arrive(bar(L::kBarTurn + 0));
-        auto take_turn = [&]() {
-            const bool t_ok = mbar_wait(bar(L::kBarTurn + i), turn_waits & 1u, abort_flag);
-            ++turn_waits;
-            return t_ok;
-        };
-        auto pass_turn = [&]() {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::kBarTurn + (i ^ 1)));
-        };
         for (int iter = 0; ok; ++iter) {
             const int buf = iter & 1;
             if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) break;
@@ -593,17 +576,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int n = 0; n < hdr.T && ok; ++n) {
                 const uint32_t e = entries[n];
                 const uint32_t tags = sched_entry_tags(e);
-                if (!((tags >> i) & 1u)) {  // not this q-block's tile: hand the turn on
-                    if (!take_turn()) {
-                        ok = false;
-                        break;
-                    }
-                    pass_turn();
-                    continue;
-                }
+                if (!((tags >> i) & 1u)) continue;  // not this q-block's tile
                 const int kb = static_cast<int>(sched_entry_kb(e));
                 const bool partial = (tags >> (2 + i)) & 1u;
-                if (!mbar_wait(bar(L::kBarSFull + i), s_waits & 1u, abort_flag) || !take_turn()) {
+                if (!mbar_wait(bar(L::kBarSFull + i), s_waits & 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -737,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_wait_st();
                 tc_fence_before();
-                pass_turn();
+                __syncwarp();
                 if (lane == 0) mbar_arrive(bar(L::kBarPFull + i));
                 ++processed;
             }
