@@ -476,10 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const bool last = --pv_left[i] == 0;
                             tc_fence_after();
                             if (elect_one()) {
-#pragma unroll 1
-                                for (int kk = 0; kk < 8; ++kk)
-                                    mma_ts(tm_o[i], tm_s[i] + 8u * kk, vd + ((kk * 2048u) >> 4), idesc_pv,
-                                           kk > 0 ? 1u : acc0);
+                                mma_ts_run8(tm_o[i], tm_s[i], vd, idesc_pv, acc0);
                                 mma_commit(bar(L::kBarKvEmpty + vslot));
                                 if (last) mma_commit(bar(L::kBarOFull + i));
                             }
@@ -499,11 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const bool last = --s_left[i] == 0;
                         tc_fence_after();
                         if (elect_one()) {
-#pragma unroll 1
-                            for (int kk = 0; kk < D / 16; ++kk) {
-                                const uint32_t off = ((kk >> 2) * 16384u + (kk & 3) * 32u) >> 4;
-                                mma_ss(tm_s[i], q_desc[i] + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
-                            }
+                            mma_ss_run<D / 16>(tm_s[i], q_desc[i], kd, idesc_s, 0u);
                             mma_commit(bar(L::kBarSFull + i));
                             mma_commit(bar(L::kBarKvEmpty + kslot));
                             if (last) mma_commit(bar(L::kBarQEmpty + i));

@@ -232,6 +232,82 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
+// A K-major SS product over K = 16 * KSTEPS (KSTEPS = 4 or 8) in one asm
+// block: steps 0-3 walk 32 B along a 128-byte swizzle row, steps 4-7 start
+// the second 64-column block 16 KB further on (descriptor units of 16 B).
+// Only the first step may start a fresh accumulator. Issuing the run from
+// one block keeps the descriptor arithmetic in two 64-bit temporaries.
+template <int KSTEPS>
+__device__ __forceinline__ void mma_ss_run(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    static_assert(KSTEPS == 4 || KSTEPS == 8, "K must be 64 or 128");
+    if constexpr (KSTEPS == 4) {
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\t.reg .b64 a, b;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "setp.ne.b32 q, 1, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+            "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+            "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+            "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t}"
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\t.reg .b64 a, b;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "setp.ne.b32 q, 1, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+            "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+            "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+            "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+            "add.s64 a, %1, 1024;\n\tadd.s64 b, %2, 1024;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+            "add.s64 a, %1, 1026;\n\tadd.s64 b, %2, 1026;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+            "add.s64 a, %1, 1028;\n\tadd.s64 b, %2, 1028;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+            "add.s64 a, %1, 1030;\n\tadd.s64 b, %2, 1030;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t}"
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    }
+}
+
+// A TS product over K = 128 in one asm block: A (bf16 pairs) from TMEM
+// columns a_tmem + 8k, B MN-major from shared memory 2 KB further per step
+// (16 rows of a 128-byte swizzle layout; 128 descriptor units).
+__device__ __forceinline__ void mma_ts_run8(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, 1, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "add.u32 a, %1, 8;\n\tadd.s64 b, %2, 128;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
+        "add.u32 a, %1, 16;\n\tadd.s64 b, %2, 256;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
+        "add.u32 a, %1, 24;\n\tadd.s64 b, %2, 384;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
+        "add.u32 a, %1, 32;\n\tadd.s64 b, %2, 512;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
+        "add.u32 a, %1, 40;\n\tadd.s64 b, %2, 640;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
+        "add.u32 a, %1, 48;\n\tadd.s64 b, %2, 768;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
+        "add.u32 a, %1, 56;\n\tadd.s64 b, %2, 896;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on an mbarrier once every tcgen05 op this thread issued so far is done.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
