@@ -464,7 +464,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t vslot = (kpos - 1u) % kRing, kslot = kpos % kRing;
                 const uint64_t vd = sdesc_sw128(sbase + L::kRingBase + vslot * L::kTileBytes, 16384, 1024);
                 const uint64_t kd = sdesc_sw128(sbase + L::kRingBase + kslot * L::kTileBytes, 16, 1024);
-                if (n > 0 && !slot_wait(kpos - 1u)) { ok = false; break; }
+                // the V tile of entry n-1 and the K tile of entry n, both up front
+                // so that each q-block's PV and S go out back to back
+                if (n > 0 && n < hdr.T) {
+                    if (!mbar_wait2(bar(L::kBarKvFull + (kpos - 1u) % kRing), ((kpos - 1u) / kRing) & 1u,
+                                    bar(L::kBarKvFull + kslot), (kpos / kRing) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                } else if ((n > 0 || n < hdr.T) && !slot_wait(n > 0 ? kpos - 1u : kpos)) {
+                    ok = false;  // (a unit with no entries waits for nothing)
+                    break;
+                }
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     // finish entry n-1 for q-block i (V at ring position kpos - 1)
@@ -487,7 +498,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (n == hdr.T) continue;
                     // start entry n for q-block i (K at ring position kpos)
-                    if (i == 0 && !slot_wait(kpos)) { ok = false; break; }
                     if ((tags >> i) & 1u) {
                         if (s_left[i] == (i == 0 ? hdr.n0 : hdr.n1)) {  // first tile of this unit: Q
                             if (!mbar_wait(bar(L::kBarQFull + i), q_uses[i] & 1u, abort_flag)) { ok = false; break; }

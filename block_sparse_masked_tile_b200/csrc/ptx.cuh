@@ -96,6 +96,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// Waits for two phases. Both probes are in flight before either result is
+// used, so two phases that are already complete cost one probe latency.
+__device__ __forceinline__ bool mbar_wait2(uint32_t bar_a, uint32_t parity_a, uint32_t bar_b, uint32_t parity_b,
+                                           volatile int* abort_flag) {
+    const bool a = mbar_try_wait(bar_a, parity_a);
+    const bool b = mbar_try_wait(bar_b, parity_b);
+    if (a && b) return true;
+    if (!a && !mbar_wait(bar_a, parity_a, abort_flag)) return false;
+    return b || mbar_wait(bar_b, parity_b, abort_flag);
+}
+
 // --------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int x, int y, int z,
                                             uint32_t bar) {
