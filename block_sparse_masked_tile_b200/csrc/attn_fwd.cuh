@@ -15,7 +15,8 @@
 //   warps 0-3  softmax for q-block 0 of the pair (one query row per thread)
 //   warps 4-7  softmax for q-block 1
 //   warp 8     TMA producer: Q tiles, then K and V tiles into a ring of slots
-//   warp 9     allocates TMEM and issues every MMA (one elected lane)
+//   warp 9     allocates TMEM; issues the MMAs of q-block 0 (one elected lane)
+//   warp 11    issues the MMAs of q-block 1
 //   warp 10    scheduler. It merges the two rows' partial and full block
 //              lists into one ascending stream of (kb, tags) in shared
 //              memory, so each K/V tile is loaded once for both q-blocks.
@@ -26,15 +27,15 @@
 //
 // The two softmax warpgroups work on their own q-blocks and fall into a
 // ping-pong by themselves: while one runs its softmax, the tensor core runs
-// the other's products. The issuer walks the entry stream in order and, for
-// each q-block, issues PV(n) as soon as that q-block's P(n) is stored, then
-// S(next). S overwrites the TMEM
+// the other's products. Two issuer warps walk the entry stream in order and,
+// taking turns, issue each q-block's PV(n) as soon as its P(n) is stored,
+// then its S(n+1). S overwrites the TMEM
 // columns that P(n) occupies, and MMAs from one thread run in issue order.
 // A tcgen05.commit fires once every earlier MMA of the thread is done, so
 // when a warpgroup sees S(next) ready, its PV(n) has finished: O can be
 // rescaled and P can overwrite S with no further barrier. A K/V ring slot is
-// free once both q-blocks are done with it: the issuer commits after the MMA
-// that read the slot, or arrives directly for a q-block that skips it.
+// free once both q-blocks are done with it: each issuer commits after the
+// MMA that read the slot, or arrives directly if its q-block skips it.
 //
 // The online softmax is in base 2 with a lazy reference max. O and l are
 // rescaled only when a row's max grows by more than 2^8. The final
@@ -77,7 +78,8 @@ struct AttnParams {
 
 constexpr int kThreads = 384;  // 12 warps: 3 warpgroups
 constexpr int kWarpLoad = 8;
-constexpr int kWarpMma = 9;
+constexpr int kWarpMma = 9;    // also the MMA issuer for q-block 0
+constexpr int kWarpMma1 = 11;  // MMA issuer for q-block 1
 constexpr int kWarpSched = 10;
 constexpr int kMaxKB = 1024;   // kv blocks per row supported by the schedule buffer
 constexpr int kRing = 4;       // K/V ring slots (K in even slots, V in odd slots)
@@ -115,7 +117,7 @@ struct SmemLayout {
     static constexpr int kBarQFull = 0, kBarQEmpty = 2, kBarSFull = 4, kBarPFull = 6, kBarOFull = 8,
                          kBarOEmpty = 10, kBarKvFull = 12, kBarKvEmpty = 12 + kRing,
                          kBarSchedFull = 12 + 2 * kRing, kBarSchedEmpty = 14 + 2 * kRing,
-                         kBarDone = 16 + 2 * kRing, kNumBars = 17 + 2 * kRing;
+                         kBarDone = 16 + 2 * kRing, kBarTok = 18 + 2 * kRing, kNumBars = 20 + 2 * kRing;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kTotal = kAbort + 4;
@@ -190,9 +192,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(L::kBarSchedFull + s), 32);
-            mbar_init(bar(L::kBarSchedEmpty + s), 1 + 8 + 1);  // producer, 8 softmax warps, MMA issuer
+            mbar_init(bar(L::kBarSchedEmpty + s), 1 + 8 + 2);  // producer, 8 softmax warps, 2 MMA issuers
         }
         mbar_init(bar(L::kBarDone + 0), 1);
+        mbar_init(bar(L::kBarDone + 1), 1);
+        mbar_init(bar(L::kBarTok + 0), 1);
+        mbar_init(bar(L::kBarTok + 1), 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q);
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // Register split: the launch gives every thread 168 registers (384
     // threads, one CTA per SM; build.py checks the count ptxas reports).
-    // Warpgroup 2 (scheduler, producer, MMA issuer, one idle warp) needs
+    // Warpgroup 2 (scheduler, producer, two MMA issuers) needs
     // few registers, so it gives them back and the two softmax warpgroups
     // take them: 128 * 72 + 256 * 216 = 64512 = 384 * 168. Each role sits
     // inside the branch of its warpgroup's setmaxnreg, so the compiler
@@ -430,22 +435,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
         }
-    } else if (warp == kWarpMma) {
-        // ================================================= MMA issuer warp
-        // Walks the entry stream in order. At entry n, for q-block 0 and then
-        // q-block 1, it finishes entry n-1 (O += P V once that q-block's P
-        // is in TMEM, or a plain release of the V slot if the q-block skips
-        // the entry) and starts entry n (S = Q K^T, or a plain release of
-        // the K slot). Every wait here ends: P(n-1) of a q-block needs only
-        // its S(n-1), issued before, and each load it waits for needs only
-        // slot releases made at earlier entries. The whole warp runs the
-        // loop and an elected lane issues.
+    } else if (warp == kWarpMma || warp == kWarpMma1) {
+        // ================================================= MMA issuer warps
+        // One warp per q-block of the pair. Each walks the whole entry stream
+        // in order; at step n it finishes entry n-1 for its q-block (O += P V
+        // once the q-block's P is in TMEM, or a plain release of the V slot if
+        // the q-block skips the entry) and starts entry n (S = Q K^T, or a
+        // plain release of the K slot). The two issuers hand a token back and
+        // forth, q-block 0 first, so the tensor pipe receives whole steps in
+        // the fixed order [PV0, S0], [PV1, S1], ... and each q-block's S(n)
+        // follows its PV(n-1) at once. Everything a step waits for (its P,
+        // the V and K tiles, Q) is waited for before taking the token, while
+        // the other issuer is issuing: a single warp issues an MMA in about as
+        // long as the tensor core takes to run one, so the issuer's own waits
+        // would otherwise leave the tensor pipe idle. Every wait ends: P(n-1)
+        // needs only S(n-1), issued at an earlier step; a load waited for at
+        // step n needs only slot releases of entries up to n-2; and the token
+        // comes back after the other issuer's step, whose waits are of the
+        // same kind. The whole warp runs the loop and an elected lane issues.
+        const int i = warp == kWarpMma ? 0 : 1;
         constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-        const uint64_t q_desc[2] = {sdesc_sw128(sbase + L::kQ0, 16, 1024), sdesc_sw128(sbase + L::kQ1, 16, 1024)};
+        const uint64_t q_desc = sdesc_sw128(sbase + (i == 0 ? L::kQ0 : L::kQ1), 16, 1024);
+        const uint32_t t_s = tm_s[i], t_o = tm_o[i];
         uint32_t g = 0;  // entries of earlier units (entry n uses ring positions 2(g+n), 2(g+n)+1)
-        uint32_t q_uses[2] = {0, 0}, pf_waits[2] = {0, 0};
+        uint32_t q_uses = 0, pf_waits = 0, tok_waits = 0;
         bool ok = true;
+        if (i == 1 && lane == 0) mbar_arrive(bar(L::kBarTok + 0));  // q-block 0 goes first
         auto slot_wait = [&](uint32_t pos) {
             return mbar_wait(bar(L::kBarKvFull + pos % kRing), (pos / kRing) & 1u, abort_flag);
         };
@@ -456,19 +472,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const SchedHeader hdr = *reinterpret_cast<const SchedHeader*>(sb + L::kSchedHeader);
             if (hdr.T < 0) break;
             const uint32_t* entries = reinterpret_cast<const uint32_t*>(sb + L::kSchedEntries);
-            int s_left[2] = {hdr.n0, hdr.n1}, pv_left[2] = {hdr.n0, hdr.n1};
-            uint32_t prev_tags = 0;
-            for (int n = 0; n <= hdr.T && ok; ++n) {
-                const uint32_t tags = n < hdr.T ? sched_entry_tags(entries[n]) : 0u;
+            const int ni = i == 0 ? hdr.n0 : hdr.n1;
+            int s_done = 0, pv_done = 0;
+            bool prev_in = false;
+            for (int n = 0; n <= hdr.T; ++n) {
+                const bool cur_in = n < hdr.T && ((sched_entry_tags(entries[n]) >> i) & 1u);
                 const uint32_t kpos = 2u * (g + static_cast<uint32_t>(n));
                 const uint32_t vslot = (kpos - 1u) % kRing, kslot = kpos % kRing;
-                const uint64_t vd = sdesc_sw128(sbase + L::kRingBase + vslot * L::kTileBytes, 16384, 1024);
-                const uint64_t kd = sdesc_sw128(sbase + L::kRingBase + kslot * L::kTileBytes, 16, 1024);
-                // the V tile of entry n-1 and the K tile of entry n, both up front
-                // so that each q-block's PV and S go out back to back
+                // waits of this step, before the token
                 if (n > 0 && n < hdr.T) {
-                    if (!mbar_wait2(bar(L::kBarKvFull + (kpos - 1u) % kRing), ((kpos - 1u) / kRing) & 1u,
-                                    bar(L::kBarKvFull + kslot), (kpos / kRing) & 1u, abort_flag)) {
+                    if (!mbar_wait2(bar(L::kBarKvFull + vslot), ((kpos - 1u) / kRing) & 1u, bar(L::kBarKvFull + kslot),
+                                    (kpos / kRing) & 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -476,37 +490,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;  // (a unit with no entries waits for nothing)
                     break;
                 }
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    // finish entry n-1 for q-block i (V at ring position kpos - 1)
-                    if (n > 0) {
-                        if ((prev_tags >> i) & 1u) {
-                            if (!mbar_wait(bar(L::kBarPFull + i), pf_waits[i] & 1u, abort_flag)) { ok = false; break; }
-                            ++pf_waits[i];
-                            const uint32_t acc0 = pv_left[i] < (i == 0 ? hdr.n0 : hdr.n1) ? 1u : 0u;
-                            const bool last = --pv_left[i] == 0;
-                            tc_fence_after();
-                            if (elect_one()) {
-                                mma_ts_run8(tm_o[i], tm_s[i], vd, idesc_pv, acc0);
-                                mma_commit(bar(L::kBarKvEmpty + vslot));
-                                if (last) mma_commit(bar(L::kBarOFull + i));
-                            }
-                        } else if (elect_one()) {
-                            mbar_arrive(bar(L::kBarKvEmpty + vslot));
-                        }
-                        __syncwarp();
-                    }
-                    if (n == hdr.T) continue;
-                    // start entry n for q-block i (K at ring position kpos)
-                    if ((tags >> i) & 1u) {
-                        if (s_left[i] == (i == 0 ? hdr.n0 : hdr.n1)) {  // first tile of this unit: Q
-                            if (!mbar_wait(bar(L::kBarQFull + i), q_uses[i] & 1u, abort_flag)) { ok = false; break; }
-                            ++q_uses[i];
-                        }
-                        const bool last = --s_left[i] == 0;
-                        tc_fence_after();
+                if (prev_in) {
+                    if (!mbar_wait(bar(L::kBarPFull + i), pf_waits & 1u, abort_flag)) { ok = false; break; }
+                    ++pf_waits;
+                }
+                if (cur_in && s_done == 0) {  // first tile of this unit: Q
+                    if (!mbar_wait(bar(L::kBarQFull + i), q_uses & 1u, abort_flag)) { ok = false; break; }
+                    ++q_uses;
+                }
+                if (!mbar_wait(bar(L::kBarTok + i), tok_waits & 1u, abort_flag)) { ok = false; break; }
+                ++tok_waits;
+                tc_fence_after();
+                if (n > 0) {  // finish entry n-1 (V at ring position kpos - 1)
+                    if (prev_in) {
+                        const uint64_t vd = sdesc_sw128(sbase + L::kRingBase + vslot * L::kTileBytes, 16384, 1024);
+                        const uint32_t acc0 = pv_done > 0 ? 1u : 0u;
+                        const bool last = ++pv_done == ni;
                         if (elect_one()) {
-                            mma_ss_run<D / 16>(tm_s[i], q_desc[i], kd, idesc_s, 0u);
+                            mma_ts_run8(t_o, t_s, vd, idesc_pv, acc0);
+                            mma_commit(bar(L::kBarKvEmpty + vslot));
+                            if (last) mma_commit(bar(L::kBarOFull + i));
+                        }
+                    } else if (elect_one()) {
+                        mbar_arrive(bar(L::kBarKvEmpty + vslot));
+                    }
+                    __syncwarp();
+                }
+                if (n < hdr.T) {  // start entry n (K at ring position kpos)
+                    if (cur_in) {
+                        const uint64_t kd = sdesc_sw128(sbase + L::kRingBase + kslot * L::kTileBytes, 16, 1024);
+                        const bool last = ++s_done == ni;
+                        if (elect_one()) {
+                            mma_ss_run<D / 16>(t_s, q_desc, kd, idesc_s, 0u);
                             mma_commit(bar(L::kBarSFull + i));
                             mma_commit(bar(L::kBarKvEmpty + kslot));
                             if (last) mma_commit(bar(L::kBarQEmpty + i));
@@ -516,17 +531,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     __syncwarp();
                 }
-                prev_tags = tags;
+                if (lane == 0) mbar_arrive(bar(L::kBarTok + (i ^ 1)));
+                prev_in = cur_in;
             }
             if (!ok) break;
             g += static_cast<uint32_t>(hdr.T);
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
         }
-        // every MMA must finish before TMEM is freed
-        if (elect_one()) mma_commit(bar(L::kBarDone));
+        // every MMA of this warp must finish before TMEM is freed
+        if (elect_one()) mma_commit(bar(L::kBarDone + i));
         __syncwarp();
-        mbar_wait(bar(L::kBarDone), 0, abort_flag);
+        mbar_wait(bar(L::kBarDone + i), 0, abort_flag);
     }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
