@@ -120,8 +120,13 @@ struct SmemLayout {
                          kBarDone = 16 + 2 * kRing, kBarTok = 18 + 2 * kRing, kNumBars = 20 + 2 * kRing;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
-    static constexpr int kTotal = kAbort + 4;
+    // out staging: one 32-row x 32-column bf16 block (2 KB, 64-byte swizzle)
+    // per softmax warp, written by the warp and stored by TMA
+    static constexpr int kStage = (kAbort + 4 + 1023) / 1024 * 1024;
+    static constexpr int kStageBytes = 32 * 32 * 2;
+    static constexpr int kTotal = kStage + 8 * kStageBytes;
     static constexpr int kAlloc = kTotal + 1024;  // room to align the base to 1024 B
+    static_assert(kAlloc <= 227 * 1024, "shared memory layout exceeds one CTA's limit");
 };
 
 __device__ __forceinline__ uint32_t sched_entry_kb(uint32_t e) { return e & 0xFFFFu; }
@@ -162,7 +167,8 @@ __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float
 template <int D, int SCORE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p, const MaskDnf dnf) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                    const AttnParams p, const MaskDnf dnf) {
     using L = SmemLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -203,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_out);
     }
     if (warp == kWarpMma) {
         tmem_alloc(sbase + L::kTmemSlot, 512);
@@ -745,6 +752,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++o_waits;
                 __syncwarp();
                 tc_fence_after();
+                // Each warp writes its 32 rows chunk by chunk (32 columns, 64 bytes a
+                // row) into its staging block and TMA stores the block: coalesced
+                // writes, and rows past M are clipped by the tensor map.
+                const uint32_t stage = sbase + L::kStage + static_cast<uint32_t>(warp) * L::kStageBytes;
+                const int y0 = qb * 128 + (warp & 3) * 32;
+                const int z = hdr.b * p.Hq + hdr.hq;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
@@ -754,11 +767,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         pk[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv_l, __uint_as_float(o[2 * j + 1]) * inv_l);
-                    if (row_valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+                    if (lane == 0) bulk_wait_group_read0();  // the previous block has been read
+                    __syncwarp();
+                    // 64-byte swizzle: 16-byte chunk k of row r sits at chunk k ^ ((r >> 1) & 3)
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    for (int k = 0; k < 4; ++k)
+                        st_shared_v4(stage + static_cast<uint32_t>(lane) * 64u +
+                                         static_cast<uint32_t>((k ^ ((lane >> 1) & 3)) * 16),
+                                     pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && y0 < p.M) {  // (a block wholly past M stores nothing)
+                        tma_store_3d(&tm_out, stage, 32 * c, y0, z);
+                        bulk_commit_group();
                     }
                 }
                 tc_fence_before();
@@ -775,6 +796,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
         }
+        if (lane == 0) bulk_wait_group0();  // staged out blocks are written before the CTA ends
+        __syncwarp();
     }
 
     // ------------------------------------------------------------ teardown

@@ -207,6 +207,20 @@ bsmt_status encode_bhsd(EncodeTiledFn enc, CUtensorMap* map, const void* base, i
     return BSMT_OK;
 }
 
+// out [BH, S, D] bf16 as a 3-D map with 32 x 32 x 1 boxes (64-byte rows) and
+// 64-byte swizzle; the attention epilogue stores through it.
+bsmt_status encode_out(EncodeTiledFn enc, CUtensorMap* map, void* base, int64_t BH, int64_t S, int64_t D) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D * 2), static_cast<cuuint64_t>(S * D * 2)};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(BSMT_ERR_CUDA, "cuTensorMapEncodeTiled (out) failed (%d)", static_cast<int>(r));
+    return BSMT_OK;
+}
+
 // Rows with no allowed key: out = 0, lse = -inf (used when KV_LEN == 0).
 __global__ void fill_empty_kernel(uint4* out, int64_t out_vec, float* lse, int64_t rows) {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -218,7 +232,8 @@ __global__ void fill_empty_kernel(uint4* out, int64_t out_vec, float* lse, int64
 
 template <int D, int SCORE>
 bsmt_status launch_attn(int dev, int nsm, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const bsmt::AttnParams& p, const bsmt::MaskDnf& dnf, cudaStream_t stream) {
+                        const CUtensorMap& to, const bsmt::AttnParams& p, const bsmt::MaskDnf& dnf,
+                        cudaStream_t stream) {
     auto kern = bsmt::attn_fwd_kernel<D, SCORE>;
     const int smem = bsmt::SmemLayout<D>::kAlloc;
     {
@@ -231,7 +246,7 @@ bsmt_status launch_attn(int dev, int nsm, const CUtensorMap& tq, const CUtensorM
         }
     }
     const int grid = p.num_units < nsm ? p.num_units : nsm;
-    kern<<<grid, bsmt::kThreads, smem, stream>>>(tq, tk, tv, p, dnf);
+    kern<<<grid, bsmt::kThreads, smem, stream>>>(tq, tk, tv, to, p, dnf);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
     return BSMT_OK;
@@ -239,15 +254,15 @@ bsmt_status launch_attn(int dev, int nsm, const CUtensorMap& tq, const CUtensorM
 
 template <int D>
 bsmt_status launch_attn_score(int score, int dev, int nsm, const CUtensorMap& tq, const CUtensorMap& tk,
-                              const CUtensorMap& tv, const bsmt::AttnParams& p, const bsmt::MaskDnf& dnf,
-                              cudaStream_t s) {
+                              const CUtensorMap& tv, const CUtensorMap& to, const bsmt::AttnParams& p,
+                              const bsmt::MaskDnf& dnf, cudaStream_t s) {
     switch (score) {
-        case bsmt::kScoreNone: return launch_attn<D, bsmt::kScoreNone>(dev, nsm, tq, tk, tv, p, dnf, s);
-        case bsmt::kScoreSoftcap: return launch_attn<D, bsmt::kScoreSoftcap>(dev, nsm, tq, tk, tv, p, dnf, s);
-        case bsmt::kScoreAlibi: return launch_attn<D, bsmt::kScoreAlibi>(dev, nsm, tq, tk, tv, p, dnf, s);
+        case bsmt::kScoreNone: return launch_attn<D, bsmt::kScoreNone>(dev, nsm, tq, tk, tv, to, p, dnf, s);
+        case bsmt::kScoreSoftcap: return launch_attn<D, bsmt::kScoreSoftcap>(dev, nsm, tq, tk, tv, to, p, dnf, s);
+        case bsmt::kScoreAlibi: return launch_attn<D, bsmt::kScoreAlibi>(dev, nsm, tq, tk, tv, to, p, dnf, s);
         case bsmt::kScoreSoftcapAlibi:
-            return launch_attn<D, bsmt::kScoreSoftcapAlibi>(dev, nsm, tq, tk, tv, p, dnf, s);
-        default: return launch_attn<D, bsmt::kScoreAlibiSoftcap>(dev, nsm, tq, tk, tv, p, dnf, s);
+            return launch_attn<D, bsmt::kScoreSoftcapAlibi>(dev, nsm, tq, tk, tv, to, p, dnf, s);
+        default: return launch_attn<D, bsmt::kScoreAlibiSoftcap>(dev, nsm, tq, tk, tv, to, p, dnf, s);
     }
 }
 
@@ -441,8 +456,9 @@ bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v,
     EncodeTiledFn enc = nullptr;
     st = get_encoder(&enc);
     if (st != BSMT_OK) return st;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if ((st = encode_bhsd(enc, &tq, q, B * Hq, M, D)) != BSMT_OK) return st;
+    if ((st = encode_out(enc, &to, out, B * Hq, M, D)) != BSMT_OK) return st;
     if ((st = encode_bhsd(enc, &tk, k, B * Hkv, N, D)) != BSMT_OK) return st;
     if ((st = encode_bhsd(enc, &tv, v, B * Hkv, N, D)) != BSMT_OK) return st;
 
@@ -465,8 +481,8 @@ bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v,
     p.slopes = slopes;
     p.out = static_cast<__nv_bfloat16*>(out);
     p.lse = lse;
-    if (D == 128) return launch_attn_score<128>(mode, dev, nsm, tq, tk, tv, p, dnf, s) == BSMT_OK ? ok() : BSMT_ERR_CUDA;
-    return launch_attn_score<64>(mode, dev, nsm, tq, tk, tv, p, dnf, s) == BSMT_OK ? ok() : BSMT_ERR_CUDA;
+    if (D == 128) return launch_attn_score<128>(mode, dev, nsm, tq, tk, tv, to, p, dnf, s) == BSMT_OK ? ok() : BSMT_ERR_CUDA;
+    return launch_attn_score<64>(mode, dev, nsm, tq, tk, tv, to, p, dnf, s) == BSMT_OK ? ok() : BSMT_ERR_CUDA;
 }
 
 bsmt_status bsmt_check_device_status(void* stream) {
