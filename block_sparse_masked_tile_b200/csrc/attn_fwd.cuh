@@ -376,6 +376,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (SCORE == kScoreAlibi || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap)
                     slope = p.slopes ? __ldg(p.slopes + hq) : exp2f(-8.0f * static_cast<float>(hq + 1) / static_cast<float>(p.Hq));
                 hdr->slope = slope;
+                // Pull this unit's Q tiles into L2 now; they are loaded into shared
+                // memory only when the unit before has finished with its own.
+                const int zq = b * p.Hq + hq;
+                for (int qq = 0; qq < 2; ++qq) {
+                    if ((qq == 0 ? n0 : n1) == 0) continue;
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h) tma_prefetch_3d(&tm_q, h * 64, (qb0 + qq) * 128, zq);
+                }
             }
             __syncwarp();
             mbar_arrive(bar(L::kBarSchedFull + buf));
@@ -465,12 +473,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
         const uint64_t q_desc = sdesc_sw128(sbase + (i == 0 ? L::kQ0 : L::kQ1), 16, 1024);
         const uint32_t t_s = tm_s[i], t_o = tm_o[i];
-        uint32_t g = 0;  // entries of earlier units (entry n uses ring positions 2(g+n), 2(g+n)+1)
+        // Entry e of the stream (counted over all units) uses ring positions
+        // 2e (K) and 2e+1 (V). Within a unit, a turn finishes entry e-1 and
+        // starts entry e. A unit's last entry is finished outside the token
+        // order, as soon as its P is stored: the next unit's first S then
+        // waits for neither q-block's last tile of the unit before.
+        uint32_t e = 0;  // entries started so far
         uint32_t q_uses = 0, pf_waits = 0, tok_waits = 0;
         bool ok = true;
+        bool prev_in = false, prev_first = false, prev_last = false;  // entry e-1 for this q-block
         if (i == 1 && lane == 0) mbar_arrive(bar(L::kBarTok + 0));  // q-block 0 goes first
         auto slot_wait = [&](uint32_t pos) {
             return mbar_wait(bar(L::kBarKvFull + pos % kRing), (pos / kRing) & 1u, abort_flag);
+        };
+        // One step: finish entry e-1 (if has_prev) and start entry e (if has_cur),
+        // in a token turn unless it only finishes.
+        auto step = [&](bool has_prev, bool has_cur, bool cur_in, bool cur_first, bool cur_last) -> bool {
+            const uint32_t kpos = 2u * e;
+            const uint32_t vslot = (kpos - 1u) % kRing, kslot = kpos % kRing;
+            // waits of this step, before the token
+            if (has_prev && has_cur) {
+                if (!mbar_wait2(bar(L::kBarKvFull + vslot), ((kpos - 1u) / kRing) & 1u, bar(L::kBarKvFull + kslot),
+                                (kpos / kRing) & 1u, abort_flag))
+                    return false;
+            } else if (!slot_wait(has_prev ? kpos - 1u : kpos)) {
+                return false;
+            }
+            if (has_prev && prev_in) {
+                if (!mbar_wait(bar(L::kBarPFull + i), pf_waits & 1u, abort_flag)) return false;
+                ++pf_waits;
+            }
+            if (has_cur && cur_in && cur_first) {  // first tile of its unit: Q
+                if (!mbar_wait(bar(L::kBarQFull + i), q_uses & 1u, abort_flag)) return false;
+                ++q_uses;
+            }
+            if (has_cur) {
+                if (!mbar_wait(bar(L::kBarTok + i), tok_waits & 1u, abort_flag)) return false;
+                ++tok_waits;
+            }
+            tc_fence_after();
+            if (has_prev) {  // finish entry e-1 (V at ring position kpos - 1)
+                if (prev_in) {
+                    const uint64_t vd = sdesc_sw128(sbase + L::kRingBase + vslot * L::kTileBytes, 16384, 1024);
+                    if (elect_one()) {
+                        mma_ts_run8(t_o, t_s, vd, idesc_pv, prev_first ? 0u : 1u);
+                        mma_commit(bar(L::kBarKvEmpty + vslot));
+                        if (prev_last) mma_commit(bar(L::kBarOFull + i));
+                    }
+                } else if (elect_one()) {
+                    mbar_arrive(bar(L::kBarKvEmpty + vslot));
+                }
+                __syncwarp();
+            }
+            if (has_cur) {  // start entry e (K at ring position kpos)
+                if (cur_in) {
+                    const uint64_t kd = sdesc_sw128(sbase + L::kRingBase + kslot * L::kTileBytes, 16, 1024);
+                    if (elect_one()) {
+                        mma_ss_run<D / 16>(t_s, q_desc, kd, idesc_s, 0u);
+                        mma_commit(bar(L::kBarSFull + i));
+                        mma_commit(bar(L::kBarKvEmpty + kslot));
+                        if (cur_last) mma_commit(bar(L::kBarQEmpty + i));
+                    }
+                } else if (elect_one()) {
+                    mbar_arrive(bar(L::kBarKvEmpty + kslot));
+                }
+                __syncwarp();
+            }
+            if (has_cur && lane == 0) mbar_arrive(bar(L::kBarTok + (i ^ 1)));
+            prev_in = has_cur && cur_in;
+            prev_first = cur_first;
+            prev_last = cur_last;
+            if (has_cur) ++e;
+            return true;
         };
         for (int iter = 0; ok; ++iter) {
             const int buf = iter & 1;
@@ -480,69 +554,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (hdr.T < 0) break;
             const uint32_t* entries = reinterpret_cast<const uint32_t*>(sb + L::kSchedEntries);
             const int ni = i == 0 ? hdr.n0 : hdr.n1;
-            int s_done = 0, pv_done = 0;
-            bool prev_in = false;
-            for (int n = 0; n <= hdr.T; ++n) {
-                const bool cur_in = n < hdr.T && ((sched_entry_tags(entries[n]) >> i) & 1u);
-                const uint32_t kpos = 2u * (g + static_cast<uint32_t>(n));
-                const uint32_t vslot = (kpos - 1u) % kRing, kslot = kpos % kRing;
-                // waits of this step, before the token
-                if (n > 0 && n < hdr.T) {
-                    if (!mbar_wait2(bar(L::kBarKvFull + vslot), ((kpos - 1u) / kRing) & 1u, bar(L::kBarKvFull + kslot),
-                                    (kpos / kRing) & 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                } else if ((n > 0 || n < hdr.T) && !slot_wait(n > 0 ? kpos - 1u : kpos)) {
-                    ok = false;  // (a unit with no entries waits for nothing)
-                    break;
-                }
-                if (prev_in) {
-                    if (!mbar_wait(bar(L::kBarPFull + i), pf_waits & 1u, abort_flag)) { ok = false; break; }
-                    ++pf_waits;
-                }
-                if (cur_in && s_done == 0) {  // first tile of this unit: Q
-                    if (!mbar_wait(bar(L::kBarQFull + i), q_uses & 1u, abort_flag)) { ok = false; break; }
-                    ++q_uses;
-                }
-                if (!mbar_wait(bar(L::kBarTok + i), tok_waits & 1u, abort_flag)) { ok = false; break; }
-                ++tok_waits;
-                tc_fence_after();
-                if (n > 0) {  // finish entry n-1 (V at ring position kpos - 1)
-                    if (prev_in) {
-                        const uint64_t vd = sdesc_sw128(sbase + L::kRingBase + vslot * L::kTileBytes, 16384, 1024);
-                        const uint32_t acc0 = pv_done > 0 ? 1u : 0u;
-                        const bool last = ++pv_done == ni;
-                        if (elect_one()) {
-                            mma_ts_run8(t_o, t_s, vd, idesc_pv, acc0);
-                            mma_commit(bar(L::kBarKvEmpty + vslot));
-                            if (last) mma_commit(bar(L::kBarOFull + i));
-                        }
-                    } else if (elect_one()) {
-                        mbar_arrive(bar(L::kBarKvEmpty + vslot));
-                    }
-                    __syncwarp();
-                }
-                if (n < hdr.T) {  // start entry n (K at ring position kpos)
-                    if (cur_in) {
-                        const uint64_t kd = sdesc_sw128(sbase + L::kRingBase + kslot * L::kTileBytes, 16, 1024);
-                        const bool last = ++s_done == ni;
-                        if (elect_one()) {
-                            mma_ss_run<D / 16>(t_s, q_desc, kd, idesc_s, 0u);
-                            mma_commit(bar(L::kBarSFull + i));
-                            mma_commit(bar(L::kBarKvEmpty + kslot));
-                            if (last) mma_commit(bar(L::kBarQEmpty + i));
-                        }
-                    } else if (elect_one()) {
-                        mbar_arrive(bar(L::kBarKvEmpty + kslot));
-                    }
-                    __syncwarp();
-                }
-                if (lane == 0) mbar_arrive(bar(L::kBarTok + (i ^ 1)));
-                prev_in = cur_in;
+            int s_done = 0;
+            for (int n = 0; n < hdr.T && ok; ++n) {
+                const bool cur_in = (sched_entry_tags(entries[n]) >> i) & 1u;
+                const bool cur_first = cur_in && s_done == 0;
+                if (cur_in) ++s_done;
+                ok = step(n > 0, true, cur_in, cur_first, cur_in && s_done == ni);
             }
+            if (ok && hdr.T > 0) ok = step(true, false, false, false, false);  // finish the unit's last entry
             if (!ok) break;
-            g += static_cast<uint32_t>(hdr.T);
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
         }
@@ -758,15 +778,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t stage = sbase + L::kStage + static_cast<uint32_t>(warp) * L::kStageBytes;
                 const int y0 = qb * 128 + (warp & 3) * 32;
                 const int z = hdr.b * p.Hq + hdr.hq;
+                uint32_t o[D];
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) tmem_ld32(t_o + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(o + 32 * c));
+                tc_wait_ld();
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(t_o + 32 * c, o);
-                    tc_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        pk[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv_l, __uint_as_float(o[2 * j + 1]) * inv_l);
+                        pk[j] = pack_bf16x2(__uint_as_float(o[32 * c + 2 * j]) * inv_l,
+                                            __uint_as_float(o[32 * c + 2 * j + 1]) * inv_l);
                     if (lane == 0) bulk_wait_group_read0();  // the previous block has been read
                     __syncwarp();
                     // 64-byte swizzle: 16-byte chunk k of row r sits at chunk k ^ ((r >> 1) & 3)
