@@ -93,3 +93,35 @@ def sparsity(bm: dict) -> float:
     total = bm["kv_indices"].size
     computed = int(bm["kv_num_blocks"].sum()) + int(bm["full_kv_num_blocks"].sum())
     return 100.0 * (1.0 - computed / total)
+
+
+def q_side(bm: dict) -> dict:
+    """The q-side lists of a BlockMask (tensorplay.nn.attention page, BlockMask
+    "Details" items 3 and 4): for every kv block, the q blocks whose partial
+    list (item 3: q_num_blocks, q_indices) or full list (item 4:
+    full_q_num_blocks, full_q_indices) holds it. The page calls them the
+    transpose of items 1 and 2. Lists are ascending; entries after the count
+    are 0; the shapes are [B, H, KB] and [B, H, KB, QB]."""
+    out = {}
+    for src_num, src_idx, dst_num, dst_idx in (("kv_num_blocks", "kv_indices", "q_num_blocks", "q_indices"),
+                                               ("full_kv_num_blocks", "full_kv_indices", "full_q_num_blocks",
+                                                "full_q_indices")):
+        num, idx = bm[src_num], bm[src_idx]
+        Bm, Hm, QB, KB = idx.shape
+        cols = [[[[] for _ in range(KB)] for _ in range(Hm)] for _ in range(Bm)]
+        for b in range(Bm):
+            for h in range(Hm):
+                for qb in range(QB):
+                    for j in range(num[b, h, qb]):
+                        cols[b][h][idx[b, h, qb, j]].append(qb)
+        q_num = np.zeros((Bm, Hm, KB), np.int32)
+        q_idx = np.zeros((Bm, Hm, KB, QB), np.int32)
+        for b in range(Bm):
+            for h in range(Hm):
+                for kb in range(KB):
+                    lst = sorted(cols[b][h][kb])
+                    q_num[b, h, kb] = len(lst)
+                    q_idx[b, h, kb, :len(lst)] = lst
+        out[dst_num] = q_num
+        out[dst_idx] = q_idx
+    return out

@@ -189,3 +189,44 @@ def test_sparsity_percentage():
 def test_broadcast_b_h_none():
     bm = obm.create_block_mask(("causal",), 0, None or 0, 256, 256)
     assert bm["kv_indices"].shape == (1, 1, 2, 2)
+
+
+def test_q_side_matches_tile_columns():
+    # tensorplay.nn.attention, BlockMask "Details" items 3-4: the q-side lists
+    # are the transpose of the kv-side ones; checked against the columns of the
+    # brute-force tile classification, a path that never reads the kv lists
+    ids = np.repeat(np.arange(3), [150, 200, 170]).astype(np.int32)
+    M = N = 520
+    trees = [("causal",), ("and", ("causal",), ("or", ("sink", 5), ("window", 200))),
+             ("and", ("document", ids[None], ids[None]), ("causal",)), ("prefix_lm", 300)]
+    for tree in trees:
+        bm = obm.create_block_mask(tree, 1, 2, M, N)
+        qs = obm.q_side(bm)
+        cls = obm.tile_classes(tree, 0, M, N)
+        QB, KB = cls.shape
+        for h in range(2):
+            for kb in range(KB):
+                part = np.nonzero(cls[:, kb] == 1)[0]
+                full = np.nonzero(cls[:, kb] == 2)[0]
+                assert qs["q_num_blocks"][0, h, kb] == len(part)
+                assert qs["full_q_num_blocks"][0, h, kb] == len(full)
+                assert list(qs["q_indices"][0, h, kb, :len(part)]) == list(part)
+                assert list(qs["full_q_indices"][0, h, kb, :len(full)]) == list(full)
+                assert not qs["q_indices"][0, h, kb, len(part):].any()
+                assert not qs["full_q_indices"][0, h, kb, len(full):].any()
+
+
+def test_q_side_twice_is_the_identity():
+    rng = np.random.default_rng(11)
+    for _ in range(5):
+        M, N = int(rng.integers(1, 700)), int(rng.integers(1, 700))
+        tree = ("and", ("causal",), ("window", int(rng.integers(1, 400))))
+        bm = obm.create_block_mask(tree, 2, 1, M, N)
+        qs = obm.q_side(bm)
+        back = obm.q_side({"kv_num_blocks": qs["q_num_blocks"], "kv_indices": qs["q_indices"],
+                           "full_kv_num_blocks": qs["full_q_num_blocks"],
+                           "full_kv_indices": qs["full_q_indices"]})
+        assert np.array_equal(back["q_num_blocks"], bm["kv_num_blocks"])
+        assert np.array_equal(back["q_indices"], bm["kv_indices"])
+        assert np.array_equal(back["full_q_num_blocks"], bm["full_kv_num_blocks"])
+        assert np.array_equal(back["full_q_indices"], bm["full_kv_indices"])
