@@ -63,6 +63,11 @@ class _ScoreSpec(ctypes.Structure):
     _fields_ = [("num_ops", ctypes.c_int32), ("ops", _ScoreOp * MAX_SCORE_OPS)]
 
 
+class _BlockMaskQ(ctypes.Structure):
+    _fields_ = [("q_num_blocks", ctypes.c_void_p), ("q_indices", ctypes.c_void_p),
+                ("full_q_num_blocks", ctypes.c_void_p), ("full_q_indices", ctypes.c_void_p)]
+
+
 class _BlockMask(ctypes.Structure):
     _fields_ = [("kv_num_blocks", ctypes.c_void_p), ("kv_indices", ctypes.c_void_p),
                 ("full_kv_num_blocks", ctypes.c_void_p), ("full_kv_indices", ctypes.c_void_p),
@@ -87,6 +92,10 @@ def _load() -> ctypes.CDLL:
                                             ctypes.POINTER(_MaskSpec), ctypes.POINTER(_ScoreSpec), ctypes.c_float,
                                             i32, vp, vp, vp]
     lib.bsmt_flex_attention_fwd.restype = i32
+    lib.bsmt_block_mask_transpose.argtypes = [ctypes.POINTER(_BlockMask), ctypes.POINTER(_BlockMaskQ), vp]
+    lib.bsmt_block_mask_transpose.restype = i32
+    lib.bsmt_block_mask_to_dense.argtypes = [ctypes.POINTER(_BlockMask), vp, vp]
+    lib.bsmt_block_mask_to_dense.restype = i32
     lib.bsmt_last_error.argtypes = []
     lib.bsmt_last_error.restype = ctypes.c_char_p
     lib.bsmt_check_device_status.argtypes = [vp]
@@ -313,6 +322,89 @@ class BlockMask:
         c.Q_LEN, c.KV_LEN = self.seq_lengths
         c.BLOCK_Q, c.BLOCK_KV = self.BLOCK_SIZE
         return c
+
+    def q_side(self) -> dict:
+        """The q-side lists (tensorplay.nn.attention, BlockMask "Details" items 3-4),
+        computed on the GPU on first use and kept: q_num_blocks [B, H, KB],
+        q_indices [B, H, KB, QB], full_q_num_blocks, full_q_indices."""
+        cached = getattr(self, "_q_side", None)
+        if cached is not None:
+            return cached
+        Bm, Hm, QB, KB = self.shape
+        dev = self.kv_indices.device
+        t = {"q_num_blocks": torch.empty((Bm, Hm, KB), dtype=torch.int32, device=dev),
+             "q_indices": torch.empty((Bm, Hm, KB, QB), dtype=torch.int32, device=dev),
+             "full_q_num_blocks": torch.empty((Bm, Hm, KB), dtype=torch.int32, device=dev),
+             "full_q_indices": torch.empty((Bm, Hm, KB, QB), dtype=torch.int32, device=dev)}
+        cq = _BlockMaskQ()
+        cq.q_num_blocks = t["q_num_blocks"].data_ptr()
+        cq.q_indices = t["q_indices"].data_ptr()
+        cq.full_q_num_blocks = t["full_q_num_blocks"].data_ptr()
+        cq.full_q_indices = t["full_q_indices"].data_ptr()
+        c = self._c()
+        with torch.cuda.device(dev):
+            _check(_lib.bsmt_block_mask_transpose(ctypes.byref(c), ctypes.byref(cq),
+                                                  ctypes.c_void_p(_stream_ptr(dev))))
+        self._q_side = t
+        return t
+
+    @property
+    def q_num_blocks(self) -> torch.Tensor:
+        return self.q_side()["q_num_blocks"]
+
+    @property
+    def q_indices(self) -> torch.Tensor:
+        return self.q_side()["q_indices"]
+
+    @property
+    def full_q_num_blocks(self) -> torch.Tensor:
+        return self.q_side()["full_q_num_blocks"]
+
+    @property
+    def full_q_indices(self) -> torch.Tensor:
+        return self.q_side()["full_q_indices"]
+
+    def to_dense(self) -> torch.Tensor:
+        """int32 [B, H, QB, KB]: 1 where a row's partial or full list holds the block
+        (the reconstruction loop of tensorplay.nn.attention, BlockMask "Basics")."""
+        dev = self.kv_indices.device
+        dense = torch.empty(self.shape, dtype=torch.int32, device=dev)
+        c = self._c()
+        with torch.cuda.device(dev):
+            _check(_lib.bsmt_block_mask_to_dense(ctypes.byref(c), ctypes.c_void_p(dense.data_ptr()),
+                                                 ctypes.c_void_p(_stream_ptr(dev))))
+        return dense
+
+    @classmethod
+    def from_kv_blocks(cls, kv_num_blocks: torch.Tensor, kv_indices: torch.Tensor,
+                       full_kv_num_blocks: torch.Tensor | None = None, full_kv_indices: torch.Tensor | None = None,
+                       BLOCK_SIZE: int | tuple[int, int] = 128, mask_mod: "MaskMod | None" = None,
+                       seq_lengths: tuple[int, int] | None = None) -> "BlockMask":
+        """A BlockMask from precomputed kv-side lists (tensorplay.nn.attention,
+        BlockMask.from_kv_blocks); the q-side lists are generated on the GPU.
+        Raises ValueError for lists of the wrong rank, dtype or shape."""
+        bq, bkv = _block_pair(BLOCK_SIZE)
+        if kv_indices.dim() != 4 or kv_num_blocks.dim() != 3:
+            raise ValueError("kv_num_blocks must be [B, H, QB] and kv_indices [B, H, QB, KB]")
+        if full_kv_num_blocks is None:
+            full_kv_num_blocks = torch.zeros_like(kv_num_blocks)
+            full_kv_indices = torch.zeros_like(kv_indices)
+        for name, t in (("kv_num_blocks", kv_num_blocks), ("kv_indices", kv_indices),
+                        ("full_kv_num_blocks", full_kv_num_blocks), ("full_kv_indices", full_kv_indices)):
+            if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+        Bm, Hm, QB, KB = kv_indices.shape
+        if (tuple(kv_num_blocks.shape) != (Bm, Hm, QB) or tuple(full_kv_num_blocks.shape) != (Bm, Hm, QB)
+                or tuple(full_kv_indices.shape) != (Bm, Hm, QB, KB)):
+            raise ValueError("BlockMask tensors disagree in shape")
+        if seq_lengths is None:
+            seq_lengths = (QB * bq, KB * bkv)
+        if mask_mod is None:
+            mask_mod = noop_mask()
+        bm = cls(tuple(int(x) for x in seq_lengths), kv_num_blocks, kv_indices, full_kv_num_blocks,
+                 full_kv_indices, (bq, bkv), mask_mod)
+        bm.q_side()
+        return bm
 
     def sparsity(self) -> float:
         """Percentage of blocks that are not computed (reads the counts back to the host)."""

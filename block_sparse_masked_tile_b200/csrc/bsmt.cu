@@ -18,6 +18,7 @@
 #include "attn_fwd.cuh"
 #include "bsmt.h"
 #include "mask_build.cuh"
+#include "mask_transpose.cuh"
 #include "mask_dnf.cuh"
 #include "ptx.cuh"
 
@@ -504,3 +505,91 @@ bsmt_status bsmt_check_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+namespace {
+// Shared checks of a kv-side BlockMask passed in by the caller.
+bsmt_status check_kv_side(const bsmt_block_mask* kv) {
+    if (kv == nullptr) return fail(BSMT_ERR_INVALID_ARGUMENT, "block mask is NULL");
+    if (kv->B < 0 || kv->H < 0 || kv->QB < 0 || kv->KB < 0)
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "block mask shape fields must be non-negative");
+    const int64_t rows = static_cast<int64_t>(kv->B) * kv->H * kv->QB;
+    if (rows > 0) {
+        if (!kv->kv_num_blocks || !kv->full_kv_num_blocks || (kv->KB > 0 && (!kv->kv_indices || !kv->full_kv_indices)))
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "block mask pointers must be non-NULL");
+        if (!aligned(kv->kv_num_blocks, 4) || !aligned(kv->kv_indices, 4) || !aligned(kv->full_kv_num_blocks, 4) ||
+            !aligned(kv->full_kv_indices, 4))
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "block mask pointers must be 4-byte aligned");
+    }
+    return BSMT_OK;
+}
+}  // namespace
+
+extern "C" bsmt_status bsmt_block_mask_transpose(const bsmt_block_mask* kv, bsmt_block_mask_q* out, void* stream) {
+    bsmt_status st = check_kv_side(kv);
+    if (st != BSMT_OK) return st;
+    if (out == nullptr) return fail(BSMT_ERR_INVALID_ARGUMENT, "q-side output is NULL");
+    const int64_t cols = static_cast<int64_t>(kv->B) * kv->H * kv->KB;
+    if (cols == 0) return ok();
+    if (!out->q_num_blocks || !out->full_q_num_blocks || (kv->QB > 0 && (!out->q_indices || !out->full_q_indices)))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "q-side output pointers must be non-NULL");
+    if (!aligned(out->q_num_blocks, 4) || !aligned(out->q_indices, 4) || !aligned(out->full_q_num_blocks, 4) ||
+        !aligned(out->full_q_indices, 4))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "q-side output pointers must be 4-byte aligned");
+    if (kv->QB > 12800) return fail(BSMT_ERR_UNSUPPORTED, "QB=%d above 12800", kv->QB);
+    if (kv->H > 65535 || kv->B > 65535) return fail(BSMT_ERR_UNSUPPORTED, "B or H above 65535");
+    int dev = 0, nsm = 0;
+    st = sm_count(&dev, &nsm);
+    if (st != BSMT_OK) return st;
+    const int smem = static_cast<int>(bsmt::transpose_smem_bytes(kv->QB));
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(bsmt::mask_transpose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    }
+    bsmt::TransposeParams p;
+    p.Bm = kv->B;
+    p.Hm = kv->H;
+    p.QB = kv->QB;
+    p.KB = kv->KB;
+    p.kv_num = kv->kv_num_blocks;
+    p.kv_idx = kv->kv_indices;
+    p.full_num = kv->full_kv_num_blocks;
+    p.full_idx = kv->full_kv_indices;
+    p.q_num = out->q_num_blocks;
+    p.q_idx = out->q_indices;
+    p.full_q_num = out->full_q_num_blocks;
+    p.full_q_idx = out->full_q_indices;
+    dim3 grid(static_cast<unsigned>((kv->KB + bsmt::kTransposeChunk - 1) / bsmt::kTransposeChunk),
+              static_cast<unsigned>(kv->H), static_cast<unsigned>(kv->B));
+    bsmt::mask_transpose_kernel<<<grid, bsmt::kTransposeThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "transpose launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+extern "C" bsmt_status bsmt_block_mask_to_dense(const bsmt_block_mask* kv, int32_t* dense, void* stream) {
+    bsmt_status st = check_kv_side(kv);
+    if (st != BSMT_OK) return st;
+    const int64_t rows = static_cast<int64_t>(kv->B) * kv->H * kv->QB;
+    if (rows == 0 || kv->KB == 0) return ok();
+    if (dense == nullptr || !aligned(dense, 4))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "dense output must be non-NULL and 4-byte aligned");
+    int dev = 0, nsm = 0;
+    st = sm_count(&dev, &nsm);
+    if (st != BSMT_OK) return st;
+    bsmt::DenseParams p;
+    p.Bm = kv->B;
+    p.Hm = kv->H;
+    p.QB = kv->QB;
+    p.KB = kv->KB;
+    p.kv_num = kv->kv_num_blocks;
+    p.kv_idx = kv->kv_indices;
+    p.full_num = kv->full_kv_num_blocks;
+    p.full_idx = kv->full_kv_indices;
+    p.dense = dense;
+    const int64_t blocks = (rows + 3) / 4;
+    if (blocks > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "grid too large");
+    bsmt::mask_to_dense_kernel<<<static_cast<unsigned>(blocks), 128, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "to_dense launch: %s", cudaGetErrorString(e));
+    return ok();
+}

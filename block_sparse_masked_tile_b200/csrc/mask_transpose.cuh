@@ -1,0 +1,154 @@
+// q-side BlockMask lists and the block-level dense map.
+//
+// tensorplay.nn.attention page, BlockMask "Details" items 3-4: q_num_blocks /
+// q_indices and full_q_num_blocks / full_q_indices are the transpose of the
+// kv-side lists. For every kv block they hold the q blocks whose partial
+// (resp. full) list contains it, ascending, followed by zeros.
+//
+// One CTA per (b, h, chunk of 32 kv blocks). Its warps read every q row's
+// two lists of (b, h) and set one bit per (kv block of the chunk, q block) in
+// two shared-memory bitmaps. Each warp then compacts whole kv columns: a
+// ballot/popc prefix per 32-bit word gives every set bit its position. The
+// kernel writes every element of its output columns, so it is bound by the
+// HBM writes of [B, H, KB, QB] x 2 lists.
+//
+// BlockMask "Basics" (the reconstruction loop) defines the dense map: a
+// block is 1 when either list of its row holds it.
+#pragma once
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace bsmt {
+
+constexpr int kTransposeChunk = 32;   // kv blocks per CTA
+constexpr int kTransposeThreads = 256;
+
+struct TransposeParams {
+    int32_t Bm, Hm, QB, KB;
+    const int32_t* kv_num;
+    const int32_t* kv_idx;
+    const int32_t* full_num;
+    const int32_t* full_idx;
+    int32_t* q_num;
+    int32_t* q_idx;
+    int32_t* full_q_num;
+    int32_t* full_q_idx;
+};
+
+// Shared memory: two bitmaps of kTransposeChunk x ceil(QB / 32) words.
+__host__ __device__ constexpr int64_t transpose_smem_bytes(int64_t QB) {
+    return 2 * kTransposeChunk * ((QB + 31) / 32) * 4;
+}
+
+__global__ void __launch_bounds__(kTransposeThreads) mask_transpose_kernel(const TransposeParams p) {
+    extern __shared__ uint32_t bits[];  // [2][kTransposeChunk][qw]
+    const int qw = (p.QB + 31) / 32;
+    const int kb0 = blockIdx.x * kTransposeChunk;
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = kTransposeThreads / 32;
+    for (int i = threadIdx.x; i < 2 * kTransposeChunk * qw; i += kTransposeThreads) bits[i] = 0u;
+    __syncthreads();
+
+    // scatter: q row qb's kv blocks that fall into this chunk
+    const int64_t row0 = (static_cast<int64_t>(b) * p.Hm + h) * p.QB;
+    bool bad = false;
+    for (int qb = warp; qb < p.QB; qb += nwarps) {
+#pragma unroll
+        for (int l = 0; l < 2; ++l) {
+            const int32_t* num = l == 0 ? p.kv_num : p.full_num;
+            const int32_t* idx = (l == 0 ? p.kv_idx : p.full_idx) + (row0 + qb) * p.KB;
+            int n = __ldg(num + row0 + qb);
+            if (n < 0 || n > p.KB) {
+                bad = true;
+                n = 0;
+            }
+            for (int j = lane; j < n; j += 32) {
+                const int kb = __ldg(idx + j);
+                if (kb < 0 || kb >= p.KB) {
+                    bad = true;
+                } else if (kb >= kb0 && kb < kb0 + kTransposeChunk) {
+                    atomicOr(&bits[(l * kTransposeChunk + (kb - kb0)) * qw + (qb >> 5)], 1u << (qb & 31));
+                }
+            }
+        }
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
+    __syncthreads();
+
+    // compact: one warp per (list, kv column)
+    const uint32_t below = (1u << lane) - 1u;
+    for (int c = warp; c < 2 * kTransposeChunk; c += nwarps) {
+        const int l = c / kTransposeChunk;
+        const int kb = kb0 + (c % kTransposeChunk);
+        if (kb >= p.KB) continue;
+        const uint32_t* col = bits + c * qw;
+        int32_t* out = (l == 0 ? p.q_idx : p.full_q_idx) + ((static_cast<int64_t>(b) * p.Hm + h) * p.KB + kb) * p.QB;
+        int pos = 0;
+        for (int w0 = 0; w0 < qw; w0 += 32) {
+            // lane handles word w0 + lane: its bits' positions follow the set
+            // bits of the lower lanes' words
+            const uint32_t word = (w0 + lane < qw) ? col[w0 + lane] : 0u;
+            const int cnt = __popc(word);
+            int incl = cnt;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+                if (lane >= d) incl += v;
+            }
+            int at = pos + incl - cnt;
+            uint32_t rest = word;
+            while (rest) {
+                const int bit = __ffs(rest) - 1;
+                rest &= rest - 1u;
+                out[at++] = (w0 + lane) * 32 + bit;
+            }
+            pos += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        for (int j = pos + lane; j < p.QB; j += 32) out[j] = 0;
+        if (lane == 0) (l == 0 ? p.q_num : p.full_q_num)[(static_cast<int64_t>(b) * p.Hm + h) * p.KB + kb] = pos;
+    }
+}
+
+struct DenseParams {
+    int32_t Bm, Hm, QB, KB;
+    const int32_t* kv_num;
+    const int32_t* kv_idx;
+    const int32_t* full_num;
+    const int32_t* full_idx;
+    int32_t* dense;  // [B, H, QB, KB]
+};
+
+// One warp per (b, h, q row): zero the row, then set the listed blocks. The
+// warp's own writes are ordered by __syncwarp.
+__global__ void __launch_bounds__(128) mask_to_dense_kernel(const DenseParams p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t rows = static_cast<int64_t>(p.Bm) * p.Hm * p.QB;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+    if (row >= rows) return;
+    int32_t* out = p.dense + row * p.KB;
+    for (int j = lane; j < p.KB; j += 32) out[j] = 0;
+    __syncwarp();
+    bool bad = false;
+#pragma unroll
+    for (int l = 0; l < 2; ++l) {
+        int n = __ldg((l == 0 ? p.kv_num : p.full_num) + row);
+        if (n < 0 || n > p.KB) {
+            bad = true;
+            n = 0;
+        }
+        const int32_t* idx = (l == 0 ? p.kv_idx : p.full_idx) + row * p.KB;
+        for (int j = lane; j < n; j += 32) {
+            const int kb = __ldg(idx + j);
+            if (kb < 0 || kb >= p.KB)
+                bad = true;
+            else
+                out[kb] = 1;
+        }
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
+}
+
+}  // namespace bsmt

@@ -180,6 +180,38 @@ bsmt_status bsmt_create_block_mask(const bsmt_mask_spec* spec, int64_t B, int64_
                                    int64_t Q_LEN, int64_t KV_LEN, int32_t BLOCK_Q,
                                    int32_t BLOCK_KV, bsmt_block_mask* out, void* stream);
 
+/* q-side lists of a BlockMask: the transpose of its kv-side lists
+ * (tensorplay.nn.attention page, BlockMask "Details" items 3 and 4).
+ *   q_num_blocks       [B, H, KB]      number of q blocks whose PARTIAL list holds kv block kb
+ *   q_indices          [B, H, KB, QB]  those q blocks, ascending, then 0s
+ *   full_q_num_blocks  [B, H, KB]      the same for the FULL lists
+ *   full_q_indices     [B, H, KB, QB]
+ * B, H, QB, KB are the kv-side BlockMask's. Caller-owned device memory,
+ * contiguous, 4-byte aligned. */
+typedef struct bsmt_block_mask_q {
+    int32_t* q_num_blocks;
+    int32_t* q_indices;
+    int32_t* full_q_num_blocks;
+    int32_t* full_q_indices;
+} bsmt_block_mask_q;
+
+/* Writes the q-side lists of `kv` (its four kv-side tensors and shape fields
+ * are read; the lists may come from bsmt_create_block_mask or from the
+ * caller). Every element of the four outputs is written. A kv-side count
+ * outside [0, KB] or an index outside [0, KB) is skipped and reported as
+ * BSMT_ERR_DEVICE_BOUNDS by bsmt_check_device_status. QB above 12800 returns
+ * BSMT_ERR_UNSUPPORTED (the kernel's shared-memory bitmaps). Stream-ordered
+ * on `stream`. */
+bsmt_status bsmt_block_mask_transpose(const bsmt_block_mask* kv, bsmt_block_mask_q* out, void* stream);
+
+/* Block-level dense map of a BlockMask: dense[b, h, qb, kb] = 1 when the
+ * partial or the full list of row (b, h, qb) holds kb, else 0 (the
+ * reconstruction loop of tensorplay.nn.attention, BlockMask "Basics").
+ * dense is caller-owned device int32 [B, H, QB, KB], 4-byte aligned. Bad
+ * counts or indices are skipped and reported as BSMT_ERR_DEVICE_BOUNDS.
+ * Stream-ordered on `stream`. */
+bsmt_status bsmt_block_mask_to_dense(const bsmt_block_mask* kv, int32_t* dense, void* stream);
+
 /* flex_attention forward with a BlockMask:
  *   out[b,hq,i,:] = softmax_j( mod(scale * q_i . k_j) masked ) @ v
  *   lse[b,hq,i]   = natural log-sum-exp of the modified, masked scores
@@ -206,9 +238,9 @@ bsmt_status bsmt_create_block_mask(const bsmt_mask_spec* spec, int64_t B, int64_
  *   lse     device float [B, Hq, M], 4-byte aligned
  *   A tensor with no elements (M == 0, N == 0 or B == 0) may be NULL.
  *
- * Both index lists of each BlockMask row must be ascending and their union
- * must hold distinct values; the kernel checks this and reports
- * BSMT_ERR_DEVICE_BOUNDS.
+ * A block listed in both lists of a row is treated as PARTIAL; the order of
+ * a list does not matter. A count outside [0, KB] or an index outside
+ * [0, KB) is skipped and reported as BSMT_ERR_DEVICE_BOUNDS.
  */
 bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v,
                                     int64_t B, int64_t Hq, int64_t Hkv, int64_t M, int64_t N,

@@ -27,6 +27,7 @@ def declared_functions():
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
     assert names == sorted(["bsmt_block_mask_shape", "bsmt_create_block_mask", "bsmt_flex_attention_fwd",
+                            "bsmt_block_mask_transpose", "bsmt_block_mask_to_dense",
                             "bsmt_last_error", "bsmt_check_device_status", "bsmt_version"])
     lib = ctypes.CDLL(bsmt.library_path())
     for n in names:
@@ -198,3 +199,28 @@ def test_python_errors_map_to_value_error():
         bsmt._check(SHAPE)
     with pytest.raises(RuntimeError):
         bsmt._check(UNSUPPORTED)
+
+
+def test_transpose_and_to_dense_argument_errors():
+    from block_sparse_masked_tile_b200 import _BlockMaskQ
+    null = ctypes.c_void_p(0)
+    assert _lib.bsmt_block_mask_transpose(None, ctypes.byref(_BlockMaskQ()), null) == INVALID
+    assert _lib.bsmt_block_mask_to_dense(None, ctypes.c_void_p(FAKE), null) == INVALID
+    bm = _BlockMask()
+    bm.B, bm.H, bm.QB, bm.KB = 1, 1, -1, 4
+    assert _lib.bsmt_block_mask_transpose(ctypes.byref(bm), ctypes.byref(_BlockMaskQ()), null) == INVALID
+    bm.QB = 4
+    assert _lib.bsmt_block_mask_transpose(ctypes.byref(bm), ctypes.byref(_BlockMaskQ()), null) == INVALID  # NULL lists
+    bm.kv_num_blocks = bm.kv_indices = bm.full_kv_num_blocks = bm.full_kv_indices = FAKE
+    assert _lib.bsmt_block_mask_transpose(ctypes.byref(bm), None, null) == INVALID
+    assert _lib.bsmt_block_mask_transpose(ctypes.byref(bm), ctypes.byref(_BlockMaskQ()), null) == INVALID
+    q = _BlockMaskQ()
+    q.q_num_blocks = q.q_indices = q.full_q_num_blocks = q.full_q_indices = FAKE + 2  # misaligned
+    assert _lib.bsmt_block_mask_transpose(ctypes.byref(bm), ctypes.byref(q), null) == INVALID
+    q.q_num_blocks = q.q_indices = q.full_q_num_blocks = q.full_q_indices = FAKE
+    bm.QB = 20000
+    assert _lib.bsmt_block_mask_transpose(ctypes.byref(bm), ctypes.byref(q), null) == UNSUPPORTED
+    assert _lib.bsmt_block_mask_to_dense(ctypes.byref(bm), None, null) == INVALID
+    bm.QB, bm.KB = 4, 0  # no kv column: nothing to write, nothing launched
+    assert _lib.bsmt_block_mask_transpose(ctypes.byref(bm), ctypes.byref(q), null) == OK
+    assert _lib.bsmt_block_mask_to_dense(ctypes.byref(bm), None, null) == OK
