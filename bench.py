@@ -156,6 +156,66 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def _time_launches(fn, reps: int = 20) -> float:
+    """Mean ms per call of fn: reps calls are captured in a CUDA graph (so the
+    host's launch cost stays out), and the graph replay is timed with CUDA
+    events on the replay stream."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(3):
+        g.replay()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (3 * reps)
+    del g
+    return ms
+
+
+def side_kernels(bsmt, mask, w, dev, hbm_peak: float) -> dict:
+    """The HBM-bound kernels timed alone (outside the step): the block-mask
+    builder at the step's shape and at B=8, H=32 (outputs larger than L2), and
+    the q-side transpose. Algorithmic bytes are the outputs written: two count
+    tensors and two index tensors."""
+    import ctypes
+    res = {}
+    for label, B, H in (("mask_build", w.B, w.Hq), ("mask_build_b8_h32", 8, 32)):
+        if w.mask == "doc_causal" and B != w.B:
+            continue  # document ids are per batch row of the workload
+        bm = bsmt.create_block_mask(mask, B, H, w.M, w.N, device=dev)
+        ms = _time_launches(lambda: bsmt.create_block_mask(mask, B, H, w.M, w.N, device=dev, out=bm))
+        Bm, Hm, QB, KB = bm.shape
+        nbytes = 2 * 4 * Bm * Hm * QB + 2 * 4 * Bm * Hm * QB * KB
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[label] = {"B": Bm, "H": Hm, "ms": ms, "bytes": nbytes, "achieved_gbs": gbs, "peak_gbs": hbm_peak,
+                      "frac": gbs / hbm_peak, "note": "outputs larger than L2" if nbytes > 126e6 else "outputs fit in L2"}
+        if label == "mask_build":
+            qs = bm.q_side()
+            cq = bsmt._BlockMaskQ()
+            cq.q_num_blocks = qs["q_num_blocks"].data_ptr()
+            cq.q_indices = qs["q_indices"].data_ptr()
+            cq.full_q_num_blocks = qs["full_q_num_blocks"].data_ptr()
+            cq.full_q_indices = qs["full_q_indices"].data_ptr()
+            c = bm._c()
+            ms = _time_launches(lambda: bsmt._lib.bsmt_block_mask_transpose(
+                ctypes.byref(c), ctypes.byref(cq), ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
+            qbytes = 2 * 4 * Bm * Hm * KB + 2 * 4 * Bm * Hm * KB * QB
+            gbs = qbytes / (ms * 1e-3) / 1e9
+            res["q_side_transpose"] = {"ms": ms, "bytes": qbytes, "achieved_gbs": gbs, "peak_gbs": hbm_peak,
+                                       "frac": gbs / hbm_peak}
+        bsmt.check_device_status(dev)
+    return res
+
+
 def counted_flops(bm, D: int) -> int:
     """4*128*128*D per kept tile per (b, hq); the mask is built at [B, Hq]."""
     tiles = int(bm.kv_num_blocks.sum().item()) + int(bm.full_kv_num_blocks.sum().item())
@@ -327,6 +387,8 @@ def main():
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
     peaks, peak_src = load_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    side = side_kernels(bsmt, mask, w, dev, hbm_peak)
     attn_tflops = (flops / (attn_ms * 1e-3)) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     traffic = profile_traffic(w.name)
@@ -366,6 +428,7 @@ def main():
         },
         "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
+        "side_kernels": side,
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
