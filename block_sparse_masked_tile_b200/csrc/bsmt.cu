@@ -336,7 +336,7 @@ bsmt_status bsmt_create_block_mask(const bsmt_mask_spec* spec, int64_t B, int64_
     p.kv_idx = out->kv_indices;
     p.full_num = out->full_kv_num_blocks;
     p.full_idx = out->full_kv_indices;
-    const int64_t gx = (p.QB + bsmt::kBuildWarps - 1) / bsmt::kBuildWarps;
+    const int64_t gx = p.QB;  // one block per q-block row
     const int64_t blocks_xy = gx * p.Bm;
     int64_t groups = (2 * nsm + blocks_xy - 1) / blocks_xy;
     if (groups < 1) groups = 1;

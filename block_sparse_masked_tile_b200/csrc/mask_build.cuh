@@ -1,21 +1,23 @@
 // Block-mask builder kernel (create_block_mask with separate_full_blocks).
 //
 // Reference: tensorplay.nn.attention page, create_block_mask and BlockMask
-// "Details" items 1-2. One warp owns one (b, q-block) row of 128 queries;
-// lane l evaluates rows l, l+32, l+64, l+96.
+// "Details" items 1-2. One block of 8 warps owns one (b, q-block) row of
+// 128 queries and a group of heads.
 //
+// Classification: warps 0-3 take one query row per lane (rows 32w + lane).
 // Per row, the DNF mask gives a union of at most kMaxTerms kv intervals. The
 // kernel sorts and merges them into disjoint intervals. Every interval then
 // sets bit ranges over kv blocks: "any" covers the blocks the interval
 // touches, "full" the blocks it covers entirely. AND-reducing "full" and
-// OR-reducing "any" over the 128 rows with redux.sync classifies each tile
-// exactly:
+// OR-reducing "any" over the rows (redux.sync within a warp, then over the
+// four warps in shared memory) classifies each tile exactly:
 //   - FULL    = every in-range element allowed, tile inside both sequences;
 //   - PARTIAL = some element allowed but not FULL;
 //   - EMPTY   = no element allowed.
-// Compaction is a ballot/popc prefix per 32-tile word. A mask is the same
-// for every head, so the rows are computed once and written for each head
-// of the block's head group. That makes the kernel a pure HBM writer.
+// Writing: a mask is the same for every head, so all 8 warps then write the
+// row's lists for the heads of the block's group, a head per warp at a time.
+// Compaction is a ballot/popc prefix per 32-tile word; tails are zeroed with
+// 16-byte stores. The kernel is then an HBM writer.
 #pragma once
 #include "mask_dnf.cuh"
 #include "ptx.cuh"
@@ -31,31 +33,34 @@ struct BuildParams {
     int32_t* full_idx;
 };
 
-constexpr int kBuildWarps = 4;
-constexpr int kWordsPerChunk = 8;  // 256 kv blocks per pass
+constexpr int kBuildWarps = 8;       // warps per block
+constexpr int kClassifyWarps = 4;    // warps that classify (one row per lane)
+constexpr int kWordsPerChunk = 8;    // 256 kv blocks per pass
 
 __global__ void __launch_bounds__(kBuildWarps * 32) mask_build_kernel(const MaskDnf dnf, const BuildParams p) {
+    __shared__ uint32_t part_f[kClassifyWarps][kWordsPerChunk];
+    __shared__ uint32_t part_a[kClassifyWarps][kWordsPerChunk];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int qb = blockIdx.x * kBuildWarps + warp;
+    const int qb = blockIdx.x;
     const int b = blockIdx.y;
-    if (qb >= p.QB) return;  // warp-uniform; no block-wide barrier below
     const int h0 = blockIdx.z * p.heads_per_block;
     const int h1 = min(p.Hm, h0 + p.heads_per_block);
     const int64_t N = p.KV_LEN;
     const int64_t M = p.Q_LEN;
+    const bool classifier = warp < kClassifyWarps;
 
     // Document ids: row pointers and the sortedness check of this block's
     // share of kv positions (every kv position is checked by exactly one
-    // (qb, head-group 0) warp per batch row).
+    // (qb, head-group 0) block per batch row, in its warp 0).
     const int32_t* qdoc = nullptr;
     const int32_t* kvdoc = nullptr;
     if (dnf.has_doc) {
         const int db = dnf.doc_batch > 1 ? b : 0;
         qdoc = dnf.q_doc + static_cast<int64_t>(db) * M;
         kvdoc = dnf.kv_doc + static_cast<int64_t>(db) * N;
-        if (blockIdx.z == 0) {
-            // kv blocks j with j % QB == qb belong to this warp
+        if (blockIdx.z == 0 && warp == 0) {
+            // kv blocks j with j % QB == qb belong to this block
             bool bad = false;
             for (int64_t seg = static_cast<int64_t>(qb) * 128; seg < N; seg += static_cast<int64_t>(p.QB) * 128) {
 #pragma unroll
@@ -68,34 +73,57 @@ __global__ void __launch_bounds__(kBuildWarps * 32) mask_build_kernel(const Mask
         }
     }
 
-    // Per-row query index, validity and document interval [ds, de].
-    int64_t qr[4];
-    bool valid[4];
-    int64_t ds[4], de[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        qr[r] = static_cast<int64_t>(qb) * 128 + lane + 32 * r;
-        valid[r] = qr[r] < M;
-        ds[r] = 0;
-        de[r] = N - 1;
-    }
-    if (dnf.has_doc) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int32_t d = valid[r] ? __ldg(qdoc + qr[r]) : 0;
-            bool pending = valid[r];
-            unsigned todo;
-            while ((todo = __ballot_sync(0xFFFFFFFFu, pending)) != 0u) {
-                const int leader = __ffs(todo) - 1;
-                const int32_t x = __shfl_sync(0xFFFFFFFFu, d, leader);
-                const int first = warp_lower_bound(kvdoc, static_cast<int>(N), x, lane);
-                const int past = warp_lower_bound(kvdoc, static_cast<int>(N), static_cast<int64_t>(x) + 1, lane);
-                if (pending && d == x) {
-                    ds[r] = first;
-                    de[r] = past - 1;
-                    pending = false;
-                }
+    // This lane's query row (classifying warps), its validity and document
+    // interval [ds, de].
+    const int64_t qr = static_cast<int64_t>(qb) * 128 + 32 * warp + lane;
+    const bool valid = classifier && qr < M;
+    int64_t ds = 0, de = N - 1;
+    if (dnf.has_doc && classifier) {
+        const int32_t d = valid ? __ldg(qdoc + qr) : 0;
+        bool pending = valid;
+        unsigned todo;
+        while ((todo = __ballot_sync(0xFFFFFFFFu, pending)) != 0u) {
+            const int leader = __ffs(todo) - 1;
+            const int32_t x = __shfl_sync(0xFFFFFFFFu, d, leader);
+            const int first = warp_lower_bound(kvdoc, static_cast<int>(N), x, lane);
+            const int past = warp_lower_bound(kvdoc, static_cast<int>(N), static_cast<int64_t>(x) + 1, lane);
+            if (pending && d == x) {
+                ds = first;
+                de = past - 1;
+                pending = false;
             }
+        }
+    }
+    // The row's intervals, sorted by lo (insertion) and merged once.
+    int64_t lo[kMaxTerms], hi[kMaxTerms];
+    int nint = 0;
+    if (valid) {
+        int n = 0;
+        for (int t = 0; t < dnf.n_terms; ++t) {
+            int64_t l, h;
+            term_interval(dnf, t, qr, 0, N - 1, ds, de, l, h);
+            if (l > h) continue;
+            int j = n++;
+            while (j > 0 && lo[j - 1] > l) {
+                lo[j] = lo[j - 1];
+                hi[j] = hi[j - 1];
+                --j;
+            }
+            lo[j] = l;
+            hi[j] = h;
+        }
+        int i = 0;
+        while (i < n) {
+            const int64_t cl = lo[i];
+            int64_t ch = hi[i];
+            ++i;
+            while (i < n && lo[i] <= ch + 1) {
+                ch = hi[i] > ch ? hi[i] : ch;
+                ++i;
+            }
+            lo[nint] = cl;
+            hi[nint] = ch;
+            ++nint;
         }
     }
 
@@ -103,74 +131,53 @@ __global__ void __launch_bounds__(kBuildWarps * 32) mask_build_kernel(const Mask
     int cnt_p = 0, cnt_f = 0;
 
     for (int c0 = 0; c0 < p.KB; c0 += 32 * kWordsPerChunk) {
-        uint32_t fw[kWordsPerChunk], aw[kWordsPerChunk];
+        if (classifier) {
+            uint32_t fw[kWordsPerChunk], aw[kWordsPerChunk];
 #pragma unroll
-        for (int w = 0; w < kWordsPerChunk; ++w) {
-            fw[w] = 0xFFFFFFFFu;
-            aw[w] = 0u;
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            if (!valid[r]) continue;  // rows past Q_LEN add nothing; their tile is never FULL (below)
-            // intervals of this row, sorted by lo (insertion) and merged
-            int64_t lo[kMaxTerms], hi[kMaxTerms];
-            int n = 0;
-            for (int t = 0; t < dnf.n_terms; ++t) {
-                int64_t l, h;
-                term_interval(dnf, t, qr[r], 0, N - 1, ds[r], de[r], l, h);
-                if (l > h) continue;
-                int j = n++;
-                while (j > 0 && lo[j - 1] > l) {
-                    lo[j] = lo[j - 1];
-                    hi[j] = hi[j - 1];
-                    --j;
-                }
-                lo[j] = l;
-                hi[j] = h;
+            for (int w = 0; w < kWordsPerChunk; ++w) {
+                // rows past Q_LEN add nothing; their tile is never FULL (below)
+                fw[w] = valid ? 0u : 0xFFFFFFFFu;
+                aw[w] = 0u;
             }
-            uint32_t rf[kWordsPerChunk], ra[kWordsPerChunk];
-#pragma unroll
-            for (int w = 0; w < kWordsPerChunk; ++w) rf[w] = ra[w] = 0u;
-            int i = 0;
-            while (i < n) {
-                const int64_t cl = lo[i];
-                int64_t ch = hi[i];
-                ++i;
-                while (i < n && lo[i] <= ch + 1) {
-                    ch = hi[i] > ch ? hi[i] : ch;
-                    ++i;
-                }
-                const int64_t a_lo = cl >> 7, a_hi = ch >> 7;
-                const int64_t f_lo = (cl + 127) >> 7, f_hi = ((ch + 1) >> 7) - 1;
+            for (int i = 0; i < nint; ++i) {
+                const int64_t a_lo = lo[i] >> 7, a_hi = hi[i] >> 7;
+                const int64_t f_lo = (lo[i] + 127) >> 7, f_hi = ((hi[i] + 1) >> 7) - 1;
 #pragma unroll
                 for (int w = 0; w < kWordsPerChunk; ++w) {
                     const int64_t base = c0 + 32 * w;
-                    ra[w] |= range_bits(a_lo, a_hi, base);
-                    rf[w] |= range_bits(f_lo, f_hi, base);
+                    aw[w] |= range_bits(a_lo, a_hi, base);
+                    fw[w] |= range_bits(f_lo, f_hi, base);
                 }
             }
 #pragma unroll
             for (int w = 0; w < kWordsPerChunk; ++w) {
-                fw[w] &= rf[w];
-                aw[w] |= ra[w];
+                fw[w] = __reduce_and_sync(0xFFFFFFFFu, fw[w]);
+                aw[w] = __reduce_or_sync(0xFFFFFFFFu, aw[w]);
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int w = 0; w < kWordsPerChunk; ++w) {
+                    part_f[warp][w] = fw[w];
+                    part_a[warp][w] = aw[w];
+                }
             }
         }
-        // A lane whose four rows are all past Q_LEN leaves fw at all-ones;
-        // the tile then cannot be FULL because q_tile_inside is false.
+        __syncthreads();
+        uint32_t fw[kWordsPerChunk], aw[kWordsPerChunk];
 #pragma unroll
         for (int w = 0; w < kWordsPerChunk; ++w) {
-            fw[w] = __reduce_and_sync(0xFFFFFFFFu, fw[w]);
-            aw[w] = __reduce_or_sync(0xFFFFFFFFu, aw[w]);
+            fw[w] = part_f[0][w] & part_f[1][w] & part_f[2][w] & part_f[3][w];
+            aw[w] = part_a[0][w] | part_a[1][w] | part_a[2][w] | part_a[3][w];
             if (!q_tile_inside) fw[w] = 0u;
             // blocks at or past KB do not exist
-            const int64_t base = c0 + 32 * w;
-            const uint32_t exist = range_bits(0, p.KB - 1, base);
+            const uint32_t exist = range_bits(0, p.KB - 1, c0 + 32 * w);
             fw[w] &= exist;
             aw[w] &= exist;
         }
-        // write this chunk's entries for every head of the group
+        __syncthreads();  // the partial words may be rewritten by the next chunk
+        // write this chunk's entries for the heads of the group
         const uint32_t below = (1u << lane) - 1u;
-        for (int h = h0; h < h1; ++h) {
+        for (int h = h0 + warp; h < h1; h += kBuildWarps) {
             const int64_t row = (static_cast<int64_t>(b) * p.Hm + h) * p.QB + qb;
             int32_t* pidx = p.kv_idx + row * p.KB;
             int32_t* fidx = p.full_idx + row * p.KB;
@@ -193,12 +200,10 @@ __global__ void __launch_bounds__(kBuildWarps * 32) mask_build_kernel(const Mask
     }
 
     // counts and zero tails
-    for (int h = h0; h < h1; ++h) {
+    for (int h = h0 + warp; h < h1; h += kBuildWarps) {
         const int64_t row = (static_cast<int64_t>(b) * p.Hm + h) * p.QB + qb;
-        int32_t* pidx = p.kv_idx + row * p.KB;
-        int32_t* fidx = p.full_idx + row * p.KB;
-        for (int j = cnt_p + lane; j < p.KB; j += 32) pidx[j] = 0;
-        for (int j = cnt_f + lane; j < p.KB; j += 32) fidx[j] = 0;
+        zero_tail(p.kv_idx + row * p.KB, cnt_p, p.KB, lane);
+        zero_tail(p.full_idx + row * p.KB, cnt_f, p.KB, lane);
         if (lane == 0) {
             p.kv_num[row] = cnt_p;
             p.full_num[row] = cnt_f;

@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kTransposeThreads) mask_transpose_kernel(const
             }
             pos += __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
-        for (int j = pos + lane; j < p.QB; j += 32) out[j] = 0;
+        zero_tail(out, pos, p.QB, lane);
         if (lane == 0) (l == 0 ? p.q_num : p.full_q_num)[(static_cast<int64_t>(b) * p.Hm + h) * p.KB + kb] = pos;
     }
 }

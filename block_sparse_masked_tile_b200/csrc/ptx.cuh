@@ -27,6 +27,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// Zeroes row[from, n) with the warp: scalar stores up to the first 16-byte
+// boundary, 16-byte stores after it, scalar stores for the rest.
+__device__ __forceinline__ void zero_tail(int32_t* row, int from, int n, int lane) {
+    if (from >= n) return;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(row + from);
+    int head = static_cast<int>(((16u - (a & 15u)) & 15u) >> 2);  // int32 slots to the boundary
+    head = head < n - from ? head : n - from;
+    if (lane < head) row[from + lane] = 0;
+    const int v0 = from + head;
+    const int nv = (n - v0) >> 2;
+    uint4* v = reinterpret_cast<uint4*>(row + v0);
+    for (int k = lane; k < nv; k += 32) v[k] = make_uint4(0u, 0u, 0u, 0u);
+    const int t0 = v0 + 4 * nv;
+    if (t0 + lane < n) row[t0 + lane] = 0;
+}
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
