@@ -29,7 +29,7 @@ import torch
 __all__ = [
     "BsmtError", "MaskMod", "ScoreMod", "BlockMask", "noop_mask", "causal", "sliding_window", "prefix_lm",
     "sink", "document", "and_masks", "or_masks", "softcap", "alibi", "create_block_mask", "flex_attention",
-    "check_device_status", "library_path", "mask_from_tree", "score_mods_from_list",
+    "check_device_status", "library_path", "mask_from_tree", "score_mods_from_list", "splitkv_workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -96,6 +96,13 @@ def _load() -> ctypes.CDLL:
     lib.bsmt_block_mask_transpose.restype = i32
     lib.bsmt_block_mask_to_dense.argtypes = [ctypes.POINTER(_BlockMask), vp, vp]
     lib.bsmt_block_mask_to_dense.restype = i32
+    lib.bsmt_splitkv_workspace_bytes.argtypes = [i64, i64, i64, i64, i32, ctypes.POINTER(i64)]
+    lib.bsmt_splitkv_workspace_bytes.restype = i32
+    lib.bsmt_flex_attention_fwd_splitkv.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64,
+                                                    ctypes.POINTER(_BlockMask), ctypes.POINTER(_MaskSpec),
+                                                    ctypes.POINTER(_ScoreSpec), ctypes.c_float, i32, i32, vp, i64,
+                                                    vp, vp, vp]
+    lib.bsmt_flex_attention_fwd_splitkv.restype = i32
     lib.bsmt_last_error.argtypes = []
     lib.bsmt_last_error.restype = ctypes.c_char_p
     lib.bsmt_check_device_status.argtypes = [vp]
@@ -476,10 +483,23 @@ def _score_spec(mods, device: torch.device, Hq: int) -> tuple[_ScoreSpec, list]:
     return spec, keep
 
 
+def splitkv_workspace_bytes(B: int, Hq: int, M: int, D: int, num_splits: int) -> int:
+    """Bytes of device workspace split-KV needs for these sizes (0 for one split)."""
+    n = ctypes.c_int64(0)
+    _check(_lib.bsmt_splitkv_workspace_bytes(int(B), int(Hq), int(M), int(D), int(num_splits), ctypes.byref(n)))
+    return int(n.value)
+
+
 def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask: BlockMask | None = None,
                    score_mod: ScoreMod | Iterable[ScoreMod] | None = None, scale: float | None = None,
-                   enable_gqa: bool = False, out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
-    """Block-sparse masked attention forward. Returns (out bf16 [B,Hq,M,D], lse fp32 [B,Hq,M])."""
+                   enable_gqa: bool = False, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                   num_splits: int = 1, workspace: torch.Tensor | None = None):
+    """Block-sparse masked attention forward. Returns (out bf16 [B,Hq,M,D], lse fp32 [B,Hq,M]).
+
+    num_splits > 1 runs split-KV: every row's kv blocks are cut into that many
+    slices computed in parallel and merged exactly (for few q-blocks and long
+    kv). ``workspace`` (a uint8 CUDA tensor of at least
+    splitkv_workspace_bytes(...) bytes) is allocated when not given."""
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.dtype != torch.bfloat16:
             raise ValueError(f"{name} must be bfloat16 (got {t.dtype})")
@@ -514,12 +534,23 @@ def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask
             mspec = getattr(block_mask, "_spec", None)
             if mspec is None:
                 mspec, keep_m = block_mask.mask_mod._spec(device, int(block_mask.shape[0]))
-        _check(_lib.bsmt_flex_attention_fwd(
-            q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, M, N, D,
-            ctypes.byref(bm_c) if bm_c is not None else None,
-            ctypes.byref(mspec) if mspec is not None else None,
-            ctypes.byref(sspec), ctypes.c_float(0.0 if scale is None else float(scale)), int(bool(enable_gqa)),
-            out.data_ptr(), lse.data_ptr(), ctypes.c_void_p(_stream_ptr(device))))
+        common = (q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, M, N, D,
+                  ctypes.byref(bm_c) if bm_c is not None else None,
+                  ctypes.byref(mspec) if mspec is not None else None,
+                  ctypes.byref(sspec), ctypes.c_float(0.0 if scale is None else float(scale)),
+                  int(bool(enable_gqa)))
+        if num_splits == 1:
+            _check(_lib.bsmt_flex_attention_fwd(*common, out.data_ptr(), lse.data_ptr(),
+                                                ctypes.c_void_p(_stream_ptr(device))))
+        else:
+            need = splitkv_workspace_bytes(B, Hq, M, D, num_splits)
+            if workspace is None:
+                workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+            if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+                raise ValueError("workspace must be a contiguous uint8 CUDA tensor")
+            _check(_lib.bsmt_flex_attention_fwd_splitkv(
+                *common, int(num_splits), ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                out.data_ptr(), lse.data_ptr(), ctypes.c_void_p(_stream_ptr(device))))
     del keep_s, keep_m
     return out, lse
 

@@ -74,6 +74,13 @@ struct AttnParams {
     const float* slopes;  // ALiBi slopes [Hq] or null (default 2^(-8(h+1)/Hq))
     __nv_bfloat16* out;
     float* lse;
+    // split-KV: each (b, hq, q-block pair) row of entries is cut into
+    // num_splits consecutive slices, one unit each. With num_splits > 1 the
+    // epilogue writes, per slice, O / l in fp32 to ws_o [S][B*Hq*M][D] and the
+    // slice's lse to ws_lse [S][B*Hq*M]; splitkv_combine_kernel merges them.
+    int32_t num_splits;
+    float* ws_o;
+    float* ws_lse;
 };
 
 constexpr int kThreads = 384;  // 12 warps: 3 warpgroups
@@ -96,7 +103,7 @@ struct SchedHeader {
     int32_t b, hq, qb0;
     int32_t n0, n1;  // tiles visited by q-block 0 / 1
     float slope;     // ALiBi slope of hq (natural units)
-    int32_t pad;
+    int32_t split;   // slice of the entry stream (split-KV), 0 otherwise
 };
 
 template <int D>
@@ -254,8 +261,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // longest-first order: highest q-block pair first, then (b, hq)
             const int bh_count = p.B * p.Hq;
-            const int pr = p.pairs - 1 - u / bh_count;
-            const int bh = u % bh_count;
+            const int pr = p.pairs - 1 - u / (bh_count * p.num_splits);
+            const int bh = (u / p.num_splits) % bh_count;
+            const int split = u % p.num_splits;
             const int b = bh / p.Hq;
             const int hq = bh % p.Hq;
             const int qb0 = 2 * pr;
@@ -333,6 +341,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     n1 += __popc(__ballot_sync(0xFFFFFFFFu, (tags & kTagIn1) != 0));
                 }
             }
+            if (p.num_splits > 1) {
+                // keep this unit's slice [lo, hi) of the stream, moved to the front
+                // (a chunk is read before it is written, and never overlaps a later
+                // chunk's source)
+                const int lo = static_cast<int>((static_cast<int64_t>(T) * split) / p.num_splits);
+                const int hi = static_cast<int>((static_cast<int64_t>(T) * (split + 1)) / p.num_splits);
+                n0 = 0;
+                n1 = 0;
+                for (int c = 0; c < hi - lo; c += 32) {
+                    const bool in = c + lane < hi - lo;
+                    const uint32_t e = in ? entries[lo + c + lane] : 0u;
+                    __syncwarp();
+                    if (in) entries[c + lane] = e;
+                    __syncwarp();
+                    const uint32_t tags = sched_entry_tags(e);
+                    n0 += __popc(__ballot_sync(0xFFFFFFFFu, in && (tags & kTagIn0)));
+                    n1 += __popc(__ballot_sync(0xFFFFFFFFu, in && (tags & kTagIn1)));
+                }
+                T = hi - lo;
+            }
             if (dnf.has_doc && p.has_block_mask) {
                 // Each row's document interval [first, last] of kv positions with
                 // the row's document id (kv ids are non-decreasing). Rows in a run
@@ -370,6 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 hdr->b = b;
                 hdr->hq = hq;
                 hdr->qb0 = qb0;
+                hdr->split = split;
                 hdr->n0 = n0;
                 hdr->n1 = n1;
                 float slope = 0.f;
@@ -767,7 +796,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             // epilogue: out = O / l, lse = ln2 * (m + log2 l)
             __nv_bfloat16* orow = p.out + ((static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.M + q) * D;
             const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-            if (ni > 0) {
+            const float row_lse = [&] {
+                const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+                return l_sum > 0.f ? (m_use + __log2f(l_sum)) * kLn2 : -INFINITY;
+            }();
+            if (p.num_splits > 1) {
+                // split-KV: this slice's O / l in fp32 and its lse, to the workspace
+                const int64_t wrow = (static_cast<int64_t>(hdr.split) * p.B * p.Hq +
+                                      static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.M + q;
+                float4* dst = reinterpret_cast<float4*>(p.ws_o + wrow * D);
+                if (ni > 0) {
+                    if (!mbar_wait(bar(L::kBarOFull + i), o_waits & 1u, abort_flag)) break;
+                    ++o_waits;
+                    __syncwarp();
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(t_o + 32 * c, o);
+                        tc_wait_ld();
+                        if (row_valid) {
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                dst[8 * c + v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                                                             __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+                        }
+                    }
+                    tc_fence_before();
+                } else if (row_valid) {
+#pragma unroll
+                    for (int v = 0; v < D / 4; ++v) dst[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                if (row_valid) p.ws_lse[wrow] = row_lse;
+            } else if (ni > 0) {
                 if (!mbar_wait(bar(L::kBarOFull + i), o_waits & 1u, abort_flag)) break;
                 ++o_waits;
                 __syncwarp();
@@ -810,11 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
             }
-            if (row_valid) {
-                const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-                p.lse[(static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.M + q] =
-                    l_sum > 0.f ? (m_use + __log2f(l_sum)) * kLn2 : -INFINITY;
-            }
+            if (row_valid && p.num_splits == 1) p.lse[(static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.M + q] = row_lse;
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
         }
@@ -829,6 +886,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+// Merges the split-KV slices of every row: with lse_s the slices' natural
+// log-sum-exps and O_s their normalised outputs,
+//   lse = log sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) O_s,
+// which is the attention over the union of the slices. A row no slice
+// reaches keeps out = 0 and lse = -inf. One warp per row; lane l holds
+// columns [l * D/32, (l + 1) * D/32).
+template <int D>
+__global__ void __launch_bounds__(256) splitkv_combine_kernel(const float* ws_o, const float* ws_lse, int splits,
+                                                              int64_t rows, __nv_bfloat16* out, float* lse) {
+    constexpr int kPer = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    float m = -INFINITY;
+    for (int s = 0; s < splits; ++s) m = fmaxf(m, __ldg(ws_lse + s * rows + row));
+    float acc[kPer];
+#pragma unroll
+    for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
+    float total = 0.f;
+    if (m != -INFINITY) {
+        for (int s = 0; s < splits; ++s) {
+            const float ls = __ldg(ws_lse + s * rows + row);
+            if (ls == -INFINITY) continue;
+            const float w = expf(ls - m);
+            total += w;
+            const float* o = ws_o + (s * rows + row) * D + lane * kPer;
+#pragma unroll
+            for (int c = 0; c < kPer; ++c) acc[c] = fmaf(w, __ldg(o + c), acc[c]);
+        }
+    }
+    const float inv = total > 0.f ? 1.f / total : 0.f;
+    uint32_t pk[kPer / 2];
+#pragma unroll
+    for (int c = 0; c < kPer / 2; ++c) pk[c] = pack_bf16x2(acc[2 * c] * inv, acc[2 * c + 1] * inv);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(out + row * D + lane * kPer);
+#pragma unroll
+    for (int c = 0; c < kPer / 2; ++c) dst[c] = pk[c];
+    if (lane == 0) lse[row] = total > 0.f ? m + logf(total) : -INFINITY;
 }
 
 }  // namespace bsmt

@@ -351,10 +351,15 @@ bsmt_status bsmt_create_block_mask(const bsmt_mask_spec* spec, int64_t B, int64_
     return ok();
 }
 
-bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v, int64_t B, int64_t Hq, int64_t Hkv,
-                                    int64_t M, int64_t N, int64_t D, const bsmt_block_mask* bm,
-                                    const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score, float scale,
-                                    int32_t enable_gqa, void* out, float* lse, void* stream) {
+}  // extern "C"
+
+namespace {
+// The attention path. num_splits > 1 runs split-KV into the workspace
+// (ws_o, ws_lse, already checked) and merges the slices into out and lse.
+bsmt_status attention(const void* q, const void* k, const void* v, int64_t B, int64_t Hq, int64_t Hkv, int64_t M,
+                      int64_t N, int64_t D, const bsmt_block_mask* bm, const bsmt_mask_spec* mask_spec,
+                      const bsmt_score_spec* score, float scale, int32_t enable_gqa, int num_splits, float* ws_o,
+                      float* ws_lse, void* out, float* lse, void* stream) {
     if (B < 0 || Hq < 0 || Hkv < 0 || M < 0 || N < 0)
         return fail(BSMT_ERR_INVALID_ARGUMENT, "negative size (B=%lld Hq=%lld Hkv=%lld M=%lld N=%lld)",
                     static_cast<long long>(B), static_cast<long long>(Hq), static_cast<long long>(Hkv),
@@ -472,7 +477,10 @@ bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v,
     p.KB = static_cast<int32_t>(KB);
     p.pairs = static_cast<int32_t>((QB + 1) / 2);
     p.group = static_cast<int32_t>(Hq / Hkv);
-    const int64_t units = B * Hq * p.pairs;
+    p.num_splits = num_splits;
+    p.ws_o = ws_o;
+    p.ws_lse = ws_lse;
+    const int64_t units = B * Hq * p.pairs * num_splits;
     if (units > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "too many work units");
     p.num_units = static_cast<int32_t>(units);
     p.scale = scale;
@@ -482,8 +490,78 @@ bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v,
     p.slopes = slopes;
     p.out = static_cast<__nv_bfloat16*>(out);
     p.lse = lse;
-    if (D == 128) return launch_attn_score<128>(mode, dev, nsm, tq, tk, tv, to, p, dnf, s) == BSMT_OK ? ok() : BSMT_ERR_CUDA;
-    return launch_attn_score<64>(mode, dev, nsm, tq, tk, tv, to, p, dnf, s) == BSMT_OK ? ok() : BSMT_ERR_CUDA;
+    st = D == 128 ? launch_attn_score<128>(mode, dev, nsm, tq, tk, tv, to, p, dnf, s)
+                  : launch_attn_score<64>(mode, dev, nsm, tq, tk, tv, to, p, dnf, s);
+    if (st != BSMT_OK) return BSMT_ERR_CUDA;
+    if (num_splits > 1) {
+        const int64_t rows = B * Hq * M;
+        const int64_t blocks = (rows + 7) / 8;
+        if (blocks > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "grid too large");
+        if (D == 128)
+            bsmt::splitkv_combine_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+                ws_o, ws_lse, num_splits, rows, static_cast<__nv_bfloat16*>(out), lse);
+        else
+            bsmt::splitkv_combine_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+                ws_o, ws_lse, num_splits, rows, static_cast<__nv_bfloat16*>(out), lse);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "split-KV combine launch: %s", cudaGetErrorString(e));
+    }
+    return ok();
+}
+
+// Bytes of the split-KV workspace: O slices [S][B*Hq*M][D] fp32, then the
+// lse slices [S][B*Hq*M] fp32 starting at a 256-byte boundary.
+int64_t splitkv_ws_o_bytes(int64_t B, int64_t Hq, int64_t M, int64_t D, int64_t S) {
+    return (S * B * Hq * M * D * 4 + 255) / 256 * 256;
+}
+int64_t splitkv_ws_bytes(int64_t B, int64_t Hq, int64_t M, int64_t D, int64_t S) {
+    return splitkv_ws_o_bytes(B, Hq, M, D, S) + S * B * Hq * M * 4;
+}
+}  // namespace
+
+extern "C" {
+
+bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v, int64_t B, int64_t Hq, int64_t Hkv,
+                                    int64_t M, int64_t N, int64_t D, const bsmt_block_mask* bm,
+                                    const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score, float scale,
+                                    int32_t enable_gqa, void* out, float* lse, void* stream) {
+    return attention(q, k, v, B, Hq, Hkv, M, N, D, bm, mask_spec, score, scale, enable_gqa, 1, nullptr, nullptr, out,
+                     lse, stream);
+}
+
+bsmt_status bsmt_splitkv_workspace_bytes(int64_t B, int64_t Hq, int64_t M, int64_t D, int32_t num_splits,
+                                         int64_t* bytes) {
+    if (bytes == nullptr) return fail(BSMT_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    if (B < 0 || Hq < 0 || M < 0) return fail(BSMT_ERR_INVALID_ARGUMENT, "negative size");
+    if (D != 64 && D != 128) return fail(BSMT_ERR_UNSUPPORTED, "head dim D=%lld (supported: 64, 128)", static_cast<long long>(D));
+    if (num_splits < 1 || num_splits > BSMT_MAX_SPLITS)
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "num_splits=%d outside [1, %d]", num_splits, BSMT_MAX_SPLITS);
+    if (M > kMaxLen || B * Hq > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "sizes too large");
+    *bytes = num_splits == 1 ? 0 : splitkv_ws_bytes(B, Hq, M, D, num_splits);
+    return ok();
+}
+
+bsmt_status bsmt_flex_attention_fwd_splitkv(const void* q, const void* k, const void* v, int64_t B, int64_t Hq,
+                                            int64_t Hkv, int64_t M, int64_t N, int64_t D, const bsmt_block_mask* bm,
+                                            const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score,
+                                            float scale, int32_t enable_gqa, int32_t num_splits, void* workspace,
+                                            int64_t workspace_bytes, void* out, float* lse, void* stream) {
+    int64_t need = 0;
+    bsmt_status st = bsmt_splitkv_workspace_bytes(B, Hq, M, D, num_splits, &need);
+    if (st != BSMT_OK) return st;
+    float* ws_o = nullptr;
+    float* ws_lse = nullptr;
+    if (num_splits > 1 && B * Hq * M > 0) {
+        if (workspace == nullptr || !aligned(workspace, 256))
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "workspace must be non-NULL and 256-byte aligned");
+        if (workspace_bytes < need)
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "workspace holds %lld bytes, %lld needed",
+                        static_cast<long long>(workspace_bytes), static_cast<long long>(need));
+        ws_o = static_cast<float*>(workspace);
+        ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + splitkv_ws_o_bytes(B, Hq, M, D, num_splits));
+    }
+    return attention(q, k, v, B, Hq, Hkv, M, N, D, bm, mask_spec, score, scale, enable_gqa, num_splits, ws_o, ws_lse,
+                     out, lse, stream);
 }
 
 bsmt_status bsmt_check_device_status(void* stream) {

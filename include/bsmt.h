@@ -249,6 +249,39 @@ bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v,
                                     const bsmt_score_spec* score, float scale,
                                     int32_t enable_gqa, void* out, float* lse, void* stream);
 
+/* ----------------------------------------------------------- split-KV
+ * Split-KV forward for rows with few q-blocks and long kv lists (decode-like
+ * shapes): the kv entries of every (b, hq, q-block pair) are cut into
+ * num_splits consecutive slices that run as separate work units, each
+ * writing its slice's normalised output O_s (fp32) and lse_s to a
+ * workspace; a second kernel merges them exactly:
+ *   lse = log sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) O_s.
+ * This is the split reduction of Split-KV FlashAttention (FlagAttention
+ * page, "Operator overview"); the result is the same attention as
+ * bsmt_flex_attention_fwd, up to rounding. */
+#define BSMT_MAX_SPLITS 64
+
+/* Workspace bytes bsmt_flex_attention_fwd_splitkv needs for these sizes
+ * (0 when num_splits == 1). Host-only; launches nothing. */
+bsmt_status bsmt_splitkv_workspace_bytes(int64_t B, int64_t Hq, int64_t M, int64_t D, int32_t num_splits,
+                                         int64_t* bytes);
+
+/* bsmt_flex_attention_fwd with split-KV. Arguments as there, plus:
+ *   num_splits       1 .. BSMT_MAX_SPLITS (1 runs the plain path)
+ *   workspace        caller-owned device memory, 256-byte aligned, at least
+ *                    bsmt_splitkv_workspace_bytes bytes; the call writes it
+ *                    and reads it back (no part needs to start zeroed). It
+ *                    may be reused once the stream has passed this call.
+ *   workspace_bytes  its size
+ * A workspace that is NULL, misaligned or too small returns
+ * BSMT_ERR_INVALID_ARGUMENT before any launch. */
+bsmt_status bsmt_flex_attention_fwd_splitkv(const void* q, const void* k, const void* v, int64_t B, int64_t Hq,
+                                            int64_t Hkv, int64_t M, int64_t N, int64_t D,
+                                            const bsmt_block_mask* block_mask, const bsmt_mask_spec* mask_spec,
+                                            const bsmt_score_spec* score, float scale, int32_t enable_gqa,
+                                            int32_t num_splits, void* workspace, int64_t workspace_bytes, void* out,
+                                            float* lse, void* stream);
+
 /* Thread-local message for the last failed call on this thread ("" if none). */
 const char* bsmt_last_error(void);
 

@@ -28,6 +28,7 @@ def test_every_declared_symbol_is_exported():
     names = declared_functions()
     assert names == sorted(["bsmt_block_mask_shape", "bsmt_create_block_mask", "bsmt_flex_attention_fwd",
                             "bsmt_block_mask_transpose", "bsmt_block_mask_to_dense",
+                            "bsmt_splitkv_workspace_bytes", "bsmt_flex_attention_fwd_splitkv",
                             "bsmt_last_error", "bsmt_check_device_status", "bsmt_version"])
     lib = ctypes.CDLL(bsmt.library_path())
     for n in names:
@@ -224,3 +225,22 @@ def test_transpose_and_to_dense_argument_errors():
     bm.QB, bm.KB = 4, 0  # no kv column: nothing to write, nothing launched
     assert _lib.bsmt_block_mask_transpose(ctypes.byref(bm), ctypes.byref(q), null) == OK
     assert _lib.bsmt_block_mask_to_dense(ctypes.byref(bm), None, null) == OK
+
+
+def test_splitkv_workspace_and_argument_errors():
+    n = ctypes.c_int64(-1)
+    assert _lib.bsmt_splitkv_workspace_bytes(2, 4, 300, 128, 1, ctypes.byref(n)) == OK and n.value == 0
+    assert _lib.bsmt_splitkv_workspace_bytes(2, 4, 300, 128, 8, ctypes.byref(n)) == OK
+    o_bytes = (8 * 2 * 4 * 300 * 128 * 4 + 255) // 256 * 256
+    assert n.value == o_bytes + 8 * 2 * 4 * 300 * 4
+    assert _lib.bsmt_splitkv_workspace_bytes(2, 4, 300, 96, 8, ctypes.byref(n)) == UNSUPPORTED
+    assert _lib.bsmt_splitkv_workspace_bytes(2, 4, 300, 128, 0, ctypes.byref(n)) == INVALID
+    assert _lib.bsmt_splitkv_workspace_bytes(2, 4, 300, 128, 65, ctypes.byref(n)) == INVALID
+    assert _lib.bsmt_splitkv_workspace_bytes(2, 4, 300, 128, 8, None) == INVALID
+    f = _lib.bsmt_flex_attention_fwd_splitkv
+    args = (FAKE, FAKE, FAKE, 1, 2, 2, 128, 4096, 128, None, None, None, ctypes.c_float(0.0), 0)
+    null = ctypes.c_void_p(0)
+    assert f(*args, 4, None, 1 << 30, FAKE, FAKE, null) == INVALID                  # no workspace
+    assert f(*args, 4, ctypes.c_void_p(FAKE + 16), 1 << 30, FAKE, FAKE, null) == INVALID  # misaligned
+    assert f(*args, 4, ctypes.c_void_p(FAKE), 1024, FAKE, FAKE, null) == INVALID    # too small
+    assert f(*args, 0, ctypes.c_void_p(FAKE), 1 << 30, FAKE, FAKE, null) == INVALID  # no splits
