@@ -213,6 +213,23 @@ def side_kernels(bsmt, mask, w, dev, hbm_peak: float) -> dict:
             res["q_side_transpose"] = {"ms": ms, "bytes": qbytes, "achieved_gbs": gbs, "peak_gbs": hbm_peak,
                                        "frac": gbs / hbm_peak}
         bsmt.check_device_status(dev)
+    # split-KV on a decode-like shape: one q-block per head over a long kv
+    # cache, no mask (every tile computed), plain path vs 8 slices
+    Bd, Hqd, Hkvd, Md, Nd, Dd, S = 1, 32, 8, 128, 32768, 128, 8
+    g = torch.Generator(device="cpu").manual_seed(7)
+    qd, kd, vd = (torch.randn(shape, generator=g).to(torch.bfloat16).to(dev)
+                  for shape in ((Bd, Hqd, Md, Dd), (Bd, Hkvd, Nd, Dd), (Bd, Hkvd, Nd, Dd)))
+    out = torch.empty((Bd, Hqd, Md, Dd), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((Bd, Hqd, Md), dtype=torch.float32, device=dev)
+    ws = torch.empty(bsmt.splitkv_workspace_bytes(Bd, Hqd, Md, Dd, S), dtype=torch.uint8, device=dev)
+    flops = Bd * Hqd * ((Md + 127) // 128) * ((Nd + 127) // 128) * 4 * 128 * 128 * Dd
+    ms1 = _time_launches(lambda: bsmt.flex_attention(qd, kd, vd, enable_gqa=True, out=out, lse=lse), reps=5)
+    mss = _time_launches(lambda: bsmt.flex_attention(qd, kd, vd, enable_gqa=True, out=out, lse=lse,
+                                                     num_splits=S, workspace=ws), reps=5)
+    bsmt.check_device_status(dev)
+    res["splitkv_decode"] = {"shape": f"B={Bd} Hq={Hqd} Hkv={Hkvd} M={Md} N={Nd} D={Dd}, no mask", "splits": S,
+                             "plain_ms": ms1, "plain_tflops": flops / (ms1 * 1e-3) / 1e12,
+                             "split_ms": mss, "split_tflops": flops / (mss * 1e-3) / 1e12}
     return res
 
 
