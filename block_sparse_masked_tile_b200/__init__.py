@@ -103,6 +103,11 @@ def _load() -> ctypes.CDLL:
                                                     ctypes.POINTER(_ScoreSpec), ctypes.c_float, i32, i32, vp, i64,
                                                     vp, vp, vp]
     lib.bsmt_flex_attention_fwd_splitkv.restype = i32
+    lib.bsmt_flex_attention_fwd_splitkv_static.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64,
+                                                           ctypes.POINTER(_BlockMask), ctypes.POINTER(_MaskSpec),
+                                                           ctypes.POINTER(_ScoreSpec), ctypes.c_float, i32, i32,
+                                                           vp, vp, vp]
+    lib.bsmt_flex_attention_fwd_splitkv_static.restype = i32
     lib.bsmt_last_error.argtypes = []
     lib.bsmt_last_error.restype = ctypes.c_char_p
     lib.bsmt_check_device_status.argtypes = [vp]
@@ -499,7 +504,10 @@ def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask
     num_splits > 1 runs split-KV: every row's kv blocks are cut into that many
     slices computed in parallel and merged exactly (for few q-blocks and long
     kv). ``workspace`` (a uint8 CUDA tensor of at least
-    splitkv_workspace_bytes(...) bytes) is allocated when not given."""
+    splitkv_workspace_bytes(...) bytes) is allocated when not given;
+    ``workspace="static"`` uses the library's fixed device scratch instead and
+    allocates nothing (bsmt_flex_attention_fwd_splitkv_static: sizes above the
+    scratch are rejected, and calls that overlap in time race on it)."""
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.dtype != torch.bfloat16:
             raise ValueError(f"{name} must be bfloat16 (got {t.dtype})")
@@ -542,6 +550,10 @@ def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask
         if num_splits == 1:
             _check(_lib.bsmt_flex_attention_fwd(*common, out.data_ptr(), lse.data_ptr(),
                                                 ctypes.c_void_p(_stream_ptr(device))))
+        elif isinstance(workspace, str) and workspace == "static":
+            # the library's own device scratch: no allocation (overlapping calls race)
+            _check(_lib.bsmt_flex_attention_fwd_splitkv_static(
+                *common, int(num_splits), out.data_ptr(), lse.data_ptr(), ctypes.c_void_p(_stream_ptr(device))))
         else:
             need = splitkv_workspace_bytes(B, Hq, M, D, num_splits)
             if workspace is None:

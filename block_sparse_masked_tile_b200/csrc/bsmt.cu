@@ -175,6 +175,26 @@ bsmt_status sm_count(int* dev_out, int* n_out) {
     return BSMT_OK;
 }
 
+// ------------------------------------------------------------ static scratch
+// Device scratch of the allocation-free split-KV entry point: a file-scope
+// array, so that call allocates nothing. Its address is looked up once per
+// device and kept.
+static __device__ __align__(256) unsigned char g_splitkv_scratch[BSMT_SPLITKV_SCRATCH_BYTES];
+void* g_scratch_addr[64] = {};
+
+bsmt_status scratch_address(int dev, void** addr) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_scratch_addr[dev] == nullptr) {
+        void* ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_splitkv_scratch);
+        if (e != cudaSuccess || ptr == nullptr)
+            return fail(BSMT_ERR_CUDA, "cudaGetSymbolAddress(split-KV scratch): %s", cudaGetErrorString(e));
+        g_scratch_addr[dev] = ptr;
+    }
+    *addr = g_scratch_addr[dev];
+    return BSMT_OK;
+}
+
 // ------------------------------------------------------------ tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -562,6 +582,35 @@ bsmt_status bsmt_flex_attention_fwd_splitkv(const void* q, const void* k, const 
     }
     return attention(q, k, v, B, Hq, Hkv, M, N, D, bm, mask_spec, score, scale, enable_gqa, num_splits, ws_o, ws_lse,
                      out, lse, stream);
+}
+
+bsmt_status bsmt_flex_attention_fwd_splitkv_static(const void* q, const void* k, const void* v, int64_t B,
+                                                   int64_t Hq, int64_t Hkv, int64_t M, int64_t N, int64_t D,
+                                                   const bsmt_block_mask* bm, const bsmt_mask_spec* mask_spec,
+                                                   const bsmt_score_spec* score, float scale, int32_t enable_gqa,
+                                                   int32_t num_splits, void* out, float* lse, void* stream) {
+    int64_t need = 0;
+    bsmt_status st = bsmt_splitkv_workspace_bytes(B, Hq, M, D, num_splits, &need);
+    if (st != BSMT_OK) return st;
+    if (need > BSMT_SPLITKV_SCRATCH_BYTES)
+        return fail(BSMT_ERR_UNSUPPORTED,
+                    "split-KV scratch: %lld bytes needed for B=%lld Hq=%lld M=%lld D=%lld with %d splits, the static "
+                    "scratch holds %lld; use bsmt_flex_attention_fwd_splitkv with a workspace",
+                    static_cast<long long>(need), static_cast<long long>(B), static_cast<long long>(Hq),
+                    static_cast<long long>(M), static_cast<long long>(D), num_splits,
+                    static_cast<long long>(BSMT_SPLITKV_SCRATCH_BYTES));
+    void* scratch = nullptr;
+    if (need > 0) {
+        int dev = 0, nsm = 0;
+        st = sm_count(&dev, &nsm);
+        if (st != BSMT_OK) return st;
+        st = scratch_address(dev, &scratch);
+        if (st != BSMT_OK) return st;
+    }
+    // nothing in the scratch must start at zero: every slice writes each of
+    // its rows (O and lse) before the merge kernel reads them
+    return bsmt_flex_attention_fwd_splitkv(q, k, v, B, Hq, Hkv, M, N, D, bm, mask_spec, score, scale, enable_gqa,
+                                           num_splits, scratch, BSMT_SPLITKV_SCRATCH_BYTES, out, lse, stream);
 }
 
 bsmt_status bsmt_check_device_status(void* stream) {

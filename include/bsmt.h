@@ -282,6 +282,26 @@ bsmt_status bsmt_flex_attention_fwd_splitkv(const void* q, const void* k, const 
                                             int32_t num_splits, void* workspace, int64_t workspace_bytes, void* out,
                                             float* lse, void* stream);
 
+/* Split-KV without a caller workspace: the same computation as
+ * bsmt_flex_attention_fwd_splitkv, with the workspace taken from a static
+ * device array inside the library (BSMT_SPLITKV_SCRATCH_BYTES per device),
+ * so the call allocates no memory. The pages have no counterpart of this
+ * entry point; it is an allocation-free form of the split-KV call.
+ *   - Sizes whose workspace (bsmt_splitkv_workspace_bytes) exceeds the
+ *     scratch return BSMT_ERR_UNSUPPORTED with the sizes in the message.
+ *   - The scratch is shared by every call on the device: calls on one stream
+ *     run in order, but calls that overlap (other streams, other host threads)
+ *     race on it and give wrong results. Serialise them, or use the
+ *     workspace form.
+ *   - The scratch address is looked up once per device (checked) and kept. */
+#define BSMT_SPLITKV_SCRATCH_BYTES (32LL << 20)
+bsmt_status bsmt_flex_attention_fwd_splitkv_static(const void* q, const void* k, const void* v, int64_t B,
+                                                   int64_t Hq, int64_t Hkv, int64_t M, int64_t N, int64_t D,
+                                                   const bsmt_block_mask* block_mask,
+                                                   const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score,
+                                                   float scale, int32_t enable_gqa, int32_t num_splits, void* out,
+                                                   float* lse, void* stream);
+
 /* Thread-local message for the last failed call on this thread ("" if none). */
 const char* bsmt_last_error(void);
 

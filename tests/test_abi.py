@@ -29,6 +29,7 @@ def test_every_declared_symbol_is_exported():
     assert names == sorted(["bsmt_block_mask_shape", "bsmt_create_block_mask", "bsmt_flex_attention_fwd",
                             "bsmt_block_mask_transpose", "bsmt_block_mask_to_dense",
                             "bsmt_splitkv_workspace_bytes", "bsmt_flex_attention_fwd_splitkv",
+                            "bsmt_flex_attention_fwd_splitkv_static",
                             "bsmt_last_error", "bsmt_check_device_status", "bsmt_version"])
     lib = ctypes.CDLL(bsmt.library_path())
     for n in names:
@@ -244,3 +245,15 @@ def test_splitkv_workspace_and_argument_errors():
     assert f(*args, 4, ctypes.c_void_p(FAKE + 16), 1 << 30, FAKE, FAKE, null) == INVALID  # misaligned
     assert f(*args, 4, ctypes.c_void_p(FAKE), 1024, FAKE, FAKE, null) == INVALID    # too small
     assert f(*args, 0, ctypes.c_void_p(FAKE), 1 << 30, FAKE, FAKE, null) == INVALID  # no splits
+
+
+def test_static_scratch_rejects_sizes_above_its_limit():
+    f = _lib.bsmt_flex_attention_fwd_splitkv_static
+    null = ctypes.c_void_p(0)
+    # 64 splits x 16 x 64 heads x 4096 rows x 129 floats is far above 32 MiB; rejected before any CUDA call
+    r = f(FAKE, FAKE, FAKE, 16, 64, 64, 4096, 8192, 128, None, None, None, ctypes.c_float(0.0), 0, 64,
+          FAKE, FAKE, null)
+    assert r == UNSUPPORTED
+    assert "static" in _lib.bsmt_last_error().decode() and "workspace" in _lib.bsmt_last_error().decode()
+    assert f(FAKE, FAKE, FAKE, 1, 2, 2, 128, 4096, 96, None, None, None, ctypes.c_float(0.0), 0, 4,
+             FAKE, FAKE, null) == UNSUPPORTED  # D = 96
