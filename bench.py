@@ -376,16 +376,14 @@ def main():
         doc_host = [torch.as_tensor(data["mask"][1][1]).pin_memory()]
 
     def e2e_step():
-        qd, kd, vd = (x.to(dev, non_blocking=True) for x in (hq_, hk_, hv_))
+        # the public host-tensor call: block mask built on the device, copies in
+        # and out pipelined with the attention of independent pieces
         m = mask
         if doc_host:
             dd = doc_host[0].to(dev, non_blocking=True)
             m = bsmt.and_masks(bsmt.document(dd), bsmt.causal())
-        b2 = bsmt.create_block_mask(m, w.B, w.Hq, w.M, w.N, device=dev)
-        o2, l2 = bsmt.flex_attention(qd, kd, vd, block_mask=b2, score_mod=mods, scale=w.scale,
-                                     enable_gqa=w.enable_gqa)
-        ho.copy_(o2, non_blocking=True)
-        hl.copy_(l2, non_blocking=True)
+        bsmt.flex_attention_host(hq_, hk_, hv_, mask_mod=m, score_mod=mods, scale=w.scale,
+                                 enable_gqa=w.enable_gqa, device=dev, out=ho, lse=hl)
         torch.cuda.current_stream(dev).synchronize()
 
     e2e_step()
