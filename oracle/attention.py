@@ -145,3 +145,32 @@ def flex_attention_sampled(q, k, v, samples, mask=None, score_mods=(), scale=Non
             outs[i] = o[j]
             lses[i] = s[j]
     return outs, lses
+
+
+def flex_attention_varlen(q, k, v, cu_q, cu_k, causal=False, score_mods=(), scale=None, enable_gqa=False):
+    """Attention over packed variable-length sequences (L-GATr "attention
+    backends" page: packed events attend within their own event; the varlen
+    kernels' cu_seqlens form). q [total_q, Hq, D], k/v [total_k, Hkv, D];
+    sequence i holds q tokens cu_q[i]:cu_q[i+1] and k tokens cu_k[i]:cu_k[i+1].
+    Each sequence is plain attention of its own tokens, computed by
+    flex_attention on a [1, H, L, D] view, causal (kv <= q, positions within
+    the sequence) when asked. Tokens past the last sequence attend to nothing.
+    Returns (out [total_q, Hq, D], lse [Hq, total_q])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cu_q = [int(x) for x in cu_q]
+    cu_k = [int(x) for x in cu_k]
+    Mt, Hq, D = q.shape
+    out = np.zeros((Mt, Hq, v.shape[2]), np.float64)
+    lse = np.full((Hq, Mt), -np.inf, np.float64)
+    for i in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[i], cu_q[i + 1], cu_k[i], cu_k[i + 1]
+        if q1 <= q0:
+            continue
+        qs = q[q0:q1].transpose(1, 0, 2)[None]
+        ks = k[k0:k1].transpose(1, 0, 2)[None]
+        vs = v[k0:k1].transpose(1, 0, 2)[None]
+        tree = ("causal",) if causal else None
+        o, l = flex_attention(qs, ks, vs, tree, score_mods, scale, enable_gqa)
+        out[q0:q1] = o[0].transpose(1, 0, 2)
+        lse[:, q0:q1] = l[0]
+    return out, lse

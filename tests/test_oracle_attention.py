@@ -185,3 +185,56 @@ def test_sampled_matches_full():
     for i, (b, h, r) in enumerate(samples):
         np.testing.assert_allclose(so[i], out[b, h, r], rtol=1e-13, atol=1e-14)
         assert sl[i] == pytest.approx(lse[b, h, r], rel=1e-13)
+
+
+def _ids_from_cu(cu, total):
+    ids = np.full(total, len(cu) - 1, np.int32)
+    for i in range(len(cu) - 1):
+        ids[cu[i]:cu[i + 1]] = i
+    return ids
+
+
+def test_varlen_equals_document_mask_and_sdpa():
+    # L-GATr page: packed events attend within their event. The slicing
+    # definition must equal the document-mask definition over the whole pack,
+    # and each sequence must equal plain SDPA on its own tokens.
+    rng = np.random.default_rng(5)
+    Hq, Hkv, D = 4, 2, 16
+    cu_q = [0, 37, 37, 120, 200]       # an empty sequence in the middle
+    cu_k = [0, 50, 61, 150, 260]
+    Mt, Nt = 210, 260                  # 10 q tokens past the last sequence
+    q = torch.from_numpy(rng.standard_normal((Mt, Hq, D))).to(torch.bfloat16)
+    k = torch.from_numpy(rng.standard_normal((Nt, Hkv, D))).to(torch.bfloat16)
+    v = torch.from_numpy(rng.standard_normal((Nt, Hkv, D))).to(torch.bfloat16)
+    out, lse = oa.flex_attention_varlen(q, k, v, cu_q, cu_k, False, (), None, True)
+    qi, ki = _ids_from_cu(cu_q, Mt), _ids_from_cu(cu_k, Nt)
+    tree = ("document", qi[None], ki[None])
+    o2, l2 = oa.flex_attention(q.permute(1, 0, 2)[None], k.permute(1, 0, 2)[None], v.permute(1, 0, 2)[None],
+                               tree, (), None, True)
+    assert np.allclose(out, o2[0].transpose(1, 0, 2), atol=1e-12)
+    assert np.array_equal(np.isneginf(lse), np.isneginf(l2[0]))
+    fin = np.isfinite(lse)
+    assert np.allclose(lse[fin], l2[0][fin], atol=1e-12)
+    assert np.all(out[200:] == 0) and np.all(np.isneginf(lse[:, 200:]))
+    for i in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[i], cu_q[i + 1], cu_k[i], cu_k[i + 1]
+        if q1 == q0:
+            continue
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[q0:q1].double().permute(1, 0, 2), k[k0:k1].double().permute(1, 0, 2).repeat_interleave(2, 0),
+            v[k0:k1].double().permute(1, 0, 2).repeat_interleave(2, 0))
+        assert np.allclose(out[q0:q1], ref.permute(1, 0, 2).numpy(), atol=1e-10)
+
+
+def test_varlen_causal_equals_document_and_causal():
+    rng = np.random.default_rng(6)
+    cu = [0, 70, 71, 200, 333]
+    q = torch.from_numpy(rng.standard_normal((333, 2, 16))).to(torch.bfloat16)
+    k = torch.from_numpy(rng.standard_normal((333, 2, 16))).to(torch.bfloat16)
+    v = torch.from_numpy(rng.standard_normal((333, 2, 16))).to(torch.bfloat16)
+    out, lse = oa.flex_attention_varlen(q, k, v, cu, cu, True)
+    ids = _ids_from_cu(cu, 333)
+    tree = ("and", ("document", ids[None], ids[None]), ("causal",))
+    o2, l2 = oa.flex_attention(q.permute(1, 0, 2)[None], k.permute(1, 0, 2)[None], v.permute(1, 0, 2)[None], tree)
+    assert np.allclose(out, o2[0].transpose(1, 0, 2), atol=1e-12)
+    assert np.allclose(lse, l2[0], atol=1e-12)
