@@ -30,7 +30,7 @@ __all__ = [
     "BsmtError", "MaskMod", "ScoreMod", "BlockMask", "noop_mask", "causal", "sliding_window", "prefix_lm",
     "sink", "document", "and_masks", "or_masks", "softcap", "alibi", "create_block_mask", "flex_attention",
     "check_device_status", "library_path", "mask_from_tree", "score_mods_from_list", "splitkv_workspace_bytes",
-    "flex_attention_host",
+    "flex_attention_host", "flex_attention_varlen", "seqlens_to_doc_ids",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -109,6 +109,12 @@ def _load() -> ctypes.CDLL:
                                                            ctypes.POINTER(_ScoreSpec), ctypes.c_float, i32, i32,
                                                            vp, vp, vp]
     lib.bsmt_flex_attention_fwd_splitkv_static.restype = i32
+    lib.bsmt_seqlens_to_doc_ids.argtypes = [vp, i32, i64, vp, vp]
+    lib.bsmt_seqlens_to_doc_ids.restype = i32
+    lib.bsmt_flex_attention_fwd_packed.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, ctypes.POINTER(_BlockMask),
+                                                   ctypes.POINTER(_MaskSpec), ctypes.POINTER(_ScoreSpec),
+                                                   ctypes.c_float, i32, vp, vp, vp]
+    lib.bsmt_flex_attention_fwd_packed.restype = i32
     lib.bsmt_last_error.argtypes = []
     lib.bsmt_last_error.restype = ctypes.c_char_p
     lib.bsmt_check_device_status.argtypes = [vp]
@@ -205,6 +211,9 @@ def noop_mask() -> MaskMod:
 
 def causal() -> MaskMod:
     return _leaf(MASK_CAUSAL)
+
+
+_causal_mask = causal  # (flex_attention_varlen's causal flag shadows the name)
 
 
 def sliding_window(window: int) -> MaskMod:
@@ -680,6 +689,66 @@ def _select_heads(mods, h0: int, h1: int, Hq: int):
         else:
             res.append(m)
     return res
+
+
+def seqlens_to_doc_ids(cu_seqlens: torch.Tensor, total: int) -> torch.Tensor:
+    """int32 [total] on the device: each packed token's sequence ordinal
+    (bsmt_seqlens_to_doc_ids)."""
+    cu = cu_seqlens.to(dtype=torch.int32).contiguous()
+    if not cu.is_cuda or cu.dim() != 1 or cu.numel() < 1:
+        raise ValueError("cu_seqlens must be a 1-D CUDA tensor with at least one entry")
+    ids = torch.empty(int(total), dtype=torch.int32, device=cu.device)
+    with torch.cuda.device(cu.device):
+        _check(_lib.bsmt_seqlens_to_doc_ids(ctypes.c_void_p(cu.data_ptr()), cu.numel() - 1, int(total),
+                                            ctypes.c_void_p(ids.data_ptr()), ctypes.c_void_p(_stream_ptr(cu.device))))
+    return ids
+
+
+def flex_attention_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                          cu_seqlens_k: torch.Tensor, causal: bool = False,
+                          score_mod: ScoreMod | Iterable[ScoreMod] | None = None, scale: float | None = None,
+                          enable_gqa: bool = False, out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
+    """Attention over packed variable-length sequences (the cu_seqlens form):
+    q [total_q, Hq, D], k/v [total_k, Hkv, D] bf16; token t of the pack
+    belongs to sequence i for cu_seqlens[i] <= t < cu_seqlens[i+1], and attends
+    only to keys of its own sequence. ``causal`` needs q and k to share
+    cu_seqlens (equal lengths, top-left aligned). Returns (out [total_q, Hq, D],
+    lse [Hq, total_q]).
+
+    The sequence ordinals become DOCUMENT ids on the device, the BlockMask is
+    built over the whole pack (B = H = 1), and the packed layout goes straight
+    to the attention kernel through its tensor maps."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or t.dim() != 3 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 3-D CUDA tensor [tokens, H, D]")
+    M, Hq, D = q.shape
+    N, Hkv, Dk = k.shape
+    if v.shape != k.shape or Dk != D:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    device = q.device
+    if causal and not (cu_seqlens_q is cu_seqlens_k or torch.equal(cu_seqlens_q, cu_seqlens_k)):
+        raise ValueError("causal varlen attention needs q and k to share cu_seqlens")
+    q_ids = seqlens_to_doc_ids(cu_seqlens_q, M)
+    kv_ids = q_ids if (cu_seqlens_k is cu_seqlens_q and N == M) else seqlens_to_doc_ids(cu_seqlens_k, N)
+    mm = document(q_ids, kv_ids)
+    if causal:
+        mm = and_masks(mm, _causal_mask())
+    bm = create_block_mask(mm, 1, 1, M, N, device=device)
+    if out is None:
+        out = torch.empty((M, Hq, D), dtype=torch.bfloat16, device=device)
+    if lse is None:
+        lse = torch.empty((Hq, M), dtype=torch.float32, device=device)
+    if out.shape != (M, Hq, D) or lse.shape != (Hq, M):
+        raise ValueError("out must be [total_q, Hq, D] and lse [Hq, total_q]")
+    with torch.cuda.device(device):
+        sspec, keep_s = _score_spec(score_mod, device, Hq)
+        c = bm._c()
+        _check(_lib.bsmt_flex_attention_fwd_packed(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), Hq, Hkv, M, N, D, ctypes.byref(c), ctypes.byref(bm._spec),
+            ctypes.byref(sspec), ctypes.c_float(0.0 if scale is None else float(scale)), int(bool(enable_gqa)),
+            out.data_ptr(), lse.data_ptr(), ctypes.c_void_p(_stream_ptr(device))))
+    del keep_s
+    return out, lse
 
 
 def check_device_status(device=None) -> None:

@@ -74,6 +74,9 @@ struct AttnParams {
     const float* slopes;  // ALiBi slopes [Hq] or null (default 2^(-8(h+1)/Hq))
     __nv_bfloat16* out;
     float* lse;
+    // out element (b, hq, i, d) sits at out + (b*Hq + hq)*out_sbh + i*out_ss + d:
+    // (M*D, D) for [B, Hq, M, D], (D, Hq*D) for the packed [M, Hq, D] (B = 1)
+    int64_t out_sbh, out_ss;
     // split-KV: each (b, hq, q-block pair) row of entries is cut into
     // num_splits consecutive slices, one unit each. With num_splits > 1 the
     // epilogue writes, per slice, O / l in fp32 to ws_o [S][B*Hq*M][D] and the
@@ -794,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             // epilogue: out = O / l, lse = ln2 * (m + log2 l)
-            __nv_bfloat16* orow = p.out + ((static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.M + q) * D;
+            __nv_bfloat16* orow = p.out + (static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.out_sbh + q * p.out_ss;
             const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
             const float row_lse = [&] {
                 const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
@@ -896,7 +899,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // columns [l * D/32, (l + 1) * D/32).
 template <int D>
 __global__ void __launch_bounds__(256) splitkv_combine_kernel(const float* ws_o, const float* ws_lse, int splits,
-                                                              int64_t rows, __nv_bfloat16* out, float* lse) {
+                                                              int64_t rows, int64_t M, int64_t out_sbh,
+                                                              int64_t out_ss, __nv_bfloat16* out, float* lse) {
     constexpr int kPer = D / 32;
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -922,7 +926,7 @@ __global__ void __launch_bounds__(256) splitkv_combine_kernel(const float* ws_o,
     uint32_t pk[kPer / 2];
 #pragma unroll
     for (int c = 0; c < kPer / 2; ++c) pk[c] = pack_bf16x2(acc[2 * c] * inv, acc[2 * c + 1] * inv);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(out + row * D + lane * kPer);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(out + (row / M) * out_sbh + (row % M) * out_ss + lane * kPer);
 #pragma unroll
     for (int c = 0; c < kPer / 2; ++c) dst[c] = pk[c];
     if (lane == 0) lse[row] = total > 0.f ? m + logf(total) : -INFINITY;

@@ -19,6 +19,7 @@
 #include "bsmt.h"
 #include "mask_build.cuh"
 #include "mask_transpose.cuh"
+#include "varlen.cuh"
 #include "mask_dnf.cuh"
 #include "ptx.cuh"
 
@@ -215,10 +216,13 @@ bsmt_status get_encoder(EncodeTiledFn* fn) {
     return BSMT_OK;
 }
 
-// bf16 tensor [BH, S, D] as a 3-D map with 64 x 128 x 1 boxes and 128-byte swizzle.
-bsmt_status encode_bhsd(EncodeTiledFn enc, CUtensorMap* map, const void* base, int64_t BH, int64_t S, int64_t D) {
+// bf16 tensor of (BH, S, D) as a 3-D map with 64 x 128 x 1 boxes and 128-byte
+// swizzle. Row s of head bh starts at base + (bh * sbh + s * ss) elements:
+// (S*D, D) for [BH, S, D], (D, H*D) for a packed [S, H, D].
+bsmt_status encode_bhsd(EncodeTiledFn enc, CUtensorMap* map, const void* base, int64_t BH, int64_t S, int64_t D,
+                        int64_t sbh, int64_t ss) {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D * 2), static_cast<cuuint64_t>(S * D * 2)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ss * 2), static_cast<cuuint64_t>(sbh * 2)};
     const cuuint32_t box[3] = {64, 128, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -230,9 +234,10 @@ bsmt_status encode_bhsd(EncodeTiledFn enc, CUtensorMap* map, const void* base, i
 
 // out [BH, S, D] bf16 as a 3-D map with 32 x 32 x 1 boxes (64-byte rows) and
 // 64-byte swizzle; the attention epilogue stores through it.
-bsmt_status encode_out(EncodeTiledFn enc, CUtensorMap* map, void* base, int64_t BH, int64_t S, int64_t D) {
+bsmt_status encode_out(EncodeTiledFn enc, CUtensorMap* map, void* base, int64_t BH, int64_t S, int64_t D,
+                       int64_t sbh, int64_t ss) {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D * 2), static_cast<cuuint64_t>(S * D * 2)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ss * 2), static_cast<cuuint64_t>(sbh * 2)};
     const cuuint32_t box[3] = {32, 32, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
@@ -379,7 +384,7 @@ namespace {
 bsmt_status attention(const void* q, const void* k, const void* v, int64_t B, int64_t Hq, int64_t Hkv, int64_t M,
                       int64_t N, int64_t D, const bsmt_block_mask* bm, const bsmt_mask_spec* mask_spec,
                       const bsmt_score_spec* score, float scale, int32_t enable_gqa, int num_splits, float* ws_o,
-                      float* ws_lse, void* out, float* lse, void* stream) {
+                      float* ws_lse, void* out, float* lse, void* stream, bool packed = false) {
     if (B < 0 || Hq < 0 || Hkv < 0 || M < 0 || N < 0)
         return fail(BSMT_ERR_INVALID_ARGUMENT, "negative size (B=%lld Hq=%lld Hkv=%lld M=%lld N=%lld)",
                     static_cast<long long>(B), static_cast<long long>(Hq), static_cast<long long>(Hkv),
@@ -483,10 +488,15 @@ bsmt_status attention(const void* q, const void* k, const void* v, int64_t B, in
     st = get_encoder(&enc);
     if (st != BSMT_OK) return st;
     CUtensorMap tq, tk, tv, to;
-    if ((st = encode_bhsd(enc, &tq, q, B * Hq, M, D)) != BSMT_OK) return st;
-    if ((st = encode_out(enc, &to, out, B * Hq, M, D)) != BSMT_OK) return st;
-    if ((st = encode_bhsd(enc, &tk, k, B * Hkv, N, D)) != BSMT_OK) return st;
-    if ((st = encode_bhsd(enc, &tv, v, B * Hkv, N, D)) != BSMT_OK) return st;
+    // element strides (head, row): [B, H, S, D], or the packed [S, H, D] with B = 1
+    const int64_t q_sbh = packed ? D : M * D, q_ss = packed ? Hq * D : D;
+    const int64_t kv_sbh = packed ? D : N * D, kv_ss = packed ? Hkv * D : D;
+    if ((st = encode_bhsd(enc, &tq, q, B * Hq, M, D, q_sbh, q_ss)) != BSMT_OK) return st;
+    if ((st = encode_out(enc, &to, out, B * Hq, M, D, q_sbh, q_ss)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tk, k, B * Hkv, N, D, kv_sbh, kv_ss)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tv, v, B * Hkv, N, D, kv_sbh, kv_ss)) != BSMT_OK) return st;
+    p.out_sbh = q_sbh;
+    p.out_ss = q_ss;
 
     p.B = static_cast<int32_t>(B);
     p.Hq = static_cast<int32_t>(Hq);
@@ -519,10 +529,10 @@ bsmt_status attention(const void* q, const void* k, const void* v, int64_t B, in
         if (blocks > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "grid too large");
         if (D == 128)
             bsmt::splitkv_combine_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-                ws_o, ws_lse, num_splits, rows, static_cast<__nv_bfloat16*>(out), lse);
+                ws_o, ws_lse, num_splits, rows, M, p.out_sbh, p.out_ss, static_cast<__nv_bfloat16*>(out), lse);
         else
             bsmt::splitkv_combine_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-                ws_o, ws_lse, num_splits, rows, static_cast<__nv_bfloat16*>(out), lse);
+                ws_o, ws_lse, num_splits, rows, M, p.out_sbh, p.out_ss, static_cast<__nv_bfloat16*>(out), lse);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "split-KV combine launch: %s", cudaGetErrorString(e));
     }
@@ -720,3 +730,32 @@ extern "C" bsmt_status bsmt_block_mask_to_dense(const bsmt_block_mask* kv, int32
     if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "to_dense launch: %s", cudaGetErrorString(e));
     return ok();
 }
+
+extern "C" bsmt_status bsmt_seqlens_to_doc_ids(const int32_t* cu_seqlens, int32_t num_seqs, int64_t total,
+                                               int32_t* doc_ids, void* stream) {
+    if (num_seqs < 0 || total < 0) return fail(BSMT_ERR_INVALID_ARGUMENT, "negative num_seqs or total");
+    if (total == 0) return ok();
+    if (cu_seqlens == nullptr || doc_ids == nullptr || !aligned(cu_seqlens, 4) || !aligned(doc_ids, 4))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "cu_seqlens and doc_ids must be non-NULL and 4-byte aligned");
+    if (total > kMaxLen) return fail(BSMT_ERR_UNSUPPORTED, "total above %lld", static_cast<long long>(kMaxLen));
+    int dev = 0, nsm = 0;
+    bsmt_status st = sm_count(&dev, &nsm);
+    if (st != BSMT_OK) return st;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 4 * nsm) blocks = 4 * nsm;
+    bsmt::seqlens_to_doc_ids_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        cu_seqlens, num_seqs, total, doc_ids);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "doc id launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+extern "C" bsmt_status bsmt_flex_attention_fwd_packed(const void* q, const void* k, const void* v, int64_t Hq,
+                                                      int64_t Hkv, int64_t M, int64_t N, int64_t D,
+                                                      const bsmt_block_mask* bm, const bsmt_mask_spec* mask_spec,
+                                                      const bsmt_score_spec* score, float scale, int32_t enable_gqa,
+                                                      void* out, float* lse, void* stream) {
+    return attention(q, k, v, 1, Hq, Hkv, M, N, D, bm, mask_spec, score, scale, enable_gqa, 1, nullptr, nullptr, out,
+                     lse, stream, /*packed=*/true);
+}
+

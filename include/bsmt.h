@@ -302,6 +302,34 @@ bsmt_status bsmt_flex_attention_fwd_splitkv_static(const void* q, const void* k,
                                                    float scale, int32_t enable_gqa, int32_t num_splits, void* out,
                                                    float* lse, void* stream);
 
+/* --------------------------------------------------- packed sequences
+ * Varlen attention in the cu_seqlens form (L-GATr "attention backends" page:
+ * packed events with a block-diagonal mask, and the varlen kernels'
+ * cu_seqlens_q / max_seqlen_q). The sequences are packed along one token
+ * axis; token t of the pack belongs to sequence i for
+ * cu_seqlens[i] <= t < cu_seqlens[i+1].
+ *
+ * bsmt_seqlens_to_doc_ids writes doc_ids[t] = that i (device int32 [total]),
+ * and num_seqs for tokens at or past cu_seqlens[num_seqs]. cu_seqlens
+ * (device int32 [num_seqs + 1]) must start at 0 and not decrease; the kernel
+ * checks this and reports BSMT_ERR_DEVICE_PRECONDITION. With those ids as
+ * DOCUMENT ids (and CAUSAL for causal attention when q and k share
+ * cu_seqlens), a BlockMask over (total_q, total_k) with B = H = 1 gives each
+ * token exactly the keys of its sequence. Stream-ordered on `stream`. */
+bsmt_status bsmt_seqlens_to_doc_ids(const int32_t* cu_seqlens, int32_t num_seqs, int64_t total, int32_t* doc_ids,
+                                    void* stream);
+
+/* bsmt_flex_attention_fwd on packed tensors, B = 1:
+ *   q    device bf16 [M, Hq, D] (M = total query tokens), contiguous, 16-byte aligned
+ *   k, v device bf16 [N, Hkv, D]
+ *   out  device bf16 [M, Hq, D]
+ *   lse  device float [Hq, M]
+ * Everything else as in bsmt_flex_attention_fwd (block_mask has B = 1). */
+bsmt_status bsmt_flex_attention_fwd_packed(const void* q, const void* k, const void* v, int64_t Hq, int64_t Hkv,
+                                           int64_t M, int64_t N, int64_t D, const bsmt_block_mask* block_mask,
+                                           const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score, float scale,
+                                           int32_t enable_gqa, void* out, float* lse, void* stream);
+
 /* Thread-local message for the last failed call on this thread ("" if none). */
 const char* bsmt_last_error(void);
 

@@ -29,7 +29,8 @@ def test_every_declared_symbol_is_exported():
     assert names == sorted(["bsmt_block_mask_shape", "bsmt_create_block_mask", "bsmt_flex_attention_fwd",
                             "bsmt_block_mask_transpose", "bsmt_block_mask_to_dense",
                             "bsmt_splitkv_workspace_bytes", "bsmt_flex_attention_fwd_splitkv",
-                            "bsmt_flex_attention_fwd_splitkv_static",
+                            "bsmt_flex_attention_fwd_splitkv_static", "bsmt_seqlens_to_doc_ids",
+                            "bsmt_flex_attention_fwd_packed",
                             "bsmt_last_error", "bsmt_check_device_status", "bsmt_version"])
     lib = ctypes.CDLL(bsmt.library_path())
     for n in names:
@@ -257,3 +258,16 @@ def test_static_scratch_rejects_sizes_above_its_limit():
     assert "static" in _lib.bsmt_last_error().decode() and "workspace" in _lib.bsmt_last_error().decode()
     assert f(FAKE, FAKE, FAKE, 1, 2, 2, 128, 4096, 96, None, None, None, ctypes.c_float(0.0), 0, 4,
              FAKE, FAKE, null) == UNSUPPORTED  # D = 96
+
+
+def test_varlen_argument_errors():
+    null = ctypes.c_void_p(0)
+    assert _lib.bsmt_seqlens_to_doc_ids(None, 2, 10, None, null) == INVALID
+    assert _lib.bsmt_seqlens_to_doc_ids(ctypes.c_void_p(FAKE), -1, 10, ctypes.c_void_p(FAKE), null) == INVALID
+    assert _lib.bsmt_seqlens_to_doc_ids(ctypes.c_void_p(FAKE + 2), 2, 10, ctypes.c_void_p(FAKE), null) == INVALID
+    assert _lib.bsmt_seqlens_to_doc_ids(None, 0, 0, None, null) == OK  # nothing to write
+    f = _lib.bsmt_flex_attention_fwd_packed
+    assert f(FAKE, FAKE, FAKE, 4, 3, 128, 128, 128, None, None, None, ctypes.c_float(0.0), 1, FAKE, FAKE,
+             null) == SHAPE  # Hq not a multiple of Hkv
+    assert f(FAKE, FAKE, FAKE, 4, 4, 128, 128, 80, None, None, None, ctypes.c_float(0.0), 0, FAKE, FAKE,
+             null) == UNSUPPORTED

@@ -1,0 +1,60 @@
+"""GPU parity: packed variable-length attention (cu_seqlens) vs the fp64
+oracle, including empty sequences, tokens past the last sequence, GQA,
+causal and score mods."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_masked_tile_b200 as bsmt
+from oracle import attention as oa
+
+pytestmark = pytest.mark.gpu
+
+
+def packed(seed, Mt, Nt, Hq, Hkv, D):
+    g = torch.Generator("cpu").manual_seed(seed)
+    return tuple(torch.randn(shape, generator=g).to(torch.bfloat16)
+                 for shape in ((Mt, Hq, D), (Nt, Hkv, D), (Nt, Hkv, D)))
+
+
+def check(seed, cu_q, cu_k, Mt, Nt, Hq, Hkv, D, causal, mods=()):
+    q, k, v = packed(seed, Mt, Nt, Hq, Hkv, D)
+    cq = torch.tensor(cu_q, dtype=torch.int32).cuda()
+    ck = cq if cu_k is cu_q else torch.tensor(cu_k, dtype=torch.int32).cuda()
+    out, lse = bsmt.flex_attention_varlen(q.cuda(), k.cuda(), v.cuda(), cq, ck, causal=causal,
+                                          score_mod=bsmt.score_mods_from_list(mods), enable_gqa=Hq != Hkv)
+    bsmt.check_device_status()
+    ro, rl = oa.flex_attention_varlen(q, k, v, cu_q, cu_k, causal, mods, None, Hq != Hkv)
+    err = np.abs(out.float().cpu().numpy() - ro).max()
+    assert err < 2e-2, err
+    got_l = lse.cpu().numpy()
+    assert np.array_equal(np.isneginf(got_l), np.isneginf(rl))
+    fin = np.isfinite(rl)
+    assert np.abs(got_l[fin] - rl[fin]).max() < 1e-2
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_causal_shared_seqlens(D):
+    cu = [0, 300, 301, 1000, 1500, 2600]
+    check(1, cu, cu, 2600, 2600, 4, 2, D, True)
+
+
+def test_non_causal_different_lengths_and_tail():
+    cu_q = [0, 129, 129, 400, 700]
+    cu_k = [0, 500, 777, 800, 1900]
+    check(2, cu_q, cu_k, 760, 1900, 2, 2, 128, False)   # q tokens 700..759 belong to no sequence
+
+
+def test_score_mods_and_many_sequences():
+    rng = np.random.default_rng(3)
+    lens = rng.integers(1, 300, size=40)
+    cu = [0] + list(np.cumsum(lens))
+    check(3, cu, cu, int(cu[-1]), int(cu[-1]), 4, 4, 64, True, (("softcap", 20.0),))
+    check(4, cu, cu, int(cu[-1]), int(cu[-1]), 4, 1, 128, True, (("alibi", None),))
+
+
+def test_unsorted_cu_seqlens_are_reported():
+    cu = torch.tensor([0, 100, 50, 200], dtype=torch.int32).cuda()
+    bsmt.seqlens_to_doc_ids(cu, 200)
+    with pytest.raises(RuntimeError, match="DEVICE_PRECONDITION"):
+        bsmt.check_device_status()
