@@ -52,6 +52,8 @@ def parse(argv=None):
     ap.add_argument("--workload", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-side-kernels", action="store_true",
+                    help="skip the side measurements (builder, transpose, split-KV, varlen) after the step")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller cases for profiling only)")
     return ap.parse_args(argv)
@@ -227,6 +229,19 @@ def side_kernels(bsmt, mask, w, dev, hbm_peak: float) -> dict:
     mss = _time_launches(lambda: bsmt.flex_attention(qd, kd, vd, enable_gqa=True, out=out, lse=lse,
                                                      num_splits=S, workspace=ws), reps=5)
     bsmt.check_device_status(dev)
+    # varlen: the packed-document workload in the cu_seqlens form (tokens, H, D)
+    lens = workloads.document_lengths(16384, workloads.get(4).seed)
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device=dev)
+    T, Hv = int(sum(lens)), 32
+    qv, kv_, vv = (torch.randn((T, Hv, 128), generator=g).to(torch.bfloat16).to(dev) for _ in range(3))
+    ids = bsmt.seqlens_to_doc_ids(cu, T)
+    bmv = bsmt.create_block_mask(bsmt.and_masks(bsmt.document(ids), bsmt.causal()), 1, 1, T, T, device=dev)
+    vflops = counted_flops(bmv, 128) * Hv
+    msv = _time_launches(lambda: bsmt.flex_attention_varlen(qv, kv_, vv, cu, cu, causal=True), reps=5)
+    bsmt.check_device_status(dev)
+    res["varlen_doc_causal"] = {"shape": f"{len(lens)} packed sequences, {T} tokens, H=32, D=128, causal",
+                                "ms": msv, "tflops": vflops / (msv * 1e-3) / 1e12,
+                                "note": "includes doc-id and block-mask kernels per call"}
     res["splitkv_decode"] = {"shape": f"B={Bd} Hq={Hqd} Hkv={Hkvd} M={Md} N={Nd} D={Dd}, no mask", "splits": S,
                              "plain_ms": ms1, "plain_tflops": flops / (ms1 * 1e-3) / 1e12,
                              "split_ms": mss, "split_tflops": flops / (mss * 1e-3) / 1e12}
@@ -403,7 +418,7 @@ def main():
 
     peaks, peak_src = load_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    side = side_kernels(bsmt, mask, w, dev, hbm_peak)
+    side = None if args.no_side_kernels else side_kernels(bsmt, mask, w, dev, hbm_peak)
     attn_tflops = (flops / (attn_ms * 1e-3)) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     traffic = profile_traffic(w.name)

@@ -726,8 +726,13 @@ def flex_attention_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_
     if v.shape != k.shape or Dk != D:
         raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
     device = q.device
-    if causal and not (cu_seqlens_q is cu_seqlens_k or torch.equal(cu_seqlens_q, cu_seqlens_k)):
-        raise ValueError("causal varlen attention needs q and k to share cu_seqlens")
+    mods = [score_mod] if isinstance(score_mod, ScoreMod) else list(score_mod or ())
+    # Causal masking and ALiBi see packed positions. These equal positions
+    # within the sequence only when q and k share cu_seqlens (the sequence
+    # start cancels in kv_idx - q_idx).
+    if (causal or any(m.kind == SCORE_ALIBI for m in mods)) and not (
+            cu_seqlens_q is cu_seqlens_k or torch.equal(cu_seqlens_q, cu_seqlens_k)):
+        raise ValueError("causal or ALiBi varlen attention needs q and k to share cu_seqlens")
     q_ids = seqlens_to_doc_ids(cu_seqlens_q, M)
     kv_ids = q_ids if (cu_seqlens_k is cu_seqlens_q and N == M) else seqlens_to_doc_ids(cu_seqlens_k, N)
     mm = document(q_ids, kv_ids)
@@ -741,7 +746,7 @@ def flex_attention_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_
     if out.shape != (M, Hq, D) or lse.shape != (Hq, M):
         raise ValueError("out must be [total_q, Hq, D] and lse [Hq, total_q]")
     with torch.cuda.device(device):
-        sspec, keep_s = _score_spec(score_mod, device, Hq)
+        sspec, keep_s = _score_spec(mods, device, Hq)
         c = bm._c()
         _check(_lib.bsmt_flex_attention_fwd_packed(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), Hq, Hkv, M, N, D, ctypes.byref(c), ctypes.byref(bm._spec),

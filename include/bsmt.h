@@ -324,7 +324,10 @@ bsmt_status bsmt_seqlens_to_doc_ids(const int32_t* cu_seqlens, int32_t num_seqs,
  *   k, v device bf16 [N, Hkv, D]
  *   out  device bf16 [M, Hq, D]
  *   lse  device float [Hq, M]
- * Everything else as in bsmt_flex_attention_fwd (block_mask has B = 1). */
+ * Everything else as in bsmt_flex_attention_fwd (block_mask has B = 1).
+ * Positions seen by the mask and by ALiBi are packed token indices; they
+ * equal positions within the sequence only when q and k share cu_seqlens
+ * (the Python binding requires that for causal and for ALiBi). */
 bsmt_status bsmt_flex_attention_fwd_packed(const void* q, const void* k, const void* v, int64_t Hq, int64_t Hkv,
                                            int64_t M, int64_t N, int64_t D, const bsmt_block_mask* block_mask,
                                            const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score, float scale,

@@ -58,3 +58,11 @@ def test_unsorted_cu_seqlens_are_reported():
     bsmt.seqlens_to_doc_ids(cu, 200)
     with pytest.raises(RuntimeError, match="DEVICE_PRECONDITION"):
         bsmt.check_device_status()
+
+
+def test_alibi_needs_shared_seqlens():
+    q, k, v = (t.cuda() for t in packed(5, 200, 300, 2, 2, 64))
+    cq = torch.tensor([0, 100, 200], dtype=torch.int32).cuda()
+    ck = torch.tensor([0, 150, 300], dtype=torch.int32).cuda()
+    with pytest.raises(ValueError, match="share cu_seqlens"):
+        bsmt.flex_attention_varlen(q, k, v, cq, ck, score_mod=bsmt.alibi())
