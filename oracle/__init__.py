@@ -25,6 +25,11 @@ What it computes is the plain definition of each operation:
   applies score_mod before the softmax (attention-gym page, "A gallery that
   grew into a toolkit"), sets masked scores to -inf and takes the softmax.
   A row with no allowed key gives output 0 and lse = -inf.
+* ``backward.flex_attention_backward`` takes the gradients of
+  sum(out * dout) with respect to q, k and v through the same steps in fp64
+  (FlagAttention page, "Operator overview": forward and backward with GQA;
+  tensorplay.nn.attention page, BlockMask "Details" items 3-4: dK and dV walk
+  the mask along the query dimension).
 
 Parity: every function here is pinned by tests in ``tests/test_oracle_*.py``
 against closed forms, library routines on special cases and invariants. The
