@@ -80,7 +80,7 @@ class _BlockMask(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(_LIB_PATH):
         raise ImportError(
-            f"{_LIB_PATH} is missing: build it with `python -m block_sparse_masked_tile_b200.build` "
+            f"{_LIB_PATH} is missing: build it with `python block_sparse_masked_tile_b200/build.py` "
             "(there is no fallback implementation)")
     lib = ctypes.CDLL(_LIB_PATH)
     i64, i32, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p

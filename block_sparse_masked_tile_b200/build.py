@@ -1,6 +1,9 @@
 """Build libbsmt.so in-tree for sm_100a with nvcc.
 
-Usage: python -m block_sparse_masked_tile_b200.build [--verbose-ptxas]
+Usage: python block_sparse_masked_tile_b200/build.py [--verbose-ptxas]
+
+Run it as a script (or load it by path): importing it through the package
+would first try to load the library it builds.
 """
 from __future__ import annotations
 
@@ -15,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbsmt.so")
 SOURCES = ["bsmt.cu"]
-HEADERS = ["ptx.cuh", "mask_dnf.cuh", "mask_build.cuh", "attn_fwd.cuh"]
+HEADERS = sorted(f for f in os.listdir(CSRC) if f.endswith(".cuh"))
 
 
 def nvcc() -> str:
