@@ -13,6 +13,8 @@ The API follows the tensorplay.nn.attention page:
   and full_kv_num_blocks/full_kv_indices (full blocks).
 * ``flex_attention(q, k, v, block_mask, score_mod, scale, enable_gqa)``
   returns ``(out, lse)``.
+* ``flex_attention_backward(q, k, v, out, lse, dout, block_mask, ...)``
+  returns ``(dq, dk, dv)``, the gradients of sum(out * dout).
 * Mask builders: ``noop_mask``, ``causal``, ``sliding_window``,
   ``prefix_lm``, ``sink``, ``document``, ``and_masks`` and ``or_masks``.
 * Score mods: ``softcap`` and ``alibi``.
@@ -30,7 +32,8 @@ __all__ = [
     "BsmtError", "MaskMod", "ScoreMod", "BlockMask", "noop_mask", "causal", "sliding_window", "prefix_lm",
     "sink", "document", "and_masks", "or_masks", "softcap", "alibi", "create_block_mask", "flex_attention",
     "check_device_status", "library_path", "mask_from_tree", "score_mods_from_list", "splitkv_workspace_bytes",
-    "flex_attention_host", "flex_attention_varlen", "seqlens_to_doc_ids",
+    "flex_attention_host", "flex_attention_varlen", "seqlens_to_doc_ids", "flex_attention_backward",
+    "backward_workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -115,6 +118,13 @@ def _load() -> ctypes.CDLL:
                                                    ctypes.POINTER(_MaskSpec), ctypes.POINTER(_ScoreSpec),
                                                    ctypes.c_float, i32, vp, vp, vp]
     lib.bsmt_flex_attention_fwd_packed.restype = i32
+    lib.bsmt_flex_attention_bwd_workspace_bytes.argtypes = [i64, i64, i64, ctypes.POINTER(i64)]
+    lib.bsmt_flex_attention_bwd_workspace_bytes.restype = i32
+    lib.bsmt_flex_attention_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64,
+                                            ctypes.POINTER(_BlockMask), ctypes.POINTER(_BlockMaskQ),
+                                            ctypes.POINTER(_MaskSpec), ctypes.POINTER(_ScoreSpec), ctypes.c_float, i32,
+                                            vp, vp, vp, vp, i64, vp]
+    lib.bsmt_flex_attention_bwd.restype = i32
     lib.bsmt_last_error.argtypes = []
     lib.bsmt_last_error.restype = ctypes.c_char_p
     lib.bsmt_check_device_status.argtypes = [vp]
@@ -595,6 +605,70 @@ def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask
                 out.data_ptr(), lse.data_ptr(), ctypes.c_void_p(_stream_ptr(device))))
     del keep_s, keep_m
     return out, lse
+
+
+def backward_workspace_bytes(B: int, Hq: int, M: int) -> int:
+    """Bytes of device workspace flex_attention_backward needs (lse and delta per query row)."""
+    n = ctypes.c_int64(0)
+    _check(_lib.bsmt_flex_attention_bwd_workspace_bytes(int(B), int(Hq), int(M), ctypes.byref(n)))
+    return int(n.value)
+
+
+def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                            lse: torch.Tensor, dout: torch.Tensor, block_mask: BlockMask | None = None,
+                            score_mod: ScoreMod | Iterable[ScoreMod] | None = None, scale: float | None = None,
+                            enable_gqa: bool = False, workspace: torch.Tensor | None = None):
+    """Gradients (dq, dk, dv) of sum(out * dout) for the forward
+    ``out, lse = flex_attention(q, k, v, block_mask, score_mod, scale, enable_gqa)``.
+    Pass the same arguments as the forward plus its out and lse. dk and dv
+    walk the block mask's q-side lists (computed on first use), dq its
+    kv-side lists. ``workspace``: a uint8 CUDA tensor of at least
+    backward_workspace_bytes(B, Hq, M) bytes, allocated when not given."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 4-D CUDA tensor")
+    B, Hq, M, D = q.shape
+    Bk, Hkv, N, Dk = k.shape
+    if k.shape != v.shape or Bk != B or Dk != D:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    if out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("out and dout must have q's shape")
+    if lse.shape != (B, Hq, M) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, M] tensor")
+    device = q.device
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    need = backward_workspace_bytes(B, Hq, M)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 CUDA tensor")
+    with torch.cuda.device(device):
+        sspec, keep_s = _score_spec(score_mod, device, Hq)
+        bm_c = bmq_c = mspec = None
+        keep_m = []
+        if block_mask is not None:
+            bm_c = block_mask._c()
+            qs = block_mask.q_side()
+            bmq_c = _BlockMaskQ()
+            bmq_c.q_num_blocks = qs["q_num_blocks"].data_ptr()
+            bmq_c.q_indices = qs["q_indices"].data_ptr()
+            bmq_c.full_q_num_blocks = qs["full_q_num_blocks"].data_ptr()
+            bmq_c.full_q_indices = qs["full_q_indices"].data_ptr()
+            mspec = getattr(block_mask, "_spec", None)
+            if mspec is None:
+                mspec, keep_m = block_mask.mask_mod._spec(device, int(block_mask.shape[0]))
+        _check(_lib.bsmt_flex_attention_bwd(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+            B, Hq, Hkv, M, N, D,
+            ctypes.byref(bm_c) if bm_c is not None else None, ctypes.byref(bmq_c) if bmq_c is not None else None,
+            ctypes.byref(mspec) if mspec is not None else None, ctypes.byref(sspec),
+            ctypes.c_float(0.0 if scale is None else float(scale)), int(bool(enable_gqa)),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+            ctypes.c_void_p(_stream_ptr(device))))
+    del keep_s, keep_m
+    return dq, dk, dv
 
 
 def flex_attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask_mod: MaskMod | None = None,

@@ -57,8 +57,9 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     return LIB
 
 
-# The attention kernel is sized for 168 registers per thread (384 threads, one
-# CTA per SM); a different count means the launch or the layout changed.
+# The attention kernels (forward and backward) are sized for 168 registers per
+# thread (384 threads, one CTA per SM, split further by setmaxnreg); a
+# different count means the launch or the layout changed.
 LAUNCH_REGS = 168
 
 
@@ -68,7 +69,8 @@ def check_attention_registers(ptxas_log: str) -> None:
     for line in ptxas_log.splitlines():
         if "Compiling entry function" in line:
             current = line
-        elif "Used" in line and "registers" in line and current and "attn_fwd_kernel" in current:
+        elif "Used" in line and "registers" in line and current and (
+                "attn_fwd_kernel" in current or "attn_bwd_kernel" in current):
             regs = int(line.split("Used")[1].split("registers")[0])
             seen += 1
             if regs != LAUNCH_REGS:

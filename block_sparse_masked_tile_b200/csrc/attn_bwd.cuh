@@ -1,0 +1,714 @@
+// Block-sparse masked attention backward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// The gradients of sum(out * dout) with respect to q, k and v, for the
+// forward of attn_fwd.cuh. The structure follows the tensorplay.nn.attention
+// page (BlockMask "Details" items 3-4): dK and dV walk the mask along the
+// query axis, using the q-side lists (q_num_blocks / q_indices and their full
+// counterparts). dQ walks it along the key axis, using the kv-side lists as
+// the forward does. Tiles that the lists leave out add nothing. mask_mod runs
+// on PARTIAL tiles only; score_mod and its derivative run on every visited
+// tile.
+//
+// With s = scale * q.k, z = score_mod(s), P = exp(z - lse) (lse from the
+// forward), dP = dO V^T and delta = rowsum(dO * out):
+//   dS = P * (dP - delta) * dz/ds,  dV = P^T dO,  dK = scale * dS^T Q,
+//   dQ = scale * dS K.
+// One kernel template serves both directions (flag KVSIDE):
+//   KVSIDE: a unit is (b, hkv, kv-block). K and V stay in shared memory while
+//     the Q and dO tiles stream in: every q-block listed for the kv-block, for
+//     every query head of the GQA group. Products are taken transposed, with
+//     one kv row per TMEM lane:
+//     S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q.
+//   !KVSIDE: a unit is (b, hq, q-block). Q and dO stay; K and V of the listed
+//     kv-blocks stream in: S = Q K^T, dP = dO V^T, dQ += dS K.
+// dQ has its own kernel, so it needs neither an fp32 accumulator in global
+// memory nor atomics, and the result does not depend on scheduling.
+//
+// Pipeline. Every streamed 128-row tile is processed as two halves of 64
+// rows. Half h of every entry uses TMEM buffer h (64 columns of S, 64 of dP)
+// and softmax warpgroup h. One MMA warp issues, for half c, S(c) and dP(c),
+// then the accumulating products of half c-1 once its warpgroup has stored
+// P and dS back to TMEM. While one warpgroup computes, the tensor core runs
+// the other half's products. MMAs issued by one thread run in order, so
+// S(c) overwrites buffer c & 1 only after the products of half c-2 that read
+// it.
+//
+// CTA of 384 threads (one per SM; every CTA takes all 512 TMEM columns):
+//   warps 0-3  half 0 (thread = TMEM lane = tile row)
+//   warps 4-7  half 1
+//   warp 8     builds the entry list, then loads tiles with TMA
+//   warp 9     allocates TMEM and issues the MMAs (one elected lane)
+//   warps 10-11 idle; they complete the third warpgroup, whose registers
+//              setmaxnreg hands to the two softmax warpgroups
+// TMEM columns: S0 [0,64), dP0 [64,128), S1 [128,192), dP1 [192,256),
+// acc0 [256, 256+D) (dV or dQ), acc1 [256+D, 256+2D) (dK). P and dS as bf16
+// pairs overwrite the first 32 columns of their S and dP.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "attn_fwd.cuh"
+#include "mask_dnf.cuh"
+#include "ptx.cuh"
+
+namespace bsmt {
+
+struct BwdParams {
+    int32_t B, Hq, Hkv, M, N, QB, KB, group;
+    int32_t Bm, Hm, has_block_mask;
+    // kv-side lists (dq kernel) or q-side lists (dk/dv kernel): rows
+    // [Bm, Hm, list_rows], each list list_len entries long
+    const int32_t* num;
+    const int32_t* idx;
+    const int32_t* full_num;
+    const int32_t* full_idx;
+    int32_t list_rows, list_len;
+    float scale, scale_log2, cap, inv_cap;
+    const float* slopes;  // ALiBi slopes [Hq] or null (default 2^(-8(h+1)/Hq))
+    // (lse * log2(e), delta) per query row, padded to whole q-blocks:
+    // [B*Hq][QB*128]. lse2 is +inf for padding rows and rows with no key.
+    const float2* ld;
+    __nv_bfloat16* g0;  // dq (dq kernel) or dk [B, Hkv, N, D]
+    __nv_bfloat16* g1;  // dv [B, Hkv, N, D]
+    int32_t num_units;
+};
+
+constexpr int kBwdThreads = 384;
+constexpr int kBwdWarpLoad = 8;
+constexpr int kBwdWarpMma = 9;
+constexpr int kBwdMaxEntries = 4096;  // entries of one unit (list length x GQA group)
+constexpr uint32_t kBwdPartial = 0x80000000u;
+constexpr int kBwdRowTerms = 4;  // mask alternatives kept per row in registers
+
+template <int D>
+struct BwdSmem {
+    static constexpr int kTile = 128 * D * 2;
+    static constexpr int kF0 = 0;                   // K (dk/dv) or Q (dq)
+    static constexpr int kF1 = kTile;               // V or dO
+    static constexpr int kStage = 2 * kTile;        // stage s: T0 at kStage + 2 s kTile, T1 one tile further
+    static constexpr int kLd = kStage + 4 * kTile;  // stage s: 128 float2 (lse2, delta) at kLd + 1024 s
+    static constexpr int kEntries = kLd + 2048;
+    static constexpr int kFlags = kEntries + 4 * kBwdMaxEntries;
+    static constexpr int kBars = kFlags + kBwdMaxEntries;
+    static constexpr int kBarFixed = 0, kBarTFull = 1, kBarTEmpty = 3, kBarSFull = 5, kBarPFull = 7, kBarAcc = 9,
+                         kNumBars = 10;
+    static constexpr int kTmemSlot = kBars + 8 * kNumBars;
+    static constexpr int kAbort = kTmemSlot + 4;
+    static constexpr int kCount = kAbort + 4;
+    static constexpr int kTotal = kCount + 8;
+    // never less than 120 KB, so that a second CTA cannot share the SM (and
+    // wait in tcgen05.alloc for the TMEM the first one holds)
+    static constexpr int kAlloc = (kTotal + 1024 > 120 * 1024) ? kTotal + 1024 : 120 * 1024;
+    static_assert(kAlloc <= 227 * 1024, "shared memory layout exceeds one CTA's limit");
+};
+
+// Score (log2 units) and dz/ds for one element: x = q.k, dkv = kv_idx - q_idx.
+template <int SCORE>
+__device__ __forceinline__ void bwd_score(const BwdParams& p, float x, float dkv, float slope, float sl2, float& z2,
+                                          float& dz) {
+    if constexpr (SCORE == kScoreNone) {
+        z2 = x * p.scale_log2;
+        dz = 1.f;
+    } else if constexpr (SCORE == kScoreSoftcap) {
+        const float t = tanh_approx(x * (p.scale * p.inv_cap));
+        z2 = (p.cap * kLog2e) * t;
+        dz = fmaf(-t, t, 1.f);
+    } else if constexpr (SCORE == kScoreAlibi) {
+        z2 = fmaf(x, p.scale_log2, sl2 * dkv);
+        dz = 1.f;
+    } else if constexpr (SCORE == kScoreSoftcapAlibi) {
+        const float t = tanh_approx(x * (p.scale * p.inv_cap));
+        z2 = fmaf(p.cap * kLog2e, t, sl2 * dkv);
+        dz = fmaf(-t, t, 1.f);
+    } else {  // ALiBi, then soft-cap
+        const float t = tanh_approx(fmaf(x, p.scale, slope * dkv) * p.inv_cap);
+        z2 = (p.cap * kLog2e) * t;
+        dz = fmaf(-t, t, 1.f);
+    }
+}
+
+// The q interval [lo, hi] one non-document leaf allows for a fixed key kv
+// (the leaves of mask_dnf.cuh read along the other axis):
+//   CAUSAL kv <= q             -> q >= kv
+//   WINDOW q - kv < W          -> q <= kv + W - 1
+//   PREFIX_LM kv < P or q >= kv -> every q when kv < P, else q >= kv
+//   SINK kv < S                -> every q when kv < S, else none
+__device__ __forceinline__ void leaf_clamp_q(int32_t kind, int32_t arg, int64_t kv, int64_t& lo, int64_t& hi) {
+    switch (kind) {
+        case BSMT_MASK_CAUSAL:
+            lo = lo > kv ? lo : kv;
+            break;
+        case BSMT_MASK_WINDOW: {
+            const int64_t h = kv + static_cast<int64_t>(arg) - 1;
+            hi = hi < h ? hi : h;
+            break;
+        }
+        case BSMT_MASK_PREFIX_LM:
+            if (kv >= static_cast<int64_t>(arg)) lo = lo > kv ? lo : kv;
+            break;
+        case BSMT_MASK_SINK:
+            if (kv >= static_cast<int64_t>(arg)) hi = -1;
+            break;
+        default:  // NOOP; DOCUMENT is applied by the caller
+            break;
+    }
+}
+
+// q interval of term t for key kv, within [0, M-1] (document leaves excluded).
+__device__ __forceinline__ void term_q_interval(const MaskDnf& m, int t, int64_t kv, int64_t M, int64_t& lo,
+                                                int64_t& hi) {
+    lo = 0;
+    hi = M - 1;
+    for (int i = m.term_begin[t]; i < m.term_begin[t + 1]; ++i)
+        if (m.leaves[i].kind != BSMT_MASK_DOCUMENT) leaf_clamp_q(m.leaves[i].kind, m.leaves[i].arg, kv, lo, hi);
+}
+
+// (lse2, delta) per padded query row: lse2 = lse * log2(e) (+inf where lse is
+// -inf and for rows past M, so that P = 0 there), delta = sum_d out * dout in
+// fp32. One warp per row; lane l reads D/32 consecutive elements.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* out, const __nv_bfloat16* dout,
+                                                       const float* lse, int64_t rows_pad, int32_t M, int32_t QB,
+                                                       float2* ld) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (row >= rows_pad) return;
+    const int64_t per_bh = static_cast<int64_t>(QB) * 128;
+    const int64_t bh = row / per_bh;
+    const int i = static_cast<int>(row - bh * per_bh);
+    float acc = 0.f, l2 = INFINITY;
+    if (i < M) {
+        const int64_t base = (bh * M + i) * D + lane * (D / 32);
+        if constexpr (D == 128) {
+            const uint2 a = *reinterpret_cast<const uint2*>(out + base);
+            const uint2 g = *reinterpret_cast<const uint2*>(dout + base);
+            const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
+            const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
+            const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g.x));
+            const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g.y));
+            acc = fmaf(a0.x, g0.x, fmaf(a0.y, g0.y, fmaf(a1.x, g1.x, a1.y * g1.y)));
+        } else {
+            const uint32_t a = *reinterpret_cast<const uint32_t*>(out + base);
+            const uint32_t g = *reinterpret_cast<const uint32_t*>(dout + base);
+            const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a));
+            const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g));
+            acc = fmaf(a0.x, g0.x, a0.y * g0.y);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+        const float L = __ldg(lse + bh * M + i);
+        l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
+    }
+    if (lane == 0) ld[row] = make_float2(l2, acc);
+}
+
+template <int D, int SCORE, bool KVSIDE>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p, const MaskDnf dnf) {
+    using L = BwdSmem<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * static_cast<uint32_t>(i); };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+    uint32_t* entries = reinterpret_cast<uint32_t*>(smem + L::kEntries);
+    int32_t* count_slot = reinterpret_cast<int32_t*>(smem + L::kCount);
+
+    // ------------------------------------------------------------ the unit
+    // dk/dv: kv-blocks in ascending order (under a causal mask the first ones
+    // have the most q-blocks); dq: q-blocks in descending order.
+    int b, hq, hkv, blk;
+    {
+        const int u = blockIdx.x;
+        if constexpr (KVSIDE) {
+            const int n_bh = p.B * p.Hkv;
+            blk = u / n_bh;
+            const int bh = u - blk * n_bh;
+            b = bh / p.Hkv;
+            hkv = bh - b * p.Hkv;
+            hq = hkv * p.group;
+        } else {
+            const int n_bh = p.B * p.Hq;
+            const int r = u / n_bh;
+            blk = p.QB - 1 - r;
+            const int bh = u - r * n_bh;
+            b = bh / p.Hq;
+            hq = bh - b * p.Hq;
+            hkv = hq / p.group;
+        }
+    }
+
+    // ------------------------------------------------------------ set-up
+    if (warp == kBwdWarpLoad) {
+        if (lane == 0) {
+            mbar_init(bar(L::kBarFixed), 1);
+            for (int s = 0; s < 2; ++s) {
+                mbar_init(bar(L::kBarTFull + s), 1);
+                mbar_init(bar(L::kBarTEmpty + s), 1);
+                mbar_init(bar(L::kBarSFull + s), 1);
+                mbar_init(bar(L::kBarPFull + s), 4);
+            }
+            mbar_init(bar(L::kBarAcc), 1);
+            *abort_flag = 0;
+            fence_mbar_init();
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            prefetch_tmap(&tm_do);
+        }
+        // Entry list of the unit: for each query head of the group (dk/dv) or
+        // the unit's head (dq), the blocks of the partial and the full list,
+        // merged in ascending order. A block in both lists counts as partial;
+        // with a ragged KV_LEN the last kv block is partial (dq).
+        uint8_t* flags = smem + L::kFlags;
+        for (int j = lane; j < p.list_len; j += 32) flags[j] = 0;
+        __syncwarp();
+        const int heads = KVSIDE ? p.group : 1;
+        const bool ragged_last = !KVSIDE && (p.N & 127) != 0;
+        const uint32_t below = (1u << lane) - 1u;
+        int T = 0;
+        bool bad = false;
+        for (int g = 0; g < heads; ++g) {
+            if (!p.has_block_mask) {
+                for (int c = 0; c < p.list_len; c += 32) {
+                    const int j = c + lane;
+                    if (j < p.list_len) {
+                        const bool part = ragged_last && j == p.list_len - 1;
+                        entries[T + j] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(g) << 16) |
+                                         (part ? kBwdPartial : 0u);
+                    }
+                }
+                T += p.list_len;
+                continue;
+            }
+            const int hl = KVSIDE ? hq + g : hq;
+            const int bb = p.Bm > 1 ? b : 0;
+            const int hh = p.Hm > 1 ? hl : 0;
+            const int64_t row = (static_cast<int64_t>(bb) * p.Hm + hh) * p.list_rows + blk;
+            int v = 0;
+            if (lane == 0) v = __ldg(p.num + row);
+            if (lane == 1) v = __ldg(p.full_num + row);
+            if (v < 0 || v > p.list_len) {
+                bad = true;
+                v = 0;
+            }
+            const int cnt0 = __shfl_sync(0xFFFFFFFFu, v, 0);
+            const int cnt1 = __shfl_sync(0xFFFFFFFFu, v, 1);
+            const int32_t* l0 = p.idx + row * p.list_len;
+            const int32_t* l1 = p.full_idx + row * p.list_len;
+            for (int j = lane; j < cnt0; j += 32) {
+                const int x = __ldg(l0 + j);
+                if (x >= 0 && x < p.list_len) flags[x] |= 1u;
+                else bad = true;
+            }
+            __syncwarp();
+            for (int j = lane; j < cnt1; j += 32) {
+                const int x = __ldg(l1 + j);
+                if (x >= 0 && x < p.list_len) flags[x] |= 2u;
+                else bad = true;
+            }
+            __syncwarp();
+            for (int c = 0; c < p.list_len; c += 32) {
+                const int j = c + lane;
+                uint32_t f = 0;
+                if (j < p.list_len) {
+                    f = flags[j];
+                    flags[j] = 0;
+                }
+                const bool part = (f & 1u) || (f != 0u && ragged_last && j == p.list_len - 1);
+                const unsigned bal = __ballot_sync(0xFFFFFFFFu, f != 0u);
+                if (f)
+                    entries[T + __popc(bal & below)] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(g) << 16) |
+                                                       (part ? kBwdPartial : 0u);
+                T += __popc(bal);
+            }
+            __syncwarp();
+        }
+        if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
+        if (lane == 0) *count_slot = T;
+    }
+    if (warp == kBwdWarpMma) {
+        tmem_alloc(sbase + L::kTmemSlot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
+    const int T = *reinterpret_cast<volatile int32_t*>(count_slot);
+
+    // Register split: every thread is launched with 168 registers (build.py
+    // checks the count); warpgroup 2 gives some back and the softmax
+    // warpgroups take them: 128 * 80 + 256 * 208 = 63488 <= 384 * 168.
+    if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
+    if (warp == kBwdWarpLoad) {
+        // ================================================= TMA producer warp
+        if (T > 0) {
+            const uint32_t tile = L::kTile;
+            const int zf = KVSIDE ? b * p.Hkv + hkv : b * p.Hq + hq;
+            if (lane == 0) {
+                const uint32_t fb = bar(L::kBarFixed);
+                mbar_arrive_expect_tx(fb, 2 * tile);
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h) {
+                    tma_load_3d(sbase + L::kF0 + h * 16384, KVSIDE ? &tm_k : &tm_q, h * 64, blk * 128, zf, fb);
+                    tma_load_3d(sbase + L::kF1 + h * 16384, KVSIDE ? &tm_v : &tm_do, h * 64, blk * 128, zf, fb);
+                }
+            }
+            for (int e = 0; e < T; ++e) {
+                const int s = e & 1;
+                if (!mbar_wait(bar(L::kBarTEmpty + s), static_cast<uint32_t>((e >> 1) & 1) ^ 1u, abort_flag)) break;
+                const uint32_t ent = entries[e];
+                const int eb = static_cast<int>(ent & 0xFFFFu);
+                const int g = static_cast<int>((ent >> 16) & 0xFFu);
+                if (lane == 0) {
+                    const uint32_t fb = bar(L::kBarTFull + s);
+                    mbar_arrive_expect_tx(fb, 2 * tile + (KVSIDE ? 1024u : 0u));
+                    const uint32_t t0 = sbase + L::kStage + static_cast<uint32_t>(s) * 2u * tile;
+                    const int zt = KVSIDE ? b * p.Hq + hq + g : b * p.Hkv + hkv;
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h) {
+                        tma_load_3d(t0 + h * 16384, KVSIDE ? &tm_q : &tm_k, h * 64, eb * 128, zt, fb);
+                        tma_load_3d(t0 + tile + h * 16384, KVSIDE ? &tm_do : &tm_v, h * 64, eb * 128, zt, fb);
+                    }
+                    if constexpr (KVSIDE)
+                        bulk_load_1d(sbase + L::kLd + 1024u * static_cast<uint32_t>(s),
+                                     p.ld + (static_cast<int64_t>(b * p.Hq + hq + g) * p.QB + eb) * 128, 1024u, fb);
+                }
+                __syncwarp();
+            }
+        }
+    } else if (warp == kBwdWarpMma) {
+        // ================================================= MMA issuer warp
+        if (T > 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+            constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+            const uint64_t f0d = sdesc_sw128(sbase + L::kF0, 16, 1024);
+            const uint64_t f1d = sdesc_sw128(sbase + L::kF1, 16, 1024);
+            bool ok = mbar_wait(bar(L::kBarFixed), 0, abort_flag);
+            // accumulating products of half c, once its warpgroup stored P and dS
+            auto issue_acc = [&](int c) -> bool {
+                const int h = c & 1, e = c >> 1, s = e & 1;
+                if (!mbar_wait(bar(L::kBarPFull + h), static_cast<uint32_t>(e & 1), abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t t0 = sbase + L::kStage + static_cast<uint32_t>(s) * 2u * L::kTile + h * 8192u;
+                const uint32_t t1 = t0 + L::kTile;
+                const uint32_t buf = tmem + 128u * static_cast<uint32_t>(h);
+                if (elect_one()) {
+                    if constexpr (KVSIDE) {
+                        mma_ts_run4(tmem + 256u, buf, sdesc_sw128(t1, 16384, 1024), idesc_acc, c > 0);      // dV += P^T dO
+                        mma_ts_run4(tmem + 256u + D, buf + 64u, sdesc_sw128(t0, 16384, 1024), idesc_acc, c > 0);  // dK += dS^T Q
+                    } else {
+                        mma_ts_run4(tmem + 256u, buf + 64u, sdesc_sw128(t0, 16384, 1024), idesc_acc, c > 0);  // dQ += dS K
+                    }
+                    if (h == 1) mma_commit(bar(L::kBarTEmpty + s));
+                }
+                __syncwarp();
+                return true;
+            };
+            for (int e = 0; e < T && ok; ++e) {
+                const int s = e & 1;
+                if (!(ok = mbar_wait(bar(L::kBarTFull + s), static_cast<uint32_t>((e >> 1) & 1), abort_flag))) break;
+                tc_fence_after();
+                const uint32_t t0 = sbase + L::kStage + static_cast<uint32_t>(s) * 2u * L::kTile;
+                const uint32_t t1 = t0 + L::kTile;
+                for (int h = 0; h < 2 && ok; ++h) {
+                    const uint32_t buf = tmem + 128u * static_cast<uint32_t>(h);
+                    if (elect_one()) {
+                        mma_ss_run<D / 16>(buf, f0d, sdesc_sw128(t0 + h * 8192u, 16, 1024), idesc_s, 0u);
+                        mma_ss_run<D / 16>(buf + 64u, f1d, sdesc_sw128(t1 + h * 8192u, 16, 1024), idesc_s, 0u);
+                        mma_commit(bar(L::kBarSFull + h));
+                    }
+                    __syncwarp();
+                    const int c = 2 * e + h;
+                    if (c > 0) ok = issue_acc(c - 1);
+                }
+            }
+            if (ok) issue_acc(2 * T - 1);
+            if (elect_one()) mma_commit(bar(L::kBarAcc));
+            __syncwarp();
+            mbar_wait(bar(L::kBarAcc), 0, abort_flag);
+        }
+    }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
+        // ================================================= softmax warpgroups
+        const int h = warp >> 2;
+        const int r = threadIdx.x & 127;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t t_s = tmem + 128u * static_cast<uint32_t>(h) + lane_base;
+        const uint32_t t_dp = t_s + 64u;
+        const int64_t row_idx = static_cast<int64_t>(blk) * 128 + r;  // this thread's kv (dk/dv) or q (dq)
+        const int db = dnf.doc_batch > 1 ? b : 0;
+        const bool masked_path = p.has_block_mask != 0;
+        const bool fast = masked_path && dnf.n_terms <= kBwdRowTerms;
+        // Per-row mask data, fixed for the unit. dk/dv: q intervals per term
+        // for this key, and the key's document id. dq: kv intervals per term
+        // for this query (the document leaf as the query's document span).
+        int iv_lo[kBwdRowTerms], iv_hi[kBwdRowTerms];
+#pragma unroll
+        for (int t = 0; t < kBwdRowTerms; ++t) {
+            iv_lo[t] = 1;
+            iv_hi[t] = 0;
+        }
+        int32_t my_doc = 0;
+        bool my_doc_ok = false;
+        int64_t row_ds = 0, row_de = -1;
+        float lse2_row = INFINITY, delta_row = 0.f, slope_unit = 0.f;
+        constexpr bool kAlibi = SCORE == kScoreAlibi || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap;
+        if constexpr (KVSIDE) {
+            if (dnf.has_doc && masked_path && row_idx < p.N) {
+                my_doc = __ldg(dnf.kv_doc + static_cast<int64_t>(db) * p.N + row_idx);
+                my_doc_ok = true;
+            }
+            if (fast) {
+#pragma unroll
+                for (int t = 0; t < kBwdRowTerms; ++t) {
+                    if (t < dnf.n_terms && row_idx < p.N) {
+                        int64_t lo, hi;
+                        term_q_interval(dnf, t, row_idx, p.M, lo, hi);
+                        if (hi >= lo) {
+                            iv_lo[t] = static_cast<int>(lo);
+                            iv_hi[t] = static_cast<int>(hi);
+                        }
+                    }
+                }
+            }
+        } else {
+            const float2 ldr = p.ld[static_cast<int64_t>(b * p.Hq + hq) * p.QB * 128 + row_idx];
+            lse2_row = ldr.x;
+            delta_row = ldr.y;
+            if constexpr (kAlibi)
+                slope_unit = p.slopes ? __ldg(p.slopes + hq)
+                                      : exp2f(-8.0f * static_cast<float>(hq + 1) / static_cast<float>(p.Hq));
+            if (dnf.has_doc && masked_path) {
+                // the span [first, last] of kv positions with this row's document
+                // id (kv ids are non-decreasing); one warp search per distinct id
+                const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
+                const int32_t* kd_row = dnf.kv_doc + static_cast<int64_t>(db) * p.N;
+                const bool valid = row_idx < p.M;
+                const int32_t d = valid ? __ldg(qd_row + row_idx) : 0;
+                bool pending = valid;
+                unsigned todo;
+                while ((todo = __ballot_sync(0xFFFFFFFFu, pending)) != 0u) {
+                    const int32_t x = __shfl_sync(0xFFFFFFFFu, d, __ffs(todo) - 1);
+                    const int first = warp_lower_bound(kd_row, p.N, x, lane);
+                    const int past = warp_lower_bound(kd_row, p.N, static_cast<int64_t>(x) + 1, lane);
+                    if (pending && d == x) {
+                        row_ds = first;
+                        row_de = past - 1;
+                        pending = false;
+                    }
+                }
+            }
+            if (fast) {
+#pragma unroll
+                for (int t = 0; t < kBwdRowTerms; ++t) {
+                    if (t < dnf.n_terms) {
+                        int64_t lo, hi;
+                        term_interval(dnf, t, row_idx, 0, p.N - 1, row_ds, row_de, lo, hi);
+                        if (hi >= lo) {
+                            iv_lo[t] = static_cast<int>(lo);
+                            iv_hi[t] = static_cast<int>(hi);
+                        }
+                    }
+                }
+            }
+        }
+        const float2* ld_smem = reinterpret_cast<const float2*>(smem + L::kLd);
+
+        bool ok = true;
+        for (int e = 0; e < T && ok; ++e) {
+            const uint32_t ent = entries[e];
+            const int eb = static_cast<int>(ent & 0xFFFFu);
+            const int g = static_cast<int>((ent >> 16) & 0xFFu);
+            const bool partial = (ent & kBwdPartial) != 0u;
+            const int64_t c0 = static_cast<int64_t>(eb) * 128 + 64 * h;  // first column (q or kv) of this half
+            // mask words over the half's 64 columns (bit j: column c0 + j allowed)
+            uint32_t w0 = 0xFFFFFFFFu, w1 = 0xFFFFFFFFu;
+            if (partial) {
+                w0 = 0u;
+                w1 = 0u;
+                if constexpr (KVSIDE) {
+                    uint32_t d0 = 0xFFFFFFFFu, d1 = 0xFFFFFFFFu;
+                    if (dnf.term_has_doc) {
+                        d0 = 0u;
+                        d1 = 0u;
+                        if (my_doc_ok) {
+                            const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
+#pragma unroll 8
+                            for (int j = 0; j < 64; ++j) {
+                                const int64_t q = c0 + j;
+                                const bool m = q < p.M && __ldg(qd_row + q) == my_doc;
+                                if (j < 32) d0 |= (m ? 1u : 0u) << j;
+                                else d1 |= (m ? 1u : 0u) << (j - 32);
+                            }
+                        }
+                    }
+                    const int ic0 = static_cast<int>(c0);
+                    if (fast) {
+#pragma unroll
+                        for (int t = 0; t < kBwdRowTerms; ++t) {
+                            uint32_t a0 = range_bits32(iv_lo[t] - ic0, iv_hi[t] - ic0);
+                            uint32_t a1 = range_bits32(iv_lo[t] - ic0 - 32, iv_hi[t] - ic0 - 32);
+                            if ((dnf.term_has_doc >> t) & 1u) {
+                                a0 &= d0;
+                                a1 &= d1;
+                            }
+                            w0 |= a0;
+                            w1 |= a1;
+                        }
+                    } else if (row_idx < p.N) {
+                        for (int t = 0; t < dnf.n_terms; ++t) {
+                            int64_t lo, hi;
+                            term_q_interval(dnf, t, row_idx, p.M, lo, hi);
+                            uint32_t a0 = range_bits(lo, hi, c0);
+                            uint32_t a1 = range_bits(lo, hi, c0 + 32);
+                            if ((dnf.term_has_doc >> t) & 1u) {
+                                a0 &= d0;
+                                a1 &= d1;
+                            }
+                            w0 |= a0;
+                            w1 |= a1;
+                        }
+                    }
+                } else {
+                    const int64_t c1 = (c0 + 63 < p.N - 1) ? c0 + 63 : p.N - 1;
+                    if (fast) {
+                        const int ic0 = static_cast<int>(c0), ic1 = static_cast<int>(c1);
+#pragma unroll
+                        for (int t = 0; t < kBwdRowTerms; ++t) {
+                            const int lo = (iv_lo[t] > ic0 ? iv_lo[t] : ic0) - ic0;
+                            const int hi = (iv_hi[t] < ic1 ? iv_hi[t] : ic1) - ic0;
+                            w0 |= range_bits32(lo, hi);
+                            w1 |= range_bits32(lo - 32, hi - 32);
+                        }
+                    } else if (masked_path) {
+                        for (int t = 0; t < dnf.n_terms; ++t) {
+                            int64_t lo, hi;
+                            term_interval(dnf, t, row_idx, c0, c1, row_ds, row_de, lo, hi);
+                            w0 |= range_bits(lo, hi, c0);
+                            w1 |= range_bits(lo, hi, c0 + 32);
+                        }
+                    } else {
+                        w0 = range_bits(c0, c1, c0);
+                        w1 = range_bits(c0, c1, c0 + 32);
+                    }
+                }
+            }
+            float slope = slope_unit;
+            if constexpr (KVSIDE && kAlibi)
+                slope = p.slopes ? __ldg(p.slopes + hq + g)
+                                 : exp2f(-8.0f * static_cast<float>(hq + g + 1) / static_cast<float>(p.Hq));
+            const float sl2 = slope * kLog2e;
+            // kv - q at column 0 of the half; it moves by -1 (dk/dv) or +1 (dq) per column
+            const float dkv0 = KVSIDE ? static_cast<float>(row_idx - c0) : static_cast<float>(c0 - row_idx);
+            constexpr float kStep = KVSIDE ? -1.f : 1.f;
+
+            if (!mbar_wait(bar(L::kBarSFull + h), static_cast<uint32_t>(e & 1), abort_flag)) {
+                ok = false;
+                break;
+            }
+            __syncwarp();  // tcgen05.ld/st are warp-collective: reconverge after the wait
+            tc_fence_after();
+            float x[64], dp[64];
+            tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(x));
+            tmem_ld32(t_s + 32u, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+            tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dp));
+            tmem_ld32(t_dp + 32u, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
+            tc_wait_ld();
+            const float2* ldc = ld_smem + 128 * (e & 1) + 64 * h;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const uint32_t w = c == 0 ? w0 : w1;
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    float pv[2], dv[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int j = 32 * c + 2 * jj + u;
+                        float l2 = lse2_row, dl = delta_row;
+                        if constexpr (KVSIDE) {
+                            const float2 t = ldc[j];
+                            l2 = t.x;
+                            dl = t.y;
+                        }
+                        float z2, dz;
+                        bwd_score<SCORE>(p, x[j], fmaf(kStep, static_cast<float>(j), dkv0), slope, sl2, z2, dz);
+                        const bool allowed = (w >> (2 * jj + u)) & 1u;
+                        const float pj = allowed ? ex2_approx(z2 - l2) : 0.f;
+                        pv[u] = pj;
+                        dv[u] = pj * (dp[j] - dl) * dz;
+                    }
+                    pk[jj] = pack_bf16x2(pv[0], pv[1]);
+                    dk[jj] = pack_bf16x2(dv[0], dv[1]);
+                }
+                if constexpr (KVSIDE) tmem_st16(t_s + 16u * c, pk);
+                tmem_st16(t_dp + 16u * c, dk);
+            }
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::kBarPFull + h));
+        }
+        // ------------------------------------------------------ epilogue
+        // dk/dv: warpgroup 0 writes dV, warpgroup 1 writes dK (times scale).
+        // dq: warpgroup h writes columns [h D/2, (h+1) D/2) of dQ (times scale).
+        if (ok && T > 0) ok = mbar_wait(bar(L::kBarAcc), 0, abort_flag);
+        __syncwarp();
+        tc_fence_after();
+        if (ok) {
+            constexpr int kCols = KVSIDE ? D : D / 2;
+            const int64_t rows = KVSIDE ? p.N : p.M;
+            const bool valid = row_idx < rows;
+            __nv_bfloat16* dst;
+            uint32_t src;
+            float mul;
+            if constexpr (KVSIDE) {
+                dst = (h == 0 ? p.g1 : p.g0) + (static_cast<int64_t>(b * p.Hkv + hkv) * p.N + row_idx) * D;
+                src = tmem + 256u + (h == 0 ? 0u : static_cast<uint32_t>(D)) + lane_base;
+                mul = h == 0 ? 1.f : p.scale;
+            } else {
+                dst = p.g0 + (static_cast<int64_t>(b * p.Hq + hq) * p.M + row_idx) * D + h * (D / 2);
+                src = tmem + 256u + static_cast<uint32_t>(h * (D / 2)) + lane_base;
+                mul = p.scale;
+            }
+#pragma unroll
+            for (int c = 0; c < kCols / 32; ++c) {
+                uint32_t a[32];
+                if (T > 0) {
+                    tmem_ld32(src + 32u * c, a);
+                    tc_wait_ld();
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) a[j] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    pk[j] = pack_bf16x2(__uint_as_float(a[2 * j]) * mul, __uint_as_float(a[2 * j + 1]) * mul);
+                if (valid) {
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) d4[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                }
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kBwdWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace bsmt

@@ -15,6 +15,7 @@
 #include <string>
 #include <vector>
 
+#include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "bsmt.h"
 #include "mask_build.cuh"
@@ -256,6 +257,43 @@ __global__ void fill_empty_kernel(uint4* out, int64_t out_vec, float* lse, int64
         lse[i] = -INFINITY;
 }
 
+// Score mods -> compile-time mode (kScore*), the soft-cap and the ALiBi slopes.
+bsmt_status parse_score(const bsmt_score_spec* score, int* mode_out, float* cap_out, const float** slopes_out) {
+    int mode = bsmt::kScoreNone;
+    float cap = 1.f;
+    const float* slopes = nullptr;
+    if (score != nullptr) {
+        if (score->num_ops < 0 || score->num_ops > BSMT_MAX_SCORE_OPS)
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: num_ops=%d outside [0, %d]", score->num_ops, BSMT_MAX_SCORE_OPS);
+        int kinds[2] = {0, 0};
+        int nk = 0;
+        for (int i = 0; i < score->num_ops; ++i) {
+            const bsmt_score_op& op = score->ops[i];
+            if (op.kind == BSMT_SCORE_NONE) continue;
+            if (op.kind == BSMT_SCORE_SOFTCAP) {
+                if (!(op.value > 0.f) || std::isinf(op.value))
+                    return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: soft-cap must be finite and > 0");
+                cap = op.value;
+            } else if (op.kind == BSMT_SCORE_ALIBI) {
+                if (op.slopes && !aligned(op.slopes, 4))
+                    return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: ALiBi slopes must be 4-byte aligned");
+                slopes = op.slopes;
+            } else {
+                return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: unknown kind %d", op.kind);
+            }
+            if (nk == 1 && kinds[0] == op.kind)
+                return fail(BSMT_ERR_UNSUPPORTED, "score spec: the same score mod twice");
+            kinds[nk++] = op.kind;
+        }
+        if (nk == 1) mode = kinds[0] == BSMT_SCORE_SOFTCAP ? bsmt::kScoreSoftcap : bsmt::kScoreAlibi;
+        if (nk == 2) mode = kinds[0] == BSMT_SCORE_SOFTCAP ? bsmt::kScoreSoftcapAlibi : bsmt::kScoreAlibiSoftcap;
+    }
+    *mode_out = mode;
+    *cap_out = cap;
+    *slopes_out = slopes;
+    return BSMT_OK;
+}
+
 template <int D, int SCORE>
 bsmt_status launch_attn(int dev, int nsm, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const CUtensorMap& to, const bsmt::AttnParams& p, const bsmt::MaskDnf& dnf,
@@ -416,31 +454,9 @@ bsmt_status attention(const void* q, const void* k, const void* v, int64_t B, in
     int mode = bsmt::kScoreNone;
     float cap = 1.f;
     const float* slopes = nullptr;
-    if (score != nullptr) {
-        if (score->num_ops < 0 || score->num_ops > BSMT_MAX_SCORE_OPS)
-            return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: num_ops=%d outside [0, %d]", score->num_ops, BSMT_MAX_SCORE_OPS);
-        int kinds[2] = {0, 0};
-        int nk = 0;
-        for (int i = 0; i < score->num_ops; ++i) {
-            const bsmt_score_op& op = score->ops[i];
-            if (op.kind == BSMT_SCORE_NONE) continue;
-            if (op.kind == BSMT_SCORE_SOFTCAP) {
-                if (!(op.value > 0.f) || std::isinf(op.value))
-                    return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: soft-cap must be finite and > 0");
-                cap = op.value;
-            } else if (op.kind == BSMT_SCORE_ALIBI) {
-                if (op.slopes && !aligned(op.slopes, 4))
-                    return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: ALiBi slopes must be 4-byte aligned");
-                slopes = op.slopes;
-            } else {
-                return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: unknown kind %d", op.kind);
-            }
-            if (nk == 1 && kinds[0] == op.kind)
-                return fail(BSMT_ERR_UNSUPPORTED, "score spec: the same score mod twice");
-            kinds[nk++] = op.kind;
-        }
-        if (nk == 1) mode = kinds[0] == BSMT_SCORE_SOFTCAP ? bsmt::kScoreSoftcap : bsmt::kScoreAlibi;
-        if (nk == 2) mode = kinds[0] == BSMT_SCORE_SOFTCAP ? bsmt::kScoreSoftcapAlibi : bsmt::kScoreAlibiSoftcap;
+    {
+        const bsmt_status sst = parse_score(score, &mode, &cap, &slopes);
+        if (sst != BSMT_OK) return sst;
     }
 
     bsmt::MaskDnf dnf;
@@ -759,3 +775,226 @@ extern "C" bsmt_status bsmt_flex_attention_fwd_packed(const void* q, const void*
                      lse, stream, /*packed=*/true);
 }
 
+
+// ------------------------------------------------------------------ backward
+namespace {
+bool g_bwd_attr_set[64][20] = {{false}};
+
+__global__ void zero_kernel(uint4* p, int64_t n) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n; i += stride)
+        p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+bsmt_status zero_bf16(void* p, int64_t elems, int nsm, cudaStream_t s) {
+    if (elems == 0) return BSMT_OK;
+    zero_kernel<<<2 * nsm, 256, 0, s>>>(static_cast<uint4*>(p), elems / 8);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "zero launch: %s", cudaGetErrorString(e));
+    return BSMT_OK;
+}
+
+template <int D, int SCORE, bool KVSIDE>
+bsmt_status launch_bwd(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const bsmt::BwdParams& p, const bsmt::MaskDnf& dnf, cudaStream_t s) {
+    auto kern = bsmt::attn_bwd_kernel<D, SCORE, KVSIDE>;
+    const int smem = bsmt::BwdSmem<D>::kAlloc;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        const int slot = (D == 128 ? 10 : 0) + 2 * SCORE + (KVSIDE ? 1 : 0);
+        if (!g_bwd_attr_set[dev][slot]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+            g_bwd_attr_set[dev][slot] = true;
+        }
+    }
+    kern<<<static_cast<unsigned>(p.num_units), bsmt::kBwdThreads, smem, s>>>(tq, tk, tv, tdo, p, dnf);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
+    return BSMT_OK;
+}
+
+template <int D, bool KVSIDE>
+bsmt_status launch_bwd_score(int mode, int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tdo, const bsmt::BwdParams& p, const bsmt::MaskDnf& dnf,
+                             cudaStream_t s) {
+    switch (mode) {
+        case bsmt::kScoreNone: return launch_bwd<D, bsmt::kScoreNone, KVSIDE>(dev, tq, tk, tv, tdo, p, dnf, s);
+        case bsmt::kScoreSoftcap: return launch_bwd<D, bsmt::kScoreSoftcap, KVSIDE>(dev, tq, tk, tv, tdo, p, dnf, s);
+        case bsmt::kScoreAlibi: return launch_bwd<D, bsmt::kScoreAlibi, KVSIDE>(dev, tq, tk, tv, tdo, p, dnf, s);
+        case bsmt::kScoreSoftcapAlibi:
+            return launch_bwd<D, bsmt::kScoreSoftcapAlibi, KVSIDE>(dev, tq, tk, tv, tdo, p, dnf, s);
+        default: return launch_bwd<D, bsmt::kScoreAlibiSoftcap, KVSIDE>(dev, tq, tk, tv, tdo, p, dnf, s);
+    }
+}
+
+int64_t bwd_ws_bytes(int64_t B, int64_t Hq, int64_t M) { return B * Hq * ((M + 127) / 128) * 128 * 8; }
+}  // namespace
+
+extern "C" bsmt_status bsmt_flex_attention_bwd_workspace_bytes(int64_t B, int64_t Hq, int64_t M, int64_t* bytes) {
+    if (bytes == nullptr) return fail(BSMT_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    if (B < 0 || Hq < 0 || M < 0) return fail(BSMT_ERR_INVALID_ARGUMENT, "negative size");
+    if (M > kMaxLen || B * Hq > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "sizes too large");
+    *bytes = bwd_ws_bytes(B, Hq, M);
+    return ok();
+}
+
+extern "C" bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, const void* v, const void* out,
+                                               const void* dout, const float* lse, int64_t B, int64_t Hq, int64_t Hkv,
+                                               int64_t M, int64_t N, int64_t D, const bsmt_block_mask* bm,
+                                               const bsmt_block_mask_q* bmq, const bsmt_mask_spec* mask_spec,
+                                               const bsmt_score_spec* score, float scale, int32_t enable_gqa,
+                                               void* dq, void* dk, void* dv, void* workspace, int64_t workspace_bytes,
+                                               void* stream) {
+    if (B < 0 || Hq < 0 || Hkv < 0 || M < 0 || N < 0)
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "negative size (B=%lld Hq=%lld Hkv=%lld M=%lld N=%lld)",
+                    static_cast<long long>(B), static_cast<long long>(Hq), static_cast<long long>(Hkv),
+                    static_cast<long long>(M), static_cast<long long>(N));
+    if (D != 64 && D != 128) return fail(BSMT_ERR_UNSUPPORTED, "head dim D=%lld (supported: 64, 128)", static_cast<long long>(D));
+    if (Hkv < 1 || Hq < 1) return fail(BSMT_ERR_SHAPE_MISMATCH, "Hq=%lld and Hkv=%lld must be >= 1", static_cast<long long>(Hq), static_cast<long long>(Hkv));
+    if (Hq % Hkv != 0)
+        return fail(BSMT_ERR_SHAPE_MISMATCH, "Hq=%lld is not a multiple of Hkv=%lld", static_cast<long long>(Hq),
+                    static_cast<long long>(Hkv));
+    if (Hq != Hkv && !enable_gqa)
+        return fail(BSMT_ERR_SHAPE_MISMATCH, "Hq=%lld != Hkv=%lld requires enable_gqa", static_cast<long long>(Hq),
+                    static_cast<long long>(Hkv));
+    if (M > kMaxLen || N > kMaxLen) return fail(BSMT_ERR_UNSUPPORTED, "sequence length above %lld", static_cast<long long>(kMaxLen));
+    if (B * Hq > 0x7FFFFFFF || B * Hkv > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "B*H above 2^31");
+    const int64_t QB = (M + 127) / 128, KB = (N + 127) / 128;
+    const int64_t group = Hq / Hkv;
+    if (KB > bsmt::kBwdMaxEntries)
+        return fail(BSMT_ERR_UNSUPPORTED, "KV_LEN=%lld: at most %d kv blocks per row", static_cast<long long>(N),
+                    bsmt::kBwdMaxEntries);
+    if (group * QB > bsmt::kBwdMaxEntries || group > 255)
+        return fail(BSMT_ERR_UNSUPPORTED, "Q_LEN=%lld with %lld query heads per kv head: at most %d q-blocks x heads",
+                    static_cast<long long>(M), static_cast<long long>(group), bsmt::kBwdMaxEntries);
+    const bool q_has = B * Hq * M > 0, kv_has = B * Hkv * N > 0;
+    if ((q_has && (!q || !out || !dout || !lse || !dq)) || (kv_has && (!k || !v || !dk || !dv)))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "q, k, v, out, dout, lse, dq, dk and dv must be non-NULL when they hold elements");
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(dout, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "q, k, v, out, dout, dq, dk and dv must be 16-byte aligned");
+    if (!aligned(lse, 4)) return fail(BSMT_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
+    if (std::isnan(scale) || std::isinf(scale)) return fail(BSMT_ERR_INVALID_ARGUMENT, "scale must be finite");
+    if (scale <= 0.f) scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    int mode = bsmt::kScoreNone;
+    float cap = 1.f;
+    const float* slopes = nullptr;
+    bsmt_status st = parse_score(score, &mode, &cap, &slopes);
+    if (st != BSMT_OK) return st;
+
+    bsmt::MaskDnf dnf;
+    std::memset(&dnf, 0, sizeof(dnf));
+    bsmt::BwdParams pq, pk;  // dq kernel (kv-side lists), dk/dv kernel (q-side lists)
+    std::memset(&pq, 0, sizeof(pq));
+    std::memset(&pk, 0, sizeof(pk));
+    if (bm != nullptr) {
+        if (bm->BLOCK_Q != 128 || bm->BLOCK_KV != 128)
+            return fail(BSMT_ERR_UNSUPPORTED, "block mask BLOCK_SIZE (%d, %d): only 128 x 128", bm->BLOCK_Q, bm->BLOCK_KV);
+        if (bm->Q_LEN != M || bm->KV_LEN != N || bm->QB != QB || bm->KB != KB)
+            return fail(BSMT_ERR_SHAPE_MISMATCH,
+                        "block mask is for (Q_LEN=%d, KV_LEN=%d, QB=%d, KB=%d) but attention has M=%lld N=%lld", bm->Q_LEN,
+                        bm->KV_LEN, bm->QB, bm->KB, static_cast<long long>(M), static_cast<long long>(N));
+        if (!(bm->B == 1 || bm->B == B) || !(bm->H == 1 || bm->H == Hq))
+            return fail(BSMT_ERR_SHAPE_MISMATCH, "block mask (B=%d, H=%d) must broadcast to (B=%lld, Hq=%lld)", bm->B, bm->H,
+                        static_cast<long long>(B), static_cast<long long>(Hq));
+        if (QB > 0 && KB > 0) {
+            if (!bm->kv_num_blocks || !bm->kv_indices || !bm->full_kv_num_blocks || !bm->full_kv_indices)
+                return fail(BSMT_ERR_INVALID_ARGUMENT, "block mask pointers must be non-NULL");
+            if (bmq == nullptr || !bmq->q_num_blocks || !bmq->q_indices || !bmq->full_q_num_blocks ||
+                !bmq->full_q_indices)
+                return fail(BSMT_ERR_INVALID_ARGUMENT, "the backward needs the q-side lists of the block mask");
+            if (!aligned(bmq->q_num_blocks, 4) || !aligned(bmq->q_indices, 4) || !aligned(bmq->full_q_num_blocks, 4) ||
+                !aligned(bmq->full_q_indices, 4))
+                return fail(BSMT_ERR_INVALID_ARGUMENT, "q-side list pointers must be 4-byte aligned");
+        }
+        st = build_dnf(mask_spec, B, &dnf);
+        if (st != BSMT_OK) return st;
+        for (bsmt::BwdParams* pp : {&pq, &pk}) {
+            pp->has_block_mask = 1;
+            pp->Bm = bm->B;
+            pp->Hm = bm->H;
+        }
+        pq.num = bm->kv_num_blocks;
+        pq.idx = bm->kv_indices;
+        pq.full_num = bm->full_kv_num_blocks;
+        pq.full_idx = bm->full_kv_indices;
+        if (bmq != nullptr) {
+            pk.num = bmq->q_num_blocks;
+            pk.idx = bmq->q_indices;
+            pk.full_num = bmq->full_q_num_blocks;
+            pk.full_idx = bmq->full_q_indices;
+        }
+    } else {
+        dnf.n_terms = 1;
+    }
+    if (B == 0 || (M == 0 && N == 0)) return ok();
+    const int64_t need = bwd_ws_bytes(B, Hq, M);
+    if (need > 0 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "workspace must be non-NULL, 256-byte aligned and hold %lld bytes (has %lld)",
+                    static_cast<long long>(need), static_cast<long long>(workspace_bytes));
+    int dev = 0, nsm = 0;
+    st = sm_count(&dev, &nsm);
+    if (st != BSMT_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M == 0) {  // no queries: nothing reaches k or v
+        if ((st = zero_bf16(dk, B * Hkv * N * D, nsm, s)) != BSMT_OK) return st;
+        return (st = zero_bf16(dv, B * Hkv * N * D, nsm, s)) != BSMT_OK ? st : ok();
+    }
+    if (N == 0) return (st = zero_bf16(dq, B * Hq * M * D, nsm, s)) != BSMT_OK ? st : ok();
+    if (B * Hkv * KB > 0x7FFFFFFF || B * Hq * QB > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "too many work units");
+
+    // (lse2, delta) per padded query row
+    float2* ld = static_cast<float2*>(workspace);
+    const int64_t rows_pad = B * Hq * QB * 128;
+    if (D == 128)
+        bsmt::bwd_prep_kernel<128><<<static_cast<unsigned>(rows_pad / 8), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, rows_pad,
+            static_cast<int32_t>(M), static_cast<int32_t>(QB), ld);
+    else
+        bsmt::bwd_prep_kernel<64><<<static_cast<unsigned>(rows_pad / 8), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, rows_pad,
+            static_cast<int32_t>(M), static_cast<int32_t>(QB), ld);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "backward prep launch: %s", cudaGetErrorString(e));
+
+    EncodeTiledFn enc = nullptr;
+    if ((st = get_encoder(&enc)) != BSMT_OK) return st;
+    CUtensorMap tq, tk, tv, tdo;
+    if ((st = encode_bhsd(enc, &tq, q, B * Hq, M, D, M * D, D)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tdo, dout, B * Hq, M, D, M * D, D)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tk, k, B * Hkv, N, D, N * D, D)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tv, v, B * Hkv, N, D, N * D, D)) != BSMT_OK) return st;
+    for (bsmt::BwdParams* pp : {&pq, &pk}) {
+        pp->B = static_cast<int32_t>(B);
+        pp->Hq = static_cast<int32_t>(Hq);
+        pp->Hkv = static_cast<int32_t>(Hkv);
+        pp->M = static_cast<int32_t>(M);
+        pp->N = static_cast<int32_t>(N);
+        pp->QB = static_cast<int32_t>(QB);
+        pp->KB = static_cast<int32_t>(KB);
+        pp->group = static_cast<int32_t>(group);
+        pp->scale = scale;
+        pp->scale_log2 = scale * bsmt::kLog2e;
+        pp->cap = cap;
+        pp->inv_cap = 1.f / cap;
+        pp->slopes = slopes;
+        pp->ld = ld;
+    }
+    pk.list_rows = static_cast<int32_t>(KB);
+    pk.list_len = static_cast<int32_t>(QB);
+    pk.g0 = static_cast<__nv_bfloat16*>(dk);
+    pk.g1 = static_cast<__nv_bfloat16*>(dv);
+    pk.num_units = static_cast<int32_t>(B * Hkv * KB);
+    pq.list_rows = static_cast<int32_t>(QB);
+    pq.list_len = static_cast<int32_t>(KB);
+    pq.g0 = static_cast<__nv_bfloat16*>(dq);
+    pq.num_units = static_cast<int32_t>(B * Hq * QB);
+    st = D == 128 ? launch_bwd_score<128, true>(mode, dev, tq, tk, tv, tdo, pk, dnf, s)
+                  : launch_bwd_score<64, true>(mode, dev, tq, tk, tv, tdo, pk, dnf, s);
+    if (st != BSMT_OK) return st;
+    st = D == 128 ? launch_bwd_score<128, false>(mode, dev, tq, tk, tv, tdo, pq, dnf, s)
+                  : launch_bwd_score<64, false>(mode, dev, tq, tk, tv, tdo, pq, dnf, s);
+    if (st != BSMT_OK) return st;
+    return ok();
+}

@@ -152,6 +152,15 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int
         : "memory");
 }
 
+// Contiguous copy global -> shared (no tensor map), completing on an
+// mbarrier's transaction count. Both addresses 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 // Brings a tile of a 3-D tensor map into L2 (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int x, int y, int z) {
     asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
@@ -369,6 +378,26 @@ __device__ __forceinline__ void mma_ts_run8(uint32_t d_tmem, uint32_t a_tmem, ui
         "add.u32 a, %1, 48;\n\tadd.s64 b, %2, 768;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
         "add.u32 a, %1, 56;\n\tadd.s64 b, %2, 896;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// A TS product over K = 64 in one asm block: the first four steps of
+// mma_ts_run8 (A from TMEM columns a_tmem + 8k, B MN-major 2 KB further per
+// step).
+__device__ __forceinline__ void mma_ts_run4(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, 1, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "add.u32 a, %1, 8;\n\tadd.s64 b, %2, 128;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
+        "add.u32 a, %1, 16;\n\tadd.s64 b, %2, 256;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
+        "add.u32 a, %1, 24;\n\tadd.s64 b, %2, 384;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t}"
         ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");

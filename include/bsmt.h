@@ -1,6 +1,6 @@
 /*
- * bsmt.h: C ABI of libbsmt, block-sparse masked-tile attention forward for
- * NVIDIA B200 (sm_100a).
+ * bsmt.h: C ABI of libbsmt, block-sparse masked-tile attention (forward and
+ * backward) for NVIDIA B200 (sm_100a).
  *
  * The library builds a block-sparse BlockMask from a composable mask
  * description. It then runs scaled-dot-product attention. The attention
@@ -332,6 +332,51 @@ bsmt_status bsmt_flex_attention_fwd_packed(const void* q, const void* k, const v
                                            int64_t M, int64_t N, int64_t D, const bsmt_block_mask* block_mask,
                                            const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score, float scale,
                                            int32_t enable_gqa, void* out, float* lse, void* stream);
+
+/* ------------------------------------------------------------- backward
+ * Gradients of the forward above: with dout the gradient arriving at out,
+ * dq, dk and dv are the gradients of sum(out * dout) with respect to q, k
+ * and v. With s = scale * q.k, z = score_mod(s), P = exp(z - lse) and
+ * delta_i = sum_d out[i,d] * dout[i,d]:
+ *   dS = P * (dout v^T - delta) * dz/ds
+ *   dv = P^T dout,  dk = scale * dS^T q,  dq = scale * dS k
+ * summed, for dk and dv, over the query heads of each kv head's GQA group.
+ * Masked elements have P = 0; a row with no allowed key (lse = -inf) passes
+ * no gradient. The structure follows the tensorplay.nn.attention page,
+ * BlockMask "Details" items 3-4: dk and dv walk the q-side lists of the
+ * block mask, dq walks its kv-side lists; mask_mod runs on PARTIAL tiles
+ * only (the FlagAttention page, "Operator overview", lists forward and
+ * backward for the same layouts).
+ *
+ * bsmt_flex_attention_bwd_workspace_bytes gives the workspace size:
+ * 8 * B * Hq * ceil(M / 128) * 128 bytes (lse and delta per query row).
+ * Host-only; launches nothing. */
+bsmt_status bsmt_flex_attention_bwd_workspace_bytes(int64_t B, int64_t Hq, int64_t M, int64_t* bytes);
+
+/* Arguments:
+ *   q, k, v, B, Hq, Hkv, M, N, D, mask_spec, score, scale, enable_gqa
+ *           as for bsmt_flex_attention_fwd (the same values as the forward)
+ *   out     device bf16 [B, Hq, M, D], the forward's output, 16-byte aligned
+ *   dout    device bf16 [B, Hq, M, D], 16-byte aligned
+ *   lse     device float [B, Hq, M], the forward's lse, 4-byte aligned
+ *   block_mask    the forward's BlockMask, or NULL for every tile
+ *   block_mask_q  its q-side lists (bsmt_block_mask_transpose); required
+ *           when block_mask is not NULL, ignored otherwise
+ *   dq      device bf16 [B, Hq, M, D]; dk, dv device bf16 [B, Hkv, N, D];
+ *           16-byte aligned, fully written (zeros where no key or query
+ *           reaches)
+ *   workspace  caller-owned device memory, 256-byte aligned, at least
+ *           bsmt_flex_attention_bwd_workspace_bytes bytes; written and read
+ *           back by the call, reusable once the stream has passed it
+ * Limits: ceil(N/128) <= 4096 and (Hq/Hkv) * ceil(M/128) <= 4096, else
+ * BSMT_ERR_UNSUPPORTED. Bad list entries are skipped and reported as
+ * BSMT_ERR_DEVICE_BOUNDS. Stream-ordered on `stream`. */
+bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                                    const float* lse, int64_t B, int64_t Hq, int64_t Hkv, int64_t M, int64_t N,
+                                    int64_t D, const bsmt_block_mask* block_mask,
+                                    const bsmt_block_mask_q* block_mask_q, const bsmt_mask_spec* mask_spec,
+                                    const bsmt_score_spec* score, float scale, int32_t enable_gqa, void* dq,
+                                    void* dk, void* dv, void* workspace, int64_t workspace_bytes, void* stream);
 
 /* Thread-local message for the last failed call on this thread ("" if none). */
 const char* bsmt_last_error(void);

@@ -218,3 +218,10 @@ def random_mask_tree(rng: np.random.Generator, B: int, M: int, N: int, depth: in
         return (op,) + tuple(node(d - 1) for _ in range(n))
 
     return node(depth)
+
+
+def grad_output(seed: int, B: int, Hq: int, M: int, D: int) -> torch.Tensor:
+    """The gradient arriving at out for backward cases: float32 N(0, 1) rounded
+    to bfloat16, [B, Hq, M, D], from its own seeded generator."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    return torch.randn((B, Hq, M, D), generator=g, dtype=torch.float32).to(torch.bfloat16)
