@@ -10,7 +10,7 @@ metric: TFLOP/s counting only the FLOPs of tiles that are not skipped,
 4 * 128 * 128 * D per kept (FULL or PARTIAL) 128x128 tile per (b, hq).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                       [--workload INDEX] [--no-cpu-baseline]
+                       [--workload INDEX] [--no-cpu-baseline] [--backward-only] [--batch B]
 For N > 1 run it under torch.distributed.run. Each rank then processes its
 own batch of the same shape (weak scaling; the units are independent).
 """
@@ -54,6 +54,9 @@ def parse(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-side-kernels", action="store_true",
                     help="skip the side measurements (builder, transpose, split-KV, varlen) after the step")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="run only the backward (prep, dk/dv and dq kernels) --steps times after one forward, "
+                         "and print its timing (for profiling the backward kernels)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller cases for profiling only)")
     return ap.parse_args(argv)
@@ -181,6 +184,35 @@ def _time_launches(fn, reps: int = 20) -> float:
     ms = e0.elapsed_time(e1) / (3 * reps)
     del g
     return ms
+
+
+BWD_PRODUCTS = 5  # dQ, dK, dV and the recomputed S and dP: 2*128*128*D FLOPs each per kept tile
+
+
+def time_backward(bsmt, w, q, k, v, out, lse, bm, mods, dev, flops_fwd: int, reps: int = 5) -> dict:
+    """The backward (prep + dk/dv + dq kernels) on the step's inputs, timed as
+    CUDA-graph replays. Counted FLOPs: BWD_PRODUCTS products of 2*128*128*D per
+    kept tile, i.e. 2.5x the forward count; the two kernels execute 7 products
+    (S and dP are computed by both)."""
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 50)
+    dout = torch.randn(out.shape, generator=g).to(torch.bfloat16).to(dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(bsmt.backward_workspace_bytes(w.B, w.Hq, w.M), dtype=torch.uint8, device=dev)
+    bm.q_side()
+    # ALiBi slopes on the device before capture (no host copies inside the graph)
+    mods = [bsmt.ScoreMod(m.kind, m.value, None if m.slopes is None else m.slopes.to(dev)) for m in mods]
+
+    def call():
+        bsmt.flex_attention_backward(q, k, v, out, lse, dout, block_mask=bm, score_mod=mods, scale=w.scale,
+                                     enable_gqa=w.enable_gqa, workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    ms = _time_launches(call, reps=reps)
+    bsmt.check_device_status(dev)
+    flops = flops_fwd * BWD_PRODUCTS // 2
+    return {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12, "counted_gflop": flops / 1e9,
+            "executed_tensor_tflops": flops * 7 / 5 / (ms * 1e-3) / 1e12,
+            "note": "flex_attention_backward: lse/delta prep, dk/dv kernel (q-side lists), dq kernel (kv-side "
+                    "lists); counted as 5 products per kept tile (2.5x forward)"}
 
 
 def side_kernels(bsmt, mask, w, dev, hbm_peak: float) -> dict:
@@ -362,6 +394,13 @@ def main():
     bsmt.check_device_status(dev)
     flops = counted_flops(bm, w.D)
     sparsity = bm.sparsity()
+    if args.backward_only:
+        r = time_backward(bsmt, w, q, k, v, out, lse, bm, mods, dev, flops, reps=max(1, args.steps))
+        if rank == 0:
+            print(json.dumps({"workload": w.name, "B": w.B, "backward": r}), flush=True)
+        if dist:
+            dist.destroy_process_group()
+        return
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -419,6 +458,8 @@ def main():
     peaks, peak_src = load_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     side = None if args.no_side_kernels else side_kernels(bsmt, mask, w, dev, hbm_peak)
+    if side is not None:
+        side["backward"] = time_backward(bsmt, w, q, k, v, out, lse, bm, mods, dev, flops)
     attn_tflops = (flops / (attn_ms * 1e-3)) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     traffic = profile_traffic(w.name)

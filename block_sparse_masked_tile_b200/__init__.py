@@ -617,13 +617,17 @@ def backward_workspace_bytes(B: int, Hq: int, M: int) -> int:
 def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                             lse: torch.Tensor, dout: torch.Tensor, block_mask: BlockMask | None = None,
                             score_mod: ScoreMod | Iterable[ScoreMod] | None = None, scale: float | None = None,
-                            enable_gqa: bool = False, workspace: torch.Tensor | None = None):
+                            enable_gqa: bool = False, workspace: torch.Tensor | None = None,
+                            dq: torch.Tensor | None = None, dk: torch.Tensor | None = None,
+                            dv: torch.Tensor | None = None):
     """Gradients (dq, dk, dv) of sum(out * dout) for the forward
     ``out, lse = flex_attention(q, k, v, block_mask, score_mod, scale, enable_gqa)``.
     Pass the same arguments as the forward plus its out and lse. dk and dv
     walk the block mask's q-side lists (computed on first use), dq its
     kv-side lists. ``workspace``: a uint8 CUDA tensor of at least
-    backward_workspace_bytes(B, Hq, M) bytes, allocated when not given."""
+    backward_workspace_bytes(B, Hq, M) bytes, allocated when not given.
+    ``dq``, ``dk``, ``dv``: output tensors to write (contiguous bf16 of q's and
+    k's shapes), allocated when not given."""
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
         if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous bf16 4-D CUDA tensor")
@@ -636,9 +640,12 @@ def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
     if lse.shape != (B, Hq, M) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [B, Hq, M] tensor")
     device = q.device
-    dq = torch.empty_like(q)
-    dk = torch.empty_like(k)
-    dv = torch.empty_like(v)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        if t.shape != ref.shape or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device != device:
+            raise ValueError(f"{name} must be a contiguous bf16 tensor of shape {tuple(ref.shape)} on {device}")
     need = backward_workspace_bytes(B, Hq, M)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
