@@ -65,8 +65,9 @@ struct BwdParams {
     int32_t list_rows, list_len;
     float scale, scale_log2, cap, inv_cap;
     const float* slopes;  // ALiBi slopes [Hq] or null (default 2^(-8(h+1)/Hq))
-    // (lse * log2(e), delta) per query row, padded to whole q-blocks:
-    // [B*Hq][QB*128]. lse2 is +inf for padding rows and rows with no key.
+    // (-lse * log2(e), -delta) per query row, padded to whole q-blocks:
+    // [B*Hq][QB*128]. The first is -inf for padding rows and rows with no
+    // key, so that P = 2^(z2 - lse2) = 0 there.
     const float2* ld;
     __nv_bfloat16* g0;  // dq (dq kernel) or dk [B, Hkv, N, D]
     __nv_bfloat16* g1;  // dv [B, Hkv, N, D]
@@ -78,7 +79,6 @@ constexpr int kBwdWarpLoad = 8;
 constexpr int kBwdWarpMma = 9;
 constexpr int kBwdMaxEntries = 4096;  // entries of one unit (list length x GQA group)
 constexpr uint32_t kBwdPartial = 0x80000000u;
-constexpr int kBwdRowTerms = 4;  // mask alternatives kept per row in registers
 
 template <int D>
 struct BwdSmem {
@@ -102,28 +102,84 @@ struct BwdSmem {
     static_assert(kAlloc <= 227 * 1024, "shared memory layout exceeds one CTA's limit");
 };
 
-// Score (log2 units) and dz/ds for one element: x = q.k, dkv = kv_idx - q_idx.
-template <int SCORE>
-__device__ __forceinline__ void bwd_score(const BwdParams& p, float x, float dkv, float slope, float sl2, float& z2,
-                                          float& dz) {
-    if constexpr (SCORE == kScoreNone) {
-        z2 = x * p.scale_log2;
-        dz = 1.f;
-    } else if constexpr (SCORE == kScoreSoftcap) {
-        const float t = tanh_approx(x * (p.scale * p.inv_cap));
-        z2 = (p.cap * kLog2e) * t;
-        dz = fmaf(-t, t, 1.f);
-    } else if constexpr (SCORE == kScoreAlibi) {
-        z2 = fmaf(x, p.scale_log2, sl2 * dkv);
-        dz = 1.f;
-    } else if constexpr (SCORE == kScoreSoftcapAlibi) {
-        const float t = tanh_approx(x * (p.scale * p.inv_cap));
-        z2 = fmaf(p.cap * kLog2e, t, sl2 * dkv);
-        dz = fmaf(-t, t, 1.f);
-    } else {  // ALiBi, then soft-cap
-        const float t = tanh_approx(fmaf(x, p.scale, slope * dkv) * p.inv_cap);
-        z2 = (p.cap * kLog2e) * t;
-        dz = fmaf(-t, t, 1.f);
+__device__ __forceinline__ float2 mul2f(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2f(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2f(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// Per-half constants of the score mods. Column j of the half has
+// kv_idx - q_idx = dkv0 + step * j (step = -1 on the dk/dv side, where
+// columns are queries; +1 on the dq side).
+struct BwdHalf {
+    float bias0, bstep;  // ALiBi bias of column 0 and its change per column (log2 units;
+                         // natural units when ALiBi comes before the soft-cap)
+};
+
+// P and dS of one 32-column chunk of a half, two columns at a time on the
+// packed f32x2 pipe. x: raw q.k; dp: dO.v; nl/nd: -lse2 and -delta of each
+// column (dk/dv side, from shared memory as float4 pairs) or of the row
+// (dq side). For the score mods, with s = scale * x:
+//   none         z2 = log2e * s
+//   soft-cap     t = tanh(s / cap), z2 = cap * log2e * t, dz/ds = 1 - t^2
+//   ALiBi        z2 = log2e * (s + slope * (kv - q))
+//   both orders  the compositions of the two
+// P = 2^(z2 - lse2), masked to 0 outside w (MASKED only), and
+// dS = P * (dP - delta) * dz/ds. Both are packed to bf16 pairs.
+template <int SCORE, bool KVSIDE, bool MASKED>
+__device__ __forceinline__ void bwd_chunk(const BwdParams& p, const float* x, const float* dp, const float4* ld4,
+                                          float2 nl_row, float2 nd_row, const BwdHalf& hb, int c0, uint32_t w,
+                                          uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+    const float2 s2 = make_float2(p.scale_log2, p.scale_log2);
+    const float2 c1 = make_float2(p.scale * p.inv_cap, p.scale * p.inv_cap);
+    const float2 c2 = make_float2(p.cap * kLog2e, p.cap * kLog2e);
+    const float2 one = make_float2(1.f, 1.f);
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+        const int j = c0 + 2 * jj;
+        float2 nl = nl_row, nd = nd_row;
+        if constexpr (KVSIDE) {
+            const float4 t = ld4[j >> 1];
+            nl = make_float2(t.x, t.z);
+            nd = make_float2(t.y, t.w);
+        }
+        const float2 X = make_float2(x[j], x[j + 1]);
+        float2 A, G = one;
+        if constexpr (SCORE == kScoreNone) {
+            A = fma2f(X, s2, nl);
+        } else if constexpr (SCORE == kScoreSoftcap) {
+            const float2 u = mul2f(X, c1);
+            const float2 t = make_float2(tanh_approx(u.x), tanh_approx(u.y));
+            A = fma2f(c2, t, nl);
+            G = fma2f(make_float2(-t.x, -t.y), t, one);
+        } else if constexpr (SCORE == kScoreAlibi) {
+            const float2 bias = fma2f(make_float2(static_cast<float>(j), static_cast<float>(j + 1)),
+                                      make_float2(hb.bstep, hb.bstep), make_float2(hb.bias0, hb.bias0));
+            A = fma2f(X, s2, add2f(bias, nl));
+        } else if constexpr (SCORE == kScoreSoftcapAlibi) {
+            const float2 bias = fma2f(make_float2(static_cast<float>(j), static_cast<float>(j + 1)),
+                                      make_float2(hb.bstep, hb.bstep), make_float2(hb.bias0, hb.bias0));
+            const float2 u = mul2f(X, c1);
+            const float2 t = make_float2(tanh_approx(u.x), tanh_approx(u.y));
+            A = fma2f(c2, t, add2f(bias, nl));
+            G = fma2f(make_float2(-t.x, -t.y), t, one);
+        } else {  // ALiBi, then soft-cap: bias in natural units, inside the tanh
+            const float2 bias = fma2f(make_float2(static_cast<float>(j), static_cast<float>(j + 1)),
+                                      make_float2(hb.bstep, hb.bstep), make_float2(hb.bias0, hb.bias0));
+            const float2 u = mul2f(fma2f(X, make_float2(p.scale, p.scale), bias),
+                                   make_float2(p.inv_cap, p.inv_cap));
+            const float2 t = make_float2(tanh_approx(u.x), tanh_approx(u.y));
+            A = fma2f(c2, t, nl);
+            G = fma2f(make_float2(-t.x, -t.y), t, one);
+        }
+        if constexpr (MASKED) {
+            if (!((w >> (2 * jj)) & 1u)) A.x = -INFINITY;
+            if (!((w >> (2 * jj + 1)) & 1u)) A.y = -INFINITY;
+        }
+        const float2 P = make_float2(ex2_approx(A.x), ex2_approx(A.y));
+        float2 T = mul2f(add2f(make_float2(dp[j], dp[j + 1]), nd), P);
+        if constexpr (SCORE == kScoreSoftcap || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap)
+            T = mul2f(T, G);
+        pk[jj] = pack_bf16x2(P.x, P.y);
+        dk[jj] = pack_bf16x2(T.x, T.y);
     }
 }
 
@@ -163,9 +219,9 @@ __device__ __forceinline__ void term_q_interval(const MaskDnf& m, int t, int64_t
         if (m.leaves[i].kind != BSMT_MASK_DOCUMENT) leaf_clamp_q(m.leaves[i].kind, m.leaves[i].arg, kv, lo, hi);
 }
 
-// (lse2, delta) per padded query row: lse2 = lse * log2(e) (+inf where lse is
-// -inf and for rows past M, so that P = 0 there), delta = sum_d out * dout in
-// fp32. One warp per row; lane l reads D/32 consecutive elements.
+// (-lse2, -delta) per padded query row: lse2 = lse * log2(e) (+inf where lse
+// is -inf and for rows past M, so that P = 0 there), delta = sum_d out * dout
+// in fp32. One warp per row; lane l reads D/32 consecutive elements.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* out, const __nv_bfloat16* dout,
                                                        const float* lse, int64_t rows_pad, int32_t M, int32_t QB,
@@ -199,7 +255,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* out,
         const float L = __ldg(lse + bh * M + i);
         l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
     }
-    if (lane == 0) ld[row] = make_float2(l2, acc);
+    if (lane == 0) ld[row] = make_float2(-l2, -acc);
 }
 
 template <int D, int SCORE, bool KVSIDE>
@@ -446,43 +502,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int64_t row_idx = static_cast<int64_t>(blk) * 128 + r;  // this thread's kv (dk/dv) or q (dq)
         const int db = dnf.doc_batch > 1 ? b : 0;
         const bool masked_path = p.has_block_mask != 0;
-        const bool fast = masked_path && dnf.n_terms <= kBwdRowTerms;
-        // Per-row mask data, fixed for the unit. dk/dv: q intervals per term
-        // for this key, and the key's document id. dq: kv intervals per term
-        // for this query (the document leaf as the query's document span).
-        int iv_lo[kBwdRowTerms], iv_hi[kBwdRowTerms];
-#pragma unroll
-        for (int t = 0; t < kBwdRowTerms; ++t) {
-            iv_lo[t] = 1;
-            iv_hi[t] = 0;
-        }
+        // Per-row mask data, fixed for the unit: the key's document id (dk/dv) or
+        // the query's document span (dq). The term intervals are recomputed on
+        // each partial half from the mask program (registers go to the tiles).
         int32_t my_doc = 0;
         bool my_doc_ok = false;
         int64_t row_ds = 0, row_de = -1;
-        float lse2_row = INFINITY, delta_row = 0.f, slope_unit = 0.f;
+        float2 nl_row = make_float2(-INFINITY, -INFINITY), nd_row = make_float2(0.f, 0.f);
+        float slope_unit = 0.f;
         constexpr bool kAlibi = SCORE == kScoreAlibi || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap;
         if constexpr (KVSIDE) {
             if (dnf.has_doc && masked_path && row_idx < p.N) {
                 my_doc = __ldg(dnf.kv_doc + static_cast<int64_t>(db) * p.N + row_idx);
                 my_doc_ok = true;
             }
-            if (fast) {
-#pragma unroll
-                for (int t = 0; t < kBwdRowTerms; ++t) {
-                    if (t < dnf.n_terms && row_idx < p.N) {
-                        int64_t lo, hi;
-                        term_q_interval(dnf, t, row_idx, p.M, lo, hi);
-                        if (hi >= lo) {
-                            iv_lo[t] = static_cast<int>(lo);
-                            iv_hi[t] = static_cast<int>(hi);
-                        }
-                    }
-                }
-            }
         } else {
             const float2 ldr = p.ld[static_cast<int64_t>(b * p.Hq + hq) * p.QB * 128 + row_idx];
-            lse2_row = ldr.x;
-            delta_row = ldr.y;
+            nl_row = make_float2(ldr.x, ldr.x);
+            nd_row = make_float2(ldr.y, ldr.y);
             if constexpr (kAlibi)
                 slope_unit = p.slopes ? __ldg(p.slopes + hq)
                                       : exp2f(-8.0f * static_cast<float>(hq + 1) / static_cast<float>(p.Hq));
@@ -503,19 +540,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         row_ds = first;
                         row_de = past - 1;
                         pending = false;
-                    }
-                }
-            }
-            if (fast) {
-#pragma unroll
-                for (int t = 0; t < kBwdRowTerms; ++t) {
-                    if (t < dnf.n_terms) {
-                        int64_t lo, hi;
-                        term_interval(dnf, t, row_idx, 0, p.N - 1, row_ds, row_de, lo, hi);
-                        if (hi >= lo) {
-                            iv_lo[t] = static_cast<int>(lo);
-                            iv_hi[t] = static_cast<int>(hi);
-                        }
                     }
                 }
             }
@@ -550,20 +574,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             }
                         }
                     }
-                    const int ic0 = static_cast<int>(c0);
-                    if (fast) {
-#pragma unroll
-                        for (int t = 0; t < kBwdRowTerms; ++t) {
-                            uint32_t a0 = range_bits32(iv_lo[t] - ic0, iv_hi[t] - ic0);
-                            uint32_t a1 = range_bits32(iv_lo[t] - ic0 - 32, iv_hi[t] - ic0 - 32);
-                            if ((dnf.term_has_doc >> t) & 1u) {
-                                a0 &= d0;
-                                a1 &= d1;
-                            }
-                            w0 |= a0;
-                            w1 |= a1;
-                        }
-                    } else if (row_idx < p.N) {
+                    if (row_idx < p.N) {
                         for (int t = 0; t < dnf.n_terms; ++t) {
                             int64_t lo, hi;
                             term_q_interval(dnf, t, row_idx, p.M, lo, hi);
@@ -579,16 +590,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     }
                 } else {
                     const int64_t c1 = (c0 + 63 < p.N - 1) ? c0 + 63 : p.N - 1;
-                    if (fast) {
-                        const int ic0 = static_cast<int>(c0), ic1 = static_cast<int>(c1);
-#pragma unroll
-                        for (int t = 0; t < kBwdRowTerms; ++t) {
-                            const int lo = (iv_lo[t] > ic0 ? iv_lo[t] : ic0) - ic0;
-                            const int hi = (iv_hi[t] < ic1 ? iv_hi[t] : ic1) - ic0;
-                            w0 |= range_bits32(lo, hi);
-                            w1 |= range_bits32(lo - 32, hi - 32);
-                        }
-                    } else if (masked_path) {
+                    if (masked_path) {
                         for (int t = 0; t < dnf.n_terms; ++t) {
                             int64_t lo, hi;
                             term_interval(dnf, t, row_idx, c0, c1, row_ds, row_de, lo, hi);
@@ -605,10 +607,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if constexpr (KVSIDE && kAlibi)
                 slope = p.slopes ? __ldg(p.slopes + hq + g)
                                  : exp2f(-8.0f * static_cast<float>(hq + g + 1) / static_cast<float>(p.Hq));
-            const float sl2 = slope * kLog2e;
             // kv - q at column 0 of the half; it moves by -1 (dk/dv) or +1 (dq) per column
             const float dkv0 = KVSIDE ? static_cast<float>(row_idx - c0) : static_cast<float>(c0 - row_idx);
             constexpr float kStep = KVSIDE ? -1.f : 1.f;
+            BwdHalf hb;
+            if constexpr (SCORE == kScoreAlibiSoftcap) {
+                hb.bias0 = slope * dkv0;
+                hb.bstep = slope * kStep;
+            } else {
+                hb.bias0 = slope * kLog2e * dkv0;
+                hb.bstep = slope * kLog2e * kStep;
+            }
 
             if (!mbar_wait(bar(L::kBarSFull + h), static_cast<uint32_t>(e & 1), abort_flag)) {
                 ok = false;
@@ -622,33 +631,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dp));
             tmem_ld32(t_dp + 32u, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
             tc_wait_ld();
-            const float2* ldc = ld_smem + 128 * (e & 1) + 64 * h;
+            const float4* ld4 = reinterpret_cast<const float4*>(ld_smem + 128 * (e & 1) + 64 * h);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                const uint32_t w = c == 0 ? w0 : w1;
                 uint32_t pk[16], dk[16];
-#pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                    float pv[2], dv[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int j = 32 * c + 2 * jj + u;
-                        float l2 = lse2_row, dl = delta_row;
-                        if constexpr (KVSIDE) {
-                            const float2 t = ldc[j];
-                            l2 = t.x;
-                            dl = t.y;
-                        }
-                        float z2, dz;
-                        bwd_score<SCORE>(p, x[j], fmaf(kStep, static_cast<float>(j), dkv0), slope, sl2, z2, dz);
-                        const bool allowed = (w >> (2 * jj + u)) & 1u;
-                        const float pj = allowed ? ex2_approx(z2 - l2) : 0.f;
-                        pv[u] = pj;
-                        dv[u] = pj * (dp[j] - dl) * dz;
-                    }
-                    pk[jj] = pack_bf16x2(pv[0], pv[1]);
-                    dk[jj] = pack_bf16x2(dv[0], dv[1]);
-                }
+                if (partial)
+                    bwd_chunk<SCORE, KVSIDE, true>(p, x, dp, ld4, nl_row, nd_row, hb, 32 * c, c == 0 ? w0 : w1, pk, dk);
+                else
+                    bwd_chunk<SCORE, KVSIDE, false>(p, x, dp, ld4, nl_row, nd_row, hb, 32 * c, 0u, pk, dk);
                 if constexpr (KVSIDE) tmem_st16(t_s + 16u * c, pk);
                 tmem_st16(t_dp + 16u * c, dk);
             }
