@@ -24,25 +24,31 @@
 // dQ has its own kernel, so it needs neither an fp32 accumulator in global
 // memory nor atomics, and the result does not depend on scheduling.
 //
-// Pipeline. Every streamed 128-row tile is processed as two halves of 64
-// rows. Half h of every entry uses TMEM buffer h (64 columns of S, 64 of dP)
-// and softmax warpgroup h. One MMA warp issues, for half c, S(c) and dP(c),
-// then the accumulating products of half c-1 once its warpgroup has stored
-// P and dS back to TMEM. While one warpgroup computes, the tensor core runs
-// the other half's products. MMAs issued by one thread run in order, so
-// S(c) overwrites buffer c & 1 only after the products of half c-2 that read
-// it.
+// Pipeline. Each entry (one streamed 128-row tile pair) has one S and one
+// dP buffer in TMEM, written by 128 x 128 products. The softmax warps work in
+// two phases per entry: the P phase reads S and writes P (bf16, for dV), the
+// dS phase reads dP and writes dS; P * dz/ds stays in registers between them.
+// The MMA warp issues, for the dk/dv kernel,
+//   S(n) dP(n) | dV(n) S(n+1) | dK(n) dP(n+1) | dV(n+1) S(n+2) | ...
+// waiting for the P phase of n before dV(n) and for the dS phase of n before
+// dK(n). So the P phase of n+1 runs while the tensor core does dK(n) and
+// dP(n+1), and the dS phase while it does dV(n+1) and S(n+2). The dq kernel
+// issues S(n) dP(n) | S(n+1) | dQ(n) dP(n+1) | ... the same way. MMAs issued
+// by one thread run in order, so S(n+1) overwrites S (and P) only after dV(n)
+// has read P, and dP(n+1) overwrites dP (and dS) only after dK(n) or dQ(n).
 //
 // CTA of 384 threads (one per SM; every CTA takes all 512 TMEM columns):
-//   warps 0-3  half 0 (thread = TMEM lane = tile row)
-//   warps 4-7  half 1
+//   warps 0-3  columns 0-63 of each entry (thread = TMEM lane = tile row)
+//   warps 4-7  columns 64-127
 //   warp 8     builds the entry list, then loads tiles with TMA
 //   warp 9     allocates TMEM and issues the MMAs (one elected lane)
 //   warps 10-11 idle; they complete the third warpgroup, whose registers
 //              setmaxnreg hands to the two softmax warpgroups
-// TMEM columns: S0 [0,64), dP0 [64,128), S1 [128,192), dP1 [192,256),
-// acc0 [256, 256+D) (dV or dQ), acc1 [256+D, 256+2D) (dK). P and dS as bf16
-// pairs overwrite the first 32 columns of their S and dP.
+// TMEM columns: S [0,128), dP [128,256), acc0 [256, 256+D) (dV or dQ), acc1
+// [256+D, 256+2D) (dK). Warpgroup g writes its P and dS as bf16 pairs over
+// the first 32 of its own 64 columns of S and dP, so the accumulating
+// products read their A operand as two runs of K = 64: columns 0-31 and
+// 64-95.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -90,8 +96,8 @@ struct BwdSmem {
     static constexpr int kEntries = kLd + 2048;
     static constexpr int kFlags = kEntries + 4 * kBwdMaxEntries;
     static constexpr int kBars = kFlags + kBwdMaxEntries;
-    static constexpr int kBarFixed = 0, kBarTFull = 1, kBarTEmpty = 3, kBarSFull = 5, kBarPFull = 7, kBarAcc = 9,
-                         kNumBars = 10;
+    static constexpr int kBarFixed = 0, kBarTFull = 1, kBarTEmpty = 3, kBarSFull = 5, kBarDpFull = 6,
+                         kBarPFull = 7, kBarDsFull = 8, kBarAcc = 9, kNumBars = 10;
     static constexpr int kTmemSlot = kBars + 8 * kNumBars;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kCount = kAbort + 4;
@@ -106,28 +112,29 @@ __device__ __forceinline__ float2 mul2f(float2 a, float2 b) { return __fmul2_rn(
 __device__ __forceinline__ float2 add2f(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 fma2f(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
-// Per-half constants of the score mods. Column j of the half has
+// ALiBi constants of one warpgroup's 64 columns of an entry. Column j has
 // kv_idx - q_idx = dkv0 + step * j (step = -1 on the dk/dv side, where
 // columns are queries; +1 on the dq side).
-struct BwdHalf {
+struct BwdCols {
     float bias0, bstep;  // ALiBi bias of column 0 and its change per column (log2 units;
                          // natural units when ALiBi comes before the soft-cap)
 };
 
-// P and dS of one 32-column chunk of a half, two columns at a time on the
-// packed f32x2 pipe. x: raw q.k; dp: dO.v; nl/nd: -lse2 and -delta of each
-// column (dk/dv side, from shared memory as float4 pairs) or of the row
-// (dq side). For the score mods, with s = scale * x:
+// P phase of one 32-column chunk, two columns at a time on the packed f32x2
+// pipe. x: raw q.k; nl: -lse2 of each column (dk/dv side, from shared memory
+// as float4 (nl, nd) pairs) or of the row (dq side). For the score mods, with
+// s = scale * x:
 //   none         z2 = log2e * s
 //   soft-cap     t = tanh(s / cap), z2 = cap * log2e * t, dz/ds = 1 - t^2
 //   ALiBi        z2 = log2e * (s + slope * (kv - q))
 //   both orders  the compositions of the two
-// P = 2^(z2 - lse2), masked to 0 outside w (MASKED only), and
-// dS = P * (dP - delta) * dz/ds. Both are packed to bf16 pairs.
+// P = 2^(z2 - lse2), masked to 0 outside w (MASKED only). pk gets P as bf16
+// pairs; pg keeps P * dz/ds in fp32 for the dS phase. On unmasked chunks the
+// first 8 columns take 2^x on the FMA pipe (exp2_poly2), the rest on MUFU:
+// the P phase is the one that has to fit in the shadow of two products.
 template <int SCORE, bool KVSIDE, bool MASKED>
-__device__ __forceinline__ void bwd_chunk(const BwdParams& p, const float* x, const float* dp, const float4* ld4,
-                                          float2 nl_row, float2 nd_row, const BwdHalf& hb, int c0, uint32_t w,
-                                          uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+__device__ __forceinline__ void bwd_p_chunk(const BwdParams& p, const float* x, const float4* ld4, float2 nl_row,
+                                            const BwdCols& hb, int c0, uint32_t w, float* pg, uint32_t (&pk)[16]) {
     const float2 s2 = make_float2(p.scale_log2, p.scale_log2);
     const float2 c1 = make_float2(p.scale * p.inv_cap, p.scale * p.inv_cap);
     const float2 c2 = make_float2(p.cap * kLog2e, p.cap * kLog2e);
@@ -135,11 +142,10 @@ __device__ __forceinline__ void bwd_chunk(const BwdParams& p, const float* x, co
 #pragma unroll
     for (int jj = 0; jj < 16; ++jj) {
         const int j = c0 + 2 * jj;
-        float2 nl = nl_row, nd = nd_row;
+        float2 nl = nl_row;
         if constexpr (KVSIDE) {
             const float4 t = ld4[j >> 1];
             nl = make_float2(t.x, t.z);
-            nd = make_float2(t.y, t.w);
         }
         const float2 X = make_float2(x[j], x[j + 1]);
         float2 A, G = one;
@@ -170,15 +176,40 @@ __device__ __forceinline__ void bwd_chunk(const BwdParams& p, const float* x, co
             A = fma2f(c2, t, nl);
             G = fma2f(make_float2(-t.x, -t.y), t, one);
         }
+        float2 P;
         if constexpr (MASKED) {
             if (!((w >> (2 * jj)) & 1u)) A.x = -INFINITY;
             if (!((w >> (2 * jj + 1)) & 1u)) A.y = -INFINITY;
+            P = make_float2(ex2_approx(A.x), ex2_approx(A.y));
+        } else if (2 * jj < 8) {
+            // (an A of -inf only comes from rows past the end of the sequence
+            // here, whose dO and dP rows are zero; 2^-125 there adds nothing)
+            exp2_poly2(P.x, P.y, A.x, A.y);
+        } else {
+            P = make_float2(ex2_approx(A.x), ex2_approx(A.y));
         }
-        const float2 P = make_float2(ex2_approx(A.x), ex2_approx(A.y));
-        float2 T = mul2f(add2f(make_float2(dp[j], dp[j + 1]), nd), P);
-        if constexpr (SCORE == kScoreSoftcap || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap)
-            T = mul2f(T, G);
         pk[jj] = pack_bf16x2(P.x, P.y);
+        if constexpr (SCORE == kScoreSoftcap || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap)
+            P = mul2f(P, G);
+        pg[j] = P.x;
+        pg[j + 1] = P.y;
+    }
+}
+
+// dS phase of one 32-column chunk: dS = (P dz/ds) * (dP - delta), as bf16
+// pairs. nd: -delta of each column (dk/dv side) or of the row (dq side).
+template <bool KVSIDE>
+__device__ __forceinline__ void bwd_ds_chunk(const float* dp, const float4* ld4, float2 nd_row, const float* pg,
+                                             int c0, uint32_t (&dk)[16]) {
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+        const int j = c0 + 2 * jj;
+        float2 nd = nd_row;
+        if constexpr (KVSIDE) {
+            const float4 t = ld4[j >> 1];
+            nd = make_float2(t.y, t.w);
+        }
+        const float2 T = mul2f(add2f(make_float2(dp[j], dp[j + 1]), nd), make_float2(pg[j], pg[j + 1]));
         dk[jj] = pack_bf16x2(T.x, T.y);
     }
 }
@@ -305,9 +336,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int s = 0; s < 2; ++s) {
                 mbar_init(bar(L::kBarTFull + s), 1);
                 mbar_init(bar(L::kBarTEmpty + s), 1);
-                mbar_init(bar(L::kBarSFull + s), 1);
-                mbar_init(bar(L::kBarPFull + s), 4);
             }
+            mbar_init(bar(L::kBarSFull), 1);
+            mbar_init(bar(L::kBarDpFull), 1);
+            mbar_init(bar(L::kBarPFull), 8);   // every softmax warp
+            mbar_init(bar(L::kBarDsFull), 8);
             mbar_init(bar(L::kBarAcc), 1);
             *abort_flag = 0;
             fence_mbar_init();
@@ -442,50 +475,84 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     } else if (warp == kBwdWarpMma) {
         // ================================================= MMA issuer warp
         if (T > 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
             constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
             const uint64_t f0d = sdesc_sw128(sbase + L::kF0, 16, 1024);
             const uint64_t f1d = sdesc_sw128(sbase + L::kF1, 16, 1024);
-            bool ok = mbar_wait(bar(L::kBarFixed), 0, abort_flag);
-            // accumulating products of half c, once its warpgroup stored P and dS
-            auto issue_acc = [&](int c) -> bool {
-                const int h = c & 1, e = c >> 1, s = e & 1;
-                if (!mbar_wait(bar(L::kBarPFull + h), static_cast<uint32_t>(e & 1), abort_flag)) return false;
+            const uint32_t tm_s = tmem, tm_dp = tmem + 128u, tm_a0 = tmem + 256u, tm_a1 = tmem + 256u + D;
+            auto t0_of = [&](int n) -> uint32_t {  // streamed tile T0 of entry n (T1 one tile further)
+                return sbase + L::kStage + static_cast<uint32_t>(n & 1) * 2u * L::kTile;
+            };
+            auto wait_tiles = [&](int n) -> bool {
+                if (!mbar_wait(bar(L::kBarTFull + (n & 1)), static_cast<uint32_t>((n >> 1) & 1), abort_flag))
+                    return false;
                 tc_fence_after();
-                const uint32_t t0 = sbase + L::kStage + static_cast<uint32_t>(s) * 2u * L::kTile + h * 8192u;
-                const uint32_t t1 = t0 + L::kTile;
-                const uint32_t buf = tmem + 128u * static_cast<uint32_t>(h);
-                if (elect_one()) {
-                    if constexpr (KVSIDE) {
-                        mma_ts_run4(tmem + 256u, buf, sdesc_sw128(t1, 16384, 1024), idesc_acc, c > 0);      // dV += P^T dO
-                        mma_ts_run4(tmem + 256u + D, buf + 64u, sdesc_sw128(t0, 16384, 1024), idesc_acc, c > 0);  // dK += dS^T Q
-                    } else {
-                        mma_ts_run4(tmem + 256u, buf + 64u, sdesc_sw128(t0, 16384, 1024), idesc_acc, c > 0);  // dQ += dS K
-                    }
-                    if (h == 1) mma_commit(bar(L::kBarTEmpty + s));
-                }
-                __syncwarp();
                 return true;
             };
-            for (int e = 0; e < T && ok; ++e) {
-                const int s = e & 1;
-                if (!(ok = mbar_wait(bar(L::kBarTFull + s), static_cast<uint32_t>((e >> 1) & 1), abort_flag))) break;
+            auto wait_phase = [&](int which, int n) -> bool {
+                if (!mbar_wait(bar(which), static_cast<uint32_t>(n & 1), abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t t0 = sbase + L::kStage + static_cast<uint32_t>(s) * 2u * L::kTile;
-                const uint32_t t1 = t0 + L::kTile;
-                for (int h = 0; h < 2 && ok; ++h) {
-                    const uint32_t buf = tmem + 128u * static_cast<uint32_t>(h);
+                return true;
+            };
+            // S(n) = F0 T0(n)^T and dP(n) = F1 T1(n)^T, each 128 x 128 over K = D
+            auto issue_s = [&](int n) {
+                if (elect_one()) {
+                    mma_ss_run<D / 16>(tm_s, f0d, sdesc_sw128(t0_of(n), 16, 1024), idesc_s, 0u);
+                    mma_commit(bar(L::kBarSFull));
+                }
+                __syncwarp();
+            };
+            auto issue_dp = [&](int n) {
+                if (elect_one()) {
+                    mma_ss_run<D / 16>(tm_dp, f1d, sdesc_sw128(t0_of(n) + L::kTile, 16, 1024), idesc_s, 0u);
+                    mma_commit(bar(L::kBarDpFull));
+                }
+                __syncwarp();
+            };
+            // acc += A B over K = 128 rows of the streamed tile: A from TMEM columns
+            // a, a+8, ... in two runs (columns 0-31 hold tile rows 0-63, columns
+            // 64-95 rows 64-127), B MN-major from tile rows 0-63 and 64-127
+            auto issue_acc = [&](uint32_t acc, uint32_t a, uint32_t tile, bool first) {
+                mma_ts_run4(acc, a, sdesc_sw128(tile, 16384, 1024), idesc_acc, first ? 0u : 1u);
+                mma_ts_run4(acc, a + 64u, sdesc_sw128(tile + 8192u, 16384, 1024), idesc_acc, 1u);
+            };
+            bool ok = mbar_wait(bar(L::kBarFixed), 0, abort_flag) && wait_tiles(0);
+            if (ok) {
+                issue_s(0);
+                issue_dp(0);
+            }
+            for (int n = 0; n < T && ok; ++n) {
+                const uint32_t t0 = t0_of(n);
+                if constexpr (KVSIDE) {
+                    // dV(n) += P(n)^T dO(n), then S(n+1), then dK(n) += dS(n)^T Q(n), then dP(n+1)
+                    if (!(ok = wait_phase(L::kBarPFull, n))) break;
+                    if (elect_one()) issue_acc(tm_a0, tm_s, t0 + L::kTile, n == 0);
+                    __syncwarp();
+                    if (n + 1 < T) {
+                        if (!(ok = wait_tiles(n + 1))) break;
+                        issue_s(n + 1);
+                    }
+                    if (!(ok = wait_phase(L::kBarDsFull, n))) break;
                     if (elect_one()) {
-                        mma_ss_run<D / 16>(buf, f0d, sdesc_sw128(t0 + h * 8192u, 16, 1024), idesc_s, 0u);
-                        mma_ss_run<D / 16>(buf + 64u, f1d, sdesc_sw128(t1 + h * 8192u, 16, 1024), idesc_s, 0u);
-                        mma_commit(bar(L::kBarSFull + h));
+                        issue_acc(tm_a1, tm_dp, t0, n == 0);
+                        mma_commit(bar(L::kBarTEmpty + (n & 1)));
                     }
                     __syncwarp();
-                    const int c = 2 * e + h;
-                    if (c > 0) ok = issue_acc(c - 1);
+                } else {
+                    // S(n+1) once the P phase of n has read S(n), then dQ(n) += dS(n) K(n), then dP(n+1)
+                    if (n + 1 < T) {
+                        if (!(ok = wait_phase(L::kBarPFull, n) && wait_tiles(n + 1))) break;
+                        issue_s(n + 1);
+                    }
+                    if (!(ok = wait_phase(L::kBarDsFull, n))) break;
+                    if (elect_one()) {
+                        issue_acc(tm_a0, tm_dp, t0, n == 0);
+                        mma_commit(bar(L::kBarTEmpty + (n & 1)));
+                    }
+                    __syncwarp();
                 }
+                if (n + 1 < T) issue_dp(n + 1);
             }
-            if (ok) issue_acc(2 * T - 1);
             if (elect_one()) mma_commit(bar(L::kBarAcc));
             __syncwarp();
             mbar_wait(bar(L::kBarAcc), 0, abort_flag);
@@ -494,17 +561,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
         // ================================================= softmax warpgroups
-        const int h = warp >> 2;
+        const int h = warp >> 2;  // this warpgroup's 64 columns of every entry: [64 h, 64 h + 64)
         const int r = threadIdx.x & 127;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t t_s = tmem + 128u * static_cast<uint32_t>(h) + lane_base;
-        const uint32_t t_dp = t_s + 64u;
+        const uint32_t t_s = tmem + 64u * static_cast<uint32_t>(h) + lane_base;
+        const uint32_t t_dp = t_s + 128u;
         const int64_t row_idx = static_cast<int64_t>(blk) * 128 + r;  // this thread's kv (dk/dv) or q (dq)
         const int db = dnf.doc_batch > 1 ? b : 0;
         const bool masked_path = p.has_block_mask != 0;
         // Per-row mask data, fixed for the unit: the key's document id (dk/dv) or
         // the query's document span (dq). The term intervals are recomputed on
-        // each partial half from the mask program (registers go to the tiles).
+        // each partial tile from the mask program (registers go to the tiles).
         int32_t my_doc = 0;
         bool my_doc_ok = false;
         int64_t row_ds = 0, row_de = -1;
@@ -552,8 +619,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int eb = static_cast<int>(ent & 0xFFFFu);
             const int g = static_cast<int>((ent >> 16) & 0xFFu);
             const bool partial = (ent & kBwdPartial) != 0u;
-            const int64_t c0 = static_cast<int64_t>(eb) * 128 + 64 * h;  // first column (q or kv) of this half
-            // mask words over the half's 64 columns (bit j: column c0 + j allowed)
+            const int64_t c0 = static_cast<int64_t>(eb) * 128 + 64 * h;  // first column (q or kv) of this warpgroup
+            // mask words over the warpgroup's 64 columns (bit j: column c0 + j allowed)
             uint32_t w0 = 0xFFFFFFFFu, w1 = 0xFFFFFFFFu;
             if (partial) {
                 w0 = 0u;
@@ -607,10 +674,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if constexpr (KVSIDE && kAlibi)
                 slope = p.slopes ? __ldg(p.slopes + hq + g)
                                  : exp2f(-8.0f * static_cast<float>(hq + g + 1) / static_cast<float>(p.Hq));
-            // kv - q at column 0 of the half; it moves by -1 (dk/dv) or +1 (dq) per column
+            // kv - q at the warpgroup's column 0; it moves by -1 (dk/dv) or +1 (dq) per column
             const float dkv0 = KVSIDE ? static_cast<float>(row_idx - c0) : static_cast<float>(c0 - row_idx);
             constexpr float kStep = KVSIDE ? -1.f : 1.f;
-            BwdHalf hb;
+            BwdCols hb;
             if constexpr (SCORE == kScoreAlibiSoftcap) {
                 hb.bias0 = slope * dkv0;
                 hb.bstep = slope * kStep;
@@ -619,33 +686,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 hb.bstep = slope * kLog2e * kStep;
             }
 
-            if (!mbar_wait(bar(L::kBarSFull + h), static_cast<uint32_t>(e & 1), abort_flag)) {
+            const float4* ld4 = reinterpret_cast<const float4*>(ld_smem + 128 * (e & 1) + 64 * h);
+            float pg[64];  // P * dz/ds of this thread's 64 columns, from the P phase to the dS phase
+            // ---- P phase: S -> P (bf16 into TMEM for dV on the dk/dv side)
+            if (!mbar_wait(bar(L::kBarSFull), static_cast<uint32_t>(e & 1), abort_flag)) {
                 ok = false;
                 break;
             }
             __syncwarp();  // tcgen05.ld/st are warp-collective: reconverge after the wait
             tc_fence_after();
-            float x[64], dp[64];
-            tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(x));
-            tmem_ld32(t_s + 32u, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-            tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dp));
-            tmem_ld32(t_dp + 32u, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
-            tc_wait_ld();
-            const float4* ld4 = reinterpret_cast<const float4*>(ld_smem + 128 * (e & 1) + 64 * h);
+            {
+                float x[64];
+                tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(x));
+                tmem_ld32(t_s + 32u, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+                tc_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t pk[16], dk[16];
-                if (partial)
-                    bwd_chunk<SCORE, KVSIDE, true>(p, x, dp, ld4, nl_row, nd_row, hb, 32 * c, c == 0 ? w0 : w1, pk, dk);
-                else
-                    bwd_chunk<SCORE, KVSIDE, false>(p, x, dp, ld4, nl_row, nd_row, hb, 32 * c, 0u, pk, dk);
-                if constexpr (KVSIDE) tmem_st16(t_s + 16u * c, pk);
-                tmem_st16(t_dp + 16u * c, dk);
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pk[16];
+                    if (partial)
+                        bwd_p_chunk<SCORE, KVSIDE, true>(p, x, ld4, nl_row, hb, 32 * c, c == 0 ? w0 : w1, pg, pk);
+                    else
+                        bwd_p_chunk<SCORE, KVSIDE, false>(p, x, ld4, nl_row, hb, 32 * c, 0u, pg, pk);
+                    if constexpr (KVSIDE) tmem_st16(t_s + 16u * c, pk);
+                }
+            }
+            if constexpr (KVSIDE) tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::kBarPFull));
+            // ---- dS phase: dP -> dS (bf16 into TMEM for dK or dQ)
+            if (!mbar_wait(bar(L::kBarDpFull), static_cast<uint32_t>(e & 1), abort_flag)) {
+                ok = false;
+                break;
+            }
+            __syncwarp();
+            tc_fence_after();
+            {
+                float dp[64];
+                tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dp));
+                tmem_ld32(t_dp + 32u, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
+                tc_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t dk[16];
+                    bwd_ds_chunk<KVSIDE>(dp, ld4, nd_row, pg, 32 * c, dk);
+                    tmem_st16(t_dp + 16u * c, dk);
+                }
             }
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::kBarPFull + h));
+            if (lane == 0) mbar_arrive(bar(L::kBarDsFull));
         }
         // ------------------------------------------------------ epilogue
         // dk/dv: warpgroup 0 writes dV, warpgroup 1 writes dK (times scale).
