@@ -252,41 +252,65 @@ __device__ __forceinline__ void term_q_interval(const MaskDnf& m, int t, int64_t
 
 // (-lse2, -delta) per padded query row: lse2 = lse * log2(e) (+inf where lse
 // is -inf and for rows past M, so that P = 0 there), delta = sum_d out * dout
-// in fp32. One warp per row; lane l reads D/32 consecutive elements.
+// in fp32. A row is read by D/8 lanes, 16 bytes of out and of dout each; a
+// warp covers kRowsPerWarp rows with all its loads issued before the sums,
+// so that enough bytes are in flight to keep HBM busy.
+constexpr int kPrepRowsPerWarp = 8;
+
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* out, const __nv_bfloat16* dout,
                                                        const float* lse, int64_t rows_pad, int32_t M, int32_t QB,
                                                        float2* ld) {
+    constexpr int kLanesPerRow = D / 8;          // 16 (D = 128) or 8 (D = 64)
+    constexpr int kRowsPerIter = 32 / kLanesPerRow;
+    constexpr int kIters = kPrepRowsPerWarp / kRowsPerIter;
     const int lane = threadIdx.x & 31;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (row >= rows_pad) return;
+    const int sub = lane / kLanesPerRow;         // row within an iteration
+    const int part = lane % kLanesPerRow;        // 16-byte piece of the row
+    const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kPrepRowsPerWarp;
     const int64_t per_bh = static_cast<int64_t>(QB) * 128;
-    const int64_t bh = row / per_bh;
-    const int i = static_cast<int>(row - bh * per_bh);
-    float acc = 0.f, l2 = INFINITY;
-    if (i < M) {
-        const int64_t base = (bh * M + i) * D + lane * (D / 32);
-        if constexpr (D == 128) {
-            const uint2 a = *reinterpret_cast<const uint2*>(out + base);
-            const uint2 g = *reinterpret_cast<const uint2*>(dout + base);
-            const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
-            const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
-            const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g.x));
-            const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g.y));
-            acc = fmaf(a0.x, g0.x, fmaf(a0.y, g0.y, fmaf(a1.x, g1.x, a1.y * g1.y)));
+    uint4 a[kIters], g[kIters];
+    bool in[kIters];
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+        const int64_t row = row0 + it * kRowsPerIter + sub;
+        const int64_t bh = row / per_bh;
+        const int i = static_cast<int>(row - bh * per_bh);
+        in[it] = row < rows_pad && i < M;
+        if (in[it]) {
+            const int64_t base = (bh * M + i) * D + part * 8;
+            a[it] = __ldg(reinterpret_cast<const uint4*>(out + base));
+            g[it] = __ldg(reinterpret_cast<const uint4*>(dout + base));
         } else {
-            const uint32_t a = *reinterpret_cast<const uint32_t*>(out + base);
-            const uint32_t g = *reinterpret_cast<const uint32_t*>(dout + base);
-            const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a));
-            const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g));
-            acc = fmaf(a0.x, g0.x, a0.y * g0.y);
+            a[it] = make_uint4(0u, 0u, 0u, 0u);
+            g[it] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+        const uint32_t av[4] = {a[it].x, a[it].y, a[it].z, a[it].w};
+        const uint32_t gv[4] = {g[it].x, g[it].y, g[it].z, g[it].w};
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[k]));
+            const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv[k]));
+            acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-        const float L = __ldg(lse + bh * M + i);
-        l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
+        for (int o = kLanesPerRow / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+        const int64_t row = row0 + it * kRowsPerIter + sub;
+        if (part == 0 && row < rows_pad) {
+            const int64_t bh = row / per_bh;
+            const int i = static_cast<int>(row - bh * per_bh);
+            float l2 = INFINITY;
+            if (in[it]) {
+                const float L = __ldg(lse + bh * M + i);
+                l2 = (L == -INFINITY) ? INFINITY : L * kLog2e;
+            }
+            ld[row] = make_float2(-l2, in[it] ? -acc : 0.f);
+        }
     }
-    if (lane == 0) ld[row] = make_float2(-l2, -acc);
 }
 
 template <int D, int SCORE, bool KVSIDE>

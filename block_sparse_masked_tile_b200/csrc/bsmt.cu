@@ -947,12 +947,14 @@ extern "C" bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, con
     // (lse2, delta) per padded query row
     float2* ld = static_cast<float2*>(workspace);
     const int64_t rows_pad = B * Hq * QB * 128;
+    const int64_t prep_blocks = (rows_pad + 8 * bsmt::kPrepRowsPerWarp - 1) / (8 * bsmt::kPrepRowsPerWarp);
+    if (prep_blocks > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "too many query rows");
     if (D == 128)
-        bsmt::bwd_prep_kernel<128><<<static_cast<unsigned>(rows_pad / 8), 256, 0, s>>>(
+        bsmt::bwd_prep_kernel<128><<<static_cast<unsigned>(prep_blocks), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, rows_pad,
             static_cast<int32_t>(M), static_cast<int32_t>(QB), ld);
     else
-        bsmt::bwd_prep_kernel<64><<<static_cast<unsigned>(rows_pad / 8), 256, 0, s>>>(
+        bsmt::bwd_prep_kernel<64><<<static_cast<unsigned>(prep_blocks), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, rows_pad,
             static_cast<int32_t>(M), static_cast<int32_t>(QB), ld);
     cudaError_t e = cudaGetLastError();
