@@ -535,11 +535,39 @@ def splitkv_workspace_bytes(B: int, Hq: int, M: int, D: int, num_splits: int) ->
     return int(n.value)
 
 
+class _FlexAttentionFn(torch.autograd.Function):
+    """flex_attention as a differentiable op: the forward kernel, then
+    flex_attention_backward for dq, dk and dv. lse is an output without a
+    gradient."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, block_mask, score_mod, scale, enable_gqa, out, lse):
+        out, lse = _flex_attention_fwd(q, k, v, block_mask, score_mod, scale, enable_gqa, out, lse, 1, None)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.args = (block_mask, score_mod, scale, enable_gqa)
+        ctx.mark_non_differentiable(lse)
+        return out, lse
+
+    @staticmethod
+    def backward(ctx, dout, _dlse):
+        q, k, v, out, lse = ctx.saved_tensors
+        block_mask, score_mod, scale, enable_gqa = ctx.args
+        if dout is None:
+            return (None,) * 9
+        dq, dk, dv = flex_attention_backward(q, k, v, out, lse, dout.to(torch.bfloat16).contiguous(), block_mask,
+                                             score_mod, scale, enable_gqa)
+        return dq, dk, dv, None, None, None, None, None, None
+
+
 def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask: BlockMask | None = None,
                    score_mod: ScoreMod | Iterable[ScoreMod] | None = None, scale: float | None = None,
                    enable_gqa: bool = False, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
                    num_splits: int = 1, workspace: torch.Tensor | None = None):
     """Block-sparse masked attention forward. Returns (out bf16 [B,Hq,M,D], lse fp32 [B,Hq,M]).
+
+    When autograd is on and q, k or v requires grad, the call is recorded
+    for backpropagation: out's gradient flows to q, k and v through
+    flex_attention_backward (one split only; lse has no gradient).
 
     num_splits > 1 runs split-KV: every row's kv blocks are cut into that many
     slices computed in parallel and merged exactly (for few q-blocks and long
@@ -548,6 +576,14 @@ def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask
     ``workspace="static"`` uses the library's fixed device scratch instead and
     allocates nothing (bsmt_flex_attention_fwd_splitkv_static: sizes above the
     scratch are rejected, and calls that overlap in time race on it)."""
+    if torch.is_grad_enabled() and any(t.requires_grad for t in (q, k, v)):
+        if num_splits != 1:
+            raise ValueError("split-KV has no backward; use num_splits=1 when q, k or v requires grad")
+        return _FlexAttentionFn.apply(q, k, v, block_mask, score_mod, scale, enable_gqa, out, lse)
+    return _flex_attention_fwd(q, k, v, block_mask, score_mod, scale, enable_gqa, out, lse, num_splits, workspace)
+
+
+def _flex_attention_fwd(q, k, v, block_mask, score_mod, scale, enable_gqa, out, lse, num_splits, workspace):
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.dtype != torch.bfloat16:
             raise ValueError(f"{name} must be bfloat16 (got {t.dtype})")
