@@ -37,13 +37,19 @@
 // by one thread run in order, so S(n+1) overwrites S (and P) only after dV(n)
 // has read P, and dP(n+1) overwrites dP (and dS) only after dK(n) or dQ(n).
 //
-// CTA of 384 threads (one per SM; every CTA takes all 512 TMEM columns):
+// Persistent CTAs, one per SM (every CTA takes all 512 TMEM columns), take
+// units from a work counter in the workspace. 384 threads:
 //   warps 0-3  columns 0-63 of each entry (thread = TMEM lane = tile row)
 //   warps 4-7  columns 64-127
-//   warp 8     builds the entry list, then loads tiles with TMA
+//   warp 8     loads tiles with TMA (the next unit's K/V or Q/dO as soon as
+//              the current unit's last S and dP are issued)
 //   warp 9     allocates TMEM and issues the MMAs (one elected lane)
-//   warps 10-11 idle; they complete the third warpgroup, whose registers
+//   warp 10    scheduler: takes the next unit and builds its entry list in
+//              the other of two buffers
+//   warp 11    idle; it completes the third warpgroup, whose registers
 //              setmaxnreg hands to the two softmax warpgroups
+// The epilogue reads the accumulators whole and releases them before its
+// stores, so the next unit's products overlap the previous unit's stores.
 // TMEM columns: S [0,128), dP [128,256), acc0 [256, 256+D) (dV or dQ), acc1
 // [256+D, 256+2D) (dK). Warpgroup g writes its P and dS as bf16 pairs over
 // the first 32 of its own 64 columns of S and dP, so the accumulating
@@ -78,13 +84,21 @@ struct BwdParams {
     __nv_bfloat16* g0;  // dq (dq kernel) or dk [B, Hkv, N, D]
     __nv_bfloat16* g1;  // dv [B, Hkv, N, D]
     int32_t num_units;
+    int32_t* next_unit;  // work counter, zero at launch (the prep kernel clears it)
 };
 
 constexpr int kBwdThreads = 384;
 constexpr int kBwdWarpLoad = 8;
 constexpr int kBwdWarpMma = 9;
-constexpr int kBwdMaxEntries = 4096;  // entries of one unit (list length x GQA group)
+constexpr int kBwdWarpSched = 10;
+constexpr int kBwdMaxEntries = 2048;  // entries of one unit (list length x GQA group)
 constexpr uint32_t kBwdPartial = 0x80000000u;
+
+// A scheduled unit in shared memory (two buffers, filled by the scheduler warp).
+struct BwdUnit {
+    int32_t T;  // entries; -1 ends the work
+    int32_t b, hq, hkv, blk;
+};
 
 template <int D>
 struct BwdSmem {
@@ -92,16 +106,18 @@ struct BwdSmem {
     static constexpr int kF0 = 0;                   // K (dk/dv) or Q (dq)
     static constexpr int kF1 = kTile;               // V or dO
     static constexpr int kStage = 2 * kTile;        // stage s: T0 at kStage + 2 s kTile, T1 one tile further
-    static constexpr int kLd = kStage + 4 * kTile;  // stage s: 128 float2 (lse2, delta) at kLd + 1024 s
-    static constexpr int kEntries = kLd + 2048;
-    static constexpr int kFlags = kEntries + 4 * kBwdMaxEntries;
+    static constexpr int kLd = kStage + 4 * kTile;  // stage s: 128 float2 (-lse2, -delta) at kLd + 1024 s
+    static constexpr int kList = kLd + 2048;        // unit buffer u: entries at kList + u * kListBytes
+    static constexpr int kListBytes = 4 * kBwdMaxEntries;
+    static constexpr int kHdr = kList + 2 * kListBytes;  // BwdUnit[2], 32 bytes each
+    static constexpr int kFlags = kHdr + 64;
     static constexpr int kBars = kFlags + kBwdMaxEntries;
-    static constexpr int kBarFixed = 0, kBarTFull = 1, kBarTEmpty = 3, kBarSFull = 5, kBarDpFull = 6,
-                         kBarPFull = 7, kBarDsFull = 8, kBarAcc = 9, kNumBars = 10;
+    static constexpr int kBarFixedFull = 0, kBarFixedEmpty = 1, kBarTFull = 2, kBarTEmpty = 4, kBarSFull = 6,
+                         kBarDpFull = 7, kBarPFull = 8, kBarDsFull = 9, kBarAccFull = 10, kBarAccEmpty = 11,
+                         kBarListFull = 12, kBarListEmpty = 14, kBarDone = 16, kNumBars = 17;
     static constexpr int kTmemSlot = kBars + 8 * kNumBars;
     static constexpr int kAbort = kTmemSlot + 4;
-    static constexpr int kCount = kAbort + 4;
-    static constexpr int kTotal = kCount + 8;
+    static constexpr int kTotal = kAbort + 4;
     // never less than 120 KB, so that a second CTA cannot share the SM (and
     // wait in tcgen05.alloc for the TMEM the first one holds)
     static constexpr int kAlloc = (kTotal + 1024 > 120 * 1024) ? kTotal + 1024 : 120 * 1024;
@@ -252,7 +268,8 @@ __device__ __forceinline__ void term_q_interval(const MaskDnf& m, int t, int64_t
 
 // (-lse2, -delta) per padded query row: lse2 = lse * log2(e) (+inf where lse
 // is -inf and for rows past M, so that P = 0 there), delta = sum_d out * dout
-// in fp32. A row is read by D/8 lanes, 16 bytes of out and of dout each; a
+// in fp32; it also zeroes the two backward kernels' work counters. A row is
+// read by D/8 lanes, 16 bytes of out and of dout each; a
 // warp covers kRowsPerWarp rows with all its loads issued before the sums,
 // so that enough bytes are in flight to keep HBM busy.
 constexpr int kPrepRowsPerWarp = 8;
@@ -260,7 +277,8 @@ constexpr int kPrepRowsPerWarp = 8;
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* out, const __nv_bfloat16* dout,
                                                        const float* lse, int64_t rows_pad, int32_t M, int32_t QB,
-                                                       float2* ld) {
+                                                       float2* ld, int32_t* counters) {
+    if (blockIdx.x == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0;  // work counters of the two kernels
     constexpr int kLanesPerRow = D / 8;          // 16 (D = 128) or 8 (D = 64)
     constexpr int kRowsPerIter = 32 / kLanesPerRow;
     constexpr int kIters = kPrepRowsPerWarp / kRowsPerIter;
@@ -326,123 +344,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int lane = threadIdx.x & 31;
     auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * static_cast<uint32_t>(i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
-    uint32_t* entries = reinterpret_cast<uint32_t*>(smem + L::kEntries);
-    int32_t* count_slot = reinterpret_cast<int32_t*>(smem + L::kCount);
-
-    // ------------------------------------------------------------ the unit
-    // dk/dv: kv-blocks in ascending order (under a causal mask the first ones
-    // have the most q-blocks); dq: q-blocks in descending order.
-    int b, hq, hkv, blk;
-    {
-        const int u = blockIdx.x;
-        if constexpr (KVSIDE) {
-            const int n_bh = p.B * p.Hkv;
-            blk = u / n_bh;
-            const int bh = u - blk * n_bh;
-            b = bh / p.Hkv;
-            hkv = bh - b * p.Hkv;
-            hq = hkv * p.group;
-        } else {
-            const int n_bh = p.B * p.Hq;
-            const int r = u / n_bh;
-            blk = p.QB - 1 - r;
-            const int bh = u - r * n_bh;
-            b = bh / p.Hq;
-            hq = bh - b * p.Hq;
-            hkv = hq / p.group;
-        }
-    }
+    auto list_of = [&](int buf) -> uint32_t* { return reinterpret_cast<uint32_t*>(smem + L::kList + buf * L::kListBytes); };
+    auto hdr_of = [&](int buf) -> BwdUnit* { return reinterpret_cast<BwdUnit*>(smem + L::kHdr + 32 * buf); };
 
     // ------------------------------------------------------------ set-up
-    if (warp == kBwdWarpLoad) {
-        if (lane == 0) {
-            mbar_init(bar(L::kBarFixed), 1);
-            for (int s = 0; s < 2; ++s) {
-                mbar_init(bar(L::kBarTFull + s), 1);
-                mbar_init(bar(L::kBarTEmpty + s), 1);
-            }
-            mbar_init(bar(L::kBarSFull), 1);
-            mbar_init(bar(L::kBarDpFull), 1);
-            mbar_init(bar(L::kBarPFull), 8);   // every softmax warp
-            mbar_init(bar(L::kBarDsFull), 8);
-            mbar_init(bar(L::kBarAcc), 1);
-            *abort_flag = 0;
-            fence_mbar_init();
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
-            prefetch_tmap(&tm_do);
+    if (warp == kBwdWarpLoad && lane == 0) {
+        mbar_init(bar(L::kBarFixedFull), 1);
+        mbar_init(bar(L::kBarFixedEmpty), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(L::kBarTFull + s), 1);
+            mbar_init(bar(L::kBarTEmpty + s), 1);
+            mbar_init(bar(L::kBarListFull + s), 32);     // every scheduler lane
+            mbar_init(bar(L::kBarListEmpty + s), 1 + 1 + 8);  // producer, MMA warp, softmax warps
         }
-        // Entry list of the unit: for each query head of the group (dk/dv) or
-        // the unit's head (dq), the blocks of the partial and the full list,
-        // merged in ascending order. A block in both lists counts as partial;
-        // with a ragged KV_LEN the last kv block is partial (dq).
-        uint8_t* flags = smem + L::kFlags;
-        for (int j = lane; j < p.list_len; j += 32) flags[j] = 0;
-        __syncwarp();
-        const int heads = KVSIDE ? p.group : 1;
-        const bool ragged_last = !KVSIDE && (p.N & 127) != 0;
-        const uint32_t below = (1u << lane) - 1u;
-        int T = 0;
-        bool bad = false;
-        for (int g = 0; g < heads; ++g) {
-            if (!p.has_block_mask) {
-                for (int c = 0; c < p.list_len; c += 32) {
-                    const int j = c + lane;
-                    if (j < p.list_len) {
-                        const bool part = ragged_last && j == p.list_len - 1;
-                        entries[T + j] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(g) << 16) |
-                                         (part ? kBwdPartial : 0u);
-                    }
-                }
-                T += p.list_len;
-                continue;
-            }
-            const int hl = KVSIDE ? hq + g : hq;
-            const int bb = p.Bm > 1 ? b : 0;
-            const int hh = p.Hm > 1 ? hl : 0;
-            const int64_t row = (static_cast<int64_t>(bb) * p.Hm + hh) * p.list_rows + blk;
-            int v = 0;
-            if (lane == 0) v = __ldg(p.num + row);
-            if (lane == 1) v = __ldg(p.full_num + row);
-            if (v < 0 || v > p.list_len) {
-                bad = true;
-                v = 0;
-            }
-            const int cnt0 = __shfl_sync(0xFFFFFFFFu, v, 0);
-            const int cnt1 = __shfl_sync(0xFFFFFFFFu, v, 1);
-            const int32_t* l0 = p.idx + row * p.list_len;
-            const int32_t* l1 = p.full_idx + row * p.list_len;
-            for (int j = lane; j < cnt0; j += 32) {
-                const int x = __ldg(l0 + j);
-                if (x >= 0 && x < p.list_len) flags[x] |= 1u;
-                else bad = true;
-            }
-            __syncwarp();
-            for (int j = lane; j < cnt1; j += 32) {
-                const int x = __ldg(l1 + j);
-                if (x >= 0 && x < p.list_len) flags[x] |= 2u;
-                else bad = true;
-            }
-            __syncwarp();
-            for (int c = 0; c < p.list_len; c += 32) {
-                const int j = c + lane;
-                uint32_t f = 0;
-                if (j < p.list_len) {
-                    f = flags[j];
-                    flags[j] = 0;
-                }
-                const bool part = (f & 1u) || (f != 0u && ragged_last && j == p.list_len - 1);
-                const unsigned bal = __ballot_sync(0xFFFFFFFFu, f != 0u);
-                if (f)
-                    entries[T + __popc(bal & below)] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(g) << 16) |
-                                                       (part ? kBwdPartial : 0u);
-                T += __popc(bal);
-            }
-            __syncwarp();
-        }
-        if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
-        if (lane == 0) *count_slot = T;
+        mbar_init(bar(L::kBarSFull), 1);
+        mbar_init(bar(L::kBarDpFull), 1);
+        mbar_init(bar(L::kBarPFull), 8);  // every softmax warp
+        mbar_init(bar(L::kBarDsFull), 8);
+        mbar_init(bar(L::kBarAccFull), 1);
+        mbar_init(bar(L::kBarAccEmpty), 8);
+        mbar_init(bar(L::kBarDone), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
     }
     if (warp == kBwdWarpMma) {
         tmem_alloc(sbase + L::kTmemSlot, 512);
@@ -452,135 +379,303 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
-    const int T = *reinterpret_cast<volatile int32_t*>(count_slot);
 
     // Register split: every thread is launched with 168 registers (build.py
     // checks the count); warpgroup 2 gives some back and the softmax
     // warpgroups take them: 128 * 80 + 256 * 208 = 63488 <= 384 * 168.
     if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
-    if (warp == kBwdWarpLoad) {
-        // ================================================= TMA producer warp
-        if (T > 0) {
-            const uint32_t tile = L::kTile;
-            const int zf = KVSIDE ? b * p.Hkv + hkv : b * p.Hq + hq;
-            if (lane == 0) {
-                const uint32_t fb = bar(L::kBarFixed);
-                mbar_arrive_expect_tx(fb, 2 * tile);
-#pragma unroll
-                for (int h = 0; h < D / 64; ++h) {
-                    tma_load_3d(sbase + L::kF0 + h * 16384, KVSIDE ? &tm_k : &tm_q, h * 64, blk * 128, zf, fb);
-                    tma_load_3d(sbase + L::kF1 + h * 16384, KVSIDE ? &tm_v : &tm_do, h * 64, blk * 128, zf, fb);
-                }
+    if (warp == kBwdWarpSched) {
+        // ================================================= scheduler warp
+        // Takes units from the work counter in order (dk/dv: kv-blocks
+        // ascending, which under a causal mask puts the longest first; dq:
+        // q-blocks descending) and writes each unit's entry list: for each
+        // query head of the GQA group (dk/dv) or the unit's head (dq), the
+        // blocks of the partial and the full list, merged in ascending order.
+        // A block in both lists counts as partial; with a ragged KV_LEN the
+        // last kv block is partial (dq).
+        uint8_t* flags = smem + L::kFlags;
+        for (int j = lane; j < p.list_len; j += 32) flags[j] = 0;
+        __syncwarp();
+        const int heads = KVSIDE ? p.group : 1;
+        const bool ragged_last = !KVSIDE && (p.N & 127) != 0;
+        const uint32_t below = (1u << lane) - 1u;
+        for (int it = 0;; ++it) {
+            const int buf = it & 1;
+            if (!mbar_wait(bar(L::kBarListEmpty + buf), static_cast<uint32_t>((it >> 1) & 1) ^ 1u, abort_flag)) break;
+            int u = 0;
+            if (lane == 0) u = atomicAdd(p.next_unit, 1);
+            u = __shfl_sync(0xFFFFFFFFu, u, 0);
+            BwdUnit* hdr = hdr_of(buf);
+            if (u >= p.num_units) {
+                if (lane == 0) hdr->T = -1;
+                __syncwarp();
+                mbar_arrive(bar(L::kBarListFull + buf));
+                break;
             }
-            for (int e = 0; e < T; ++e) {
-                const int s = e & 1;
-                if (!mbar_wait(bar(L::kBarTEmpty + s), static_cast<uint32_t>((e >> 1) & 1) ^ 1u, abort_flag)) break;
-                const uint32_t ent = entries[e];
-                const int eb = static_cast<int>(ent & 0xFFFFu);
-                const int g = static_cast<int>((ent >> 16) & 0xFFu);
-                if (lane == 0) {
-                    const uint32_t fb = bar(L::kBarTFull + s);
-                    mbar_arrive_expect_tx(fb, 2 * tile + (KVSIDE ? 1024u : 0u));
-                    const uint32_t t0 = sbase + L::kStage + static_cast<uint32_t>(s) * 2u * tile;
-                    const int zt = KVSIDE ? b * p.Hq + hq + g : b * p.Hkv + hkv;
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h) {
-                        tma_load_3d(t0 + h * 16384, KVSIDE ? &tm_q : &tm_k, h * 64, eb * 128, zt, fb);
-                        tma_load_3d(t0 + tile + h * 16384, KVSIDE ? &tm_do : &tm_v, h * 64, eb * 128, zt, fb);
+            int b, hq, hkv, blk;
+            if constexpr (KVSIDE) {
+                const int n_bh = p.B * p.Hkv;
+                blk = u / n_bh;
+                const int bh = u - blk * n_bh;
+                b = bh / p.Hkv;
+                hkv = bh - b * p.Hkv;
+                hq = hkv * p.group;
+            } else {
+                const int n_bh = p.B * p.Hq;
+                const int r = u / n_bh;
+                blk = p.QB - 1 - r;
+                const int bh = u - r * n_bh;
+                b = bh / p.Hq;
+                hq = bh - b * p.Hq;
+                hkv = hq / p.group;
+            }
+            uint32_t* entries = list_of(buf);
+            int T = 0;
+            bool bad = false;
+            for (int g = 0; g < heads; ++g) {
+                if (!p.has_block_mask) {
+                    for (int c = 0; c < p.list_len; c += 32) {
+                        const int j = c + lane;
+                        if (j < p.list_len) {
+                            const bool part = ragged_last && j == p.list_len - 1;
+                            entries[T + j] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(g) << 16) |
+                                             (part ? kBwdPartial : 0u);
+                        }
                     }
-                    if constexpr (KVSIDE)
-                        bulk_load_1d(sbase + L::kLd + 1024u * static_cast<uint32_t>(s),
-                                     p.ld + (static_cast<int64_t>(b * p.Hq + hq + g) * p.QB + eb) * 128, 1024u, fb);
+                    T += p.list_len;
+                    continue;
+                }
+                const int hl = KVSIDE ? hq + g : hq;
+                const int bb = p.Bm > 1 ? b : 0;
+                const int hh = p.Hm > 1 ? hl : 0;
+                const int64_t row = (static_cast<int64_t>(bb) * p.Hm + hh) * p.list_rows + blk;
+                int v = 0;
+                if (lane == 0) v = __ldg(p.num + row);
+                if (lane == 1) v = __ldg(p.full_num + row);
+                if (v < 0 || v > p.list_len) {
+                    bad = true;
+                    v = 0;
+                }
+                const int cnt0 = __shfl_sync(0xFFFFFFFFu, v, 0);
+                const int cnt1 = __shfl_sync(0xFFFFFFFFu, v, 1);
+                const int32_t* l0 = p.idx + row * p.list_len;
+                const int32_t* l1 = p.full_idx + row * p.list_len;
+                for (int j = lane; j < cnt0; j += 32) {
+                    const int x = __ldg(l0 + j);
+                    if (x >= 0 && x < p.list_len) flags[x] |= 1u;
+                    else bad = true;
+                }
+                __syncwarp();
+                for (int j = lane; j < cnt1; j += 32) {
+                    const int x = __ldg(l1 + j);
+                    if (x >= 0 && x < p.list_len) flags[x] |= 2u;
+                    else bad = true;
+                }
+                __syncwarp();
+                for (int c = 0; c < p.list_len; c += 32) {
+                    const int j = c + lane;
+                    uint32_t f = 0;
+                    if (j < p.list_len) {
+                        f = flags[j];
+                        flags[j] = 0;
+                    }
+                    const bool part = (f & 1u) || (f != 0u && ragged_last && j == p.list_len - 1);
+                    const unsigned bal = __ballot_sync(0xFFFFFFFFu, f != 0u);
+                    if (f)
+                        entries[T + __popc(bal & below)] = static_cast<uint32_t>(j) |
+                                                           (static_cast<uint32_t>(g) << 16) |
+                                                           (part ? kBwdPartial : 0u);
+                    T += __popc(bal);
                 }
                 __syncwarp();
             }
+            if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
+            if (lane == 0) {
+                hdr->T = T;
+                hdr->b = b;
+                hdr->hq = hq;
+                hdr->hkv = hkv;
+                hdr->blk = blk;
+            }
+            __syncwarp();
+            mbar_arrive(bar(L::kBarListFull + buf));
+        }
+    } else if (warp == kBwdWarpLoad) {
+        // ================================================= TMA producer warp
+        const uint32_t tile = L::kTile;
+        uint32_t ge = 0, fixed_uses = 0;  // entries and units with entries so far
+        for (int it = 0;; ++it) {
+            const int buf = it & 1;
+            if (!mbar_wait(bar(L::kBarListFull + buf), static_cast<uint32_t>((it >> 1) & 1), abort_flag)) break;
+            const BwdUnit hdr = *hdr_of(buf);
+            if (hdr.T < 0) break;
+            const uint32_t* entries = list_of(buf);
+            bool ok = true;
+            if (hdr.T > 0) {
+                // K, V (dk/dv) or Q, dO (dq) of the unit, once the last unit's S and dP are issued
+                if (fixed_uses > 0 &&
+                    !mbar_wait(bar(L::kBarFixedEmpty), (fixed_uses - 1) & 1u, abort_flag))
+                    break;
+                ++fixed_uses;
+                const int zf = KVSIDE ? hdr.b * p.Hkv + hdr.hkv : hdr.b * p.Hq + hdr.hq;
+                if (lane == 0) {
+                    const uint32_t fb = bar(L::kBarFixedFull);
+                    mbar_arrive_expect_tx(fb, 2 * tile);
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h) {
+                        tma_load_3d(sbase + L::kF0 + h * 16384, KVSIDE ? &tm_k : &tm_q, h * 64, hdr.blk * 128, zf, fb);
+                        tma_load_3d(sbase + L::kF1 + h * 16384, KVSIDE ? &tm_v : &tm_do, h * 64, hdr.blk * 128, zf, fb);
+                    }
+                }
+                for (int e = 0; e < hdr.T; ++e, ++ge) {
+                    const uint32_t s = ge & 1u;
+                    if (!mbar_wait(bar(L::kBarTEmpty + s), ((ge >> 1) & 1u) ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t ent = entries[e];
+                    const int eb = static_cast<int>(ent & 0xFFFFu);
+                    const int g = static_cast<int>((ent >> 16) & 0xFFu);
+                    if (lane == 0) {
+                        const uint32_t fb = bar(L::kBarTFull + s);
+                        mbar_arrive_expect_tx(fb, 2 * tile + (KVSIDE ? 1024u : 0u));
+                        const uint32_t t0 = sbase + L::kStage + s * 2u * tile;
+                        const int zt = KVSIDE ? hdr.b * p.Hq + hdr.hq + g : hdr.b * p.Hkv + hdr.hkv;
+#pragma unroll
+                        for (int h = 0; h < D / 64; ++h) {
+                            tma_load_3d(t0 + h * 16384, KVSIDE ? &tm_q : &tm_k, h * 64, eb * 128, zt, fb);
+                            tma_load_3d(t0 + tile + h * 16384, KVSIDE ? &tm_do : &tm_v, h * 64, eb * 128, zt, fb);
+                        }
+                        if constexpr (KVSIDE)
+                            bulk_load_1d(sbase + L::kLd + 1024u * s,
+                                         p.ld + (static_cast<int64_t>(hdr.b * p.Hq + hdr.hq + g) * p.QB + eb) * 128,
+                                         1024u, fb);
+                    }
+                    __syncwarp();
+                }
+            }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::kBarListEmpty + buf));
         }
     } else if (warp == kBwdWarpMma) {
         // ================================================= MMA issuer warp
-        if (T > 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
-            const uint64_t f0d = sdesc_sw128(sbase + L::kF0, 16, 1024);
-            const uint64_t f1d = sdesc_sw128(sbase + L::kF1, 16, 1024);
-            const uint32_t tm_s = tmem, tm_dp = tmem + 128u, tm_a0 = tmem + 256u, tm_a1 = tmem + 256u + D;
-            auto t0_of = [&](int n) -> uint32_t {  // streamed tile T0 of entry n (T1 one tile further)
-                return sbase + L::kStage + static_cast<uint32_t>(n & 1) * 2u * L::kTile;
-            };
-            auto wait_tiles = [&](int n) -> bool {
-                if (!mbar_wait(bar(L::kBarTFull + (n & 1)), static_cast<uint32_t>((n >> 1) & 1), abort_flag))
-                    return false;
-                tc_fence_after();
-                return true;
-            };
-            auto wait_phase = [&](int which, int n) -> bool {
-                if (!mbar_wait(bar(which), static_cast<uint32_t>(n & 1), abort_flag)) return false;
-                tc_fence_after();
-                return true;
-            };
-            // S(n) = F0 T0(n)^T and dP(n) = F1 T1(n)^T, each 128 x 128 over K = D
-            auto issue_s = [&](int n) {
-                if (elect_one()) {
-                    mma_ss_run<D / 16>(tm_s, f0d, sdesc_sw128(t0_of(n), 16, 1024), idesc_s, 0u);
-                    mma_commit(bar(L::kBarSFull));
-                }
-                __syncwarp();
-            };
-            auto issue_dp = [&](int n) {
-                if (elect_one()) {
-                    mma_ss_run<D / 16>(tm_dp, f1d, sdesc_sw128(t0_of(n) + L::kTile, 16, 1024), idesc_s, 0u);
-                    mma_commit(bar(L::kBarDpFull));
-                }
-                __syncwarp();
-            };
-            // acc += A B over K = 128 rows of the streamed tile: A from TMEM columns
-            // a, a+8, ... in two runs (columns 0-31 hold tile rows 0-63, columns
-            // 64-95 rows 64-127), B MN-major from tile rows 0-63 and 64-127
-            auto issue_acc = [&](uint32_t acc, uint32_t a, uint32_t tile, bool first) {
-                mma_ts_run4(acc, a, sdesc_sw128(tile, 16384, 1024), idesc_acc, first ? 0u : 1u);
-                mma_ts_run4(acc, a + 64u, sdesc_sw128(tile + 8192u, 16384, 1024), idesc_acc, 1u);
-            };
-            bool ok = mbar_wait(bar(L::kBarFixed), 0, abort_flag) && wait_tiles(0);
-            if (ok) {
-                issue_s(0);
-                issue_dp(0);
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, false, true);
+        const uint64_t f0d = sdesc_sw128(sbase + L::kF0, 16, 1024);
+        const uint64_t f1d = sdesc_sw128(sbase + L::kF1, 16, 1024);
+        const uint32_t tm_s = tmem, tm_dp = tmem + 128u, tm_a0 = tmem + 256u, tm_a1 = tmem + 256u + D;
+        auto t0_of = [&](uint32_t g) -> uint32_t {  // streamed tile T0 of entry g (T1 one tile further)
+            return sbase + L::kStage + (g & 1u) * 2u * L::kTile;
+        };
+        auto wait_tiles = [&](uint32_t g) -> bool {
+            if (!mbar_wait(bar(L::kBarTFull + (g & 1u)), (g >> 1) & 1u, abort_flag)) return false;
+            tc_fence_after();
+            return true;
+        };
+        auto wait_phase = [&](int which, uint32_t parity) -> bool {
+            if (!mbar_wait(bar(which), parity & 1u, abort_flag)) return false;
+            tc_fence_after();
+            return true;
+        };
+        // S(g) = F0 T0(g)^T and dP(g) = F1 T1(g)^T, each 128 x 128 over K = D
+        auto issue_s = [&](uint32_t g) {
+            if (elect_one()) {
+                mma_ss_run<D / 16>(tm_s, f0d, sdesc_sw128(t0_of(g), 16, 1024), idesc_s, 0u);
+                mma_commit(bar(L::kBarSFull));
             }
-            for (int n = 0; n < T && ok; ++n) {
-                const uint32_t t0 = t0_of(n);
-                if constexpr (KVSIDE) {
-                    // dV(n) += P(n)^T dO(n), then S(n+1), then dK(n) += dS(n)^T Q(n), then dP(n+1)
-                    if (!(ok = wait_phase(L::kBarPFull, n))) break;
-                    if (elect_one()) issue_acc(tm_a0, tm_s, t0 + L::kTile, n == 0);
-                    __syncwarp();
-                    if (n + 1 < T) {
-                        if (!(ok = wait_tiles(n + 1))) break;
-                        issue_s(n + 1);
-                    }
-                    if (!(ok = wait_phase(L::kBarDsFull, n))) break;
-                    if (elect_one()) {
-                        issue_acc(tm_a1, tm_dp, t0, n == 0);
-                        mma_commit(bar(L::kBarTEmpty + (n & 1)));
-                    }
-                    __syncwarp();
-                } else {
-                    // S(n+1) once the P phase of n has read S(n), then dQ(n) += dS(n) K(n), then dP(n+1)
-                    if (n + 1 < T) {
-                        if (!(ok = wait_phase(L::kBarPFull, n) && wait_tiles(n + 1))) break;
-                        issue_s(n + 1);
-                    }
-                    if (!(ok = wait_phase(L::kBarDsFull, n))) break;
-                    if (elect_one()) {
-                        issue_acc(tm_a0, tm_dp, t0, n == 0);
-                        mma_commit(bar(L::kBarTEmpty + (n & 1)));
-                    }
-                    __syncwarp();
-                }
-                if (n + 1 < T) issue_dp(n + 1);
-            }
-            if (elect_one()) mma_commit(bar(L::kBarAcc));
             __syncwarp();
-            mbar_wait(bar(L::kBarAcc), 0, abort_flag);
+        };
+        auto issue_dp = [&](uint32_t g) {
+            if (elect_one()) {
+                mma_ss_run<D / 16>(tm_dp, f1d, sdesc_sw128(t0_of(g) + L::kTile, 16, 1024), idesc_s, 0u);
+                mma_commit(bar(L::kBarDpFull));
+            }
+            __syncwarp();
+        };
+        // acc += A B over K = 128 rows of the streamed tile: A from TMEM columns
+        // a, a+8, ... in two runs (columns 0-31 hold tile rows 0-63, columns
+        // 64-95 rows 64-127), B MN-major from tile rows 0-63 and 64-127
+        auto issue_acc = [&](uint32_t acc, uint32_t a, uint32_t tile, bool first) {
+            mma_ts_run4(acc, a, sdesc_sw128(tile, 16384, 1024), idesc_acc, first ? 0u : 1u);
+            mma_ts_run4(acc, a + 64u, sdesc_sw128(tile + 8192u, 16384, 1024), idesc_acc, 1u);
+        };
+        uint32_t ge = 0, units = 0;  // entries and units with entries so far
+        bool pend_p = false;         // the P phase of entry ge - 1 is not yet waited for
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+            const int buf = it & 1;
+            if (!mbar_wait(bar(L::kBarListFull + buf), static_cast<uint32_t>((it >> 1) & 1), abort_flag)) break;
+            const BwdUnit hdr = *hdr_of(buf);
+            if (hdr.T < 0) break;
+            const int T = hdr.T;
+            if (T > 0) {
+                // the unit's fixed tiles; S(first) overwrites S once the last P phase has read it
+                if (!(ok = wait_phase(L::kBarFixedFull, units))) break;
+                if (pend_p && !(ok = wait_phase(L::kBarPFull, ge - 1))) break;
+                if (!(ok = wait_tiles(ge))) break;
+                issue_s(ge);
+                issue_dp(ge);
+                if (T == 1 && elect_one()) mma_commit(bar(L::kBarFixedEmpty));
+                __syncwarp();
+                for (int n = 0; n < T && ok; ++n) {
+                    const uint32_t g = ge + n;
+                    const uint32_t t0 = t0_of(g);
+                    // The first accumulating product of a unit overwrites the
+                    // accumulators: the previous unit's epilogue must have read them.
+                    const bool acc_wait = n == 0 && units > 0;
+                    if constexpr (KVSIDE) {
+                        // dV(g) += P(g)^T dO(g), S(g+1), dK(g) += dS(g)^T Q(g), dP(g+1)
+                        if (!(ok = wait_phase(L::kBarPFull, g))) break;
+                        if (acc_wait && !(ok = wait_phase(L::kBarAccEmpty, units - 1))) break;
+                        if (elect_one()) issue_acc(tm_a0, tm_s, t0 + L::kTile, n == 0);
+                        __syncwarp();
+                        if (n + 1 < T) {
+                            if (!(ok = wait_tiles(g + 1))) break;
+                            issue_s(g + 1);
+                        }
+                        if (!(ok = wait_phase(L::kBarDsFull, g))) break;
+                        if (elect_one()) {
+                            issue_acc(tm_a1, tm_dp, t0, n == 0);
+                            mma_commit(bar(L::kBarTEmpty + (g & 1u)));
+                        }
+                        __syncwarp();
+                    } else {
+                        // S(g+1) once the P phase of g has read S(g), dQ(g) += dS(g) K(g), dP(g+1)
+                        if (n + 1 < T) {
+                            if (!(ok = wait_phase(L::kBarPFull, g) && wait_tiles(g + 1))) break;
+                            issue_s(g + 1);
+                        }
+                        if (!(ok = wait_phase(L::kBarDsFull, g))) break;
+                        if (acc_wait && !(ok = wait_phase(L::kBarAccEmpty, units - 1))) break;
+                        if (elect_one()) {
+                            issue_acc(tm_a0, tm_dp, t0, n == 0);
+                            mma_commit(bar(L::kBarTEmpty + (g & 1u)));
+                        }
+                        __syncwarp();
+                    }
+                    if (n + 1 < T) {
+                        issue_dp(g + 1);
+                        // the unit's last S and dP are issued: its fixed tiles may be replaced
+                        if (n + 2 == T && elect_one()) mma_commit(bar(L::kBarFixedEmpty));
+                        __syncwarp();
+                    }
+                }
+                if (!ok) break;
+                if (elect_one()) mma_commit(bar(L::kBarAccFull));
+                __syncwarp();
+                pend_p = !KVSIDE;  // the dq side does not wait for its last P phase
+                ge += T;
+                ++units;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::kBarListEmpty + buf));
         }
+        // every MMA of this warp must finish before TMEM is freed
+        if (elect_one()) mma_commit(bar(L::kBarDone));
+        __syncwarp();
+        mbar_wait(bar(L::kBarDone), 0, abort_flag);
     }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
@@ -590,220 +685,236 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_s = tmem + 64u * static_cast<uint32_t>(h) + lane_base;
         const uint32_t t_dp = t_s + 128u;
-        const int64_t row_idx = static_cast<int64_t>(blk) * 128 + r;  // this thread's kv (dk/dv) or q (dq)
-        const int db = dnf.doc_batch > 1 ? b : 0;
+        const int db_of = dnf.doc_batch > 1 ? 1 : 0;
         const bool masked_path = p.has_block_mask != 0;
-        // Per-row mask data, fixed for the unit: the key's document id (dk/dv) or
-        // the query's document span (dq). The term intervals are recomputed on
-        // each partial tile from the mask program (registers go to the tiles).
-        int32_t my_doc = 0;
-        bool my_doc_ok = false;
-        int64_t row_ds = 0, row_de = -1;
-        float2 nl_row = make_float2(-INFINITY, -INFINITY), nd_row = make_float2(0.f, 0.f);
-        float slope_unit = 0.f;
         constexpr bool kAlibi = SCORE == kScoreAlibi || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap;
-        if constexpr (KVSIDE) {
-            if (dnf.has_doc && masked_path && row_idx < p.N) {
-                my_doc = __ldg(dnf.kv_doc + static_cast<int64_t>(db) * p.N + row_idx);
-                my_doc_ok = true;
-            }
-        } else {
-            const float2 ldr = p.ld[static_cast<int64_t>(b * p.Hq + hq) * p.QB * 128 + row_idx];
-            nl_row = make_float2(ldr.x, ldr.x);
-            nd_row = make_float2(ldr.y, ldr.y);
-            if constexpr (kAlibi)
-                slope_unit = p.slopes ? __ldg(p.slopes + hq)
-                                      : exp2f(-8.0f * static_cast<float>(hq + 1) / static_cast<float>(p.Hq));
-            if (dnf.has_doc && masked_path) {
-                // the span [first, last] of kv positions with this row's document
-                // id (kv ids are non-decreasing); one warp search per distinct id
-                const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
-                const int32_t* kd_row = dnf.kv_doc + static_cast<int64_t>(db) * p.N;
-                const bool valid = row_idx < p.M;
-                const int32_t d = valid ? __ldg(qd_row + row_idx) : 0;
-                bool pending = valid;
-                unsigned todo;
-                while ((todo = __ballot_sync(0xFFFFFFFFu, pending)) != 0u) {
-                    const int32_t x = __shfl_sync(0xFFFFFFFFu, d, __ffs(todo) - 1);
-                    const int first = warp_lower_bound(kd_row, p.N, x, lane);
-                    const int past = warp_lower_bound(kd_row, p.N, static_cast<int64_t>(x) + 1, lane);
-                    if (pending && d == x) {
-                        row_ds = first;
-                        row_de = past - 1;
-                        pending = false;
+        const float2* ld_smem = reinterpret_cast<const float2*>(smem + L::kLd);
+        uint32_t ge = 0, units = 0;
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+            const int buf = it & 1;
+            if (!mbar_wait(bar(L::kBarListFull + buf), static_cast<uint32_t>((it >> 1) & 1), abort_flag)) break;
+            const BwdUnit hdr = *hdr_of(buf);
+            if (hdr.T < 0) break;
+            const uint32_t* entries = list_of(buf);
+            const int T = hdr.T;
+            const int b = hdr.b, hq = hdr.hq, hkv = hdr.hkv;
+            const int db = db_of ? b : 0;
+            const int64_t row_idx = static_cast<int64_t>(hdr.blk) * 128 + r;  // this thread's kv (dk/dv) or q (dq)
+            // Per-row data, fixed for the unit: the key's document id (dk/dv), or
+            // the query's -lse2, -delta and document span (dq). Term intervals
+            // are recomputed on each partial tile from the mask program.
+            int32_t my_doc = 0;
+            bool my_doc_ok = false;
+            int64_t row_ds = 0, row_de = -1;
+            float2 nl_row = make_float2(-INFINITY, -INFINITY), nd_row = make_float2(0.f, 0.f);
+            float slope_unit = 0.f;
+            if constexpr (KVSIDE) {
+                if (dnf.has_doc && masked_path && row_idx < p.N) {
+                    my_doc = __ldg(dnf.kv_doc + static_cast<int64_t>(db) * p.N + row_idx);
+                    my_doc_ok = true;
+                }
+            } else if (T > 0) {
+                const float2 ldr = p.ld[static_cast<int64_t>(b * p.Hq + hq) * p.QB * 128 + row_idx];
+                nl_row = make_float2(ldr.x, ldr.x);
+                nd_row = make_float2(ldr.y, ldr.y);
+                if constexpr (kAlibi)
+                    slope_unit = p.slopes ? __ldg(p.slopes + hq)
+                                          : exp2f(-8.0f * static_cast<float>(hq + 1) / static_cast<float>(p.Hq));
+                if (dnf.has_doc && masked_path) {
+                    // the span [first, last] of kv positions with this row's document
+                    // id (kv ids are non-decreasing); one warp search per distinct id
+                    const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
+                    const int32_t* kd_row = dnf.kv_doc + static_cast<int64_t>(db) * p.N;
+                    const bool valid = row_idx < p.M;
+                    const int32_t d = valid ? __ldg(qd_row + row_idx) : 0;
+                    bool pending = valid;
+                    unsigned todo;
+                    while ((todo = __ballot_sync(0xFFFFFFFFu, pending)) != 0u) {
+                        const int32_t x = __shfl_sync(0xFFFFFFFFu, d, __ffs(todo) - 1);
+                        const int first = warp_lower_bound(kd_row, p.N, x, lane);
+                        const int past = warp_lower_bound(kd_row, p.N, static_cast<int64_t>(x) + 1, lane);
+                        if (pending && d == x) {
+                            row_ds = first;
+                            row_de = past - 1;
+                            pending = false;
+                        }
                     }
                 }
             }
-        }
-        const float2* ld_smem = reinterpret_cast<const float2*>(smem + L::kLd);
-
-        bool ok = true;
-        for (int e = 0; e < T && ok; ++e) {
-            const uint32_t ent = entries[e];
-            const int eb = static_cast<int>(ent & 0xFFFFu);
-            const int g = static_cast<int>((ent >> 16) & 0xFFu);
-            const bool partial = (ent & kBwdPartial) != 0u;
-            const int64_t c0 = static_cast<int64_t>(eb) * 128 + 64 * h;  // first column (q or kv) of this warpgroup
-            // mask words over the warpgroup's 64 columns (bit j: column c0 + j allowed)
-            uint32_t w0 = 0xFFFFFFFFu, w1 = 0xFFFFFFFFu;
-            if (partial) {
-                w0 = 0u;
-                w1 = 0u;
-                if constexpr (KVSIDE) {
-                    uint32_t d0 = 0xFFFFFFFFu, d1 = 0xFFFFFFFFu;
-                    if (dnf.term_has_doc) {
-                        d0 = 0u;
-                        d1 = 0u;
-                        if (my_doc_ok) {
-                            const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
+            for (int n = 0; n < T && ok; ++n) {
+                const uint32_t g_ent = ge + n;
+                const uint32_t ent = entries[n];
+                const int eb = static_cast<int>(ent & 0xFFFFu);
+                const int g = static_cast<int>((ent >> 16) & 0xFFu);
+                const bool partial = (ent & kBwdPartial) != 0u;
+                const int64_t c0 = static_cast<int64_t>(eb) * 128 + 64 * h;  // first column (q or kv) of this warpgroup
+                // mask words over the warpgroup's 64 columns (bit j: column c0 + j allowed)
+                uint32_t w0 = 0xFFFFFFFFu, w1 = 0xFFFFFFFFu;
+                if (partial) {
+                    w0 = 0u;
+                    w1 = 0u;
+                    if constexpr (KVSIDE) {
+                        uint32_t d0 = 0xFFFFFFFFu, d1 = 0xFFFFFFFFu;
+                        if (dnf.term_has_doc) {
+                            d0 = 0u;
+                            d1 = 0u;
+                            if (my_doc_ok) {
+                                const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
 #pragma unroll 8
-                            for (int j = 0; j < 64; ++j) {
-                                const int64_t q = c0 + j;
-                                const bool m = q < p.M && __ldg(qd_row + q) == my_doc;
-                                if (j < 32) d0 |= (m ? 1u : 0u) << j;
-                                else d1 |= (m ? 1u : 0u) << (j - 32);
+                                for (int j = 0; j < 64; ++j) {
+                                    const int64_t q = c0 + j;
+                                    const bool m = q < p.M && __ldg(qd_row + q) == my_doc;
+                                    if (j < 32) d0 |= (m ? 1u : 0u) << j;
+                                    else d1 |= (m ? 1u : 0u) << (j - 32);
+                                }
                             }
                         }
-                    }
-                    if (row_idx < p.N) {
-                        for (int t = 0; t < dnf.n_terms; ++t) {
-                            int64_t lo, hi;
-                            term_q_interval(dnf, t, row_idx, p.M, lo, hi);
-                            uint32_t a0 = range_bits(lo, hi, c0);
-                            uint32_t a1 = range_bits(lo, hi, c0 + 32);
-                            if ((dnf.term_has_doc >> t) & 1u) {
-                                a0 &= d0;
-                                a1 &= d1;
+                        if (row_idx < p.N) {
+                            for (int t = 0; t < dnf.n_terms; ++t) {
+                                int64_t lo, hi;
+                                term_q_interval(dnf, t, row_idx, p.M, lo, hi);
+                                uint32_t a0 = range_bits(lo, hi, c0);
+                                uint32_t a1 = range_bits(lo, hi, c0 + 32);
+                                if ((dnf.term_has_doc >> t) & 1u) {
+                                    a0 &= d0;
+                                    a1 &= d1;
+                                }
+                                w0 |= a0;
+                                w1 |= a1;
                             }
-                            w0 |= a0;
-                            w1 |= a1;
-                        }
-                    }
-                } else {
-                    const int64_t c1 = (c0 + 63 < p.N - 1) ? c0 + 63 : p.N - 1;
-                    if (masked_path) {
-                        for (int t = 0; t < dnf.n_terms; ++t) {
-                            int64_t lo, hi;
-                            term_interval(dnf, t, row_idx, c0, c1, row_ds, row_de, lo, hi);
-                            w0 |= range_bits(lo, hi, c0);
-                            w1 |= range_bits(lo, hi, c0 + 32);
                         }
                     } else {
-                        w0 = range_bits(c0, c1, c0);
-                        w1 = range_bits(c0, c1, c0 + 32);
+                        const int64_t c1 = (c0 + 63 < p.N - 1) ? c0 + 63 : p.N - 1;
+                        if (masked_path) {
+                            for (int t = 0; t < dnf.n_terms; ++t) {
+                                int64_t lo, hi;
+                                term_interval(dnf, t, row_idx, c0, c1, row_ds, row_de, lo, hi);
+                                w0 |= range_bits(lo, hi, c0);
+                                w1 |= range_bits(lo, hi, c0 + 32);
+                            }
+                        } else {
+                            w0 = range_bits(c0, c1, c0);
+                            w1 = range_bits(c0, c1, c0 + 32);
+                        }
                     }
                 }
-            }
-            float slope = slope_unit;
-            if constexpr (KVSIDE && kAlibi)
-                slope = p.slopes ? __ldg(p.slopes + hq + g)
-                                 : exp2f(-8.0f * static_cast<float>(hq + g + 1) / static_cast<float>(p.Hq));
-            // kv - q at the warpgroup's column 0; it moves by -1 (dk/dv) or +1 (dq) per column
-            const float dkv0 = KVSIDE ? static_cast<float>(row_idx - c0) : static_cast<float>(c0 - row_idx);
-            constexpr float kStep = KVSIDE ? -1.f : 1.f;
-            BwdCols hb;
-            if constexpr (SCORE == kScoreAlibiSoftcap) {
-                hb.bias0 = slope * dkv0;
-                hb.bstep = slope * kStep;
-            } else {
-                hb.bias0 = slope * kLog2e * dkv0;
-                hb.bstep = slope * kLog2e * kStep;
-            }
-
-            const float4* ld4 = reinterpret_cast<const float4*>(ld_smem + 128 * (e & 1) + 64 * h);
-            float pg[64];  // P * dz/ds of this thread's 64 columns, from the P phase to the dS phase
-            // ---- P phase: S -> P (bf16 into TMEM for dV on the dk/dv side)
-            if (!mbar_wait(bar(L::kBarSFull), static_cast<uint32_t>(e & 1), abort_flag)) {
-                ok = false;
-                break;
-            }
-            __syncwarp();  // tcgen05.ld/st are warp-collective: reconverge after the wait
-            tc_fence_after();
-            {
-                float x[64];
-                tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(x));
-                tmem_ld32(t_s + 32u, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-                tc_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t pk[16];
-                    if (partial)
-                        bwd_p_chunk<SCORE, KVSIDE, true>(p, x, ld4, nl_row, hb, 32 * c, c == 0 ? w0 : w1, pg, pk);
-                    else
-                        bwd_p_chunk<SCORE, KVSIDE, false>(p, x, ld4, nl_row, hb, 32 * c, 0u, pg, pk);
-                    if constexpr (KVSIDE) tmem_st16(t_s + 16u * c, pk);
-                }
-            }
-            if constexpr (KVSIDE) tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::kBarPFull));
-            // ---- dS phase: dP -> dS (bf16 into TMEM for dK or dQ)
-            if (!mbar_wait(bar(L::kBarDpFull), static_cast<uint32_t>(e & 1), abort_flag)) {
-                ok = false;
-                break;
-            }
-            __syncwarp();
-            tc_fence_after();
-            {
-                float dp[64];
-                tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dp));
-                tmem_ld32(t_dp + 32u, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
-                tc_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t dk[16];
-                    bwd_ds_chunk<KVSIDE>(dp, ld4, nd_row, pg, 32 * c, dk);
-                    tmem_st16(t_dp + 16u * c, dk);
-                }
-            }
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::kBarDsFull));
-        }
-        // ------------------------------------------------------ epilogue
-        // dk/dv: warpgroup 0 writes dV, warpgroup 1 writes dK (times scale).
-        // dq: warpgroup h writes columns [h D/2, (h+1) D/2) of dQ (times scale).
-        if (ok && T > 0) ok = mbar_wait(bar(L::kBarAcc), 0, abort_flag);
-        __syncwarp();
-        tc_fence_after();
-        if (ok) {
-            constexpr int kCols = KVSIDE ? D : D / 2;
-            const int64_t rows = KVSIDE ? p.N : p.M;
-            const bool valid = row_idx < rows;
-            __nv_bfloat16* dst;
-            uint32_t src;
-            float mul;
-            if constexpr (KVSIDE) {
-                dst = (h == 0 ? p.g1 : p.g0) + (static_cast<int64_t>(b * p.Hkv + hkv) * p.N + row_idx) * D;
-                src = tmem + 256u + (h == 0 ? 0u : static_cast<uint32_t>(D)) + lane_base;
-                mul = h == 0 ? 1.f : p.scale;
-            } else {
-                dst = p.g0 + (static_cast<int64_t>(b * p.Hq + hq) * p.M + row_idx) * D + h * (D / 2);
-                src = tmem + 256u + static_cast<uint32_t>(h * (D / 2)) + lane_base;
-                mul = p.scale;
-            }
-#pragma unroll
-            for (int c = 0; c < kCols / 32; ++c) {
-                uint32_t a[32];
-                if (T > 0) {
-                    tmem_ld32(src + 32u * c, a);
-                    tc_wait_ld();
+                float slope = slope_unit;
+                if constexpr (KVSIDE && kAlibi)
+                    slope = p.slopes ? __ldg(p.slopes + hq + g)
+                                     : exp2f(-8.0f * static_cast<float>(hq + g + 1) / static_cast<float>(p.Hq));
+                // kv - q at the warpgroup's column 0; it moves by -1 (dk/dv) or +1 (dq) per column
+                const float dkv0 = KVSIDE ? static_cast<float>(row_idx - c0) : static_cast<float>(c0 - row_idx);
+                constexpr float kStep = KVSIDE ? -1.f : 1.f;
+                BwdCols hb;
+                if constexpr (SCORE == kScoreAlibiSoftcap) {
+                    hb.bias0 = slope * dkv0;
+                    hb.bstep = slope * kStep;
                 } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) a[j] = 0u;
+                    hb.bias0 = slope * kLog2e * dkv0;
+                    hb.bstep = slope * kLog2e * kStep;
                 }
-                uint32_t pk[16];
+                const float4* ld4 = reinterpret_cast<const float4*>(ld_smem + 128 * (g_ent & 1u) + 64 * h);
+                float pg[64];  // P * dz/ds of this thread's 64 columns, from the P phase to the dS phase
+                // ---- P phase: S -> P (bf16 into TMEM for dV on the dk/dv side)
+                if (!mbar_wait(bar(L::kBarSFull), g_ent & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                __syncwarp();  // tcgen05.ld/st are warp-collective: reconverge after the wait
+                tc_fence_after();
+                {
+                    float x[64];
+                    tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(x));
+                    tmem_ld32(t_s + 32u, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+                    tc_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    pk[j] = pack_bf16x2(__uint_as_float(a[2 * j]) * mul, __uint_as_float(a[2 * j + 1]) * mul);
-                if (valid) {
-                    uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t pk[16];
+                        if (partial)
+                            bwd_p_chunk<SCORE, KVSIDE, true>(p, x, ld4, nl_row, hb, 32 * c, c == 0 ? w0 : w1, pg, pk);
+                        else
+                            bwd_p_chunk<SCORE, KVSIDE, false>(p, x, ld4, nl_row, hb, 32 * c, 0u, pg, pk);
+                        if constexpr (KVSIDE) tmem_st16(t_s + 16u * c, pk);
+                    }
+                }
+                if constexpr (KVSIDE) tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::kBarPFull));
+                // ---- dS phase: dP -> dS (bf16 into TMEM for dK or dQ)
+                if (!mbar_wait(bar(L::kBarDpFull), g_ent & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                __syncwarp();
+                tc_fence_after();
+                {
+                    float dp[64];
+                    tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dp));
+                    tmem_ld32(t_dp + 32u, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
+                    tc_wait_ld();
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) d4[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t dk[16];
+                        bwd_ds_chunk<KVSIDE>(dp, ld4, nd_row, pg, 32 * c, dk);
+                        tmem_st16(t_dp + 16u * c, dk);
+                    }
+                }
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::kBarDsFull));
+            }
+            if (!ok) break;
+            ge += T;
+            // -------------------------------------------------- epilogue
+            // dk/dv: warpgroup 0 writes dV, warpgroup 1 writes dK (times scale).
+            // dq: warpgroup h writes columns [h D/2, (h+1) D/2) of dQ (times
+            // scale). The accumulator is read whole and released before the
+            // stores, so that the next unit's products can start.
+            constexpr int kCols = KVSIDE ? D : D / 2;
+            uint32_t a[kCols];
+            if (T > 0) {
+                if (!(ok = mbar_wait(bar(L::kBarAccFull), units & 1u, abort_flag))) break;
+                ++units;
+                __syncwarp();
+                tc_fence_after();
+                const uint32_t src = tmem + 256u + (KVSIDE ? (h == 0 ? 0u : static_cast<uint32_t>(D))
+                                                           : static_cast<uint32_t>(h * (D / 2))) + lane_base;
+#pragma unroll
+                for (int c = 0; c < kCols / 32; ++c) tmem_ld32(src + 32u * c, *reinterpret_cast<uint32_t(*)[32]>(a + 32 * c));
+                tc_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::kBarAccEmpty));
+            } else {
+#pragma unroll
+                for (int j = 0; j < kCols; ++j) a[j] = 0u;
+            }
+            const int64_t rows = KVSIDE ? p.N : p.M;
+            if (row_idx < rows) {
+                __nv_bfloat16* dst;
+                float mul;
+                if constexpr (KVSIDE) {
+                    dst = (h == 0 ? p.g1 : p.g0) + (static_cast<int64_t>(b * p.Hkv + hkv) * p.N + row_idx) * D;
+                    mul = h == 0 ? 1.f : p.scale;
+                } else {
+                    dst = p.g0 + (static_cast<int64_t>(b * p.Hq + hq) * p.M + row_idx) * D + h * (D / 2);
+                    mul = p.scale;
+                }
+                uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+                for (int v = 0; v < kCols / 8; ++v) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        pk[k] = pack_bf16x2(__uint_as_float(a[8 * v + 2 * k]) * mul, __uint_as_float(a[8 * v + 2 * k + 1]) * mul);
+                    d4[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(L::kBarListEmpty + buf));
         }
     }
 

@@ -808,7 +808,11 @@ bsmt_status launch_bwd(int dev, const CUtensorMap& tq, const CUtensorMap& tk, co
             g_bwd_attr_set[dev][slot] = true;
         }
     }
-    kern<<<static_cast<unsigned>(p.num_units), bsmt::kBwdThreads, smem, s>>>(tq, tk, tv, tdo, p, dnf);
+    int nsm = 0;
+    cudaError_t ea = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (ea != cudaSuccess) return fail(BSMT_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(ea));
+    const int grid = p.num_units < nsm ? p.num_units : nsm;  // persistent: units come from a work counter
+    kern<<<static_cast<unsigned>(grid), bsmt::kBwdThreads, smem, s>>>(tq, tk, tv, tdo, p, dnf);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
     return BSMT_OK;
@@ -828,7 +832,10 @@ bsmt_status launch_bwd_score(int mode, int dev, const CUtensorMap& tq, const CUt
     }
 }
 
-int64_t bwd_ws_bytes(int64_t B, int64_t Hq, int64_t M) { return B * Hq * ((M + 127) / 128) * 128 * 8; }
+// Workspace of the backward: (-lse2, -delta) per padded query row, then the
+// two kernels' work counters at the next 256-byte boundary.
+int64_t bwd_ld_bytes(int64_t B, int64_t Hq, int64_t M) { return (B * Hq * ((M + 127) / 128) * 128 * 8 + 255) / 256 * 256; }
+int64_t bwd_ws_bytes(int64_t B, int64_t Hq, int64_t M) { return bwd_ld_bytes(B, Hq, M) + 256; }
 }  // namespace
 
 extern "C" bsmt_status bsmt_flex_attention_bwd_workspace_bytes(int64_t B, int64_t Hq, int64_t M, int64_t* bytes) {
@@ -944,19 +951,20 @@ extern "C" bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, con
     if (N == 0) return (st = zero_bf16(dq, B * Hq * M * D, nsm, s)) != BSMT_OK ? st : ok();
     if (B * Hkv * KB > 0x7FFFFFFF || B * Hq * QB > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "too many work units");
 
-    // (lse2, delta) per padded query row
+    // (-lse2, -delta) per padded query row, and the work counters
     float2* ld = static_cast<float2*>(workspace);
+    int32_t* counters = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + bwd_ld_bytes(B, Hq, M));
     const int64_t rows_pad = B * Hq * QB * 128;
     const int64_t prep_blocks = (rows_pad + 8 * bsmt::kPrepRowsPerWarp - 1) / (8 * bsmt::kPrepRowsPerWarp);
     if (prep_blocks > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "too many query rows");
     if (D == 128)
         bsmt::bwd_prep_kernel<128><<<static_cast<unsigned>(prep_blocks), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, rows_pad,
-            static_cast<int32_t>(M), static_cast<int32_t>(QB), ld);
+            static_cast<int32_t>(M), static_cast<int32_t>(QB), ld, counters);
     else
         bsmt::bwd_prep_kernel<64><<<static_cast<unsigned>(prep_blocks), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, rows_pad,
-            static_cast<int32_t>(M), static_cast<int32_t>(QB), ld);
+            static_cast<int32_t>(M), static_cast<int32_t>(QB), ld, counters);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "backward prep launch: %s", cudaGetErrorString(e));
 
@@ -988,10 +996,12 @@ extern "C" bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, con
     pk.g0 = static_cast<__nv_bfloat16*>(dk);
     pk.g1 = static_cast<__nv_bfloat16*>(dv);
     pk.num_units = static_cast<int32_t>(B * Hkv * KB);
+    pk.next_unit = counters;
     pq.list_rows = static_cast<int32_t>(QB);
     pq.list_len = static_cast<int32_t>(KB);
     pq.g0 = static_cast<__nv_bfloat16*>(dq);
     pq.num_units = static_cast<int32_t>(B * Hq * QB);
+    pq.next_unit = counters + 1;
     st = D == 128 ? launch_bwd_score<128, true>(mode, dev, tq, tk, tv, tdo, pk, dnf, s)
                   : launch_bwd_score<64, true>(mode, dev, tq, tk, tv, tdo, pk, dnf, s);
     if (st != BSMT_OK) return st;

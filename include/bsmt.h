@@ -349,8 +349,9 @@ bsmt_status bsmt_flex_attention_fwd_packed(const void* q, const void* k, const v
  * backward for the same layouts).
  *
  * bsmt_flex_attention_bwd_workspace_bytes gives the workspace size:
- * 8 * B * Hq * ceil(M / 128) * 128 bytes (lse and delta per query row).
- * Host-only; launches nothing. */
+ * 8 * B * Hq * ceil(M / 128) * 128 bytes (lse and delta per query row),
+ * rounded up to 256, plus 256 bytes of work counters. Host-only; launches
+ * nothing. */
 bsmt_status bsmt_flex_attention_bwd_workspace_bytes(int64_t B, int64_t Hq, int64_t M, int64_t* bytes);
 
 /* Arguments:
@@ -368,8 +369,9 @@ bsmt_status bsmt_flex_attention_bwd_workspace_bytes(int64_t B, int64_t Hq, int64
  *   workspace  caller-owned device memory, 256-byte aligned, at least
  *           bsmt_flex_attention_bwd_workspace_bytes bytes; written and read
  *           back by the call, reusable once the stream has passed it
- * Limits: ceil(N/128) <= 4096 and (Hq/Hkv) * ceil(M/128) <= 4096, else
- * BSMT_ERR_UNSUPPORTED. Bad list entries are skipped and reported as
+ * Limits: ceil(N/128) <= 2048 and (Hq/Hkv) * ceil(M/128) <= 2048, else
+ * BSMT_ERR_UNSUPPORTED. Calls that share a workspace must not overlap in
+ * time (it holds the kernels' work counters). Bad list entries are skipped and reported as
  * BSMT_ERR_DEVICE_BOUNDS. Stream-ordered on `stream`. */
 bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                                     const float* lse, int64_t B, int64_t Hq, int64_t Hkv, int64_t M, int64_t N,
