@@ -824,12 +824,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 __syncwarp();  // tcgen05.ld/st are warp-collective: reconverge after the wait
                 tc_fence_after();
                 {
+                    // the second 32 columns load while the first are computed
                     float x[64];
                     tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(x));
-                    tmem_ld32(t_s + 32u, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
                     tc_wait_ld();
+                    tmem_ld32(t_s + 32u, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
+                        if (c == 1) tc_wait_ld();
                         uint32_t pk[16];
                         if (partial)
                             bwd_p_chunk<SCORE, KVSIDE, true>(p, x, ld4, nl_row, hb, 32 * c, c == 0 ? w0 : w1, pg, pk);
@@ -852,10 +854,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 {
                     float dp[64];
                     tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dp));
-                    tmem_ld32(t_dp + 32u, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
                     tc_wait_ld();
+                    tmem_ld32(t_dp + 32u, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
+                        if (c == 1) tc_wait_ld();
                         uint32_t dk[16];
                         bwd_ds_chunk<KVSIDE>(dp, ld4, nd_row, pg, 32 * c, dk);
                         tmem_st16(t_dp + 16u * c, dk);
