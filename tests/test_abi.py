@@ -272,3 +272,55 @@ def test_varlen_argument_errors():
              null) == SHAPE  # Hq not a multiple of Hkv
     assert f(FAKE, FAKE, FAKE, 4, 4, 128, 128, 80, None, None, None, ctypes.c_float(0.0), 0, FAKE, FAKE,
              null) == UNSUPPORTED
+
+
+def bwd(B=1, Hq=2, Hkv=2, M=256, N=256, D=64, bm=None, bmq=None, spec=None, score=None, scale=0.0, gqa=0,
+        ptr=FAKE, lse=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    return _lib.bsmt_flex_attention_bwd(ptr, ptr, ptr, ptr, ptr, lse, B, Hq, Hkv, M, N, D, bm, bmq, spec, score,
+                                        ctypes.c_float(scale), gqa, ptr, ptr, ptr, ws, ws_bytes, None)
+
+
+def bwd_ws(B, Hq, M):
+    n = ctypes.c_int64(0)
+    assert _lib.bsmt_flex_attention_bwd_workspace_bytes(B, Hq, M, ctypes.byref(n)) == OK
+    return n.value
+
+
+def test_backward_workspace_bytes():
+    # 8 bytes per padded query row, rounded to 256, plus 256 bytes of counters
+    assert bwd_ws(2, 32, 32768) == 2 * 32 * 32768 * 8 + 256
+    assert bwd_ws(1, 1, 1) == 128 * 8 + 256
+    assert bwd_ws(1, 3, 0) == 256
+    assert _lib.bsmt_flex_attention_bwd_workspace_bytes(1, 1, 1, None) == INVALID
+    assert _lib.bsmt_flex_attention_bwd_workspace_bytes(-1, 1, 1, ctypes.byref(ctypes.c_int64())) == INVALID
+
+
+def test_backward_argument_errors():
+    """Every check of the backward entry point runs on the host before any
+    CUDA call, so these need no GPU."""
+    assert bwd(D=96) == UNSUPPORTED
+    assert bwd(Hq=3, Hkv=2, gqa=1) == SHAPE
+    assert bwd(Hq=4, Hkv=2, gqa=0) == SHAPE
+    assert bwd(M=-1) == INVALID
+    assert bwd(ptr=FAKE + 8) == INVALID                      # misaligned tensors
+    assert bwd(lse=FAKE + 2) == INVALID
+    assert bwd(scale=float("nan")) == INVALID
+    assert bwd(N=2049 * 128) == UNSUPPORTED                  # more than 2048 kv blocks per dq row
+    assert bwd(Hq=8, Hkv=1, gqa=1, M=257 * 128) == UNSUPPORTED  # 8 heads x 257 q-blocks > 2048 entries
+    # a block mask without its q-side lists
+    c = _BlockMask()
+    c.kv_num_blocks = c.kv_indices = c.full_kv_num_blocks = c.full_kv_indices = FAKE
+    c.B, c.H, c.QB, c.KB, c.Q_LEN, c.KV_LEN, c.BLOCK_Q, c.BLOCK_KV = 1, 1, 2, 2, 256, 256, 128, 128
+    assert bwd(bm=ctypes.byref(c), spec=ctypes.byref(spec_of([(C, 0)]))) == INVALID
+    assert "q-side" in _lib.bsmt_last_error().decode()
+    cq = bsmt._BlockMaskQ()
+    cq.q_num_blocks = cq.q_indices = cq.full_q_num_blocks = cq.full_q_indices = FAKE
+    c.QB = 3  # shape fields that disagree with M
+    assert bwd(bm=ctypes.byref(c), bmq=ctypes.byref(cq), spec=ctypes.byref(spec_of([(C, 0)]))) == SHAPE
+    # a workspace that is too small or misaligned (checked before any launch)
+    c.QB = 2
+    assert bwd(bm=ctypes.byref(c), bmq=ctypes.byref(cq), spec=ctypes.byref(spec_of([(C, 0)])), ws_bytes=100) == INVALID
+    assert bwd(ws=FAKE + 16) == INVALID
+    # nothing to compute: no work and no CUDA call
+    assert bwd(B=0) == OK
+    assert bwd(M=0, N=0) == OK
