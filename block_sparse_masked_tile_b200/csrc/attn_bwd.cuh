@@ -877,7 +877,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // scale). The accumulator is read whole and released before the
             // stores, so that the next unit's products can start.
             constexpr int kCols = KVSIDE ? D : D / 2;
-            uint32_t a[kCols];
+            constexpr int kBatch = kCols < 64 ? kCols : 64;  // columns read, packed and stored at a time
+            const bool valid = row_idx < (KVSIDE ? p.N : p.M);
+            const float mul = (KVSIDE && h == 0) ? 1.f : p.scale;
+            __nv_bfloat16* dst;
+            if constexpr (KVSIDE)
+                dst = (h == 0 ? p.g1 : p.g0) + (static_cast<int64_t>(b * p.Hkv + hkv) * p.N + row_idx) * D;
+            else
+                dst = p.g0 + (static_cast<int64_t>(b * p.Hq + hq) * p.M + row_idx) * D + h * (D / 2);
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
             if (T > 0) {
                 if (!(ok = mbar_wait(bar(L::kBarAccFull), units & 1u, abort_flag))) break;
                 ++units;
@@ -886,35 +894,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const uint32_t src = tmem + 256u + (KVSIDE ? (h == 0 ? 0u : static_cast<uint32_t>(D))
                                                            : static_cast<uint32_t>(h * (D / 2))) + lane_base;
 #pragma unroll
-                for (int c = 0; c < kCols / 32; ++c) tmem_ld32(src + 32u * c, *reinterpret_cast<uint32_t(*)[32]>(a + 32 * c));
-                tc_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(L::kBarAccEmpty));
-            } else {
+                for (int c0 = 0; c0 < kCols; c0 += kBatch) {
+                    uint32_t a[kBatch];
 #pragma unroll
-                for (int j = 0; j < kCols; ++j) a[j] = 0u;
-            }
-            const int64_t rows = KVSIDE ? p.N : p.M;
-            if (row_idx < rows) {
-                __nv_bfloat16* dst;
-                float mul;
-                if constexpr (KVSIDE) {
-                    dst = (h == 0 ? p.g1 : p.g0) + (static_cast<int64_t>(b * p.Hkv + hkv) * p.N + row_idx) * D;
-                    mul = h == 0 ? 1.f : p.scale;
-                } else {
-                    dst = p.g0 + (static_cast<int64_t>(b * p.Hq + hq) * p.M + row_idx) * D + h * (D / 2);
-                    mul = p.scale;
+                    for (int c = 0; c < kBatch / 32; ++c)
+                        tmem_ld32(src + static_cast<uint32_t>(c0 + 32 * c), *reinterpret_cast<uint32_t(*)[32]>(a + 32 * c));
+                    tc_wait_ld();
+                    if (c0 + kBatch == kCols) {
+                        // the whole accumulator is in registers: the next unit may overwrite it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(L::kBarAccEmpty));
+                    }
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < kBatch / 8; ++v) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                pk[k] = pack_bf16x2(__uint_as_float(a[8 * v + 2 * k]) * mul,
+                                                    __uint_as_float(a[8 * v + 2 * k + 1]) * mul);
+                            d4[c0 / 8 + v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
                 }
-                uint4* d4 = reinterpret_cast<uint4*>(dst);
+            } else if (valid) {
 #pragma unroll
-                for (int v = 0; v < kCols / 8; ++v) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        pk[k] = pack_bf16x2(__uint_as_float(a[8 * v + 2 * k]) * mul, __uint_as_float(a[8 * v + 2 * k + 1]) * mul);
-                    d4[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
+                for (int v = 0; v < kCols / 8; ++v) d4[v] = make_uint4(0u, 0u, 0u, 0u);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarListEmpty + buf));
