@@ -93,6 +93,10 @@ constexpr int kBwdWarpMma = 9;
 constexpr int kBwdWarpSched = 10;
 constexpr int kBwdMaxEntries = 2048;  // entries of one unit (list length x GQA group)
 constexpr uint32_t kBwdPartial = 0x80000000u;
+// Columns of every 32-column chunk of a full tile whose 2^x the P phase takes
+// on the FMA pipe (exp2_poly2) instead of MUFU. 8 measured faster than 16 on
+// B200 (the phase is bound by latency more than by MUFU).
+constexpr int kBwdEmuCols = 8;
 
 // A scheduled unit in shared memory (two buffers, filled by the scheduler warp).
 struct BwdUnit {
@@ -197,7 +201,7 @@ __device__ __forceinline__ void bwd_p_chunk(const BwdParams& p, const float* x, 
             if (!((w >> (2 * jj)) & 1u)) A.x = -INFINITY;
             if (!((w >> (2 * jj + 1)) & 1u)) A.y = -INFINITY;
             P = make_float2(ex2_approx(A.x), ex2_approx(A.y));
-        } else if (2 * jj < 8) {
+        } else if (2 * jj < kBwdEmuCols) {
             // (an A of -inf only comes from rows past the end of the sequence
             // here, whose dO and dP rows are zero; 2^-125 there adds nothing)
             exp2_poly2(P.x, P.y, A.x, A.y);
