@@ -274,6 +274,19 @@ def side_kernels(bsmt, mask, w, dev, hbm_peak: float) -> dict:
     res["varlen_doc_causal"] = {"shape": f"{len(lens)} packed sequences, {T} tokens, H=32, D=128, causal",
                                 "ms": msv, "tflops": vflops / (msv * 1e-3) / 1e12,
                                 "note": "includes doc-id and block-mask kernels per call"}
+    # the same forward kernel on long rows of full tiles (no mask) and causal
+    long_rows = []
+    for (Bl, Hl, Sl, Dl, causal_l) in ((1, 32, 8192, 128, False), (1, 32, 8192, 128, True)):
+        ql, kl, vl = (torch.randn((Bl, Hl, Sl, Dl), generator=g).to(torch.bfloat16).to(dev) for _ in range(3))
+        bml = bsmt.create_block_mask(bsmt.causal(), Bl, Hl, Sl, Sl, device=dev) if causal_l else None
+        tiles = (int(bml.kv_num_blocks.sum()) + int(bml.full_kv_num_blocks.sum())) if causal_l \
+            else Bl * Hl * ((Sl + 127) // 128) ** 2
+        msl = _time_launches(lambda: bsmt.flex_attention(ql, kl, vl, block_mask=bml), reps=5)
+        long_rows.append({"shape": f"B={Bl} H={Hl} S={Sl} D={Dl}", "mask": "causal" if causal_l else "none",
+                          "ms": msl, "tflops": tiles * 4 * 128 * 128 * Dl / (msl * 1e-3) / 1e12})
+        del ql, kl, vl
+    bsmt.check_device_status(dev)
+    res["long_rows"] = long_rows
     res["splitkv_decode"] = {"shape": f"B={Bd} Hq={Hqd} Hkv={Hkvd} M={Md} N={Nd} D={Dd}, no mask", "splits": S,
                              "plain_ms": ms1, "plain_tflops": flops / (ms1 * 1e-3) / 1e12,
                              "split_ms": mss, "split_tflops": flops / (mss * 1e-3) / 1e12}
