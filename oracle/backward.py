@@ -154,3 +154,31 @@ def backward_dkv_sampled(q, k, v, dout, samples, mask=None, score_mods=(), scale
                 dks[i] += gk[j]
                 dvs[i] += gv[j]
     return dks, dvs
+
+
+def flex_attention_varlen_backward(q, k, v, dout, cu_q, cu_k, causal=False, score_mods=(), scale=None,
+                                   enable_gqa=False):
+    """Gradients (dq [total_q, Hq, D], dk, dv [total_k, Hkv, D]) of
+    sum(out * dout) for the packed variable-length attention of
+    ``oracle.attention.flex_attention_varlen``. Each sequence is an
+    independent plain attention, so its gradients are flex_attention_backward
+    of its own tokens on a [1, H, L, D] view; tokens outside every sequence
+    get zero gradients."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    cu_q = [int(x) for x in cu_q]
+    cu_k = [int(x) for x in cu_k]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for i in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[i], cu_q[i + 1], cu_k[i], cu_k[i + 1]
+        if q1 <= q0 or k1 <= k0:
+            continue
+        view = lambda x, a, b: x[a:b].transpose(1, 0, 2)[None]  # noqa: E731
+        gq, gk, gv = flex_attention_backward(view(q, q0, q1), view(k, k0, k1), view(v, k0, k1),
+                                             view(dout, q0, q1), ("causal",) if causal else None, score_mods,
+                                             scale, enable_gqa)
+        dq[q0:q1] = gq[0].transpose(1, 0, 2)
+        dk[k0:k1] = gk[0].transpose(1, 0, 2)
+        dv[k0:k1] = gv[0].transpose(1, 0, 2)
+    return dq, dk, dv

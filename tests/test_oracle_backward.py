@@ -131,3 +131,35 @@ def test_sampled_equals_full():
     gk, gv = ob.backward_dkv_sampled(q, k, v, dout, ks, mask, mods, None, row_chunk=7)
     np.testing.assert_allclose(gk, np.stack([dk[s] for s in ks]), rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(gv, np.stack([dv[s] for s in ks]), rtol=1e-12, atol=1e-13)
+
+
+def test_varlen_backward_equals_document_mask_form():
+    """Packed sequences: the per-sequence backward equals the backward of the
+    whole pack under the document mask (and causal when asked), which is the
+    same attention written as one [1, H, T, D] problem."""
+    lens_q = [5, 1, 7, 3]
+    T = sum(lens_q) + 2  # two tokens past the last sequence
+    cu = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int64)
+    ids = np.full(T, len(lens_q), np.int32)
+    for i in range(len(lens_q)):
+        ids[cu[i]:cu[i + 1]] = i
+    Hq, Hkv, D = 4, 2, 8
+    q = _rand((T, Hq, D), 71).numpy()
+    k = _rand((T, Hkv, D), 72).numpy()
+    v = _rand((T, Hkv, D), 73).numpy()
+    dout = _rand((T, Hq, D), 74).numpy()
+    for causal in (False, True):
+        for mods in ((), (("softcap", 3.0),)):
+            got = ob.flex_attention_varlen_backward(q, k, v, dout, cu, cu, causal, mods, None, True)
+            # the pack: tokens past the last sequence carry their own id and attend
+            # nothing in the varlen form, so their rows are masked out here too
+            ids_q = ids.copy()
+            ids_q[cu[-1]:] = -1
+            tree = ("document", ids_q[None], ids[None])
+            if causal:
+                tree = ("and", tree, ("causal",))
+            pk = lambda x: x.transpose(1, 0, 2)[None]  # noqa: E731
+            ref = ob.flex_attention_backward(pk(q), pk(k), pk(v), pk(dout), tree, mods, None, True)
+            for g, r in zip(got, ref):
+                np.testing.assert_allclose(g, r[0].transpose(1, 0, 2), rtol=1e-10, atol=1e-12)
+            assert np.all(got[0][cu[-1]:] == 0) and np.all(got[1][cu[-1]:] == 0)
