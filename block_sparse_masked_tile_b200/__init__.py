@@ -33,7 +33,7 @@ __all__ = [
     "sink", "document", "and_masks", "or_masks", "softcap", "alibi", "create_block_mask", "flex_attention",
     "check_device_status", "library_path", "mask_from_tree", "score_mods_from_list", "splitkv_workspace_bytes",
     "flex_attention_host", "flex_attention_varlen", "seqlens_to_doc_ids", "flex_attention_backward",
-    "backward_workspace_bytes",
+    "backward_workspace_bytes", "flex_attention_varlen_backward",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -125,6 +125,11 @@ def _load() -> ctypes.CDLL:
                                             ctypes.POINTER(_MaskSpec), ctypes.POINTER(_ScoreSpec), ctypes.c_float, i32,
                                             vp, vp, vp, vp, i64, vp]
     lib.bsmt_flex_attention_bwd.restype = i32
+    lib.bsmt_flex_attention_bwd_packed.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                                   ctypes.POINTER(_BlockMask), ctypes.POINTER(_BlockMaskQ),
+                                                   ctypes.POINTER(_MaskSpec), ctypes.POINTER(_ScoreSpec),
+                                                   ctypes.c_float, i32, vp, vp, vp, vp, i64, vp]
+    lib.bsmt_flex_attention_bwd_packed.restype = i32
     lib.bsmt_last_error.argtypes = []
     lib.bsmt_last_error.restype = ctypes.c_char_p
     lib.bsmt_check_device_status.argtypes = [vp]
@@ -821,29 +826,10 @@ def seqlens_to_doc_ids(cu_seqlens: torch.Tensor, total: int) -> torch.Tensor:
     return ids
 
 
-def flex_attention_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
-                          cu_seqlens_k: torch.Tensor, causal: bool = False,
-                          score_mod: ScoreMod | Iterable[ScoreMod] | None = None, scale: float | None = None,
-                          enable_gqa: bool = False, out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
-    """Attention over packed variable-length sequences (the cu_seqlens form):
-    q [total_q, Hq, D], k/v [total_k, Hkv, D] bf16; token t of the pack
-    belongs to sequence i for cu_seqlens[i] <= t < cu_seqlens[i+1], and attends
-    only to keys of its own sequence. ``causal`` needs q and k to share
-    cu_seqlens (equal lengths, top-left aligned). Returns (out [total_q, Hq, D],
-    lse [Hq, total_q]).
-
-    The sequence ordinals become DOCUMENT ids on the device, the BlockMask is
-    built over the whole pack (B = H = 1), and the packed layout goes straight
-    to the attention kernel through its tensor maps."""
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        if t.dtype != torch.bfloat16 or t.dim() != 3 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous bf16 3-D CUDA tensor [tokens, H, D]")
-    M, Hq, D = q.shape
-    N, Hkv, Dk = k.shape
-    if v.shape != k.shape or Dk != D:
-        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
-    device = q.device
-    mods = [score_mod] if isinstance(score_mod, ScoreMod) else list(score_mod or ())
+def _varlen_block_mask(cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor, M: int, N: int, causal: bool,
+                       mods: list, device: torch.device) -> BlockMask:
+    """The BlockMask of packed sequences over (total_q, total_k), B = H = 1:
+    sequence ordinals as DOCUMENT ids, and CAUSAL when asked."""
     # Causal masking and ALiBi see packed positions. These equal positions
     # within the sequence only when q and k share cu_seqlens (the sequence
     # start cancels in kv_idx - q_idx).
@@ -855,7 +841,19 @@ def flex_attention_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_
     mm = document(q_ids, kv_ids)
     if causal:
         mm = and_masks(mm, _causal_mask())
-    bm = create_block_mask(mm, 1, 1, M, N, device=device)
+    return create_block_mask(mm, 1, 1, M, N, device=device)
+
+
+def _check_packed(**tensors) -> None:
+    for name, t in tensors.items():
+        if t.dtype != torch.bfloat16 or t.dim() != 3 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 3-D CUDA tensor [tokens, H, D]")
+
+
+def _varlen_fwd(q, k, v, bm, mods, scale, enable_gqa, out, lse):
+    M, Hq, D = q.shape
+    N, Hkv, _ = k.shape
+    device = q.device
     if out is None:
         out = torch.empty((M, Hq, D), dtype=torch.bfloat16, device=device)
     if lse is None:
@@ -871,6 +869,100 @@ def flex_attention_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_
             out.data_ptr(), lse.data_ptr(), ctypes.c_void_p(_stream_ptr(device))))
     del keep_s
     return out, lse
+
+
+def _varlen_bwd(q, k, v, out, lse, dout, bm, mods, scale, enable_gqa):
+    M, Hq, D = q.shape
+    N, Hkv, _ = k.shape
+    device = q.device
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(backward_workspace_bytes(1, Hq, M), 1), dtype=torch.uint8, device=device)
+    with torch.cuda.device(device):
+        sspec, keep_s = _score_spec(mods, device, Hq)
+        c = bm._c()
+        qs = bm.q_side()
+        cq = _BlockMaskQ()
+        cq.q_num_blocks = qs["q_num_blocks"].data_ptr()
+        cq.q_indices = qs["q_indices"].data_ptr()
+        cq.full_q_num_blocks = qs["full_q_num_blocks"].data_ptr()
+        cq.full_q_indices = qs["full_q_indices"].data_ptr()
+        _check(_lib.bsmt_flex_attention_bwd_packed(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(), Hq, Hkv, M, N,
+            D, ctypes.byref(c), ctypes.byref(cq), ctypes.byref(bm._spec), ctypes.byref(sspec),
+            ctypes.c_float(0.0 if scale is None else float(scale)), int(bool(enable_gqa)), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr(), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+            ctypes.c_void_p(_stream_ptr(device))))
+    del keep_s
+    return dq, dk, dv
+
+
+class _FlexAttentionVarlenFn(torch.autograd.Function):
+    """flex_attention_varlen as a differentiable op (lse has no gradient)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, bm, mods, scale, enable_gqa, out, lse):
+        out, lse = _varlen_fwd(q, k, v, bm, mods, scale, enable_gqa, out, lse)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.args = (bm, mods, scale, enable_gqa)
+        ctx.mark_non_differentiable(lse)
+        return out, lse
+
+    @staticmethod
+    def backward(ctx, dout, _dlse):
+        if dout is None:
+            return (None,) * 9
+        q, k, v, out, lse = ctx.saved_tensors
+        bm, mods, scale, enable_gqa = ctx.args
+        dq, dk, dv = _varlen_bwd(q, k, v, out, lse, dout.to(torch.bfloat16).contiguous(), bm, mods, scale,
+                                 enable_gqa)
+        return dq, dk, dv, None, None, None, None, None, None
+
+
+def flex_attention_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                          cu_seqlens_k: torch.Tensor, causal: bool = False,
+                          score_mod: ScoreMod | Iterable[ScoreMod] | None = None, scale: float | None = None,
+                          enable_gqa: bool = False, out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
+    """Attention over packed variable-length sequences (the cu_seqlens form):
+    q [total_q, Hq, D], k/v [total_k, Hkv, D] bf16; token t of the pack
+    belongs to sequence i for cu_seqlens[i] <= t < cu_seqlens[i+1], and attends
+    only to keys of its own sequence. ``causal`` needs q and k to share
+    cu_seqlens (equal lengths, top-left aligned). Returns (out [total_q, Hq, D],
+    lse [Hq, total_q]).
+
+    The sequence ordinals become DOCUMENT ids on the device, the BlockMask is
+    built over the whole pack (B = H = 1), and the packed layout goes straight
+    to the attention kernel through its tensor maps. With q, k or v requiring
+    grad the call is recorded for backpropagation (the packed backward)."""
+    _check_packed(q=q, k=k, v=v)
+    M, Hq, D = q.shape
+    N, Hkv, Dk = k.shape
+    if v.shape != k.shape or Dk != D:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
+    mods = [score_mod] if isinstance(score_mod, ScoreMod) else list(score_mod or ())
+    bm = _varlen_block_mask(cu_seqlens_q, cu_seqlens_k, M, N, causal, mods, q.device)
+    if torch.is_grad_enabled() and any(t.requires_grad for t in (q, k, v)):
+        return _FlexAttentionVarlenFn.apply(q, k, v, bm, mods, scale, enable_gqa, out, lse)
+    return _varlen_fwd(q, k, v, bm, mods, scale, enable_gqa, out, lse)
+
+
+def flex_attention_varlen_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                                   lse: torch.Tensor, dout: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                                   cu_seqlens_k: torch.Tensor, causal: bool = False,
+                                   score_mod: ScoreMod | Iterable[ScoreMod] | None = None,
+                                   scale: float | None = None, enable_gqa: bool = False):
+    """Gradients (dq [total_q, Hq, D], dk, dv [total_k, Hkv, D]) of
+    sum(out * dout) for ``out, lse = flex_attention_varlen(...)`` with the same
+    arguments (bsmt_flex_attention_bwd_packed)."""
+    _check_packed(q=q, k=k, v=v, out=out, dout=dout)
+    M, Hq, D = q.shape
+    N, Hkv, Dk = k.shape
+    if v.shape != k.shape or Dk != D or out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("shape mismatch among q, k, v, out and dout")
+    if lse.shape != (Hq, M) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [Hq, total_q] tensor")
+    mods = [score_mod] if isinstance(score_mod, ScoreMod) else list(score_mod or ())
+    bm = _varlen_block_mask(cu_seqlens_q, cu_seqlens_k, M, N, causal, mods, q.device)
+    return _varlen_bwd(q, k, v, out, lse, dout, bm, mods, scale, enable_gqa)
 
 
 def check_device_status(device=None) -> None:

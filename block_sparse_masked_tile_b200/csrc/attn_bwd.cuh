@@ -83,6 +83,11 @@ struct BwdParams {
     const float2* ld;
     __nv_bfloat16* g0;  // dq (dq kernel) or dk [B, Hkv, N, D]
     __nv_bfloat16* g1;  // dv [B, Hkv, N, D]
+    // Element strides of the row-major tensors: row i of head bh of q, out,
+    // dout and dq starts at bh * q_sbh + i * q_ss; of k, v, dk and dv at
+    // bh * kv_sbh + i * kv_ss. (S*D, D) for [B, H, S, D]; (D, H*D) for a
+    // packed [S, H, D] with B = 1.
+    int64_t q_sbh, q_ss, kv_sbh, kv_ss;
     int32_t num_units;
     int32_t* next_unit;  // work counter, zero at launch (the prep kernel clears it)
 };
@@ -272,7 +277,8 @@ __device__ __forceinline__ void term_q_interval(const MaskDnf& m, int t, int64_t
 
 // (-lse2, -delta) per padded query row: lse2 = lse * log2(e) (+inf where lse
 // is -inf and for rows past M, so that P = 0 there), delta = sum_d out * dout
-// in fp32; it also zeroes the two backward kernels' work counters. A row is
+// in fp32 (row i of head bh of out and dout at bh * sbh + i * ss; lse is
+// [B*Hq, M]); it also zeroes the two backward kernels' work counters. A row is
 // read by D/8 lanes, 16 bytes of out and of dout each; a
 // warp covers kRowsPerWarp rows with all its loads issued before the sums,
 // so that enough bytes are in flight to keep HBM busy.
@@ -281,7 +287,7 @@ constexpr int kPrepRowsPerWarp = 8;
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* out, const __nv_bfloat16* dout,
                                                        const float* lse, int64_t rows_pad, int32_t M, int32_t QB,
-                                                       float2* ld, int32_t* counters) {
+                                                       int64_t sbh, int64_t ss, float2* ld, int32_t* counters) {
     if (blockIdx.x == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0;  // work counters of the two kernels
     constexpr int kLanesPerRow = D / 8;          // 16 (D = 128) or 8 (D = 64)
     constexpr int kRowsPerIter = 32 / kLanesPerRow;
@@ -300,7 +306,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* out,
         const int i = static_cast<int>(row - bh * per_bh);
         in[it] = row < rows_pad && i < M;
         if (in[it]) {
-            const int64_t base = (bh * M + i) * D + part * 8;
+            const int64_t base = bh * sbh + static_cast<int64_t>(i) * ss + part * 8;
             a[it] = __ldg(reinterpret_cast<const uint4*>(out + base));
             g[it] = __ldg(reinterpret_cast<const uint4*>(dout + base));
         } else {
@@ -886,9 +892,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float mul = (KVSIDE && h == 0) ? 1.f : p.scale;
             __nv_bfloat16* dst;
             if constexpr (KVSIDE)
-                dst = (h == 0 ? p.g1 : p.g0) + (static_cast<int64_t>(b * p.Hkv + hkv) * p.N + row_idx) * D;
+                dst = (h == 0 ? p.g1 : p.g0) + static_cast<int64_t>(b * p.Hkv + hkv) * p.kv_sbh + row_idx * p.kv_ss;
             else
-                dst = p.g0 + (static_cast<int64_t>(b * p.Hq + hq) * p.M + row_idx) * D + h * (D / 2);
+                dst = p.g0 + static_cast<int64_t>(b * p.Hq + hq) * p.q_sbh + row_idx * p.q_ss + h * (D / 2);
             uint4* d4 = reinterpret_cast<uint4*>(dst);
             if (T > 0) {
                 if (!(ok = mbar_wait(bar(L::kBarAccFull), units & 1u, abort_flag))) break;

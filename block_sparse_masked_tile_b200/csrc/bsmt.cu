@@ -846,13 +846,13 @@ extern "C" bsmt_status bsmt_flex_attention_bwd_workspace_bytes(int64_t B, int64_
     return ok();
 }
 
-extern "C" bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, const void* v, const void* out,
-                                               const void* dout, const float* lse, int64_t B, int64_t Hq, int64_t Hkv,
-                                               int64_t M, int64_t N, int64_t D, const bsmt_block_mask* bm,
-                                               const bsmt_block_mask_q* bmq, const bsmt_mask_spec* mask_spec,
-                                               const bsmt_score_spec* score, float scale, int32_t enable_gqa,
-                                               void* dq, void* dk, void* dv, void* workspace, int64_t workspace_bytes,
-                                               void* stream) {
+namespace {
+// The backward path; `packed` selects the [S, H, D] layouts (B = 1).
+bsmt_status backward(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+                     int64_t B, int64_t Hq, int64_t Hkv, int64_t M, int64_t N, int64_t D, const bsmt_block_mask* bm,
+                     const bsmt_block_mask_q* bmq, const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score,
+                     float scale, int32_t enable_gqa, void* dq, void* dk, void* dv, void* workspace,
+                     int64_t workspace_bytes, void* stream, bool packed) {
     if (B < 0 || Hq < 0 || Hkv < 0 || M < 0 || N < 0)
         return fail(BSMT_ERR_INVALID_ARGUMENT, "negative size (B=%lld Hq=%lld Hkv=%lld M=%lld N=%lld)",
                     static_cast<long long>(B), static_cast<long long>(Hq), static_cast<long long>(Hkv),
@@ -954,27 +954,30 @@ extern "C" bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, con
     // (-lse2, -delta) per padded query row, and the work counters
     float2* ld = static_cast<float2*>(workspace);
     int32_t* counters = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + bwd_ld_bytes(B, Hq, M));
+    // element strides (head, row): [B, H, S, D], or the packed [S, H, D] with B = 1
+    const int64_t q_sbh = packed ? D : M * D, q_ss = packed ? Hq * D : D;
+    const int64_t kv_sbh = packed ? D : N * D, kv_ss = packed ? Hkv * D : D;
     const int64_t rows_pad = B * Hq * QB * 128;
     const int64_t prep_blocks = (rows_pad + 8 * bsmt::kPrepRowsPerWarp - 1) / (8 * bsmt::kPrepRowsPerWarp);
     if (prep_blocks > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "too many query rows");
     if (D == 128)
         bsmt::bwd_prep_kernel<128><<<static_cast<unsigned>(prep_blocks), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, rows_pad,
-            static_cast<int32_t>(M), static_cast<int32_t>(QB), ld, counters);
+            static_cast<int32_t>(M), static_cast<int32_t>(QB), q_sbh, q_ss, ld, counters);
     else
         bsmt::bwd_prep_kernel<64><<<static_cast<unsigned>(prep_blocks), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, rows_pad,
-            static_cast<int32_t>(M), static_cast<int32_t>(QB), ld, counters);
+            static_cast<int32_t>(M), static_cast<int32_t>(QB), q_sbh, q_ss, ld, counters);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "backward prep launch: %s", cudaGetErrorString(e));
 
     EncodeTiledFn enc = nullptr;
     if ((st = get_encoder(&enc)) != BSMT_OK) return st;
     CUtensorMap tq, tk, tv, tdo;
-    if ((st = encode_bhsd(enc, &tq, q, B * Hq, M, D, M * D, D)) != BSMT_OK) return st;
-    if ((st = encode_bhsd(enc, &tdo, dout, B * Hq, M, D, M * D, D)) != BSMT_OK) return st;
-    if ((st = encode_bhsd(enc, &tk, k, B * Hkv, N, D, N * D, D)) != BSMT_OK) return st;
-    if ((st = encode_bhsd(enc, &tv, v, B * Hkv, N, D, N * D, D)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tq, q, B * Hq, M, D, q_sbh, q_ss)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tdo, dout, B * Hq, M, D, q_sbh, q_ss)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tk, k, B * Hkv, N, D, kv_sbh, kv_ss)) != BSMT_OK) return st;
+    if ((st = encode_bhsd(enc, &tv, v, B * Hkv, N, D, kv_sbh, kv_ss)) != BSMT_OK) return st;
     for (bsmt::BwdParams* pp : {&pq, &pk}) {
         pp->B = static_cast<int32_t>(B);
         pp->Hq = static_cast<int32_t>(Hq);
@@ -990,6 +993,10 @@ extern "C" bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, con
         pp->inv_cap = 1.f / cap;
         pp->slopes = slopes;
         pp->ld = ld;
+        pp->q_sbh = q_sbh;
+        pp->q_ss = q_ss;
+        pp->kv_sbh = kv_sbh;
+        pp->kv_ss = kv_ss;
     }
     pk.list_rows = static_cast<int32_t>(KB);
     pk.list_len = static_cast<int32_t>(QB);
@@ -1009,4 +1016,27 @@ extern "C" bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, con
                   : launch_bwd_score<64, false>(mode, dev, tq, tk, tv, tdo, pq, dnf, s);
     if (st != BSMT_OK) return st;
     return ok();
+}
+}  // namespace
+
+extern "C" bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, const void* v, const void* out,
+                                               const void* dout, const float* lse, int64_t B, int64_t Hq, int64_t Hkv,
+                                               int64_t M, int64_t N, int64_t D, const bsmt_block_mask* bm,
+                                               const bsmt_block_mask_q* bmq, const bsmt_mask_spec* mask_spec,
+                                               const bsmt_score_spec* score, float scale, int32_t enable_gqa,
+                                               void* dq, void* dk, void* dv, void* workspace, int64_t workspace_bytes,
+                                               void* stream) {
+    return backward(q, k, v, out, dout, lse, B, Hq, Hkv, M, N, D, bm, bmq, mask_spec, score, scale, enable_gqa, dq,
+                    dk, dv, workspace, workspace_bytes, stream, false);
+}
+
+extern "C" bsmt_status bsmt_flex_attention_bwd_packed(const void* q, const void* k, const void* v, const void* out,
+                                                      const void* dout, const float* lse, int64_t Hq, int64_t Hkv,
+                                                      int64_t M, int64_t N, int64_t D, const bsmt_block_mask* bm,
+                                                      const bsmt_block_mask_q* bmq, const bsmt_mask_spec* mask_spec,
+                                                      const bsmt_score_spec* score, float scale, int32_t enable_gqa,
+                                                      void* dq, void* dk, void* dv, void* workspace,
+                                                      int64_t workspace_bytes, void* stream) {
+    return backward(q, k, v, out, dout, lse, 1, Hq, Hkv, M, N, D, bm, bmq, mask_spec, score, scale, enable_gqa, dq,
+                    dk, dv, workspace, workspace_bytes, stream, true);
 }

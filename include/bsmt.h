@@ -380,6 +380,21 @@ bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, const void* v,
                                     const bsmt_score_spec* score, float scale, int32_t enable_gqa, void* dq,
                                     void* dk, void* dv, void* workspace, int64_t workspace_bytes, void* stream);
 
+/* bsmt_flex_attention_bwd on packed tensors (the layouts of
+ * bsmt_flex_attention_fwd_packed), B = 1:
+ *   q, out, dout, dq  device bf16 [M, Hq, D], 16-byte aligned
+ *   k, v, dk, dv      device bf16 [N, Hkv, D]
+ *   lse               device float [Hq, M], from the packed forward
+ * Everything else as in bsmt_flex_attention_bwd (block_mask has B = 1); the
+ * workspace size is bsmt_flex_attention_bwd_workspace_bytes(1, Hq, M). */
+bsmt_status bsmt_flex_attention_bwd_packed(const void* q, const void* k, const void* v, const void* out,
+                                           const void* dout, const float* lse, int64_t Hq, int64_t Hkv, int64_t M,
+                                           int64_t N, int64_t D, const bsmt_block_mask* block_mask,
+                                           const bsmt_block_mask_q* block_mask_q, const bsmt_mask_spec* mask_spec,
+                                           const bsmt_score_spec* score, float scale, int32_t enable_gqa, void* dq,
+                                           void* dk, void* dv, void* workspace, int64_t workspace_bytes,
+                                           void* stream);
+
 /* Thread-local message for the last failed call on this thread ("" if none). */
 const char* bsmt_last_error(void);
 
