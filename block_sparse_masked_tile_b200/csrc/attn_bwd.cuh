@@ -48,8 +48,9 @@
 //              the other of two buffers
 //   warp 11    idle; it completes the third warpgroup, whose registers
 //              setmaxnreg hands to the two softmax warpgroups
-// The epilogue reads the accumulators whole and releases them before its
-// stores, so the next unit's products overlap the previous unit's stores.
+// The epilogue reads the accumulators in 64-column batches, storing each, and
+// releases them once the last batch is in registers, so the next unit's
+// products overlap the rest of the previous unit's stores.
 // TMEM columns: S [0,128), dP [128,256), acc0 [256, 256+D) (dV or dQ), acc1
 // [256+D, 256+2D) (dK). Warpgroup g writes its P and dS as bf16 pairs over
 // the first 32 of its own 64 columns of S and dP, so the accumulating
