@@ -226,3 +226,32 @@ def test_autograd_through_flex_attention():
     assert_grads_close([t.float().cpu().numpy() for t in (qg.grad, kg.grad, vg.grad)], oracle, "autograd")
     with pytest.raises(ValueError, match="split-KV"):
         bsmt.flex_attention(qg, kg, vg, block_mask=bm, enable_gqa=True, num_splits=2)
+
+
+def test_maximum_length_forward_and_backward():
+    """The longest sequences the library takes: KV_LEN = 1024 kv blocks (the
+    forward's limit) with GQA 2:1, so a dk/dv unit walks 2 heads x 1024
+    q-blocks = 2048 entries (the backward's limit). Sampled query rows are
+    compared for out, lse and dq; dk/dv rows for keys near the end, which
+    few queries reach under the causal mask."""
+    from oracle import attention as oa
+    from tests.gpu_helpers import assert_attention_close
+    L, D = 1024 * 128, 64
+    q, k, v = workloads.random_inputs(70, 1, 2, 1, L, L, D)
+    dout = workloads.grad_output(71, 1, 2, L, D)
+    qd, kd, vd, dd = (t.cuda() for t in (q, k, v, dout))
+    bm = bsmt.create_block_mask(bsmt.causal(), 1, 2, L, L)
+    out, lse = bsmt.flex_attention(qd, kd, vd, block_mask=bm, enable_gqa=True)
+    dq, dk, dv = bsmt.flex_attention_backward(qd, kd, vd, out, lse, dd, block_mask=bm, enable_gqa=True)
+    bsmt.check_device_status()
+    rows = [(0, 0, 0), (0, 1, 1), (0, 0, 127), (0, 1, 128), (0, 0, L // 2 + 3), (0, 1, L - 1), (0, 0, L - 129)]
+    so, sl = oa.flex_attention_sampled(q, k, v, rows, ("causal",), (), None, True)
+    go = np.stack([out[b, h, r].float().cpu().numpy() for b, h, r in rows])
+    gl = np.array([lse[b, h, r].item() for b, h, r in rows])
+    assert_attention_close(go, gl, so, sl, "maximum length")
+    ref_q = ob.backward_dq_sampled(q, k, v, dout, rows, ("causal",), (), None)
+    assert_close("dq rows", np.stack([dq[b, h, r].float().cpu().numpy() for b, h, r in rows]), ref_q, "max")
+    keys = [(0, 0, L - 1), (0, 0, L - 128), (0, 0, L - 700)]
+    ref_k, ref_v = ob.backward_dkv_sampled(q, k, v, dout, keys, ("causal",), (), None)
+    assert_close("dk rows", np.stack([dk[b, h, j].float().cpu().numpy() for b, h, j in keys]), ref_k, "max")
+    assert_close("dv rows", np.stack([dv[b, h, j].float().cpu().numpy() for b, h, j in keys]), ref_v, "max")
