@@ -130,6 +130,8 @@ def _load() -> ctypes.CDLL:
                                                    ctypes.POINTER(_MaskSpec), ctypes.POINTER(_ScoreSpec),
                                                    ctypes.c_float, i32, vp, vp, vp, vp, i64, vp]
     lib.bsmt_flex_attention_bwd_packed.restype = i32
+    lib.bsmt_selftest_wait_timeout.argtypes = [vp, vp]
+    lib.bsmt_selftest_wait_timeout.restype = i32
     lib.bsmt_last_error.argtypes = []
     lib.bsmt_last_error.restype = ctypes.c_char_p
     lib.bsmt_check_device_status.argtypes = [vp]
@@ -963,6 +965,19 @@ def flex_attention_varlen_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Te
     mods = [score_mod] if isinstance(score_mod, ScoreMod) else list(score_mod or ())
     bm = _varlen_block_mask(cu_seqlens_q, cu_seqlens_k, M, N, causal, mods, q.device)
     return _varlen_bwd(q, k, v, out, lse, dout, bm, mods, scale, enable_gqa)
+
+
+def selftest_wait_timeout(device=None) -> dict:
+    """Run the library's bounded-wait failure path on purpose
+    (bsmt_selftest_wait_timeout) and return what the kernel saw. The device
+    status word then holds DEVICE_TIMEOUT; check_device_status raises it."""
+    device = torch.device("cuda") if device is None else torch.device(device)
+    res = torch.full((3,), -1, dtype=torch.int32, device=device)
+    with torch.cuda.device(device):
+        _check(_lib.bsmt_selftest_wait_timeout(ctypes.c_void_p(res.data_ptr()), ctypes.c_void_p(_stream_ptr(device))))
+        torch.cuda.current_stream(device).synchronize()
+    r = res.cpu().tolist()
+    return {"warp0_completed": r[0], "warp1_completed": r[1], "warp0_wait_us": r[2]}
 
 
 def check_device_status(device=None) -> None:

@@ -23,6 +23,7 @@
 #include "varlen.cuh"
 #include "mask_dnf.cuh"
 #include "ptx.cuh"
+#include "selftest.cuh"
 
 namespace {
 
@@ -1039,4 +1040,16 @@ extern "C" bsmt_status bsmt_flex_attention_bwd_packed(const void* q, const void*
                                                       int64_t workspace_bytes, void* stream) {
     return backward(q, k, v, out, dout, lse, 1, Hq, Hkv, M, N, D, bm, bmq, mask_spec, score, scale, enable_gqa, dq,
                     dk, dv, workspace, workspace_bytes, stream, true);
+}
+
+extern "C" bsmt_status bsmt_selftest_wait_timeout(int32_t* result, void* stream) {
+    if (result == nullptr || !aligned(result, 4))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "result must be a non-NULL, 4-byte aligned device int32[3]");
+    int dev = 0, nsm = 0;
+    bsmt_status st = sm_count(&dev, &nsm);
+    if (st != BSMT_OK) return st;
+    bsmt::wait_timeout_selftest_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(result);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
+    return ok();
 }

@@ -395,6 +395,18 @@ bsmt_status bsmt_flex_attention_bwd_packed(const void* q, const void* k, const v
                                            void* dk, void* dv, void* workspace, int64_t workspace_bytes,
                                            void* stream);
 
+/* Self-test of the device failure path. Every pipeline wait in the kernels
+ * is bounded (2 s); one that runs out records BSMT_ERR_DEVICE_TIMEOUT in the
+ * status word and makes the CTA's other waits return, so the kernel ends
+ * and the context stays usable. This call runs that path on purpose in a
+ * one-CTA kernel: warp 0 waits on an mbarrier that nothing arrives on, warp 1
+ * on another one. Afterwards bsmt_check_device_status reports
+ * BSMT_ERR_DEVICE_TIMEOUT. result: device int32[3], written as
+ * {warp 0 wait completed (0), warp 1 wait completed (0), warp 0 wait time in
+ * microseconds (about 2e6)}. Takes about 2 s of GPU time. The pages have no
+ * counterpart; it exists to test failure detection without a fault. */
+bsmt_status bsmt_selftest_wait_timeout(int32_t* result, void* stream);
+
 /* Thread-local message for the last failed call on this thread ("" if none). */
 const char* bsmt_last_error(void);
 

@@ -32,6 +32,7 @@ def test_every_declared_symbol_is_exported():
                             "bsmt_flex_attention_fwd_splitkv_static", "bsmt_seqlens_to_doc_ids",
                             "bsmt_flex_attention_fwd_packed", "bsmt_flex_attention_bwd_workspace_bytes",
                             "bsmt_flex_attention_bwd", "bsmt_flex_attention_bwd_packed",
+                            "bsmt_selftest_wait_timeout",
                             "bsmt_last_error", "bsmt_check_device_status", "bsmt_version"])
     lib = ctypes.CDLL(bsmt.library_path())
     for n in names:

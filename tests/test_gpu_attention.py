@@ -166,3 +166,17 @@ def test_invalid_block_mask_is_reported():
     bsmt.check_device_status()
     ro, rl = oa.flex_attention(q.cpu(), k.cpu(), v.cpu(), ("causal",), (), None, False)
     assert_attention_close(out.float().cpu().numpy(), lse.cpu().numpy(), ro, rl, "after bounds error")
+
+
+def test_wait_timeout_is_reported_and_context_survives():
+    """Failure detection without a fault: a pipeline wait on an mbarrier that
+    nothing arrives on gives up after its 2 s bound, records DEVICE_TIMEOUT in
+    the status word, and the CTA's other wait returns too. The context stays
+    usable: the word clears and the next attention call is correct."""
+    r = bsmt.selftest_wait_timeout()
+    assert r["warp0_completed"] == 0 and r["warp1_completed"] == 0
+    assert 1_500_000 <= r["warp0_wait_us"] <= 10_000_000, r
+    with pytest.raises(RuntimeError, match="DEVICE_TIMEOUT"):
+        bsmt.check_device_status()
+    bsmt.check_device_status()  # read and cleared
+    run_case(47, 1, 2, 2, 384, 384, 128, ("causal",), ())
