@@ -169,6 +169,18 @@ def _check(status: int) -> None:
     raise BsmtError(status, msg)
 
 
+# BSMT_DEBUG_SYNC=1: after every kernel launch, wait for the stream and raise
+# any device-side status (bounds, precondition, timeout) at the call that
+# caused it, instead of at the next check_device_status.
+_DEBUG_SYNC = os.environ.get("BSMT_DEBUG_SYNC", "0") == "1"
+
+
+def _check_launch(status: int) -> None:
+    _check(status)
+    if _DEBUG_SYNC:
+        _check(_lib.bsmt_check_device_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))
+
+
 def _stream_ptr(device: torch.device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
@@ -392,7 +404,7 @@ class BlockMask:
         cq.full_q_indices = t["full_q_indices"].data_ptr()
         c = self._c()
         with torch.cuda.device(dev):
-            _check(_lib.bsmt_block_mask_transpose(ctypes.byref(c), ctypes.byref(cq),
+            _check_launch(_lib.bsmt_block_mask_transpose(ctypes.byref(c), ctypes.byref(cq),
                                                   ctypes.c_void_p(_stream_ptr(dev))))
         self._q_side = t
         return t
@@ -420,7 +432,7 @@ class BlockMask:
         dense = torch.empty(self.shape, dtype=torch.int32, device=dev)
         c = self._c()
         with torch.cuda.device(dev):
-            _check(_lib.bsmt_block_mask_to_dense(ctypes.byref(c), ctypes.c_void_p(dense.data_ptr()),
+            _check_launch(_lib.bsmt_block_mask_to_dense(ctypes.byref(c), ctypes.c_void_p(dense.data_ptr()),
                                                  ctypes.c_void_p(_stream_ptr(dev))))
         return dense
 
@@ -504,7 +516,7 @@ def create_block_mask(mask_mod: MaskMod, B: int | None, H: int | None, Q_LEN: in
     c = bm._c()
     with torch.cuda.device(device):
         spec, keep = mask_mod._spec(device, shp[0])
-        _check(_lib.bsmt_create_block_mask(ctypes.byref(spec), Bv, Hv, int(Q_LEN), int(KV_LEN), bq, bkv,
+        _check_launch(_lib.bsmt_create_block_mask(ctypes.byref(spec), Bv, Hv, int(Q_LEN), int(KV_LEN), bq, bkv,
                                            ctypes.byref(c), ctypes.c_void_p(_stream_ptr(device))))
     # the marshalled spec and its device copies of document ids live as long as the mask
     bm._spec = spec
@@ -631,11 +643,11 @@ def _flex_attention_fwd(q, k, v, block_mask, score_mod, scale, enable_gqa, out, 
                   ctypes.byref(sspec), ctypes.c_float(0.0 if scale is None else float(scale)),
                   int(bool(enable_gqa)))
         if num_splits == 1:
-            _check(_lib.bsmt_flex_attention_fwd(*common, out.data_ptr(), lse.data_ptr(),
+            _check_launch(_lib.bsmt_flex_attention_fwd(*common, out.data_ptr(), lse.data_ptr(),
                                                 ctypes.c_void_p(_stream_ptr(device))))
         elif isinstance(workspace, str) and workspace == "static":
             # the library's own device scratch: no allocation (overlapping calls race)
-            _check(_lib.bsmt_flex_attention_fwd_splitkv_static(
+            _check_launch(_lib.bsmt_flex_attention_fwd_splitkv_static(
                 *common, int(num_splits), out.data_ptr(), lse.data_ptr(), ctypes.c_void_p(_stream_ptr(device))))
         else:
             need = splitkv_workspace_bytes(B, Hq, M, D, num_splits)
@@ -643,7 +655,7 @@ def _flex_attention_fwd(q, k, v, block_mask, score_mod, scale, enable_gqa, out, 
                 workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
             if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
                 raise ValueError("workspace must be a contiguous uint8 CUDA tensor")
-            _check(_lib.bsmt_flex_attention_fwd_splitkv(
+            _check_launch(_lib.bsmt_flex_attention_fwd_splitkv(
                 *common, int(num_splits), ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                 out.data_ptr(), lse.data_ptr(), ctypes.c_void_p(_stream_ptr(device))))
     del keep_s, keep_m
@@ -709,7 +721,7 @@ def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
             mspec = getattr(block_mask, "_spec", None)
             if mspec is None:
                 mspec, keep_m = block_mask.mask_mod._spec(device, int(block_mask.shape[0]))
-        _check(_lib.bsmt_flex_attention_bwd(
+        _check_launch(_lib.bsmt_flex_attention_bwd(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
             B, Hq, Hkv, M, N, D,
             ctypes.byref(bm_c) if bm_c is not None else None, ctypes.byref(bmq_c) if bmq_c is not None else None,
@@ -823,7 +835,7 @@ def seqlens_to_doc_ids(cu_seqlens: torch.Tensor, total: int) -> torch.Tensor:
         raise ValueError("cu_seqlens must be a 1-D CUDA tensor with at least one entry")
     ids = torch.empty(int(total), dtype=torch.int32, device=cu.device)
     with torch.cuda.device(cu.device):
-        _check(_lib.bsmt_seqlens_to_doc_ids(ctypes.c_void_p(cu.data_ptr()), cu.numel() - 1, int(total),
+        _check_launch(_lib.bsmt_seqlens_to_doc_ids(ctypes.c_void_p(cu.data_ptr()), cu.numel() - 1, int(total),
                                             ctypes.c_void_p(ids.data_ptr()), ctypes.c_void_p(_stream_ptr(cu.device))))
     return ids
 
@@ -865,7 +877,7 @@ def _varlen_fwd(q, k, v, bm, mods, scale, enable_gqa, out, lse):
     with torch.cuda.device(device):
         sspec, keep_s = _score_spec(mods, device, Hq)
         c = bm._c()
-        _check(_lib.bsmt_flex_attention_fwd_packed(
+        _check_launch(_lib.bsmt_flex_attention_fwd_packed(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), Hq, Hkv, M, N, D, ctypes.byref(c), ctypes.byref(bm._spec),
             ctypes.byref(sspec), ctypes.c_float(0.0 if scale is None else float(scale)), int(bool(enable_gqa)),
             out.data_ptr(), lse.data_ptr(), ctypes.c_void_p(_stream_ptr(device))))
@@ -888,7 +900,7 @@ def _varlen_bwd(q, k, v, out, lse, dout, bm, mods, scale, enable_gqa):
         cq.q_indices = qs["q_indices"].data_ptr()
         cq.full_q_num_blocks = qs["full_q_num_blocks"].data_ptr()
         cq.full_q_indices = qs["full_q_indices"].data_ptr()
-        _check(_lib.bsmt_flex_attention_bwd_packed(
+        _check_launch(_lib.bsmt_flex_attention_bwd_packed(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(), Hq, Hkv, M, N,
             D, ctypes.byref(c), ctypes.byref(cq), ctypes.byref(bm._spec), ctypes.byref(sspec),
             ctypes.c_float(0.0 if scale is None else float(scale)), int(bool(enable_gqa)), dq.data_ptr(),
