@@ -187,14 +187,14 @@ def test_debug_sync_raises_at_the_call():
     caused it (here a block index past KB), not at a later check."""
     import subprocess
     import sys
-    code = ("import torch, block_sparse_masked_tile_b200 as bsmt\\n"
-            "q = torch.randn(1, 1, 256, 64, device='cuda').to(torch.bfloat16)\\n"
-            "bm = bsmt.create_block_mask(bsmt.causal(), 1, 1, 256, 256)\\n"
-            "bm.kv_indices[0, 0, 1, 0] = 99\\n"
-            "try:\\n"
-            "    bsmt.flex_attention(q, q, q, block_mask=bm)\\n"
-            "except RuntimeError as e:\\n"
-            "    print('raised', 'DEVICE_BOUNDS' in str(e))\\n")
+    code = ("import torch, block_sparse_masked_tile_b200 as bsmt\n"
+            "q = torch.randn(1, 1, 256, 64, device='cuda').to(torch.bfloat16)\n"
+            "bm = bsmt.create_block_mask(bsmt.causal(), 1, 1, 256, 256)\n"
+            "bm.kv_indices[0, 0, 1, 0] = 99\n"
+            "try:\n"
+            "    bsmt.flex_attention(q, q, q, block_mask=bm)\n"
+            "except RuntimeError as e:\n"
+            "    print('raised', 'DEVICE_BOUNDS' in str(e))\n")
     import os
     env = dict(os.environ, BSMT_DEBUG_SYNC="1")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
