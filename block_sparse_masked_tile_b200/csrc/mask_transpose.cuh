@@ -52,26 +52,63 @@ __global__ void __launch_bounds__(kTransposeThreads) mask_transpose_kernel(const
     for (int i = threadIdx.x; i < 2 * kTransposeChunk * qw; i += kTransposeThreads) bits[i] = 0u;
     __syncthreads();
 
-    // scatter: q row qb's kv blocks that fall into this chunk
+    // scatter: q row qb's kv blocks that fall into this chunk. A warp takes 32
+    // rows at a time: lane r loads row r's two counts, then the warp loads the
+    // first 32 entries of 8 rows' two lists per batch (16 independent loads in
+    // flight, each coalesced along a row) before using any of them. Rows with
+    // more than 32 entries finish in a second loop.
     const int64_t row0 = (static_cast<int64_t>(b) * p.Hm + h) * p.QB;
     bool bad = false;
-    for (int qb = warp; qb < p.QB; qb += nwarps) {
-#pragma unroll
-        for (int l = 0; l < 2; ++l) {
-            const int32_t* num = l == 0 ? p.kv_num : p.full_num;
-            const int32_t* idx = (l == 0 ? p.kv_idx : p.full_idx) + (row0 + qb) * p.KB;
-            int n = __ldg(num + row0 + qb);
-            if (n < 0 || n > p.KB) {
+    auto take = [&](int l, int qb, int kb) {
+        if (kb < 0 || kb >= p.KB) {
+            bad = true;
+        } else if (kb >= kb0 && kb < kb0 + kTransposeChunk) {
+            atomicOr(&bits[(l * kTransposeChunk + (kb - kb0)) * qw + (qb >> 5)], 1u << (qb & 31));
+        }
+    };
+    for (int base = warp * 32; base < p.QB; base += nwarps * 32) {
+        const int rows = (p.QB - base) < 32 ? (p.QB - base) : 32;
+        int n0 = 0, n1 = 0;
+        if (lane < rows) {
+            n0 = __ldg(p.kv_num + row0 + base + lane);
+            n1 = __ldg(p.full_num + row0 + base + lane);
+            if (n0 < 0 || n0 > p.KB) {
                 bad = true;
-                n = 0;
+                n0 = 0;
             }
-            for (int j = lane; j < n; j += 32) {
-                const int kb = __ldg(idx + j);
-                if (kb < 0 || kb >= p.KB) {
-                    bad = true;
-                } else if (kb >= kb0 && kb < kb0 + kTransposeChunk) {
-                    atomicOr(&bits[(l * kTransposeChunk + (kb - kb0)) * qw + (qb >> 5)], 1u << (qb & 31));
-                }
+            if (n1 < 0 || n1 > p.KB) {
+                bad = true;
+                n1 = 0;
+            }
+        }
+        for (int r0 = 0; r0 < rows; r0 += 8) {
+            int v0[8], v1[8];
+            bool h0[8], h1[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int r = r0 + k;
+                const int c0 = __shfl_sync(0xFFFFFFFFu, n0, r & 31);
+                const int c1 = __shfl_sync(0xFFFFFFFFu, n1, r & 31);
+                const int64_t row = row0 + base + r;
+                h0[k] = r < rows && lane < c0;
+                h1[k] = r < rows && lane < c1;
+                v0[k] = h0[k] ? __ldg(p.kv_idx + row * p.KB + lane) : 0;
+                v1[k] = h1[k] ? __ldg(p.full_idx + row * p.KB + lane) : 0;
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                if (h0[k]) take(0, base + r0 + k, v0[k]);
+                if (h1[k]) take(1, base + r0 + k, v1[k]);
+            }
+        }
+        // entries past the first 32 of a row (dense rows)
+        if (__any_sync(0xFFFFFFFFu, n0 > 32 || n1 > 32)) {
+            for (int r = 0; r < rows; ++r) {
+                const int c0 = __shfl_sync(0xFFFFFFFFu, n0, r);
+                const int c1 = __shfl_sync(0xFFFFFFFFu, n1, r);
+                const int64_t row = row0 + base + r;
+                for (int j = 32 + lane; j < c0; j += 32) take(0, base + r, __ldg(p.kv_idx + row * p.KB + j));
+                for (int j = 32 + lane; j < c1; j += 32) take(1, base + r, __ldg(p.full_idx + row * p.KB + j));
             }
         }
     }
