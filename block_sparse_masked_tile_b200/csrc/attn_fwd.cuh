@@ -250,7 +250,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = lane; j < kMaxKB; j += 32) flags[j] = 0;
         __syncwarp();
         int iter = 0;
-        for (int u = blockIdx.x;; u += gridDim.x, ++iter) {
+        // Units go out in a serpentine order: round k gives CTA c unit
+        // k * G + c for even k and k * G + (G - 1 - c) for odd k (G CTAs). The
+        // order runs longest first, so alternating the direction evens out
+        // each CTA's total when unit lengths fall steadily (causal rows). A
+        // CTA's units still increase, so the first past the end is its last.
+        for (int64_t k = 0;; ++k, ++iter) {
+            const int64_t G = gridDim.x;
+            const int64_t u64 = k * G + ((k & 1) ? (G - 1 - blockIdx.x) : static_cast<int64_t>(blockIdx.x));
+            const int u = u64 < p.num_units ? static_cast<int>(u64) : p.num_units;
             const int buf = iter & 1;
             const uint32_t use = static_cast<uint32_t>(iter >> 1);
             if (!mbar_wait(bar(L::kBarSchedEmpty + buf), (use & 1u) ^ 1u, abort_flag)) break;
