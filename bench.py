@@ -59,6 +59,10 @@ def parse(argv=None):
     ap.add_argument("--backward-only", action="store_true",
                     help="run only the backward (prep, dk/dv and dq kernels) --steps times after one forward, "
                          "and print its timing (for profiling the backward kernels)")
+    ap.add_argument("--builder-only", action="store_true",
+                    help="run only the block-mask builder --steps times at the workload's shape (--batch and "
+                         "--heads override B and H) and print its timing (for profiling the builder)")
+    ap.add_argument("--heads", type=int, default=0, help="override H for --builder-only")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller cases for profiling only)")
     return ap.parse_args(argv)
@@ -301,6 +305,27 @@ def counted_flops(bm, D: int) -> int:
     return tiles * 4 * 128 * 128 * D
 
 
+def run_builder_only(bsmt, args, w):
+    """The block-mask builder alone: --steps launches at (B, H) of the workload
+    (or --batch / --heads), timed through a CUDA graph. Bytes are the four
+    output tensors (and the document ids read, if any)."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    data = workloads.make(w)
+    mask = bsmt.mask_from_tree(data["mask"], device=dev)
+    H = args.heads or w.Hq
+    bm = bsmt.create_block_mask(mask, w.B, H, w.M, w.N, device=dev)
+    ms = _time_launches(lambda: bsmt.create_block_mask(mask, w.B, H, w.M, w.N, device=dev, out=bm),
+                        reps=max(1, args.steps))
+    bsmt.check_device_status(dev)
+    Bm, Hm, QB, KB = bm.shape
+    nbytes = 2 * 4 * Bm * Hm * QB + 2 * 4 * Bm * Hm * QB * KB
+    peaks, _ = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    print(json.dumps({"workload": w.name, "B": Bm, "H": Hm, "ms": ms, "bytes": nbytes,
+                      "achieved_gbs": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm}))
+
+
 # ------------------------------------------------------------------ oracle
 def cpu_baseline(w, data, max_rows: int = 16384, chunk: int = 1024, cls=None):
     """The fp64 oracle, as it stands, on a bounded sample of the workload: whole
@@ -373,6 +398,10 @@ def main():
         return
 
     import block_sparse_masked_tile_b200 as bsmt
+
+    if args.builder_only:
+        run_builder_only(bsmt, args, w)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -37,7 +37,8 @@ constexpr int kBuildWarps = 8;       // warps per block
 constexpr int kClassifyWarps = 4;    // warps that classify (one row per lane)
 constexpr int kWordsPerChunk = 8;    // 256 kv blocks per pass
 
-__global__ void __launch_bounds__(kBuildWarps * 32) mask_build_kernel(const MaskDnf dnf, const BuildParams p) {
+__global__ void __launch_bounds__(kBuildWarps * 32)
+    mask_build_kernel(const __grid_constant__ MaskDnf dnf, const BuildParams p) {
     __shared__ uint32_t part_f[kClassifyWarps][kWordsPerChunk];
     __shared__ uint32_t part_a[kClassifyWarps][kWordsPerChunk];
     const int lane = threadIdx.x & 31;
@@ -140,13 +141,15 @@ __global__ void __launch_bounds__(kBuildWarps * 32) mask_build_kernel(const Mask
                 aw[w] = 0u;
             }
             for (int i = 0; i < nint; ++i) {
-                const int64_t a_lo = lo[i] >> 7, a_hi = hi[i] >> 7;
-                const int64_t f_lo = (lo[i] + 127) >> 7, f_hi = ((hi[i] + 1) >> 7) - 1;
+                // kv-block bounds of the interval, relative to this chunk (32-bit:
+                // intervals lie in [0, KV_LEN), so blocks fit easily)
+                const int a_lo = static_cast<int>(lo[i] >> 7) - c0, a_hi = static_cast<int>(hi[i] >> 7) - c0;
+                const int f_lo = static_cast<int>((lo[i] + 127) >> 7) - c0;
+                const int f_hi = static_cast<int>((hi[i] + 1) >> 7) - 1 - c0;
 #pragma unroll
                 for (int w = 0; w < kWordsPerChunk; ++w) {
-                    const int64_t base = c0 + 32 * w;
-                    aw[w] |= range_bits(a_lo, a_hi, base);
-                    fw[w] |= range_bits(f_lo, f_hi, base);
+                    aw[w] |= range_bits32(a_lo - 32 * w, a_hi - 32 * w);
+                    fw[w] |= range_bits32(f_lo - 32 * w, f_hi - 32 * w);
                 }
             }
 #pragma unroll
@@ -175,21 +178,31 @@ __global__ void __launch_bounds__(kBuildWarps * 32) mask_build_kernel(const Mask
             aw[w] &= exist;
         }
         __syncthreads();  // the partial words may be rewritten by the next chunk
-        // write this chunk's entries for the heads of the group
+        // This lane's list positions for the chunk, the same for every head:
+        // -1 where its kv block is not in the list.
         const uint32_t below = (1u << lane) - 1u;
-        for (int h = h0 + warp; h < h1; h += kBuildWarps) {
-            const int64_t row = (static_cast<int64_t>(b) * p.Hm + h) * p.QB + qb;
-            int32_t* pidx = p.kv_idx + row * p.KB;
-            int32_t* fidx = p.full_idx + row * p.KB;
+        int pos_p[kWordsPerChunk], pos_f[kWordsPerChunk];
+        {
             int cp = cnt_p, cf = cnt_f;
 #pragma unroll
             for (int w = 0; w < kWordsPerChunk; ++w) {
                 const uint32_t pw = aw[w] & ~fw[w];
-                const int kb = c0 + 32 * w + lane;
-                if ((pw >> lane) & 1u) pidx[cp + __popc(pw & below)] = kb;
-                if ((fw[w] >> lane) & 1u) fidx[cf + __popc(fw[w] & below)] = kb;
+                pos_p[w] = ((pw >> lane) & 1u) ? cp + __popc(pw & below) : -1;
+                pos_f[w] = ((fw[w] >> lane) & 1u) ? cf + __popc(fw[w] & below) : -1;
                 cp += __popc(pw);
                 cf += __popc(fw[w]);
+            }
+        }
+        // write this chunk's entries for the heads of the group
+        for (int h = h0 + warp; h < h1; h += kBuildWarps) {
+            const int64_t row = (static_cast<int64_t>(b) * p.Hm + h) * p.QB + qb;
+            int32_t* pidx = p.kv_idx + row * p.KB;
+            int32_t* fidx = p.full_idx + row * p.KB;
+#pragma unroll
+            for (int w = 0; w < kWordsPerChunk; ++w) {
+                const int kb = c0 + 32 * w + lane;
+                if (pos_p[w] >= 0) pidx[pos_p[w]] = kb;
+                if (pos_f[w] >= 0) fidx[pos_f[w]] = kb;
             }
         }
 #pragma unroll
