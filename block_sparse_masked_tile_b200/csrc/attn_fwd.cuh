@@ -713,6 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int tc0 = static_cast<int>(c0), tc1 = static_cast<int>(c1);
 #pragma unroll
                         for (int t = 0; t < kRowTerms; ++t) {
+                            if (t >= dnf.n_terms) break;  // uniform: the mask's own term count
                             int lo = iv_lo[t], hi = iv_hi[t];
                             lo = (lo > tc0 ? lo : tc0) - tc0;
                             hi = (hi < tc1 ? hi : tc1) - tc0;
