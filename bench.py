@@ -341,10 +341,22 @@ def cpu_baseline(w, data, max_rows: int = 16384, chunk: int = 1024, cls=None):
     nblk = max(1, min(QB, max_rows // rows_per_block))
     qbs = list(range(QB - nblk, QB))
     samples = [(0, 0, qb * 128 + r) for qb in qbs for r in range(128) if qb * 128 + r < w.M]
-    # kept tiles of those q-block rows (oracle block mask, per q-block row)
+    block_mask = None
     if cls is None:
-        cls = obm.tile_classes(data["mask"], 0, w.M, w.N)
-    tiles = sum(int((cls[qb] > 0).sum()) for qb in qbs)
+        # The oracle's block mask on its own: one (b, h) slice with B = H = 1 (the
+        # workloads' masks do not depend on the head), classification and
+        # compaction; GB/s of its four outputs, as for the GPU builder.
+        t0 = time.perf_counter()
+        bmo = obm.create_block_mask(data["mask"], 1, 1, w.M, w.N)
+        t_bm = time.perf_counter() - t0
+        nbytes = sum(int(a.nbytes) for a in bmo.values())
+        cls = bmo["kv_num_blocks"][0, 0] + bmo["full_kv_num_blocks"][0, 0]  # kept tiles per q-block row
+        block_mask = {"value": nbytes / t_bm / 1e9, "unit": "GB/s", "seconds": t_bm,
+                      "sample": f"create_block_mask of one (b, h) slice: {QB} x {(w.N + 127) // 128} tiles, "
+                                f"{nbytes} bytes of outputs, one core"}
+        tiles = sum(int(cls[qb]) for qb in qbs)
+    else:
+        tiles = sum(int((cls[qb] > 0).sum()) for qb in qbs)
     flops = tiles * 4 * 128 * 128 * w.D
     t0 = time.perf_counter()
     for c0 in range(0, len(samples), chunk):
@@ -352,9 +364,12 @@ def cpu_baseline(w, data, max_rows: int = 16384, chunk: int = 1024, cls=None):
                                   data["score_mods"], w.scale, w.enable_gqa)
     dt = time.perf_counter() - t0
     threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
-    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": int(threads), "kind": "oracle",
-            "sample": f"{len(samples)} query rows = q-blocks {qbs[0]}..{qbs[-1]} of (b=0, hq=0), "
-                      f"{tiles} kept tiles, {dt:.1f} s"}
+    res = {"value": flops / dt / 1e12, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+           "sample": f"{len(samples)} query rows = q-blocks {qbs[0]}..{qbs[-1]} of (b=0, hq=0), "
+                     f"{tiles} kept tiles, {dt:.1f} s"}
+    if block_mask is not None:
+        res["block_mask"] = block_mask
+    return res
 
 
 def run_reference(args, w):
