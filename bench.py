@@ -85,18 +85,24 @@ def attn_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profile_traffic(workload_name: str):
-    """DRAM bytes per attention launch from the committed ncu summary, if it was
-    taken on the current kernel source (same hash); otherwise None."""
+def profile_figures(workload_name: str) -> dict:
+    """Figures of the committed ncu summary of the attention kernel (DRAM bytes
+    per launch, tensor and MUFU pipe shares of active cycles), if it was taken
+    on the current kernel source (same hash); otherwise None for each."""
+    keys = {"traffic": "dram_bytes_per_launch", "tensor_pipe_pct": "tensor_pipe_pct_active",
+            "mufu_pipe_pct": "mufu_pipe_pct_active"}
+    res = dict.fromkeys(keys)
     path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload_name}.md")
     if not os.path.exists(path):
-        return None
+        return res
     text = open(path).read()
     m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != attn_source_hash():
-        return None
-    return float(m_bytes.group(1))
+    if not m_hash or m_hash.group(1) != attn_source_hash():
+        return res
+    for k, tag in keys.items():
+        m = re.search(tag + r":\s*([0-9.eE+]+)", text)
+        res[k] = float(m.group(1)) if m else None
+    return res
 
 
 def reduce_over_ranks(dist, device, times_ms, units):
@@ -521,7 +527,7 @@ def main():
         side["backward"] = time_backward(bsmt, w, q, k, v, out, lse, bm, mods, dev, flops)
     attn_tflops = (flops / (attn_ms * 1e-3)) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    traffic = profile_traffic(w.name)
+    prof = profile_figures(w.name)
     line = {
         "metric": METRIC,
         "value": value,
@@ -549,8 +555,12 @@ def main():
             "peak": peak,
             "unit": "TFLOP/s",
             "frac": attn_tflops / peak,
-            "traffic": traffic,
+            "traffic": prof["traffic"],
             "kernel": "attn_fwd_kernel",
+            # the ncu capture's pipe shares (of active cycles) for the same source;
+            # MUFU shows how close the exponentials are to bounding the kernel
+            "tensor_pipe_pct": prof["tensor_pipe_pct"],
+            "mufu_pipe_pct": prof["mufu_pipe_pct"],
             "peak_source": f"{peak_src} bf16_tflops (burst); sustained "
                            f"{peaks.get('bf16_tflops_sustained')}; datasheet {DATASHEET_BF16_TFLOPS}",
             "frac_of_datasheet": attn_tflops / DATASHEET_BF16_TFLOPS,
