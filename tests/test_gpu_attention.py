@@ -71,6 +71,28 @@ def test_random_masks_and_shapes(seed):
     run_case(seed, B, Hq, Hkv, M, N, D, tree, mods)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("S", [1, 4, 31, 32, 33])
+def test_sink_tiles(D, S):
+    # Once the window no longer reaches kv-block 0, the sink tile allows only
+    # its first S columns in every row of a q-block (StreamingLLM's shape at
+    # several sink sizes).
+    run_case(40 + S, 1, 2, 1, 1024, 1024, D, ("and", ("causal",), ("or", ("sink", S), ("window", 256))), ())
+
+
+@pytest.mark.parametrize("mods", [(("softcap", 20.0),), (("alibi", None),), (("softcap", 5.0), ("alibi", None)),
+                                  (("alibi", None), ("softcap", 5.0))])
+def test_sink_tiles_score_mods_gqa_ragged(mods):
+    run_case(50, 2, 4, 2, 1000, 1100, 128, ("and", ("causal",), ("or", ("sink", 8), ("window", 300))), mods)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_sink_only(D):
+    # causal and sink(4) alone: each q-block has a single partial tile, which
+    # both starts and finishes its O
+    run_case(60, 1, 2, 2, 640, 640, D, ("and", ("causal",), ("sink", 4)), ())
+
+
 def test_broadcast_block_mask():
     run_case(21, 2, 4, 2, 512, 512, 128, ("and", ("causal",), ("window", 200)), (), mask_B=None, mask_H=None)
     tree = ("and", ("causal",), ("window", 200))

@@ -43,6 +43,11 @@ def test_masks_and_score_mods(D):
         run(10 + i, 1, 4, 4, 256, 3000, D, tree, mods, 6)
 
 
+def test_sink_tiles_split():
+    # the window leaves kv-block 0 for q-blocks 3..7; slices cut the stream anywhere
+    run(25, 1, 4, 2, 1024, 2048, 128, ("and", ("causal",), ("or", ("sink", 4), ("window", 256))), (), 3)
+
+
 def test_more_splits_than_entries_and_ragged():
     # slices beyond the entry count are empty and must merge as nothing
     run(20, 2, 2, 1, 200, 300, 128, ("causal",), (), 9)
