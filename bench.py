@@ -569,6 +569,8 @@ def main():
         "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
         "side_kernels": side,
+        # each timed step is one builder launch and one attention launch (the
+        # committed launch list of this command shows exactly these)
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
