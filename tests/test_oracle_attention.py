@@ -121,6 +121,38 @@ def test_alibi_closed_form_geometric_weights():
                 math.log((1 - math.exp(-m * (i + 1))) / (1 - math.exp(-m))), rel=1e-12)
 
 
+def test_alibi_equals_sdpa_float_bias():
+    # ALiBi adds m_h * (j - i) to the scaled score of query i and key j
+    # (transformerlab page, "alibi" row). SDPA with a float attn_mask adds the
+    # mask to scale * q.k before its softmax, so a bias tensor m_h * (j - i),
+    # with -inf where a boolean mask forbids the pair, must give the same
+    # attention. Several heads with different slopes, GQA and a sliding-window
+    # causal mask check the head index, the sign and the masking together.
+    B, Hq, Hkv, M, N, D = 2, 4, 2, 41, 53, 16
+    q, k, v = _rand((B, Hq, M, D), 31), _rand((B, Hkv, N, D), 32), _rand((B, Hkv, N, D), 33)
+    slopes = np.array([0.5, 0.25, 0.0625, 0.75], np.float32)
+    sc = float(np.float32(0.2))
+    tree = ("and", ("causal",), ("window", 17))
+    out, lse = oa.flex_attention(q, k, v, tree, (("alibi", slopes),), scale=0.2, enable_gqa=True)
+    i = torch.arange(M, dtype=torch.float64)[:, None]
+    j = torch.arange(N, dtype=torch.float64)[None, :]
+    allowed = (i >= j) & ((i - j) < 17)
+    bias = torch.tensor(slopes, dtype=torch.float64)[:, None, None] * (j - i)[None]
+    bias = bias.masked_fill(~allowed[None], float("-inf"))[None].expand(B, Hq, M, N)
+    ref = F.scaled_dot_product_attention(q, k, v, attn_mask=bias, scale=sc, enable_gqa=True)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+    kr = k.repeat_interleave(Hq // Hkv, dim=1)
+    s = sc * (q @ kr.transpose(-1, -2)) + bias
+    np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), rtol=1e-12, atol=1e-12)
+    # the default slopes 2^(-8(h+1)/Hq) through the same float-bias form
+    out_d, _ = oa.flex_attention(q, k, v, tree, (("alibi", None),), scale=0.2, enable_gqa=True)
+    dflt = torch.tensor([2.0 ** (-8.0 * (h + 1) / Hq) for h in range(Hq)], dtype=torch.float64)
+    bias_d = (dflt[:, None, None] * (j - i)[None]).masked_fill(~allowed[None], float("-inf"))[None]
+    ref_d = F.scaled_dot_product_attention(q, k, v, attn_mask=bias_d.expand(B, Hq, M, N), scale=sc,
+                                           enable_gqa=True)
+    np.testing.assert_allclose(out_d, ref_d.numpy(), rtol=1e-12, atol=1e-12)
+
+
 def test_alibi_default_slopes_and_zero_slopes():
     np.testing.assert_allclose(oa.default_alibi_slopes(16)[[0, 1, 15]],
                                [2 ** -0.5, 2 ** -1.0, 2 ** -8.0], rtol=1e-15)

@@ -230,3 +230,27 @@ def test_q_side_twice_is_the_identity():
         assert np.array_equal(back["q_indices"], bm["kv_indices"])
         assert np.array_equal(back["full_q_num_blocks"], bm["full_kv_num_blocks"])
         assert np.array_equal(back["full_q_indices"], bm["full_kv_indices"])
+
+
+def test_create_mask_per_batch_documents_and_heads():
+    # create_mask(mod_fn, B, H, Q_LEN, KV_LEN) returns the element mask of
+    # shape (B, H, M, N) (tensorplay.nn.attention page, create_mask). With
+    # document ids that differ per batch row, each [b, h] slice must be that
+    # row's block-diagonal matrix (scipy.linalg.block_diag of all-ones
+    # blocks, one per document) intersected with the lower triangle, the same
+    # for every head.
+    lens = [[3, 5, 4], [6, 6], [1, 2, 3, 6]]
+    ids = np.stack([np.repeat(np.arange(len(L)), L) for L in lens]).astype(np.int32)
+    B, H, L = 3, 2, 12
+    tree = ("and", ("document", ids, ids), ("causal",))
+    got = om.create_mask(tree, B, H, L, L)
+    assert got.shape == (B, H, L, L) and got.dtype == bool
+    for b in range(B):
+        blocks = scipy.linalg.block_diag(*[np.ones((n, n), bool) for n in lens[b]]).astype(bool)
+        want = blocks & np.tril(np.ones((L, L), bool))
+        for h in range(H):
+            assert np.array_equal(got[b, h], want), (b, h)
+    # rows of different batch rows really differ (the per-row ids are used)
+    assert not np.array_equal(got[0, 0], got[1, 0])
+    # no mask at all: every element allowed, at a non-square shape
+    assert om.create_mask(None, 1, 3, 5, 7).all()
