@@ -32,7 +32,7 @@ __all__ = [
     "BsmtError", "MaskMod", "ScoreMod", "BlockMask", "noop_mask", "causal", "sliding_window", "prefix_lm",
     "sink", "document", "and_masks", "or_masks", "softcap", "alibi", "create_block_mask", "flex_attention",
     "check_device_status", "library_path", "mask_from_tree", "score_mods_from_list", "splitkv_workspace_bytes",
-    "flex_attention_host", "flex_attention_varlen", "seqlens_to_doc_ids", "flex_attention_backward",
+    "flex_attention_host", "host_workspace_bytes", "flex_attention_varlen", "seqlens_to_doc_ids", "flex_attention_backward",
     "backward_workspace_bytes", "flex_attention_varlen_backward",
 ]
 
@@ -60,7 +60,8 @@ class _MaskSpec(ctypes.Structure):
 
 
 class _ScoreOp(ctypes.Structure):
-    _fields_ = [("kind", ctypes.c_int32), ("value", ctypes.c_float), ("slopes", ctypes.c_void_p)]
+    _fields_ = [("kind", ctypes.c_int32), ("value", ctypes.c_float), ("slopes", ctypes.c_void_p),
+                ("head_offset", ctypes.c_int32), ("num_heads", ctypes.c_int32)]
 
 
 class _ScoreSpec(ctypes.Structure):
@@ -112,6 +113,13 @@ def _load() -> ctypes.CDLL:
                                                            ctypes.POINTER(_ScoreSpec), ctypes.c_float, i32, i32,
                                                            vp, vp, vp]
     lib.bsmt_flex_attention_fwd_splitkv_static.restype = i32
+    lib.bsmt_flex_attention_host_workspace_bytes.argtypes = [i64, i64, i64, i64, i64, i64,
+                                                             ctypes.POINTER(_MaskSpec), ctypes.POINTER(i64)]
+    lib.bsmt_flex_attention_host_workspace_bytes.restype = i32
+    lib.bsmt_flex_attention_host.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.POINTER(_MaskSpec),
+                                             ctypes.POINTER(_ScoreSpec), ctypes.c_float, i32, i32, vp, i64, vp, vp,
+                                             vp]
+    lib.bsmt_flex_attention_host.restype = i32
     lib.bsmt_seqlens_to_doc_ids.argtypes = [vp, i32, i64, vp, vp]
     lib.bsmt_seqlens_to_doc_ids.restype = i32
     lib.bsmt_flex_attention_fwd_packed.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, ctypes.POINTER(_BlockMask),
@@ -219,16 +227,6 @@ class MaskMod:
             spec.doc_batch = 1
         return spec, keep
 
-    def select_batch(self, b: int) -> "MaskMod":
-        """The mask of batch row b alone (document ids of that row; other
-        primitives do not depend on b)."""
-        if self.q_doc_ids is None:
-            return self
-        qd, kd = self.q_doc_ids, self.kv_doc_ids
-        if qd.dim() == 1 or qd.shape[0] == 1:
-            return self
-        return MaskMod(self.nodes, qd[b:b + 1], kd[b:b + 1])
-
 
 def _leaf(kind: int, arg: int = 0) -> MaskMod:
     return MaskMod(((kind, int(arg)),))
@@ -333,6 +331,8 @@ class ScoreMod:
     kind: int
     value: float = 0.0
     slopes: torch.Tensor | None = field(default=None, compare=False)
+    head_offset: int = 0   # ALiBi default slopes: model index of the call's first query head
+    num_heads: int = 0     # ALiBi default slopes: the model's head count (0: the call's Hq)
 
 
 def softcap(cap: float) -> ScoreMod:
@@ -340,9 +340,12 @@ def softcap(cap: float) -> ScoreMod:
     return ScoreMod(SCORE_SOFTCAP, float(cap))
 
 
-def alibi(slopes: torch.Tensor | None = None) -> ScoreMod:
-    """s -> s + m_h * (kv_idx - q_idx); default slopes m_h = 2^(-8(h+1)/Hq)."""
-    return ScoreMod(SCORE_ALIBI, 0.0, slopes)
+def alibi(slopes: torch.Tensor | None = None, head_offset: int = 0, num_heads: int | None = None) -> ScoreMod:
+    """s -> s + m_h * (kv_idx - q_idx). Without ``slopes`` the library uses
+    m_h = 2^(-8(head_offset + h + 1) / num_heads) for the call's head h
+    (num_heads defaults to the call's Hq), so a call on a slice of a model's
+    heads gets those heads' slopes."""
+    return ScoreMod(SCORE_ALIBI, 0.0, slopes, int(head_offset), 0 if num_heads is None else int(num_heads))
 
 
 def score_mods_from_list(mods) -> list[ScoreMod]:
@@ -467,16 +470,6 @@ class BlockMask:
         bm.q_side()
         return bm
 
-    def select(self, b0: int, b1: int, h0: int, h1: int) -> "BlockMask":
-        """Rows [b0, b1) x heads [h0, h1) of this BlockMask as views (dimensions
-        of size 1 broadcast and are kept)."""
-        Bm, Hm = self.shape[:2]
-        bs = slice(0, 1) if Bm == 1 else slice(b0, b1)
-        hs = slice(0, 1) if Hm == 1 else slice(h0, h1)
-        mm = self.mask_mod.select_batch(b0) if (b1 - b0 == 1 and Bm > 1) else self.mask_mod
-        return BlockMask(self.seq_lengths, self.kv_num_blocks[bs, hs], self.kv_indices[bs, hs],
-                         self.full_kv_num_blocks[bs, hs], self.full_kv_indices[bs, hs], self.BLOCK_SIZE, mm)
-
     def sparsity(self) -> float:
         """Percentage of blocks that are not computed (reads the counts back to the host)."""
         total = self.kv_indices.numel()
@@ -538,6 +531,8 @@ def _score_spec(mods, device: torch.device, Hq: int) -> tuple[_ScoreSpec, list]:
     for i, m in enumerate(mods):
         spec.ops[i].kind = m.kind
         spec.ops[i].value = m.value
+        spec.ops[i].head_offset = m.head_offset
+        spec.ops[i].num_heads = m.num_heads
         if m.kind == SCORE_ALIBI and m.slopes is not None:
             s = m.slopes.to(device=device, dtype=torch.float32).contiguous()
             if s.numel() != Hq:
@@ -733,18 +728,36 @@ def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
     return dq, dk, dv
 
 
+def host_workspace_bytes(B: int, Hq: int, Hkv: int, M: int, N: int, D: int,
+                         mask_mod: MaskMod | None = None) -> int:
+    """Bytes of device workspace flex_attention_host needs
+    (bsmt_flex_attention_host_workspace_bytes)."""
+    spec = None
+    if mask_mod is not None:
+        spec, _ = mask_mod._spec(torch.device("cpu"), int(B))
+    n = ctypes.c_int64(0)
+    _check(_lib.bsmt_flex_attention_host_workspace_bytes(int(B), int(Hq), int(Hkv), int(M), int(N), int(D),
+                                                         ctypes.byref(spec) if spec is not None else None,
+                                                         ctypes.byref(n)))
+    return int(n.value)
+
+
 def flex_attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask_mod: MaskMod | None = None,
                         score_mod: ScoreMod | Iterable[ScoreMod] | None = None, scale: float | None = None,
                         enable_gqa: bool = False, device="cuda", out: torch.Tensor | None = None,
-                        lse: torch.Tensor | None = None, chunks: int = 16):
-    """flex_attention on host tensors: q [B,Hq,M,D], k/v [B,Hkv,N,D] bf16 in CPU
-    memory (pinned for full speed). The BlockMask of ``mask_mod`` is built on
-    the device, then the work is cut into about ``chunks`` pieces along
-    (batch row, kv-head group), which are independent. The host-to-device
-    copy of piece i+1, the attention of piece i and the device-to-host copy
-    of piece i-1 run at the same time on three streams. Returns host
-    (out bf16 [B,Hq,M,D], lse fp32 [B,Hq,M]); ``out``/``lse`` may be given
-    (pinned CPU tensors)."""
+                        lse: torch.Tensor | None = None, chunks: int = 16, workspace: torch.Tensor | None = None):
+    """flex_attention on host tensors (bsmt_flex_attention_host): q [B,Hq,M,D],
+    k/v [B,Hkv,N,D] bf16 in CPU memory (pinned for full speed). The library
+    copies the document ids and slopes in, builds the BlockMask of
+    ``mask_mod`` on the device and pipelines about ``chunks`` independent
+    pieces along (batch row, kv-head group): the host-to-device copy of piece
+    i+1, the attention of piece i and the device-to-host copy of piece i-1 run
+    at the same time. Document ids of ``mask_mod`` and ALiBi slopes are read
+    from host memory (CUDA tensors are brought to the host first). Returns
+    host (out bf16 [B,Hq,M,D], lse fp32 [B,Hq,M]) once the copies are done;
+    ``out``/``lse`` may be given (pinned CPU tensors). ``workspace``: a uint8
+    tensor on ``device`` of at least host_workspace_bytes(...) bytes,
+    allocated when not given."""
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.dtype != torch.bfloat16 or t.dim() != 4 or t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous bf16 4-D CPU tensor")
@@ -755,76 +768,35 @@ def flex_attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask_
         raise ValueError(f"shape mismatch: q {tuple(q.shape)}, k {tuple(k.shape)}, v {tuple(v.shape)}")
     if Hkv < 1 or Hq % Hkv != 0:
         raise ValueError(f"Hq={Hq} is not a multiple of Hkv={Hkv}")
-    G = Hq // Hkv
     if out is None:
         out = torch.empty((B, Hq, M, D), dtype=torch.bfloat16, pin_memory=True)
     if lse is None:
         lse = torch.empty((B, Hq, M), dtype=torch.float32, pin_memory=True)
-    if out.shape != (B, Hq, M, D) or lse.shape != (B, Hq, M) or out.is_cuda or lse.is_cuda:
-        raise ValueError("out and lse must be CPU tensors of shape [B,Hq,M,D] and [B,Hq,M]")
-    # pieces: whole batch rows, or groups of kv heads within a batch row
-    per_b = max(1, min(Hkv, round(chunks / max(B, 1))))
-    gs = -(-Hkv // per_b)  # kv heads per piece
-    pieces = [(b, g0, min(Hkv, g0 + gs)) for b in range(B) for g0 in range(0, Hkv, gs)]
+    if (out.shape != (B, Hq, M, D) or lse.shape != (B, Hq, M) or out.is_cuda or lse.is_cuda
+            or out.dtype != torch.bfloat16 or lse.dtype != torch.float32
+            or not out.is_contiguous() or not lse.is_contiguous()):
+        raise ValueError("out and lse must be contiguous CPU tensors: bf16 [B,Hq,M,D] and fp32 [B,Hq,M]")
+    host = torch.device("cpu")
+    mspec, keep_m = (None, []) if mask_mod is None else mask_mod._spec(host, B)
+    sspec, keep_s = _score_spec(score_mod, host, Hq)
+    need = host_workspace_bytes(B, Hq, Hkv, M, N, D, mask_mod)
     with torch.cuda.device(device):
-        compute = torch.cuda.current_stream(device)
-        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
-        qd = torch.empty(q.shape, dtype=q.dtype, device=device)
-        kd = torch.empty(k.shape, dtype=k.dtype, device=device)
-        vd = torch.empty(v.shape, dtype=v.dtype, device=device)
-        od = torch.empty(out.shape, dtype=out.dtype, device=device)
-        ld = torch.empty(lse.shape, dtype=lse.dtype, device=device)
-        bm = None
-        if mask_mod is not None:
-            bm = create_block_mask(mask_mod, B, Hq, M, N, device=device)
-        ev_in = []
-        s_in.wait_stream(compute)  # the buffers were allocated on the compute stream
-        with torch.cuda.stream(s_in):
-            for (b, g0, g1) in pieces:
-                qd[b, g0 * G:g1 * G].copy_(q[b, g0 * G:g1 * G], non_blocking=True)
-                kd[b, g0:g1].copy_(k[b, g0:g1], non_blocking=True)
-                vd[b, g0:g1].copy_(v[b, g0:g1], non_blocking=True)
-                e = torch.cuda.Event()
-                e.record(s_in)
-                ev_in.append(e)
-        for i, (b, g0, g1) in enumerate(pieces):
-            compute.wait_event(ev_in[i])
-            h0, h1 = g0 * G, g1 * G
-            flex_attention(qd[b:b + 1, h0:h1], kd[b:b + 1, g0:g1], vd[b:b + 1, g0:g1],
-                           block_mask=None if bm is None else bm.select(b, b + 1, h0, h1),
-                           score_mod=_select_heads(score_mod, h0, h1, Hq), scale=scale,
-                           enable_gqa=enable_gqa, out=od[b:b + 1, h0:h1], lse=ld[b:b + 1, h0:h1])
-            e = torch.cuda.Event()
-            e.record(compute)
-            s_out.wait_event(e)
-            with torch.cuda.stream(s_out):
-                out[b, h0:h1].copy_(od[b, h0:h1], non_blocking=True)
-                lse[b, h0:h1].copy_(ld[b, h0:h1], non_blocking=True)
-        s_out.synchronize()
-        compute.wait_stream(s_out)
-        for t in (qd, kd, vd, od, ld):  # keep the buffers until the copies that use them are done
-            t.record_stream(s_in)
-            t.record_stream(s_out)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+        if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous uint8 CUDA tensor")
+        stream = torch.cuda.current_stream(device)
+        _check(_lib.bsmt_flex_attention_host(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, M, N, D,
+            ctypes.byref(mspec) if mspec is not None else None, ctypes.byref(sspec),
+            ctypes.c_float(0.0 if scale is None else float(scale)), int(bool(enable_gqa)), int(chunks),
+            ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), out.data_ptr(), lse.data_ptr(),
+            ctypes.c_void_p(stream.cuda_stream)))
+        stream.synchronize()  # the host outputs are complete
+        if _DEBUG_SYNC:
+            _check(_lib.bsmt_check_device_status(ctypes.c_void_p(stream.cuda_stream)))
+    del keep_s, keep_m
     return out, lse
-
-
-def _select_heads(mods, h0: int, h1: int, Hq: int):
-    """Score mods for query heads [h0, h1): ALiBi's slopes are per head, so a
-    piece of the heads gets its own slopes (the default ones when none were
-    given)."""
-    if mods is None:
-        return None
-    lst = [mods] if isinstance(mods, ScoreMod) else list(mods)
-    res = []
-    for m in lst:
-        if m.kind == SCORE_ALIBI:
-            slopes = m.slopes
-            if slopes is None:
-                slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / Hq) for h in range(Hq)], dtype=torch.float32)
-            res.append(ScoreMod(m.kind, m.value, slopes[h0:h1]))
-        else:
-            res.append(m)
-    return res
 
 
 def seqlens_to_doc_ids(cu_seqlens: torch.Tensor, total: int) -> torch.Tensor:

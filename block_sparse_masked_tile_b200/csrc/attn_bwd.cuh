@@ -77,7 +77,8 @@ struct BwdParams {
     const int32_t* full_idx;
     int32_t list_rows, list_len;
     float scale, scale_log2, cap, inv_cap;
-    const float* slopes;  // ALiBi slopes [Hq] or null (default 2^(-8(h+1)/Hq))
+    const float* slopes;  // ALiBi slopes [Hq] or null (default 2^(-8(h0+h+1)/Ht))
+    int32_t alibi_h0, alibi_heads;  // h0 and Ht of the default slopes
     // (-lse * log2(e), -delta) per query row, padded to whole q-blocks:
     // [B*Hq][QB*128]. The first is -inf for padding rows and rows with no
     // key, so that P = 2^(z2 - lse2) = 0 there.
@@ -731,7 +732,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 nd_row = make_float2(ldr.y, ldr.y);
                 if constexpr (kAlibi)
                     slope_unit = p.slopes ? __ldg(p.slopes + hq)
-                                          : exp2f(-8.0f * static_cast<float>(hq + 1) / static_cast<float>(p.Hq));
+                                          : exp2f(-8.0f * static_cast<float>(p.alibi_h0 + hq + 1) /
+                                                  static_cast<float>(p.alibi_heads));
                 if (dnf.has_doc && masked_path) {
                     // the span [first, last] of kv positions with this row's document
                     // id (kv ids are non-decreasing); one warp search per distinct id
@@ -813,7 +815,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 float slope = slope_unit;
                 if constexpr (KVSIDE && kAlibi)
                     slope = p.slopes ? __ldg(p.slopes + hq + g)
-                                     : exp2f(-8.0f * static_cast<float>(hq + g + 1) / static_cast<float>(p.Hq));
+                                     : exp2f(-8.0f * static_cast<float>(p.alibi_h0 + hq + g + 1) /
+                                             static_cast<float>(p.alibi_heads));
                 // kv - q at the warpgroup's column 0; it moves by -1 (dk/dv) or +1 (dq) per column
                 const float dkv0 = KVSIDE ? static_cast<float>(row_idx - c0) : static_cast<float>(c0 - row_idx);
                 constexpr float kStep = KVSIDE ? -1.f : 1.f;

@@ -71,7 +71,8 @@ struct AttnParams {
     float scale_log2;  // scale * log2(e)
     float cap;         // soft-cap
     float inv_cap;     // 1 / cap
-    const float* slopes;  // ALiBi slopes [Hq] or null (default 2^(-8(h+1)/Hq))
+    const float* slopes;  // ALiBi slopes [Hq] or null (default 2^(-8(h0+h+1)/Ht))
+    int32_t alibi_h0, alibi_heads;  // h0 and Ht of the default slopes
     __nv_bfloat16* out;
     float* lse;
     // out element (b, hq, i, d) sits at out + (b*Hq + hq)*out_sbh + i*out_ss + d:
@@ -414,7 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 hdr->n1 = n1;
                 float slope = 0.f;
                 if (SCORE == kScoreAlibi || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap)
-                    slope = p.slopes ? __ldg(p.slopes + hq) : exp2f(-8.0f * static_cast<float>(hq + 1) / static_cast<float>(p.Hq));
+                    slope = p.slopes ? __ldg(p.slopes + hq)
+                                     : exp2f(-8.0f * static_cast<float>(p.alibi_h0 + hq + 1) /
+                                             static_cast<float>(p.alibi_heads));
                 hdr->slope = slope;
                 // Pull this unit's Q tiles into L2 now; they are loaded into shared
                 // memory only when the unit before has finished with its own.

@@ -258,11 +258,22 @@ __global__ void fill_empty_kernel(uint4* out, int64_t out_vec, float* lse, int64
         lse[i] = -INFINITY;
 }
 
-// Score mods -> compile-time mode (kScore*), the soft-cap and the ALiBi slopes.
-bsmt_status parse_score(const bsmt_score_spec* score, int* mode_out, float* cap_out, const float** slopes_out) {
+// Score mods -> compile-time mode (kScore*), the soft-cap and the ALiBi slopes
+// (explicit, or the default ones of heads h0 .. h0 + Hq - 1 of a model of
+// `heads` heads).
+struct ScoreArgs {
     int mode = bsmt::kScoreNone;
     float cap = 1.f;
     const float* slopes = nullptr;
+    int32_t alibi_h0 = 0, alibi_heads = 1;
+};
+
+bsmt_status parse_score(const bsmt_score_spec* score, int64_t Hq, ScoreArgs* out_args) {
+    int mode = bsmt::kScoreNone;
+    float cap = 1.f;
+    const float* slopes = nullptr;
+    int32_t h0 = 0;
+    int64_t heads = Hq;
     if (score != nullptr) {
         if (score->num_ops < 0 || score->num_ops > BSMT_MAX_SCORE_OPS)
             return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: num_ops=%d outside [0, %d]", score->num_ops, BSMT_MAX_SCORE_OPS);
@@ -279,6 +290,21 @@ bsmt_status parse_score(const bsmt_score_spec* score, int* mode_out, float* cap_
                 if (op.slopes && !aligned(op.slopes, 4))
                     return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: ALiBi slopes must be 4-byte aligned");
                 slopes = op.slopes;
+                if (slopes == nullptr) {
+                    if (op.num_heads <= 0) {
+                        if (op.head_offset != 0)
+                            return fail(BSMT_ERR_INVALID_ARGUMENT,
+                                        "score spec: ALiBi head_offset=%d needs num_heads (the model's head count)",
+                                        op.head_offset);
+                    } else if (op.head_offset < 0 || op.head_offset + Hq > op.num_heads) {
+                        return fail(BSMT_ERR_INVALID_ARGUMENT,
+                                    "score spec: ALiBi heads [%d, %lld) outside the model's %d heads", op.head_offset,
+                                    static_cast<long long>(op.head_offset + Hq), op.num_heads);
+                    } else {
+                        h0 = op.head_offset;
+                        heads = op.num_heads;
+                    }
+                }
             } else {
                 return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: unknown kind %d", op.kind);
             }
@@ -289,9 +315,11 @@ bsmt_status parse_score(const bsmt_score_spec* score, int* mode_out, float* cap_
         if (nk == 1) mode = kinds[0] == BSMT_SCORE_SOFTCAP ? bsmt::kScoreSoftcap : bsmt::kScoreAlibi;
         if (nk == 2) mode = kinds[0] == BSMT_SCORE_SOFTCAP ? bsmt::kScoreSoftcapAlibi : bsmt::kScoreAlibiSoftcap;
     }
-    *mode_out = mode;
-    *cap_out = cap;
-    *slopes_out = slopes;
+    out_args->mode = mode;
+    out_args->cap = cap;
+    out_args->slopes = slopes;
+    out_args->alibi_h0 = h0;
+    out_args->alibi_heads = static_cast<int32_t>(heads > 0 ? heads : 1);
     return BSMT_OK;
 }
 
@@ -335,7 +363,7 @@ bsmt_status launch_attn_score(int score, int dev, int nsm, const CUtensorMap& tq
 
 extern "C" {
 
-int32_t bsmt_version(void) { return (1 << 16) | 0; }
+int32_t bsmt_version(void) { return (2 << 16) | 0; }
 
 const char* bsmt_last_error(void) { return g_last_error.c_str(); }
 
@@ -423,7 +451,8 @@ namespace {
 bsmt_status attention(const void* q, const void* k, const void* v, int64_t B, int64_t Hq, int64_t Hkv, int64_t M,
                       int64_t N, int64_t D, const bsmt_block_mask* bm, const bsmt_mask_spec* mask_spec,
                       const bsmt_score_spec* score, float scale, int32_t enable_gqa, int num_splits, float* ws_o,
-                      float* ws_lse, void* out, float* lse, void* stream, bool packed = false) {
+                      float* ws_lse, void* out, float* lse, void* stream, bool packed = false,
+                      bool dry_run = false) {
     if (B < 0 || Hq < 0 || Hkv < 0 || M < 0 || N < 0)
         return fail(BSMT_ERR_INVALID_ARGUMENT, "negative size (B=%lld Hq=%lld Hkv=%lld M=%lld N=%lld)",
                     static_cast<long long>(B), static_cast<long long>(Hq), static_cast<long long>(Hkv),
@@ -452,13 +481,12 @@ bsmt_status attention(const void* q, const void* k, const void* v, int64_t B, in
     if (scale <= 0.f) scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
 
     // score mods -> compile-time mode
-    int mode = bsmt::kScoreNone;
-    float cap = 1.f;
-    const float* slopes = nullptr;
+    ScoreArgs sa;
     {
-        const bsmt_status sst = parse_score(score, &mode, &cap, &slopes);
+        const bsmt_status sst = parse_score(score, Hq, &sa);
         if (sst != BSMT_OK) return sst;
     }
+    const int mode = sa.mode;
 
     bsmt::MaskDnf dnf;
     std::memset(&dnf, 0, sizeof(dnf));
@@ -489,7 +517,7 @@ bsmt_status attention(const void* q, const void* k, const void* v, int64_t B, in
     } else {
         dnf.n_terms = 1;
     }
-    if (B == 0 || M == 0) return ok();
+    if (dry_run || B == 0 || M == 0) return ok();  // (a dry run only checks the arguments)
     int dev = 0, nsm = 0;
     bsmt_status st = sm_count(&dev, &nsm);
     if (st != BSMT_OK) return st;
@@ -532,9 +560,11 @@ bsmt_status attention(const void* q, const void* k, const void* v, int64_t B, in
     p.num_units = static_cast<int32_t>(units);
     p.scale = scale;
     p.scale_log2 = scale * bsmt::kLog2e;
-    p.cap = cap;
-    p.inv_cap = 1.f / cap;
-    p.slopes = slopes;
+    p.cap = sa.cap;
+    p.inv_cap = 1.f / sa.cap;
+    p.slopes = sa.slopes;
+    p.alibi_h0 = sa.alibi_h0;
+    p.alibi_heads = sa.alibi_heads;
     p.out = static_cast<__nv_bfloat16*>(out);
     p.lse = lse;
     st = D == 128 ? launch_attn_score<128>(mode, dev, nsm, tq, tk, tv, to, p, dnf, s)
@@ -885,11 +915,10 @@ bsmt_status backward(const void* q, const void* k, const void* v, const void* ou
     if (!aligned(lse, 4)) return fail(BSMT_ERR_INVALID_ARGUMENT, "lse must be 4-byte aligned");
     if (std::isnan(scale) || std::isinf(scale)) return fail(BSMT_ERR_INVALID_ARGUMENT, "scale must be finite");
     if (scale <= 0.f) scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
-    int mode = bsmt::kScoreNone;
-    float cap = 1.f;
-    const float* slopes = nullptr;
-    bsmt_status st = parse_score(score, &mode, &cap, &slopes);
+    ScoreArgs sa;
+    bsmt_status st = parse_score(score, Hq, &sa);
     if (st != BSMT_OK) return st;
+    const int mode = sa.mode;
 
     bsmt::MaskDnf dnf;
     std::memset(&dnf, 0, sizeof(dnf));
@@ -990,9 +1019,11 @@ bsmt_status backward(const void* q, const void* k, const void* v, const void* ou
         pp->group = static_cast<int32_t>(group);
         pp->scale = scale;
         pp->scale_log2 = scale * bsmt::kLog2e;
-        pp->cap = cap;
-        pp->inv_cap = 1.f / cap;
-        pp->slopes = slopes;
+        pp->cap = sa.cap;
+        pp->inv_cap = 1.f / sa.cap;
+        pp->slopes = sa.slopes;
+        pp->alibi_h0 = sa.alibi_h0;
+        pp->alibi_heads = sa.alibi_heads;
         pp->ld = ld;
         pp->q_sbh = q_sbh;
         pp->q_ss = q_ss;
@@ -1051,5 +1082,306 @@ extern "C" bsmt_status bsmt_selftest_wait_timeout(int32_t* result, void* stream)
     bsmt::wait_timeout_selftest_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(result);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+
+// ------------------------------------------------------------ host buffers
+namespace {
+constexpr int kMaxHostPieces = 256;
+
+// Per device: two copy streams and a pool of events for the host pipeline,
+// created on its first call there and kept.
+struct HostCtx {
+    bool ready = false;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[2 * kMaxHostPieces + 4] = {};
+};
+HostCtx g_host[64];
+std::mutex g_host_mu;  // held while a call enqueues (the pool is shared)
+
+int64_t round256(int64_t x) { return (x + 255) / 256 * 256; }
+
+// Where each device copy sits in the workspace (byte offsets, 256-aligned).
+struct HostLayout {
+    int64_t q, k, v, o, l, kvn, kvi, fn, fi, qdoc, kvdoc, slopes[BSMT_MAX_SCORE_OPS], total;
+    int64_t Bm, QB, KB;
+    bool has_doc;
+    int32_t doc_batch;
+};
+
+bool spec_has_doc(const bsmt_mask_spec* spec) {
+    if (spec == nullptr) return false;
+    for (int i = 0; i < spec->num_nodes && i < BSMT_MAX_MASK_NODES; ++i)
+        if (spec->nodes[i].kind == BSMT_MASK_DOCUMENT) return true;
+    return false;
+}
+
+bsmt_status host_layout(int64_t B, int64_t Hq, int64_t Hkv, int64_t M, int64_t N, int64_t D,
+                        const bsmt_mask_spec* spec, HostLayout* L) {
+    if (B < 0 || Hq < 0 || Hkv < 0 || M < 0 || N < 0) return fail(BSMT_ERR_INVALID_ARGUMENT, "negative size");
+    if (D != 64 && D != 128) return fail(BSMT_ERR_UNSUPPORTED, "head dim D=%lld (supported: 64, 128)", static_cast<long long>(D));
+    if (M > kMaxLen || N > kMaxLen || B * Hq > 0x7FFFFFFF || B * Hkv > 0x7FFFFFFF)
+        return fail(BSMT_ERR_UNSUPPORTED, "sizes too large");
+    L->has_doc = spec_has_doc(spec);
+    L->doc_batch = L->has_doc ? (spec->doc_batch < 1 ? 1 : spec->doc_batch) : 1;
+    if (L->has_doc && !(L->doc_batch == 1 || L->doc_batch == B))
+        return fail(BSMT_ERR_SHAPE_MISMATCH, "mask spec: doc_batch=%d must be 1 or B=%lld", L->doc_batch,
+                    static_cast<long long>(B));
+    L->Bm = (L->has_doc && L->doc_batch > 1) ? B : 1;
+    L->QB = (M + 127) / 128;
+    L->KB = (N + 127) / 128;
+    int64_t off = 0;
+    auto take = [&](int64_t bytes) {
+        const int64_t at = off;
+        off += round256(bytes);
+        return at;
+    };
+    L->q = take(B * Hq * M * D * 2);
+    L->k = take(B * Hkv * N * D * 2);
+    L->v = take(B * Hkv * N * D * 2);
+    L->o = take(B * Hq * M * D * 2);
+    L->l = take(B * Hq * M * 4);
+    const bool has_mask = spec != nullptr;
+    L->kvn = take(has_mask ? L->Bm * L->QB * 4 : 0);
+    L->fn = take(has_mask ? L->Bm * L->QB * 4 : 0);
+    L->kvi = take(has_mask ? L->Bm * L->QB * L->KB * 4 : 0);
+    L->fi = take(has_mask ? L->Bm * L->QB * L->KB * 4 : 0);
+    L->qdoc = take(L->has_doc ? int64_t(L->doc_batch) * M * 4 : 0);
+    L->kvdoc = take(L->has_doc ? int64_t(L->doc_batch) * N * 4 : 0);
+    for (int i = 0; i < BSMT_MAX_SCORE_OPS; ++i) L->slopes[i] = take(Hq * 4);
+    L->total = off;
+    return BSMT_OK;
+}
+
+bsmt_status host_ctx(int dev, HostCtx** out) {
+    HostCtx& c = g_host[dev];
+    if (!c.ready) {
+        cudaError_t e = cudaStreamCreateWithFlags(&c.s_in, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c.s_out, cudaStreamNonBlocking);
+        for (int i = 0; e == cudaSuccess && i < 2 * kMaxHostPieces + 4; ++i)
+            e = cudaEventCreateWithFlags(&c.ev[i], cudaEventDisableTiming);
+        if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "host pipeline set-up: %s", cudaGetErrorString(e));
+        c.ready = true;
+    }
+    *out = &c;
+    return BSMT_OK;
+}
+
+// One piece of the host pipeline: batch rows [b0, b1) and kv heads [g0, g1)
+// with their query heads (either one batch row or all heads).
+struct HostPiece {
+    int64_t b0, b1, g0, g1;
+};
+
+std::vector<HostPiece> host_pieces(int64_t B, int64_t Hkv, int32_t target) {
+    std::vector<HostPiece> v;
+    const int64_t t = target <= 0 ? 16 : (target > kMaxHostPieces ? kMaxHostPieces : target);
+    if (B >= t) {
+        const int64_t rows = (B + t - 1) / t;
+        for (int64_t b = 0; b < B; b += rows) v.push_back({b, b + rows < B ? b + rows : B, 0, Hkv});
+    } else {
+        int64_t per_b = t / (B > 0 ? B : 1);
+        if (per_b < 1) per_b = 1;
+        if (per_b > Hkv) per_b = Hkv;
+        const int64_t gs = (Hkv + per_b - 1) / per_b;
+        for (int64_t b = 0; b < B; ++b)
+            for (int64_t g = 0; g < Hkv; g += gs) v.push_back({b, b + 1, g, g + gs < Hkv ? g + gs : Hkv});
+    }
+    return v;
+}
+}  // namespace
+
+extern "C" bsmt_status bsmt_flex_attention_host_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t M,
+                                                                int64_t N, int64_t D, const bsmt_mask_spec* mask_spec,
+                                                                int64_t* bytes) {
+    if (bytes == nullptr) return fail(BSMT_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    HostLayout L;
+    const bsmt_status st = host_layout(B, Hq, Hkv, M, N, D, mask_spec, &L);
+    if (st != BSMT_OK) return st;
+    *bytes = L.total;
+    return ok();
+}
+
+extern "C" bsmt_status bsmt_flex_attention_host(const void* q, const void* k, const void* v, int64_t B, int64_t Hq,
+                                                int64_t Hkv, int64_t M, int64_t N, int64_t D,
+                                                const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score,
+                                                float scale, int32_t enable_gqa, int32_t pieces, void* workspace,
+                                                int64_t workspace_bytes, void* out, float* lse, void* stream) {
+    HostLayout L;
+    bsmt_status st = host_layout(B, Hq, Hkv, M, N, D, mask_spec, &L);
+    if (st != BSMT_OK) return st;
+    if (Hkv < 1 || Hq < 1 || Hq % Hkv != 0)
+        return fail(BSMT_ERR_SHAPE_MISMATCH, "Hq=%lld must be a positive multiple of Hkv=%lld", static_cast<long long>(Hq),
+                    static_cast<long long>(Hkv));
+    if (L.Bm > 65535) return fail(BSMT_ERR_UNSUPPORTED, "B=%lld above 65535", static_cast<long long>(L.Bm));
+    const bool q_has = B * Hq * M > 0, kv_has = B * Hkv * N > 0;
+    if ((q_has && (!q || !out || !lse)) || (kv_has && (!k || !v)))
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "q, k, v, out and lse must be non-NULL when they hold elements");
+    if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < L.total)
+        return fail(BSMT_ERR_INVALID_ARGUMENT, "workspace must be non-NULL, 256-byte aligned and hold %lld bytes (has %lld)",
+                    static_cast<long long>(L.total), static_cast<long long>(workspace_bytes));
+    char* ws = static_cast<char*>(workspace);
+    // device-side copies of the mask and score specs: the same programs, with
+    // their arrays in the workspace
+    bsmt_mask_spec dspec;
+    if (mask_spec != nullptr) {
+        dspec = *mask_spec;
+        if (L.has_doc) {
+            if (mask_spec->q_doc_ids == nullptr || mask_spec->kv_doc_ids == nullptr)
+                return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: DOCUMENT needs q_doc_ids and kv_doc_ids");
+            dspec.q_doc_ids = reinterpret_cast<const int32_t*>(ws + L.qdoc);
+            dspec.kv_doc_ids = reinterpret_cast<const int32_t*>(ws + L.kvdoc);
+            dspec.doc_batch = L.doc_batch;
+        }
+    }
+    bsmt_score_spec dscore;
+    std::memset(&dscore, 0, sizeof(dscore));
+    if (score != nullptr) {
+        dscore = *score;
+        if (score->num_ops < 0 || score->num_ops > BSMT_MAX_SCORE_OPS)
+            return fail(BSMT_ERR_INVALID_ARGUMENT, "score spec: num_ops=%d outside [0, %d]", score->num_ops,
+                        BSMT_MAX_SCORE_OPS);
+        for (int i = 0; i < score->num_ops; ++i)
+            if (score->ops[i].kind == BSMT_SCORE_ALIBI && score->ops[i].slopes != nullptr)
+                dscore.ops[i].slopes = reinterpret_cast<const float*>(ws + L.slopes[i]);
+    }
+    bsmt_block_mask bm;
+    std::memset(&bm, 0, sizeof(bm));
+    bm.kv_num_blocks = reinterpret_cast<int32_t*>(ws + L.kvn);
+    bm.kv_indices = reinterpret_cast<int32_t*>(ws + L.kvi);
+    bm.full_kv_num_blocks = reinterpret_cast<int32_t*>(ws + L.fn);
+    bm.full_kv_indices = reinterpret_cast<int32_t*>(ws + L.fi);
+    bm.B = static_cast<int32_t>(L.Bm);
+    bm.H = 1;
+    bm.QB = static_cast<int32_t>(L.QB);
+    bm.KB = static_cast<int32_t>(L.KB);
+    bm.Q_LEN = static_cast<int32_t>(M);
+    bm.KV_LEN = static_cast<int32_t>(N);
+    bm.BLOCK_Q = bm.BLOCK_KV = 128;
+    const bsmt_block_mask* bmp = mask_spec != nullptr ? &bm : nullptr;
+    const bsmt_mask_spec* dspec_p = mask_spec != nullptr ? &dspec : nullptr;
+    char* const wq = ws + L.q;
+    char* const wk = ws + L.k;
+    char* const wv = ws + L.v;
+    char* const wo = ws + L.o;
+    float* const wl = reinterpret_cast<float*>(ws + L.l);
+    // every argument check of the attention, at the full size, before anything is enqueued
+    st = attention(wq, wk, wv, B, Hq, Hkv, M, N, D, bmp, dspec_p, &dscore, scale, enable_gqa, 1, nullptr, nullptr,
+                   wo, wl, stream, false, /*dry_run=*/true);
+    if (st != BSMT_OK) return st;
+    if (!q_has) return ok();
+    int dev = 0, nsm = 0;
+    if ((st = sm_count(&dev, &nsm)) != BSMT_OK) return st;
+
+    std::lock_guard<std::mutex> lk(g_host_mu);
+    HostCtx* hc = nullptr;
+    if ((st = host_ctx(dev, &hc)) != BSMT_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaEvent_t* ev = hc->ev;
+    const int64_t G = Hq / Hkv;
+    const std::vector<HostPiece> pcs = host_pieces(B, Hkv, pieces);
+    const int np = static_cast<int>(pcs.size());
+    cudaError_t ce = cudaSuccess;
+    auto cuda_ok = [&](cudaError_t e) {
+        if (ce == cudaSuccess && e != cudaSuccess) ce = e;
+        return ce == cudaSuccess;
+    };
+    // `stream` waits for both copy streams at the end, error or not, so the
+    // workspace is free once `stream` has passed the call
+    auto join = [&]() {
+        cudaEventRecord(ev[2 * kMaxHostPieces + 1], hc->s_in);
+        cudaEventRecord(ev[2 * kMaxHostPieces + 2], hc->s_out);
+        cudaStreamWaitEvent(s, ev[2 * kMaxHostPieces + 1], 0);
+        cudaStreamWaitEvent(s, ev[2 * kMaxHostPieces + 2], 0);
+    };
+    cuda_ok(cudaEventRecord(ev[2 * kMaxHostPieces], s));
+    cuda_ok(cudaStreamWaitEvent(hc->s_in, ev[2 * kMaxHostPieces], 0));
+    cuda_ok(cudaStreamWaitEvent(hc->s_out, ev[2 * kMaxHostPieces], 0));
+    // 1. document ids and slopes, then the BlockMask, on the caller's stream
+    if (L.has_doc) {
+        cuda_ok(cudaMemcpyAsync(ws + L.qdoc, mask_spec->q_doc_ids, int64_t(L.doc_batch) * M * 4, cudaMemcpyHostToDevice, s));
+        cuda_ok(cudaMemcpyAsync(ws + L.kvdoc, mask_spec->kv_doc_ids, int64_t(L.doc_batch) * N * 4, cudaMemcpyHostToDevice, s));
+    }
+    for (int i = 0; score != nullptr && i < score->num_ops; ++i)
+        if (score->ops[i].kind == BSMT_SCORE_ALIBI && score->ops[i].slopes != nullptr)
+            cuda_ok(cudaMemcpyAsync(ws + L.slopes[i], score->ops[i].slopes, Hq * 4, cudaMemcpyHostToDevice, s));
+    if (ce != cudaSuccess) {
+        join();
+        return fail(BSMT_ERR_CUDA, "host pipeline: %s", cudaGetErrorString(ce));
+    }
+    if (mask_spec != nullptr) {
+        st = bsmt_create_block_mask(&dspec, L.Bm, 1, M, N, 128, 128, &bm, stream);
+        if (st != BSMT_OK) {
+            join();
+            return st;
+        }
+    }
+    // 2. inputs of every piece, in order, on the input copy stream
+    for (int i = 0; i < np; ++i) {
+        const HostPiece& pc = pcs[i];
+        const int64_t qoff = (pc.b0 * Hq + pc.g0 * G) * M * D * 2;
+        const int64_t qlen = (pc.b1 - pc.b0) * (pc.g1 - pc.g0) * G * M * D * 2;
+        const int64_t koff = (pc.b0 * Hkv + pc.g0) * N * D * 2;
+        const int64_t klen = (pc.b1 - pc.b0) * (pc.g1 - pc.g0) * N * D * 2;
+        cuda_ok(cudaMemcpyAsync(wq + qoff, static_cast<const char*>(q) + qoff, qlen, cudaMemcpyHostToDevice, hc->s_in));
+        if (klen > 0) {
+            cuda_ok(cudaMemcpyAsync(wk + koff, static_cast<const char*>(k) + koff, klen, cudaMemcpyHostToDevice,
+                                    hc->s_in));
+            cuda_ok(cudaMemcpyAsync(wv + koff, static_cast<const char*>(v) + koff, klen, cudaMemcpyHostToDevice,
+                                    hc->s_in));
+        }
+        cuda_ok(cudaEventRecord(ev[i], hc->s_in));
+    }
+    // 3. each piece's attention once its inputs are in, then its outputs back
+    for (int i = 0; i < np && ce == cudaSuccess; ++i) {
+        const HostPiece& pc = pcs[i];
+        const int64_t Bp = pc.b1 - pc.b0, Hkvp = pc.g1 - pc.g0, Hqp = Hkvp * G;
+        const int64_t qrow = pc.b0 * Hq + pc.g0 * G;  // first (b, hq) row of the piece
+        const int64_t krow = pc.b0 * Hkv + pc.g0;
+        bsmt_block_mask bmi = bm;
+        bsmt_mask_spec si;
+        if (mask_spec != nullptr) {
+            si = dspec;
+            if (L.Bm > 1) {
+                bmi.kv_num_blocks += pc.b0 * L.QB;
+                bmi.full_kv_num_blocks += pc.b0 * L.QB;
+                bmi.kv_indices += pc.b0 * L.QB * L.KB;
+                bmi.full_kv_indices += pc.b0 * L.QB * L.KB;
+                bmi.B = static_cast<int32_t>(Bp);
+            }
+            if (L.has_doc && L.doc_batch > 1) {
+                si.q_doc_ids += pc.b0 * M;
+                si.kv_doc_ids += pc.b0 * N;
+                si.doc_batch = static_cast<int32_t>(Bp);
+            }
+        }
+        bsmt_score_spec sc = dscore;
+        for (int j = 0; j < sc.num_ops; ++j) {
+            if (sc.ops[j].kind != BSMT_SCORE_ALIBI) continue;
+            if (sc.ops[j].slopes != nullptr) {
+                sc.ops[j].slopes += pc.g0 * G;
+            } else {
+                if (sc.ops[j].num_heads <= 0) sc.ops[j].num_heads = static_cast<int32_t>(Hq);
+                sc.ops[j].head_offset += static_cast<int32_t>(pc.g0 * G);
+            }
+        }
+        cuda_ok(cudaStreamWaitEvent(s, ev[i], 0));
+        if (ce != cudaSuccess) break;
+        st = attention(wq + qrow * M * D * 2, wk + krow * N * D * 2, wv + krow * N * D * 2, Bp, Hqp, Hkvp, M, N, D,
+                       mask_spec != nullptr ? &bmi : nullptr, mask_spec != nullptr ? &si : nullptr, &sc, scale,
+                       enable_gqa, 1, nullptr, nullptr, wo + qrow * M * D * 2, wl + qrow * M, stream);
+        if (st != BSMT_OK) {
+            join();
+            return st;
+        }
+        cuda_ok(cudaEventRecord(ev[kMaxHostPieces + i], s));
+        cuda_ok(cudaStreamWaitEvent(hc->s_out, ev[kMaxHostPieces + i], 0));
+        cuda_ok(cudaMemcpyAsync(static_cast<char*>(out) + qrow * M * D * 2, wo + qrow * M * D * 2, Bp * Hqp * M * D * 2,
+                                cudaMemcpyDeviceToHost, hc->s_out));
+        cuda_ok(cudaMemcpyAsync(lse + qrow * M, wl + qrow * M, Bp * Hqp * M * 4, cudaMemcpyDeviceToHost, hc->s_out));
+    }
+    join();
+    if (ce != cudaSuccess) return fail(BSMT_ERR_CUDA, "host pipeline: %s", cudaGetErrorString(ce));
     return ok();
 }

@@ -30,8 +30,12 @@
  *   - Argument checks happen on the host, before any launch. A call that
  *     returns an error has launched nothing and written nothing.
  *   - Device pointers are owned by the caller. The library never allocates,
- *     frees or keeps device memory beyond the call. Its only global device
- *     state is one status word per device.
+ *     frees or keeps device memory beyond the call. Its global device state
+ *     is one status word per device and the static split-KV scratch of
+ *     bsmt_flex_attention_fwd_splitkv_static (both part of the library's
+ *     module, so resident on every device where the module is loaded).
+ *     bsmt_flex_attention_host also keeps, per device, two copy streams and
+ *     a pool of events, created on its first call there.
  *   - Work is enqueued on the caller's stream (a cudaStream_t passed as
  *     void*; NULL is the legacy default stream). Calls do not synchronize.
  *   - Errors found on the device set the status word and leave the outputs
@@ -120,8 +124,15 @@ typedef struct bsmt_mask_spec {
  * page, "A gallery that grew into a toolkit": score_mod changes a score
  * before the softmax.
  *   SOFTCAP  value = cap > 0:  s <- cap * tanh(s / cap)
- *   ALIBI    s <- s + m_h * (j - i). The slopes m_h are device float[Hq],
- *            or NULL for m_h = 2^(-8(h+1)/Hq).
+ *   ALIBI    s <- s + m_h * (j - i) (transformerlab page, registry table,
+ *            "alibi"). The slopes m_h are device float[Hq], or NULL for the
+ *            default slopes m_h = 2^(-8(h0 + h + 1) / Ht): h0 = head_offset
+ *            and Ht = num_heads place this call's Hq heads inside a model
+ *            of Ht heads, so a call on a slice of the heads gets the slopes
+ *            of those heads. num_heads <= 0 means Hq (and head_offset must
+ *            then be 0); otherwise 0 <= head_offset and
+ *            head_offset + Hq <= num_heads, else BSMT_ERR_INVALID_ARGUMENT.
+ *            Both fields are ignored when slopes is given and for SOFTCAP.
  */
 #define BSMT_MAX_SCORE_OPS 2
 enum { BSMT_SCORE_NONE = 0, BSMT_SCORE_SOFTCAP = 1, BSMT_SCORE_ALIBI = 2 };
@@ -130,6 +141,8 @@ typedef struct bsmt_score_op {
     int32_t kind;          /* BSMT_SCORE_* */
     float value;           /* SOFTCAP: cap */
     const float* slopes;   /* ALIBI: device float[Hq] or NULL */
+    int32_t head_offset;   /* ALIBI default slopes: model head index of this call's head 0 */
+    int32_t num_heads;     /* ALIBI default slopes: the model's head count (<= 0: Hq) */
 } bsmt_score_op;
 
 typedef struct bsmt_score_spec {
@@ -301,6 +314,54 @@ bsmt_status bsmt_flex_attention_fwd_splitkv_static(const void* q, const void* k,
                                                    const bsmt_mask_spec* mask_spec, const bsmt_score_spec* score,
                                                    float scale, int32_t enable_gqa, int32_t num_splits, void* out,
                                                    float* lse, void* stream);
+
+/* --------------------------------------------------------- host buffers
+ * flex_attention on inputs and outputs in host memory, end to end: the
+ * create_block_mask / flex_attention example of the tensorplay.nn.attention
+ * page for a caller whose tensors live on the host. One call
+ *   1. copies the document ids and ALiBi slopes (if any) to the device and
+ *      builds the BlockMask of mask_spec there (bsmt_create_block_mask, with
+ *      B = 1 unless the document ids differ per batch row, and H = 1: the
+ *      mask does not depend on the head);
+ *   2. cuts the work into about `pieces` independent pieces along (batch
+ *      row, group of kv heads with their query heads), and pipelines them:
+ *      the host-to-device copy of piece i+1, the attention of piece i and the
+ *      device-to-host copy of piece i-1 run at the same time, on two copy
+ *      streams of the library and the caller's stream;
+ *   3. makes `stream` wait for the last copy, so that once `stream` has
+ *      passed the call, out and lse hold the result.
+ * Every copy is one cudaMemcpyAsync of a contiguous range.
+ *
+ * Arguments:
+ *   q          host bf16 [B, Hq, M, D], contiguous
+ *   k, v       host bf16 [B, Hkv, N, D]
+ *   mask_spec  as for bsmt_create_block_mask, but its document id arrays
+ *              are HOST int32 [doc_batch, M] and [doc_batch, N]; NULL means
+ *              no mask (every tile computed)
+ *   score      as for bsmt_flex_attention_fwd, but ALiBi slopes are HOST
+ *              float[Hq]; NULL means none
+ *   scale, enable_gqa  as for bsmt_flex_attention_fwd
+ *   pieces     the number of pieces to aim for (<= 0: 16); at most 256 are
+ *              made
+ *   workspace  caller-owned device memory, 256-byte aligned, at least
+ *              bsmt_flex_attention_host_workspace_bytes bytes: it holds the
+ *              device copies of q, k, v, out, lse, the BlockMask, the
+ *              document ids and the slopes. Reusable once `stream` has
+ *              passed the call.
+ *   out        host bf16 [B, Hq, M, D]; lse host float [B, Hq, M]
+ * Host buffers should be page-locked (cudaHostAlloc, or torch's
+ * pin_memory) so the copies run asynchronously and overlap; pageable memory
+ * gives the same result without the overlap. The host inputs must stay
+ * unchanged, and out and lse unread, until `stream` has passed the call.
+ * Calls on one device take a library lock while they enqueue. Argument
+ * errors are returned before anything is enqueued; a CUDA error in the
+ * middle returns BSMT_ERR_CUDA with the outputs unspecified. */
+bsmt_status bsmt_flex_attention_host_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t M, int64_t N,
+                                                     int64_t D, const bsmt_mask_spec* mask_spec, int64_t* bytes);
+bsmt_status bsmt_flex_attention_host(const void* q, const void* k, const void* v, int64_t B, int64_t Hq,
+                                     int64_t Hkv, int64_t M, int64_t N, int64_t D, const bsmt_mask_spec* mask_spec,
+                                     const bsmt_score_spec* score, float scale, int32_t enable_gqa, int32_t pieces,
+                                     void* workspace, int64_t workspace_bytes, void* out, float* lse, void* stream);
 
 /* --------------------------------------------------- packed sequences
  * Varlen attention in the cu_seqlens form (L-GATr "attention backends" page:

@@ -32,7 +32,8 @@ def test_every_declared_symbol_is_exported():
                             "bsmt_flex_attention_fwd_splitkv_static", "bsmt_seqlens_to_doc_ids",
                             "bsmt_flex_attention_fwd_packed", "bsmt_flex_attention_bwd_workspace_bytes",
                             "bsmt_flex_attention_bwd", "bsmt_flex_attention_bwd_packed",
-                            "bsmt_selftest_wait_timeout",
+                            "bsmt_selftest_wait_timeout", "bsmt_flex_attention_host_workspace_bytes",
+                            "bsmt_flex_attention_host",
                             "bsmt_last_error", "bsmt_check_device_status", "bsmt_version"])
     lib = ctypes.CDLL(bsmt.library_path())
     for n in names:
@@ -40,7 +41,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version():
-    assert _lib.bsmt_version() == (1 << 16)
+    assert _lib.bsmt_version() == (2 << 16)
 
 
 def shape(*args):
@@ -169,6 +170,81 @@ def test_flex_attention_score_errors():
     sc.ops[1].kind = bsmt.SCORE_ALIBI
     sc.ops[1].slopes = FAKE + 1
     assert attn(score=ctypes.byref(sc)) == INVALID
+
+
+def test_alibi_head_offset_checks():
+    # default ALiBi slopes for heads [head_offset, head_offset + Hq) of a model
+    # of num_heads heads: the range must lie inside the model
+    sc = _ScoreSpec()
+    sc.num_ops = 1
+    sc.ops[0].kind = bsmt.SCORE_ALIBI
+    for h0, nh, code in ((0, 0, OK), (0, 2, OK), (6, 8, OK), (1, 0, INVALID), (7, 8, INVALID),
+                         (-1, 8, INVALID), (0, 1, INVALID)):
+        sc.ops[0].head_offset, sc.ops[0].num_heads = h0, nh
+        assert attn(M=0, score=ctypes.byref(sc)) == code, (h0, nh, _lib.bsmt_last_error())
+    # with explicit slopes both fields are ignored
+    sc.ops[0].slopes = FAKE
+    sc.ops[0].head_offset, sc.ops[0].num_heads = 5, 1
+    assert attn(M=0, score=ctypes.byref(sc)) == OK
+
+
+def host_ws(B, Hq, Hkv, M, N, D, spec=None):
+    n = ctypes.c_int64(-1)
+    st = _lib.bsmt_flex_attention_host_workspace_bytes(B, Hq, Hkv, M, N, D,
+                                                       ctypes.byref(spec) if spec is not None else None,
+                                                       ctypes.byref(n))
+    return st, n.value
+
+
+def test_host_workspace_bytes():
+    r = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    B, Hq, Hkv, M, N, D = 2, 32, 8, 32768, 32768, 128
+    q, kv, l = B * Hq * M * D * 2, B * Hkv * N * D * 2, B * Hq * M * 4
+    slopes = 2 * r(Hq * 4)
+    assert host_ws(B, Hq, Hkv, M, N, D) == (OK, 2 * r(q) + 2 * r(kv) + r(l) + slopes)
+    # a mask adds its four tensors at B = H = 1 (the mask depends on neither)
+    QB = KB = 256
+    mask = 2 * r(QB * 4) + 2 * r(QB * KB * 4)
+    assert host_ws(B, Hq, Hkv, M, N, D, spec_of([(C, 0)])) == (OK, 2 * r(q) + 2 * r(kv) + r(l) + mask + slopes)
+    # document ids that differ per batch row: the mask keeps B rows, plus the ids
+    st, n = host_ws(2, 4, 4, 300, 500, 64, spec_of([(DOC, 0)], FAKE, FAKE, doc_batch=2))
+    q, kv, l = 2 * 4 * 300 * 64 * 2, 2 * 4 * 500 * 64 * 2, 2 * 4 * 300 * 4
+    mask = 2 * r(2 * 3 * 4) + 2 * r(2 * 3 * 4 * 4)
+    assert (st, n) == (OK, 2 * r(q) + 2 * r(kv) + r(l) + mask + r(2 * 300 * 4) + r(2 * 500 * 4) + 2 * r(16))
+    assert host_ws(2, 4, 4, 300, 500, 96)[0] == UNSUPPORTED
+    assert host_ws(3, 4, 4, 300, 500, 64, spec_of([(DOC, 0)], FAKE, FAKE, doc_batch=2))[0] == SHAPE
+    assert _lib.bsmt_flex_attention_host_workspace_bytes(1, 1, 1, 1, 1, 64, None, None) == INVALID
+
+
+def host_call(B=1, Hq=2, Hkv=2, M=256, N=256, D=64, spec=None, score=None, gqa=0, ws=FAKE, ws_bytes=1 << 40,
+              q=FAKE, out=FAKE, lse=FAKE):
+    return _lib.bsmt_flex_attention_host(q, FAKE, FAKE, B, Hq, Hkv, M, N, D,
+                                         ctypes.byref(spec) if spec is not None else None,
+                                         ctypes.byref(score) if score is not None else None, ctypes.c_float(0.0),
+                                         gqa, 16, ctypes.c_void_p(ws), ws_bytes, out, lse, None)
+
+
+def test_host_entry_argument_errors():
+    """Every check of the host-buffer entry point runs before anything is
+    enqueued (the attention's own checks at the full size included)."""
+    assert host_call(D=96) == UNSUPPORTED
+    assert host_call(Hq=3, Hkv=2, gqa=1) == SHAPE
+    assert host_call(Hq=4, Hkv=2, gqa=0) == SHAPE
+    assert host_call(M=-1) == INVALID
+    assert host_call(q=0) == INVALID
+    assert host_call(ws=0) == INVALID
+    assert host_call(ws=FAKE + 16) == INVALID                 # not 256-byte aligned
+    assert host_call(ws_bytes=1000) == INVALID                # too small
+    assert host_call(spec=spec_of([(C, 0), (AND, 2)])) == INVALID
+    assert host_call(spec=spec_of([(DOC, 0)])) == INVALID    # document without ids
+    assert host_call(N=1025 * 128) == UNSUPPORTED            # more kv blocks than a row supports
+    sc = _ScoreSpec()
+    sc.num_ops = 1
+    sc.ops[0].kind = bsmt.SCORE_SOFTCAP
+    sc.ops[0].value = -2.0
+    assert host_call(score=sc) == INVALID
+    assert host_call(B=0) == OK                                # nothing to compute, nothing enqueued
+    assert host_call(M=0) == OK
 
 
 def block_mask_c(B=1, H=1, QB=2, KB=2, M=256, N=256, bq=128):
