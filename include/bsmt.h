@@ -295,18 +295,31 @@ bsmt_status bsmt_flex_attention_fwd_splitkv(const void* q, const void* k, const 
                                             int32_t num_splits, void* workspace, int64_t workspace_bytes, void* out,
                                             float* lse, void* stream);
 
-/* Split-KV without a caller workspace: the same computation as
+/* Split-KV without a caller workspace. The pages have no counterpart of this
+ * entry point: it exists for callers that cannot allocate device memory,
+ * such as a server whose memory manager reserves the whole device up front
+ * and forbids other allocations, or a plug-in whose host framework owns
+ * every allocation. It runs the same computation as
  * bsmt_flex_attention_fwd_splitkv, with the workspace taken from a static
  * device array inside the library (BSMT_SPLITKV_SCRATCH_BYTES per device),
- * so the call allocates no memory. The pages have no counterpart of this
- * entry point; it is an allocation-free form of the split-KV call.
+ * and calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - The array is part of the library's module: every device on which the
+ *     module is loaded holds its 32 MiB until the process exits, whether or
+ *     not this call is used.
  *   - Sizes whose workspace (bsmt_splitkv_workspace_bytes) exceeds the
- *     scratch return BSMT_ERR_UNSUPPORTED with the sizes in the message.
- *   - The scratch is shared by every call on the device: calls on one stream
- *     run in order, but calls that overlap (other streams, other host threads)
- *     race on it and give wrong results. Serialise them, or use the
+ *     scratch return BSMT_ERR_UNSUPPORTED with the sizes in the message;
+ *     nothing is launched.
+ *   - The scratch is shared by every call on the device and keeps the last
+ *     call's contents. Nothing in it must start at zero: each split writes
+ *     every row it owns before the merge reads it. Calls on one stream run
+ *     in order, but calls that overlap on the GPU (other streams, other host
+ *     threads) race on it and give wrong results. Serialise them, or use the
  *     workspace form.
- *   - The scratch address is looked up once per device (checked) and kept. */
+ *   - The first call on a device does one-time set-up there, with that
+ *     device current: it looks the scratch's device address up with
+ *     cudaGetSymbolAddress (checked, then kept), sets the kernel's
+ *     shared-memory attribute and fetches the tensor-map encoder. Make that
+ *     first call before any stream capture. */
 #define BSMT_SPLITKV_SCRATCH_BYTES (32LL << 20)
 bsmt_status bsmt_flex_attention_fwd_splitkv_static(const void* q, const void* k, const void* v, int64_t B,
                                                    int64_t Hq, int64_t Hkv, int64_t M, int64_t N, int64_t D,

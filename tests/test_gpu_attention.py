@@ -159,6 +159,52 @@ def test_workload2_full_exhaustive():
     assert_attention_close(out, lse, ref_out, ref_lse, w.name)
 
 
+def _compare_slices(out, lse, tasks, results, what):
+    go = np.concatenate([out[b, hq, r0:r1] for (b, hq, r0, r1) in tasks])
+    gl = np.concatenate([lse[b, hq, r0:r1] for (b, hq, r0, r1) in tasks])
+    ro = np.concatenate([o for o, _ in results])
+    rl = np.concatenate([l for _, l in results])
+    assert_attention_close(go, gl, ro, rl, what)
+
+
+def test_workload3_full_exhaustive():
+    # causal + ALiBi at D = 64: every (b, hq) and every row, oracle in a pool
+    from tests import oracle_pool
+    w = workloads.get(3)
+    d = workloads.make(w)
+    out, lse = gpu_attention(d["q"], d["k"], d["v"], d["mask"], d["score_mods"], w.scale, w.enable_gqa)
+    tasks = oracle_pool.row_tasks([(b, h) for b in range(w.B) for h in range(w.Hq)], w.M, w.M)
+    res = oracle_pool.forward_rows(d["q"], d["k"], d["v"], tasks, d["mask"], d["score_mods"], w.scale)
+    _compare_slices(out, lse, tasks, res, w.name)
+
+
+def test_workload4_whole_heads():
+    # document and causal: every row of four query heads
+    from tests import oracle_pool
+    w = workloads.get(4)
+    d = workloads.make(w)
+    out, lse = gpu_attention(d["q"], d["k"], d["v"], d["mask"], d["score_mods"], w.scale, w.enable_gqa)
+    tasks = oracle_pool.row_tasks([(0, 0), (0, 11), (0, 20), (0, 31)], w.M, 4096)
+    res = oracle_pool.forward_rows(d["q"], d["k"], d["v"], tasks, d["mask"], d["score_mods"], w.scale)
+    _compare_slices(out, lse, tasks, res, w.name)
+
+
+def test_workload5_whole_heads_and_transition_blocks():
+    # StreamingLLM at full size: every row of two (b, hq) slices, one per
+    # batch row and in different GQA groups, and every row of q-blocks 0-10
+    # (where the window leaves the sink's block) for all four query heads of
+    # one kv head
+    from tests import oracle_pool
+    w = workloads.get(5)
+    d = workloads.make(w)
+    out, lse = gpu_attention(d["q"], d["k"], d["v"], d["mask"], d["score_mods"], w.scale, w.enable_gqa)
+    group = w.Hq // w.Hkv
+    tasks = oracle_pool.row_tasks([(0, 3), (1, 30)], w.M, 4096)
+    tasks += [(1, h, 0, 11 * 128) for h in range(5 * group, 6 * group)]
+    res = oracle_pool.forward_rows(d["q"], d["k"], d["v"], tasks, d["mask"], d["score_mods"], w.scale)
+    _compare_slices(out, lse, tasks, res, w.name)
+
+
 def test_repeatable_and_deterministic():
     w = workloads.get(1)
     d = workloads.make(w)

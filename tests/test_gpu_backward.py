@@ -203,6 +203,54 @@ def test_workloads_full_size_sampled(index):
     assert_close("dv rows", np.stack([dv[b, h, j] for b, h, j in ks]), ref_v, w.name)
 
 
+def _gpu_backward_full(w, d, dout):
+    dq, dk, dv = gpu_backward(d["q"], d["k"], d["v"], dout, d["mask"], d["score_mods"], w.scale, w.enable_gqa)
+    for t in (dq, dk, dv):
+        assert np.all(np.isfinite(t))
+    return dq, dk, dv
+
+
+def test_workload3_backward_exhaustive():
+    # causal + ALiBi at D = 64: all of dq, dk and dv, oracle in a pool
+    from tests import oracle_pool
+    w = workloads.get(3)
+    d = workloads.make(w)
+    dout = workloads.grad_output(w.seed + 50, w.B, w.Hq, w.M, w.D)
+    dq, dk, dv = _gpu_backward_full(w, d, dout)
+    tasks = oracle_pool.row_tasks([(b, h) for b in range(w.B) for h in range(w.Hq)], w.M, w.M)
+    res = oracle_pool.backward_rows(d["q"], d["k"], d["v"], dout, tasks, d["mask"], d["score_mods"], w.scale,
+                                    want_kv=True)
+    ref_q = np.zeros_like(dq)
+    ref_k, ref_v = np.zeros_like(dk), np.zeros_like(dv)
+    group = w.Hq // w.Hkv
+    for (b, hq, r0, r1), (gq, gk, gv) in zip(tasks, res):
+        ref_q[b, hq, r0:r1] = gq
+        ref_k[b, hq // group] += gk
+        ref_v[b, hq // group] += gv
+    assert_grads_close([dq, dk, dv], [ref_q, ref_k, ref_v], w.name)
+
+
+@pytest.mark.parametrize("index", [4, 5])
+def test_workload_dq_whole_heads(index):
+    # every dq row of whole (b, hq) slices (and, for the streaming workload,
+    # of q-blocks 0-10 for the four query heads of one kv head)
+    from tests import oracle_pool
+    w = workloads.get(index)
+    d = workloads.make(w)
+    dout = workloads.grad_output(w.seed + 50, w.B, w.Hq, w.M, w.D)
+    dq, _, _ = _gpu_backward_full(w, d, dout)
+    if index == 4:
+        tasks = oracle_pool.row_tasks([(0, 0), (0, 11), (0, 20), (0, 31)], w.M, 4096)
+    else:
+        group = w.Hq // w.Hkv
+        tasks = oracle_pool.row_tasks([(0, 3), (1, 30)], w.M, 4096)
+        tasks += [(1, h, 0, 11 * 128) for h in range(5 * group, 6 * group)]
+    res = oracle_pool.backward_rows(d["q"], d["k"], d["v"], dout, tasks, d["mask"], d["score_mods"], w.scale)
+    got = np.concatenate([dq[b, hq, r0:r1] for (b, hq, r0, r1) in tasks])
+    ref = np.concatenate([gq for gq, _, _ in res])
+    assert_close("dq rows", got, ref, w.name)
+
+
 def test_autograd_through_flex_attention():
     """q, k, v that require grad: flex_attention records the op and
     backpropagating sum(out * dout) gives the same bits as the direct

@@ -270,3 +270,31 @@ def test_varlen_causal_equals_document_and_causal():
     o2, l2 = oa.flex_attention(q.permute(1, 0, 2)[None], k.permute(1, 0, 2)[None], v.permute(1, 0, 2)[None], tree)
     assert np.allclose(out, o2[0].transpose(1, 0, 2), atol=1e-12)
     assert np.allclose(lse, l2[0], atol=1e-12)
+
+
+def test_pool_rows_equal_the_oracle():
+    # the spawned-pool runner of the GPU tests cuts slices into row ranges;
+    # rows are independent, so it must reproduce the oracle itself
+    from tests import oracle_pool
+    import workloads
+    q, k, v = workloads.random_inputs(90, 2, 4, 2, 300, 260, 64)
+    dout = workloads.grad_output(91, 2, 4, 300, 64)
+    tree = ("and", ("causal",), ("or", ("sink", 3), ("window", 70)))
+    mods = (("softcap", 9.0), ("alibi", None))
+    want_o, want_l = oa.flex_attention(q, k, v, tree, mods, None, True)
+    tasks = oracle_pool.row_tasks([(0, 1), (1, 3)], 300, 128)
+    got = oracle_pool.forward_rows(q, k, v, tasks, tree, mods, None, chunk=50)
+    for (b, hq, r0, r1), (o, l) in zip(tasks, got):
+        np.testing.assert_allclose(o, want_o[b, hq, r0:r1], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l, want_l[b, hq, r0:r1], rtol=0, atol=1e-12)
+    from oracle import backward as ob
+    dq, dk, dv = ob.flex_attention_backward(q, k, v, dout, tree, mods, None, True)
+    all_tasks = oracle_pool.row_tasks([(b, h) for b in range(2) for h in range(4)], 300, 100)
+    res = oracle_pool.backward_rows(q, k, v, dout, all_tasks, tree, mods, None, want_kv=True, chunk=64)
+    gk, gv = np.zeros_like(dk), np.zeros_like(dv)
+    for (b, hq, r0, r1), (gq, pk, pv) in zip(all_tasks, res):
+        np.testing.assert_allclose(gq, dq[b, hq, r0:r1], rtol=0, atol=1e-12)
+        gk[b, hq // 2] += pk
+        gv[b, hq // 2] += pv
+    np.testing.assert_allclose(gk, dk, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(gv, dv, rtol=0, atol=1e-11)
