@@ -305,6 +305,100 @@ def side_kernels(bsmt, mask, w, dev, hbm_peak: float) -> dict:
     return res
 
 
+def workload_sweep(bsmt, dev, peak_tflops: float, hbm_peak: float) -> list:
+    """Each of the five workloads on its own: the attention kernel alone (CUDA
+    graph of repeated launches, CUDA events), its counted TFLOP/s and fraction
+    of the measured bf16 peak, the builder at the workload's own shape (GB/s of
+    its four outputs) and the sparsity."""
+    res = []
+    for w in workloads.WORKLOADS:
+        data = workloads.make(w)
+        q, k, v = (t.to(dev) for t in (data["q"], data["k"], data["v"]))
+        mask = bsmt.mask_from_tree(data["mask"], device=dev)
+        mods = [bsmt.ScoreMod(m.kind, m.value, None if m.slopes is None else m.slopes.to(dev))
+                for m in bsmt.score_mods_from_list(data["score_mods"])]
+        bm = bsmt.create_block_mask(mask, w.B, w.Hq, w.M, w.N, device=dev)
+        out = torch.empty((w.B, w.Hq, w.M, w.D), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((w.B, w.Hq, w.M), dtype=torch.float32, device=dev)
+        reps = 20 if w.index <= 2 else 5
+        ms = _time_launches(lambda: bsmt.flex_attention(q, k, v, block_mask=bm, score_mod=mods, scale=w.scale,
+                                                        enable_gqa=w.enable_gqa, out=out, lse=lse), reps=reps)
+        ms_b = _time_launches(lambda: bsmt.create_block_mask(mask, w.B, w.Hq, w.M, w.N, device=dev, out=bm),
+                              reps=20)
+        bsmt.check_device_status(dev)
+        flops = counted_flops(bm, w.D)
+        tf = flops / (ms * 1e-3) / 1e12
+        Bm, Hm, QB, KB = bm.shape
+        nbytes = 2 * 4 * Bm * Hm * QB + 2 * 4 * Bm * Hm * QB * KB
+        qkv_bytes = sum(x.numel() * 2 for x in (q, k, v))
+        res.append({"index": w.index, "workload": w.name, "attn_ms": ms, "counted_gflop": flops / 1e9,
+                    "tflops": tf, "frac": tf / peak_tflops, "frac_of_datasheet": tf / DATASHEET_BF16_TFLOPS,
+                    "builder_ms": ms_b, "builder_gbs": nbytes / (ms_b * 1e-3) / 1e9,
+                    "builder_frac": nbytes / (ms_b * 1e-3) / 1e9 / hbm_peak,
+                    "sparsity_pct": bm.sparsity(),
+                    "l2": "inputs larger than L2" if qkv_bytes > 126e6 else "inputs fit in L2 (repeated launches)"})
+        del q, k, v, out, lse, bm
+    torch.cuda.empty_cache()
+    return res
+
+
+def all_partial(bsmt, bm):
+    """The same kept tiles as ``bm``, every one listed as PARTIAL (no FULL
+    list): the kernel then applies mask_mod on every tile. Built from the
+    block-level dense map (the library's to_dense kernel); each row's kept kv
+    blocks in ascending order, then zeros."""
+    dense = bm.to_dense()
+    KB = dense.shape[-1]
+    ar = torch.arange(KB, dtype=torch.int32, device=dense.device)
+    key = torch.where(dense > 0, ar, ar + KB)
+    idx = torch.sort(key, dim=-1).values
+    num = dense.sum(-1, dtype=torch.int32)
+    idx = torch.where(ar < num[..., None], idx, torch.zeros_like(idx)).to(torch.int32).contiguous()
+    return bsmt.BlockMask.from_kv_blocks(num.contiguous(), idx, torch.zeros_like(num), torch.zeros_like(idx),
+                                         mask_mod=bm.mask_mod, seq_lengths=bm.seq_lengths)
+
+
+def full_partial_ablation(bsmt, dev) -> list:
+    """The tensorplay.nn.attention page (BlockMask "Details" item 2) stores
+    full blocks apart so that mask_mod is skipped on them. Each case is timed
+    with its BlockMask and with every kept tile listed as partial (same tiles,
+    same output bits)."""
+    res = []
+    g = torch.Generator(device="cpu").manual_seed(11)
+    w5 = workloads.get(5)
+    d5 = workloads.make(w5)
+    cases = [(w5.name, d5["q"], d5["k"], d5["v"], d5["mask"], w5.enable_gqa),
+             ("causal_b1_h32_s8192_d128",) + tuple(torch.randn((1, 32, 8192, 128), generator=g).to(torch.bfloat16)
+                                                   for _ in range(3)) + (("causal",), False)]
+    for name, qh, kh, vh, tree, gqa in cases:
+        q, k, v = (t.to(dev) for t in (qh, kh, vh))
+        B, Hq, M, D = q.shape
+        N = k.shape[2]
+        mask = bsmt.mask_from_tree(tree, device=dev)
+        bm = bsmt.create_block_mask(mask, B, Hq, M, N, device=dev)
+        bmp = all_partial(bsmt, bm)
+        outs = []
+        times = []
+        for b in (bm, bmp):
+            out = torch.empty((B, Hq, M, D), dtype=torch.bfloat16, device=dev)
+            lse = torch.empty((B, Hq, M), dtype=torch.float32, device=dev)
+            times.append(_time_launches(lambda: bsmt.flex_attention(q, k, v, block_mask=b, enable_gqa=gqa, out=out,
+                                                                    lse=lse), reps=5))
+            outs.append((out, lse))
+        bsmt.check_device_status(dev)
+        flops = counted_flops(bm, D)
+        res.append({"case": name, "full_and_partial_ms": times[0], "all_partial_ms": times[1],
+                    "full_and_partial_tflops": flops / (times[0] * 1e-3) / 1e12,
+                    "all_partial_tflops": flops / (times[1] * 1e-3) / 1e12,
+                    "speedup": times[1] / times[0],
+                    "full_tiles": int(bm.full_kv_num_blocks.sum()), "partial_tiles": int(bm.kv_num_blocks.sum()),
+                    "outputs_identical": bool(torch.equal(outs[0][0], outs[1][0]) and
+                                              torch.equal(outs[0][1], outs[1][1]))})
+        del q, k, v, outs
+    torch.cuda.empty_cache()
+    return res
+
+
 def counted_flops(bm, D: int) -> int:
     """4*128*128*D per kept tile per (b, hq); the mask is built at [B, Hq]."""
     tiles = int(bm.kv_num_blocks.sum().item()) + int(bm.full_kv_num_blocks.sum().item())
@@ -338,8 +432,10 @@ def cpu_baseline(w, data, max_rows: int = 16384, chunk: int = 1024, cls=None):
     q-blocks of (b=0, hq=0) from the top of the sequence (the rows with the most
     kept tiles), in chunks of ``chunk`` rows, counted with the same tile rule as
     the GPU metric."""
-    from threadpoolctl import threadpool_info
+    from threadpoolctl import threadpool_info, threadpool_limits
     from oracle import attention as oa
+    # the oracle's matrix products use one BLAS thread per host core given to this process
+    threadpool_limits(len(os.sched_getaffinity(0)))
     from oracle import block_mask as obm
 
     rows_per_block = 128
@@ -369,8 +465,9 @@ def cpu_baseline(w, data, max_rows: int = 16384, chunk: int = 1024, cls=None):
         oa.flex_attention_sampled(data["q"], data["k"], data["v"], samples[c0:c0 + chunk], data["mask"],
                                   data["score_mods"], w.scale, w.enable_gqa)
     dt = time.perf_counter() - t0
-    threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
-    res = {"value": flops / dt / 1e12, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+    blas = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    res = {"value": flops / dt / 1e12, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "blas_threads": int(blas),
+           "kind": "oracle",
            "sample": f"{len(samples)} query rows = q-blocks {qbs[0]}..{qbs[-1]} of (b=0, hq=0), "
                      f"{tiles} kept tiles, {dt:.1f} s"}
     if block_mask is not None:
@@ -490,20 +587,24 @@ def main():
     hq_, hk_, hv_ = (x.pin_memory() for x in (data["q"], data["k"], data["v"]))
     ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    # the mask with its document ids (if any) in pinned host memory, and ALiBi
+    # slopes on the host: the host-buffer call copies them in itself
+    hmask = bsmt.mask_from_tree(data["mask"])
     doc_host = []
-    if w.mask == "doc_causal":
-        doc_host = [torch.as_tensor(data["mask"][1][1]).pin_memory()]
+    if hmask.q_doc_ids is not None:
+        doc_host = [hmask.q_doc_ids.pin_memory(), hmask.kv_doc_ids.pin_memory()]
+        hmask = bsmt.MaskMod(hmask.nodes, doc_host[0], doc_host[1])
+    hmods = bsmt.score_mods_from_list(data["score_mods"])
+    slopes_host = [m.slopes for m in hmods if m.slopes is not None]
+    hws = torch.empty(bsmt.host_workspace_bytes(w.B, w.Hq, w.Hkv, w.M, w.N, w.D, hmask), dtype=torch.uint8,
+                      device=dev)
 
     def e2e_step():
-        # the public host-tensor call: block mask built on the device, copies in
-        # and out pipelined with the attention of independent pieces
-        m = mask
-        if doc_host:
-            dd = doc_host[0].to(dev, non_blocking=True)
-            m = bsmt.and_masks(bsmt.document(dd), bsmt.causal())
-        bsmt.flex_attention_host(hq_, hk_, hv_, mask_mod=m, score_mod=mods, scale=w.scale,
-                                 enable_gqa=w.enable_gqa, device=dev, out=ho, lse=hl)
-        torch.cuda.current_stream(dev).synchronize()
+        # the public host-buffer call (bsmt_flex_attention_host): document ids
+        # and slopes in, block mask built on the device, pieces' copies in and
+        # out pipelined with their attention; returns once out/lse are on the host
+        bsmt.flex_attention_host(hq_, hk_, hv_, mask_mod=hmask, score_mod=hmods, scale=w.scale,
+                                 enable_gqa=w.enable_gqa, device=dev, out=ho, lse=hl, workspace=hws)
 
     e2e_step()
     if dist:
@@ -517,16 +618,19 @@ def main():
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
     (e2e_ms,), _ = reduce_over_ranks(dist, dev, (e2e_ms,), 0)
-    h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_)) + sum(x.numel() * 4 for x in doc_host)
+    h2d = (sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_)) + sum(x.numel() * 4 for x in doc_host)
+           + sum(x.numel() * 4 for x in slopes_host))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
     peaks, peak_src = load_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     side = None if args.no_side_kernels else side_kernels(bsmt, mask, w, dev, hbm_peak)
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     if side is not None:
         side["backward"] = time_backward(bsmt, w, q, k, v, out, lse, bm, mods, dev, flops)
+        side["workloads"] = workload_sweep(bsmt, dev, peak, hbm_peak)
+        side["full_partial_ablation"] = full_partial_ablation(bsmt, dev)
     attn_tflops = (flops / (attn_ms * 1e-3)) / 1e12
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     prof = profile_figures(w.name)
     line = {
         "metric": METRIC,
