@@ -687,23 +687,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // score_mod on every visited tile. Other modes move to base-2
                 // units here; the plain mode keeps raw scores and folds
                 // scale * log2(e) into the exponent's FFMA below.
+                // Column pairs go through the packed f32x2 FMA pipe (the same
+                // roundings as one column at a time).
                 if constexpr (SCORE != kScoreNone) {
                     const float tile_bias = sl2 * static_cast<float>(kb * 128 - q);
+                    const float tile_pos = static_cast<float>(kb * 128 - q);  // exact below 2^24
+                    const float u_mul = p.scale * p.inv_cap;
+                    const float capl2 = p.cap * kLog2e;
 #pragma unroll
-                    for (int j = 0; j < 128; ++j) {
-                        float s = x[j];
+                    for (int j = 0; j < 128; j += 2) {
+                        const float j0 = static_cast<float>(j), j1 = static_cast<float>(j + 1);
                         if constexpr (SCORE == kScoreSoftcap) {
-                            s = (p.cap * kLog2e) * tanh_approx(s * (p.scale * p.inv_cap));
+                            float u0, u1;
+                            mul2(u0, u1, x[j], x[j + 1], u_mul, u_mul);
+                            mul2(x[j], x[j + 1], capl2, capl2, tanh_approx(u0), tanh_approx(u1));
                         } else if constexpr (SCORE == kScoreAlibi) {
-                            s = fmaf(s, p.scale_log2, fmaf(sl2, static_cast<float>(j), tile_bias));
+                            float c0, c1;
+                            fma2(c0, c1, sl2, sl2, j0, j1, tile_bias, tile_bias);
+                            fma2(x[j], x[j + 1], x[j], x[j + 1], p.scale_log2, p.scale_log2, c0, c1);
                         } else if constexpr (SCORE == kScoreSoftcapAlibi) {
-                            s = fmaf((p.cap * kLog2e), tanh_approx(s * (p.scale * p.inv_cap)),
-                                     fmaf(sl2, static_cast<float>(j), tile_bias));
-                        } else {
-                            const float t = fmaf(s, p.scale, hdr.slope * static_cast<float>(kb * 128 + j - q));
-                            s = (p.cap * kLog2e) * tanh_approx(t * p.inv_cap);
+                            float u0, u1, c0, c1;
+                            mul2(u0, u1, x[j], x[j + 1], u_mul, u_mul);
+                            fma2(c0, c1, sl2, sl2, j0, j1, tile_bias, tile_bias);
+                            fma2(x[j], x[j + 1], capl2, capl2, tanh_approx(u0), tanh_approx(u1), c0, c1);
+                        } else {  // ALiBi, then the soft-cap
+                            float r0, r1, b0, b1, t0, t1;
+                            add2(r0, r1, tile_pos, tile_pos, j0, j1);       // kv - q, exact
+                            mul2(b0, b1, hdr.slope, hdr.slope, r0, r1);
+                            fma2(t0, t1, x[j], x[j + 1], p.scale, p.scale, b0, b1);
+                            mul2(t0, t1, t0, t1, p.inv_cap, p.inv_cap);
+                            mul2(x[j], x[j + 1], capl2, capl2, tanh_approx(t0), tanh_approx(t1));
                         }
-                        x[j] = s;
                     }
                 }
                 // mask_mod on partial tiles only

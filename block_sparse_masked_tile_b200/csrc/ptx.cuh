@@ -477,6 +477,12 @@ __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, f
     d1 = r.y;
 }
 
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+    const float2 r = __fmul2_rn(make_float2(a0, a1), make_float2(b0, b1));
+    d0 = r.x;
+    d1 = r.y;
+}
+
 __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
     const float2 r = __fadd2_rn(make_float2(a0, a1), make_float2(b0, b1));
     d0 = r.x;
