@@ -152,7 +152,7 @@ constexpr int kEmuCols = 8;
 
 // 2^x on the FMA pipe for a pair: round x to n, 2^f by a degree-3 polynomial
 // for f = x - n in [-1/2, 1/2] (minimax in relative error, max 1.02e-4; the
-// coefficients come from csrc/fit_exp2_poly.py), and n goes straight into the
+// coefficients come from tests/fit_exp2_poly.py), and n goes straight into the
 // exponent bits. Inputs are clamped at -125 so the exponent field stays
 // positive; 2^-125 is far below what a bf16 P or an fp32 row sum can see.
 constexpr float kExp2C1 = 0.69328314f;
