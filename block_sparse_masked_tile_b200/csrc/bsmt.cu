@@ -437,7 +437,15 @@ bsmt_status bsmt_create_block_mask(const bsmt_mask_spec* spec, int64_t B, int64_
     groups = (p.Hm + p.heads_per_block - 1) / p.heads_per_block;
     if (gx > 0x7FFFFFFF || groups > 65535) return fail(BSMT_ERR_UNSUPPORTED, "grid too large");
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(p.Bm), static_cast<unsigned>(groups));
-    bsmt::mask_build_kernel<<<grid, bsmt::kBuildWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(dnf, p);
+    // Rows staged in shared memory and written by bulk copies when their size
+    // and the lists' alignment allow it.
+    const bool staged = p.KB > 0 && p.KB % 4 == 0 && p.KB <= bsmt::kStagedMaxKB && aligned(p.kv_idx, 16) &&
+                        aligned(p.full_idx, 16);
+    if (staged)
+        bsmt::mask_build_kernel<true><<<grid, bsmt::kBuildWarps * 32, 2 * p.KB * 4, static_cast<cudaStream_t>(stream)>>>(
+            dnf, p);
+    else
+        bsmt::mask_build_kernel<false><<<grid, bsmt::kBuildWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(dnf, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "mask builder launch: %s", cudaGetErrorString(e));
     return ok();
@@ -724,7 +732,8 @@ extern "C" bsmt_status bsmt_block_mask_transpose(const bsmt_block_mask* kv, bsmt
     int dev = 0, nsm = 0;
     st = sm_count(&dev, &nsm);
     if (st != BSMT_OK) return st;
-    const int smem = static_cast<int>(bsmt::transpose_smem_bytes(kv->QB));
+    const int chunk = bsmt::transpose_chunk(kv->QB);
+    const int smem = static_cast<int>(bsmt::transpose_smem_bytes(kv->QB, chunk));
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(bsmt::mask_transpose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -734,6 +743,7 @@ extern "C" bsmt_status bsmt_block_mask_transpose(const bsmt_block_mask* kv, bsmt
     p.Hm = kv->H;
     p.QB = kv->QB;
     p.KB = kv->KB;
+    p.chunk = chunk;
     p.kv_num = kv->kv_num_blocks;
     p.kv_idx = kv->kv_indices;
     p.full_num = kv->full_kv_num_blocks;
@@ -742,8 +752,8 @@ extern "C" bsmt_status bsmt_block_mask_transpose(const bsmt_block_mask* kv, bsmt
     p.q_idx = out->q_indices;
     p.full_q_num = out->full_q_num_blocks;
     p.full_q_idx = out->full_q_indices;
-    dim3 grid(static_cast<unsigned>((kv->KB + bsmt::kTransposeChunk - 1) / bsmt::kTransposeChunk),
-              static_cast<unsigned>(kv->H), static_cast<unsigned>(kv->B));
+    dim3 grid(static_cast<unsigned>((kv->KB + chunk - 1) / chunk), static_cast<unsigned>(kv->H),
+              static_cast<unsigned>(kv->B));
     bsmt::mask_transpose_kernel<<<grid, bsmt::kTransposeThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "transpose launch: %s", cudaGetErrorString(e));

@@ -14,11 +14,16 @@
 //   - FULL    = every in-range element allowed, tile inside both sequences;
 //   - PARTIAL = some element allowed but not FULL;
 //   - EMPTY   = no element allowed.
-// Writing: a mask is the same for every head, so all 8 warps then write the
-// row's lists for the heads of the block's group, a head per warp at a time.
-// Compaction is a ballot/popc prefix per 32-tile word; tails are zeroed with
-// 16-byte stores. The kernel is then an HBM writer.
+// Writing: a mask is the same for every head. With STAGED (KB a multiple of
+// 4, at most kStagedMaxKB, 16-byte aligned lists), the row's two lists are
+// compacted once into shared memory, zero tails included, and the bulk copy
+// engine writes them to every head of the block's group: two copies per
+// head, issued by one lane. Otherwise all 8 warps write the row's lists for
+// the heads of the group, a head per warp at a time, and zero the tails with
+// 16-byte stores. Compaction is a ballot/popc prefix per 32-tile word. The
+// kernel is then an HBM writer.
 #pragma once
+#include "bulk_copy.cuh"
 #include "mask_dnf.cuh"
 #include "ptx.cuh"
 
@@ -36,13 +41,21 @@ struct BuildParams {
 constexpr int kBuildWarps = 8;       // warps per block
 constexpr int kClassifyWarps = 4;    // warps that classify (one row per lane)
 constexpr int kWordsPerChunk = 8;    // 256 kv blocks per pass
+constexpr int kStagedMaxKB = 4096;   // staged rows: 2 x 4096 int32 = 32 KB of shared memory
 
+template <bool STAGED>
 __global__ void __launch_bounds__(kBuildWarps * 32)
     mask_build_kernel(const __grid_constant__ MaskDnf dnf, const BuildParams p) {
     __shared__ uint32_t part_f[kClassifyWarps][kWordsPerChunk];
     __shared__ uint32_t part_a[kClassifyWarps][kWordsPerChunk];
+    extern __shared__ __align__(16) int32_t staged[];  // STAGED: partial row [KB], then full row [KB]
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
+    if constexpr (STAGED) {
+        uint4* z = reinterpret_cast<uint4*>(staged);
+        for (int i = threadIdx.x; i < p.KB / 2; i += kBuildWarps * 32) z[i] = make_uint4(0u, 0u, 0u, 0u);
+        // (ordered before the compaction's writes by the first chunk's __syncthreads)
+    }
     const int qb = blockIdx.x;
     const int b = blockIdx.y;
     const int h0 = blockIdx.z * p.heads_per_block;
@@ -193,8 +206,20 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
                 cf += __popc(fw[w]);
             }
         }
+        if constexpr (STAGED) {
+            // this chunk's entries, once, into the shared rows (warp 0: every
+            // warp holds the same positions)
+            if (warp == 0) {
+#pragma unroll
+                for (int w = 0; w < kWordsPerChunk; ++w) {
+                    const int kb = c0 + 32 * w + lane;
+                    if (pos_p[w] >= 0) staged[pos_p[w]] = kb;
+                    if (pos_f[w] >= 0) staged[p.KB + pos_f[w]] = kb;
+                }
+            }
+        }
         // write this chunk's entries for the heads of the group
-        for (int h = h0 + warp; h < h1; h += kBuildWarps) {
+        for (int h = h0 + warp; !STAGED && h < h1; h += kBuildWarps) {
             const int64_t row = (static_cast<int64_t>(b) * p.Hm + h) * p.QB + qb;
             int32_t* pidx = p.kv_idx + row * p.KB;
             int32_t* fidx = p.full_idx + row * p.KB;
@@ -212,6 +237,25 @@ __global__ void __launch_bounds__(kBuildWarps * 32)
         }
     }
 
+    if constexpr (STAGED) {
+        // the staged rows (entries, then zeros) to every head of the group
+        fence_proxy_async_smem();
+        __syncthreads();
+        const uint32_t src = smem_u32(staged);
+        const uint32_t row_bytes = static_cast<uint32_t>(p.KB) * 4u;
+        for (int h = h0 + warp; h < h1; h += kBuildWarps) {
+            const int64_t row = (static_cast<int64_t>(b) * p.Hm + h) * p.QB + qb;
+            if (lane == 0) {
+                bulk_store_1d(p.kv_idx + row * p.KB, src, row_bytes);
+                bulk_store_1d(p.full_idx + row * p.KB, src + row_bytes, row_bytes);
+                bulk_commit_group();
+                p.kv_num[row] = cnt_p;
+                p.full_num[row] = cnt_f;
+            }
+        }
+        if (lane == 0) bulk_wait_group0();  // the shared rows are read before the block ends
+        return;
+    }
     // counts and zero tails
     for (int h = h0 + warp; h < h1; h += kBuildWarps) {
         const int64_t row = (static_cast<int64_t>(b) * p.Hm + h) * p.QB + qb;

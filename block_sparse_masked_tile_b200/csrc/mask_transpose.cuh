@@ -5,9 +5,10 @@
 // kv-side lists. For every kv block they hold the q blocks whose partial
 // (resp. full) list contains it, ascending, followed by zeros.
 //
-// One CTA per (b, h, chunk of 32 kv blocks). Its warps read every q row's
-// two lists of (b, h) and set one bit per (kv block of the chunk, q block) in
-// two shared-memory bitmaps. Each warp then compacts whole kv columns: a
+// One CTA per (b, h, chunk of kv blocks): up to kTransposeChunk kv blocks, so
+// that a (b, h) is scanned by few CTAs. Its warps read every q row's two
+// lists of (b, h) and set one bit per (kv block of the chunk, q block) in two
+// shared-memory bitmaps. Each warp then compacts whole kv columns: a
 // ballot/popc prefix per 32-bit word gives every set bit its position. The
 // kernel writes every element of its output columns, so it is bound by the
 // HBM writes of [B, H, KB, QB] x 2 lists.
@@ -21,11 +22,12 @@
 
 namespace bsmt {
 
-constexpr int kTransposeChunk = 32;   // kv blocks per CTA
-constexpr int kTransposeThreads = 256;
+constexpr int kTransposeChunk = 128;  // kv blocks per CTA (at most)
+constexpr int kTransposeThreads = 512;
 
 struct TransposeParams {
     int32_t Bm, Hm, QB, KB;
+    int32_t chunk;  // kv blocks per CTA
     const int32_t* kv_num;
     const int32_t* kv_idx;
     const int32_t* full_num;
@@ -36,20 +38,28 @@ struct TransposeParams {
     int32_t* full_q_idx;
 };
 
-// Shared memory: two bitmaps of kTransposeChunk x ceil(QB / 32) words.
-__host__ __device__ constexpr int64_t transpose_smem_bytes(int64_t QB) {
-    return 2 * kTransposeChunk * ((QB + 31) / 32) * 4;
+// Kv blocks per CTA: kTransposeChunk, or fewer so that the two bitmaps stay
+// within 96 KB of shared memory.
+__host__ __device__ constexpr int transpose_chunk(int64_t QB) {
+    const int64_t c = (96 * 1024) / (2 * 4 * ((QB + 31) / 32 > 0 ? (QB + 31) / 32 : 1));
+    return static_cast<int>(c < 1 ? 1 : (c > kTransposeChunk ? kTransposeChunk : c));
+}
+
+// Shared memory: two bitmaps of chunk x ceil(QB / 32) words.
+__host__ __device__ constexpr int64_t transpose_smem_bytes(int64_t QB, int chunk) {
+    return 2 * static_cast<int64_t>(chunk) * ((QB + 31) / 32) * 4;
 }
 
 __global__ void __launch_bounds__(kTransposeThreads) mask_transpose_kernel(const TransposeParams p) {
-    extern __shared__ uint32_t bits[];  // [2][kTransposeChunk][qw]
+    extern __shared__ uint32_t bits[];  // [2][chunk][qw]
     const int qw = (p.QB + 31) / 32;
-    const int kb0 = blockIdx.x * kTransposeChunk;
+    const int C = p.chunk;
+    const int kb0 = blockIdx.x * C;
     const int h = blockIdx.y;
     const int b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = kTransposeThreads / 32;
-    for (int i = threadIdx.x; i < 2 * kTransposeChunk * qw; i += kTransposeThreads) bits[i] = 0u;
+    for (int i = threadIdx.x; i < 2 * C * qw; i += kTransposeThreads) bits[i] = 0u;
     __syncthreads();
 
     // scatter: q row qb's kv blocks that fall into this chunk. A warp takes 32
@@ -62,8 +72,8 @@ __global__ void __launch_bounds__(kTransposeThreads) mask_transpose_kernel(const
     auto take = [&](int l, int qb, int kb) {
         if (kb < 0 || kb >= p.KB) {
             bad = true;
-        } else if (kb >= kb0 && kb < kb0 + kTransposeChunk) {
-            atomicOr(&bits[(l * kTransposeChunk + (kb - kb0)) * qw + (qb >> 5)], 1u << (qb & 31));
+        } else if (kb >= kb0 && kb < kb0 + C) {
+            atomicOr(&bits[(l * C + (kb - kb0)) * qw + (qb >> 5)], 1u << (qb & 31));
         }
     };
     for (int base = warp * 32; base < p.QB; base += nwarps * 32) {
@@ -117,9 +127,9 @@ __global__ void __launch_bounds__(kTransposeThreads) mask_transpose_kernel(const
 
     // compact: one warp per (list, kv column)
     const uint32_t below = (1u << lane) - 1u;
-    for (int c = warp; c < 2 * kTransposeChunk; c += nwarps) {
-        const int l = c / kTransposeChunk;
-        const int kb = kb0 + (c % kTransposeChunk);
+    for (int c = warp; c < 2 * C; c += nwarps) {
+        const int l = c / C;
+        const int kb = kb0 + (c % C);
         if (kb >= p.KB) continue;
         const uint32_t* col = bits + c * qw;
         int32_t* out = (l == 0 ? p.q_idx : p.full_q_idx) + ((static_cast<int64_t>(b) * p.Hm + h) * p.KB + kb) * p.QB;
