@@ -110,6 +110,15 @@ struct SchedHeader {
     int32_t split;   // slice of the entry stream (split-KV), 0 otherwise
 };
 
+// At D = 64 the tensor core also sums each row of P: the PV product runs with
+// N = D + 16 over V followed by a block of ones, so O's column D holds the row
+// sum l (of the bf16 P the product uses). TMEM has room for the wider O only
+// at D = 64.
+template <int D>
+constexpr bool kTcRowSum = D == 64;
+template <int D>
+constexpr int kOCols = D + (kTcRowSum<D> ? 16 : 0);  // TMEM columns of one O accumulator
+
 template <int D>
 struct SmemLayout {
     static constexpr int kTileBytes = 128 * D * 2;          // one 128-row bf16 tile
@@ -135,7 +144,10 @@ struct SmemLayout {
     // per softmax warp, written by the warp and stored by TMA
     static constexpr int kStage = (kAbort + 4 + 1023) / 1024 * 1024;
     static constexpr int kStageBytes = 32 * 32 * 2;
-    static constexpr int kTotal = kStage + 8 * kStageBytes;
+    // the ones block of the row-sum product (a 128 x 64 bf16 tile of 1.0)
+    static constexpr int kOnes = kStage + 8 * kStageBytes;
+    static constexpr int kOnesBytes = kTcRowSum<D> ? 128 * 64 * 2 : 0;
+    static constexpr int kTotal = kOnes + kOnesBytes;
     static constexpr int kAlloc = kTotal + 1024;  // room to align the base to 1024 B
     static_assert(kAlloc <= 227 * 1024, "shared memory layout exceeds one CTA's limit");
 };
@@ -226,12 +238,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(sbase + L::kTmemSlot, 512);
         tmem_relinquish();
     }
+    if constexpr (kTcRowSum<D>) {
+        uint4* ones = reinterpret_cast<uint4*>(smem + L::kOnes);
+        for (int j = threadIdx.x; j < L::kOnesBytes / 16; j += kThreads)
+            ones[j] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);  // bf16 1.0 pairs
+        fence_proxy_async_smem();  // read by the tensor core (async proxy)
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tm_s[2] = {tmem + 0u, tmem + 128u};
-    const uint32_t tm_o[2] = {tmem + 256u, tmem + 256u + (D == 128 ? 128u : 64u)};
+    const uint32_t tm_o[2] = {tmem + 256u, tmem + 256u + static_cast<uint32_t>(kOCols<D>)};
 
     auto sched_base = [&](int buf) -> uint8_t* { return smem + L::kSched + buf * L::kSchedBytes; };
 
@@ -513,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // same kind. The whole warp runs the loop and an elected lane issues.
         const int i = warp == kWarpMma ? 0 : 1;
         constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kOCols<D>, false, true);
         const uint64_t q_desc = sdesc_sw128(sbase + (i == 0 ? L::kQ0 : L::kQ1), 16, 1024);
         const uint32_t t_s = tm_s[i], t_o = tm_o[i];
         // Entry e of the stream (counted over all units) uses ring positions
@@ -557,7 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             if (has_prev) {  // finish entry e-1 (V at ring position kpos - 1)
                 if (prev_in) {
-                    const uint64_t vd = sdesc_sw128(sbase + L::kRingBase + vslot * L::kTileBytes, 16384, 1024);
+                    // N's second 64-column block: V's own at D = 128, the ones block at D = 64
+                    const uint32_t vaddr = sbase + L::kRingBase + vslot * L::kTileBytes;
+                    const uint64_t vd = sdesc_sw128(vaddr, kTcRowSum<D> ? sbase + L::kOnes - vaddr : 16384u, 1024);
                     if (elect_one()) {
                         mma_ts_run8(t_o, t_s, vd, idesc_pv, prev_first ? 0u : 1u);
                         mma_commit(bar(L::kBarKvEmpty + vslot));
@@ -794,16 +814,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                             p0 = ex2_approx(a0);
                             p1 = ex2_approx(a1);
                         }
-                        add2(acc[2 * (jj & 3)], acc[2 * (jj & 3) + 1], acc[2 * (jj & 3)], acc[2 * (jj & 3) + 1], p0, p1);
+                        if constexpr (!kTcRowSum<D>)
+                            add2(acc[2 * (jj & 3)], acc[2 * (jj & 3) + 1], acc[2 * (jj & 3)], acc[2 * (jj & 3) + 1],
+                                 p0, p1);
                         pk[jj] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(t_s + 16 * c, pk);
                 }
                 // a row whose every element in this tile is masked adds nothing
-                // (the FMA-pipe exp2 returns 2^-125 rather than 0 for -inf)
-                if (mt != -INFINITY)
+                // (the FMA-pipe exp2 returns 2^-125 rather than 0 for -inf). With the
+                // tensor core's row sum such a row adds 2^-125 per column against its
+                // reference, which stays negligible; a row that never has an allowed
+                // key keeps m_ref = -inf and the epilogue treats it as empty.
+                if (!kTcRowSum<D> && mt != -INFINITY)
                     l_sum += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-                // O rescale after P is out of registers (lower register peak)
+                // O rescale after P is out of registers (lower register peak); with
+                // the tensor core's row sum, l (column D) is rescaled with O
                 if (__any_sync(0xFFFFFFFFu, need_rescale)) {
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
@@ -813,6 +839,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
                         tmem_st32(t_o + 32 * c, o);
+                    }
+                    if constexpr (kTcRowSum<D>) {
+                        uint32_t o[16];
+                        tmem_ld16(t_o + D, o);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        tmem_st16(t_o + D, o);
                     }
                 }
                 tc_wait_st();
@@ -824,6 +858,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             // epilogue: out = O / l, lse = ln2 * (m + log2 l)
             __nv_bfloat16* orow = p.out + (static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.out_sbh + q * p.out_ss;
+            if constexpr (kTcRowSum<D>) {
+                // l is O's column D, complete once the unit's last PV is (it is
+                // read again after the O-full wait below; this read only fixes
+                // the row's empty case early for the lse)
+                l_sum = 0.f;
+                if (ni > 0) {
+                    if (!mbar_wait(bar(L::kBarOFull + i), o_waits & 1u, abort_flag)) break;
+                    __syncwarp();
+                    tc_fence_after();
+                    l_sum = __uint_as_float(tmem_ld1(t_o + D));
+                    tc_wait_ld();
+                }
+                if (m_ref == -INFINITY) l_sum = 0.f;  // no allowed key in the row
+            }
             const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
             const float row_lse = [&] {
                 const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
