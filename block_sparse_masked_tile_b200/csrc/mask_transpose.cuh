@@ -8,10 +8,13 @@
 // One CTA per (b, h, chunk of kv blocks): up to kTransposeChunk kv blocks, so
 // that a (b, h) is scanned by few CTAs. Its warps read every q row's two
 // lists of (b, h) and set one bit per (kv block of the chunk, q block) in two
-// shared-memory bitmaps. Each warp then compacts whole kv columns: a
-// ballot/popc prefix per 32-bit word gives every set bit its position. The
-// kernel writes every element of its output columns, so it is bound by the
-// HBM writes of [B, H, KB, QB] x 2 lists.
+// shared-memory bitmaps. The chunk's output columns are contiguous, so the
+// whole CTA first zeroes them with 16-byte stores; then each thread takes one
+// column and writes its set bits in ascending order over the zeros. Columns
+// with more than 32 entries are left to a second pass in which a warp takes a
+// column and a popc prefix over its words places every bit. The kernel writes
+// every element of its output columns, so it is bound by the writes of
+// [B, H, KB, QB] x 2 lists.
 //
 // BlockMask "Basics" (the reconstruction loop) defines the dense map: a
 // block is 1 when either list of its row holds it.
@@ -47,19 +50,25 @@ __host__ __device__ constexpr int transpose_chunk(int64_t QB) {
 
 // Shared memory: two bitmaps of chunk x ceil(QB / 32) words.
 __host__ __device__ constexpr int64_t transpose_smem_bytes(int64_t QB, int chunk) {
-    return 2 * static_cast<int64_t>(chunk) * ((QB + 31) / 32) * 4;
+    return 2 * static_cast<int64_t>(chunk) * ((QB + 31) / 32) * 4 + (2 * chunk + 1) * 4;
 }
 
 __global__ void __launch_bounds__(kTransposeThreads) mask_transpose_kernel(const TransposeParams p) {
-    extern __shared__ uint32_t bits[];  // [2][chunk][qw]
+    // bitmaps [2][qw][chunk] (a column's words chunk apart, so that threads
+    // reading one column each read consecutive words), then the count and
+    // the list of dense columns for the second pass
+    extern __shared__ uint32_t bits[];
     const int qw = (p.QB + 31) / 32;
     const int C = p.chunk;
+    int* n_dense = reinterpret_cast<int*>(bits + 2 * C * qw);
+    int* dense_cols = n_dense + 1;
     const int kb0 = blockIdx.x * C;
     const int h = blockIdx.y;
     const int b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = kTransposeThreads / 32;
     for (int i = threadIdx.x; i < 2 * C * qw; i += kTransposeThreads) bits[i] = 0u;
+    if (threadIdx.x == 0) *n_dense = 0;
     __syncthreads();
 
     // scatter: q row qb's kv blocks that fall into this chunk. A warp takes 32
@@ -73,7 +82,7 @@ __global__ void __launch_bounds__(kTransposeThreads) mask_transpose_kernel(const
         if (kb < 0 || kb >= p.KB) {
             bad = true;
         } else if (kb >= kb0 && kb < kb0 + C) {
-            atomicOr(&bits[(l * C + (kb - kb0)) * qw + (qb >> 5)], 1u << (qb & 31));
+            atomicOr(&bits[(l * qw + (qb >> 5)) * C + (kb - kb0)], 1u << (qb & 31));
         }
     };
     for (int base = warp * 32; base < p.QB; base += nwarps * 32) {
@@ -125,37 +134,77 @@ __global__ void __launch_bounds__(kTransposeThreads) mask_transpose_kernel(const
     if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
     __syncthreads();
 
-    // compact: one warp per (list, kv column)
-    const uint32_t below = (1u << lane) - 1u;
-    for (int c = warp; c < 2 * C; c += nwarps) {
-        const int l = c / C;
-        const int kb = kb0 + (c % C);
-        if (kb >= p.KB) continue;
-        const uint32_t* col = bits + c * qw;
-        int32_t* out = (l == 0 ? p.q_idx : p.full_q_idx) + ((static_cast<int64_t>(b) * p.Hm + h) * p.KB + kb) * p.QB;
+    // zero the chunk's columns of both lists: [kb0, kb0 + cols) x QB int32,
+    // contiguous in each list
+    const int cols = (p.KB - kb0) < C ? (p.KB - kb0) : C;
+    const int64_t base_row = (static_cast<int64_t>(b) * p.Hm + h) * p.KB + kb0;
+    const int64_t n_int = static_cast<int64_t>(cols) * p.QB;
+#pragma unroll 1
+    for (int l = 0; l < 2; ++l) {
+        int32_t* blk = (l == 0 ? p.q_idx : p.full_q_idx) + base_row * p.QB;
+        const uintptr_t a = reinterpret_cast<uintptr_t>(blk);
+        int64_t head = static_cast<int64_t>(((16u - (a & 15u)) & 15u) >> 2);  // int32 slots to the boundary
+        head = head < n_int ? head : n_int;
+        if (threadIdx.x < head) blk[threadIdx.x] = 0;
+        const int64_t nv = (n_int - head) >> 2;
+        uint4* v = reinterpret_cast<uint4*>(blk + head);
+        for (int64_t k = threadIdx.x; k < nv; k += kTransposeThreads) v[k] = make_uint4(0u, 0u, 0u, 0u);
+        const int64_t tail = head + 4 * nv;
+        if (tail + threadIdx.x < n_int) blk[tail + threadIdx.x] = 0;
+    }
+    __syncthreads();  // the entries below overwrite the zeros
+
+    // one thread per (list, kv column): the set bits in ascending order
+    for (int c = threadIdx.x; c < 2 * cols; c += kTransposeThreads) {
+        const int l = c / cols;
+        const int kc = c - l * cols;
+        const uint32_t* col = bits + l * qw * C + kc;
+        int count = 0;
+        for (int w = 0; w < qw; ++w) count += __popc(col[w * C]);
+        const int64_t orow = base_row + kc;
+        if (count > 32) {  // a dense column: the second pass writes it
+            dense_cols[atomicAdd(n_dense, 1)] = c;
+        } else {
+            int32_t* out = (l == 0 ? p.q_idx : p.full_q_idx) + orow * p.QB;
+            int pos = 0;
+            for (int w = 0; w < qw && pos < count; ++w) {
+                uint32_t rest = col[w * C];
+                while (rest) {
+                    out[pos++] = w * 32 + __ffs(rest) - 1;
+                    rest &= rest - 1u;
+                }
+            }
+        }
+        (l == 0 ? p.q_num : p.full_q_num)[orow] = count;
+    }
+    __syncthreads();
+    // dense columns: one warp per column; lane takes word w0 + lane, its bits'
+    // positions following the set bits of the lower lanes' words
+    const int nd = *n_dense;
+    for (int d = warp; d < nd; d += nwarps) {
+        const int c = dense_cols[d];
+        const int l = c / cols;
+        const int kc = c - l * cols;
+        const uint32_t* col = bits + l * qw * C + kc;
+        int32_t* out = (l == 0 ? p.q_idx : p.full_q_idx) + (base_row + kc) * p.QB;
         int pos = 0;
         for (int w0 = 0; w0 < qw; w0 += 32) {
-            // lane handles word w0 + lane: its bits' positions follow the set
-            // bits of the lower lanes' words
-            const uint32_t word = (w0 + lane < qw) ? col[w0 + lane] : 0u;
+            const uint32_t word = (w0 + lane < qw) ? col[(w0 + lane) * C] : 0u;
             const int cnt = __popc(word);
             int incl = cnt;
 #pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-                if (lane >= d) incl += v;
+            for (int dd = 1; dd < 32; dd <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, dd);
+                if (lane >= dd) incl += v;
             }
             int at = pos + incl - cnt;
             uint32_t rest = word;
             while (rest) {
-                const int bit = __ffs(rest) - 1;
+                out[at++] = (w0 + lane) * 32 + __ffs(rest) - 1;
                 rest &= rest - 1u;
-                out[at++] = (w0 + lane) * 32 + bit;
             }
             pos += __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
-        zero_tail(out, pos, p.QB, lane);
-        if (lane == 0) (l == 0 ? p.q_num : p.full_q_num)[(static_cast<int64_t>(b) * p.Hm + h) * p.KB + kb] = pos;
     }
 }
 
