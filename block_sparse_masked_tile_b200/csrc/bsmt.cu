@@ -732,7 +732,7 @@ extern "C" bsmt_status bsmt_block_mask_transpose(const bsmt_block_mask* kv, bsmt
     int dev = 0, nsm = 0;
     st = sm_count(&dev, &nsm);
     if (st != BSMT_OK) return st;
-    const int chunk = bsmt::transpose_chunk(kv->QB);
+    const int chunk = bsmt::transpose_chunk(kv->QB, kv->KB, static_cast<int64_t>(kv->B) * kv->H, nsm);
     const int smem = static_cast<int>(bsmt::transpose_smem_bytes(kv->QB, chunk));
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(bsmt::mask_transpose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

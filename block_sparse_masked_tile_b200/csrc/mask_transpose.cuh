@@ -25,7 +25,7 @@
 
 namespace bsmt {
 
-constexpr int kTransposeChunk = 128;  // kv blocks per CTA (at most)
+constexpr int kTransposeChunk = 256;  // kv blocks per CTA (at most)
 constexpr int kTransposeThreads = 512;
 
 struct TransposeParams {
@@ -41,11 +41,19 @@ struct TransposeParams {
     int32_t* full_q_idx;
 };
 
-// Kv blocks per CTA: kTransposeChunk, or fewer so that the two bitmaps stay
-// within 96 KB of shared memory.
-__host__ __device__ constexpr int transpose_chunk(int64_t QB) {
-    const int64_t c = (96 * 1024) / (2 * 4 * ((QB + 31) / 32 > 0 ? (QB + 31) / 32 : 1));
-    return static_cast<int>(c < 1 ? 1 : (c > kTransposeChunk ? kTransposeChunk : c));
+// Kv blocks per CTA: every kv block of a (b, h) when the grid still has at
+// least half a CTA per SM, else KB split into as many chunks as that takes;
+// at most kTransposeChunk, and few enough for the two bitmaps to stay within
+// 96 KB of shared memory. (A (b, h) is scanned once per chunk: at B2 H32 with
+// 256 x 256 blocks, two chunks measured faster than one or three.)
+__host__ __device__ constexpr int transpose_chunk(int64_t QB, int64_t KB, int64_t BH, int64_t nsm) {
+    const int64_t want = (nsm + 1) / 2;  // CTAs
+    const int64_t per_bh = BH >= want ? 1 : (want + BH - 1) / (BH > 0 ? BH : 1);  // chunks per (b, h)
+    int64_t c = (KB + per_bh - 1) / per_bh;
+    const int64_t fit = (96 * 1024) / (2 * 4 * ((QB + 31) / 32 > 0 ? (QB + 31) / 32 : 1));
+    c = c > fit ? fit : c;
+    c = c > kTransposeChunk ? kTransposeChunk : c;
+    return static_cast<int>(c < 1 ? 1 : c);
 }
 
 // Shared memory: two bitmaps of chunk x ceil(QB / 32) words.
