@@ -108,7 +108,14 @@ struct SchedHeader {
     int32_t n0, n1;  // tiles visited by q-block 0 / 1
     float slope;     // ALiBi slope of hq (natural units)
     int32_t split;   // slice of the entry stream (split-KV), 0 otherwise
+    int32_t kb_base; // entries hold kv blocks relative to this block
+    int32_t seg;     // kSegFirst | kSegLast | kSegMany
 };
+
+// Segments of a unit: the first and the last of its windows, and whether it
+// has more than one. A unit of one segment carries exact tile counts (n0, n1)
+// up front; the segments of a longer one carry their own counts only.
+constexpr int32_t kSegFirst = 1, kSegLast = 2, kSegMany = 4;
 
 // At D = 64 the tensor core also sums each row of P: the PV product runs with
 // N = D + 16 over V followed by a block of ones, so O's column D holds the row
@@ -187,7 +194,10 @@ __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float
     y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-template <int D, int SCORE>
+// LONG: rows may span more than kMaxKB kv blocks (units in windows and
+// segments). Without it the kernel assumes KB <= kMaxKB and every unit is one
+// segment from block 0, and the segment logic folds away.
+template <int D, int SCORE, bool LONG>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
@@ -269,23 +279,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = lane; j < kMaxKB; j += 32) flags[j] = 0;
         __syncwarp();
         int iter = 0;
+        const uint32_t below = (1u << lane) - 1u;
+        const bool ragged_kv = (p.N & 127) != 0;
         // Units go out in a serpentine order: round k gives CTA c unit
         // k * G + c for even k and k * G + (G - 1 - c) for odd k (G CTAs). The
         // order runs longest first, so alternating the direction evens out
         // each CTA's total when unit lengths fall steadily (causal rows). A
         // CTA's units still increase, so the first past the end is its last.
-        for (int64_t k = 0;; ++k, ++iter) {
+        //
+        // A unit's entries hold kv blocks relative to a window base. When the
+        // unit's kv blocks span more than kMaxKB blocks (rows longer than
+        // kMaxKB blocks), it goes out as several segments, one window of
+        // kMaxKB blocks each, in kv order; the consumers carry the unit's
+        // state from one segment to the next.
+        for (int64_t k = 0;; ++k) {
             const int64_t G = gridDim.x;
             const int64_t u64 = k * G + ((k & 1) ? (G - 1 - blockIdx.x) : static_cast<int64_t>(blockIdx.x));
             const int u = u64 < p.num_units ? static_cast<int>(u64) : p.num_units;
-            const int buf = iter & 1;
-            const uint32_t use = static_cast<uint32_t>(iter >> 1);
-            if (!mbar_wait(bar(L::kBarSchedEmpty + buf), (use & 1u) ^ 1u, abort_flag)) break;
-            uint8_t* sb = sched_base(buf);
-            SchedHeader* hdr = reinterpret_cast<SchedHeader*>(sb + L::kSchedHeader);
-            uint32_t* entries = reinterpret_cast<uint32_t*>(sb + L::kSchedEntries);
             if (u >= p.num_units) {
-                if (lane == 0) hdr->T = -1;
+                const int buf = iter & 1;
+                if (!mbar_wait(bar(L::kBarSchedEmpty + buf), ((static_cast<uint32_t>(iter) >> 1) & 1u) ^ 1u,
+                               abort_flag))
+                    break;
+                if (lane == 0) reinterpret_cast<SchedHeader*>(sched_base(buf) + L::kSchedHeader)->T = -1;
                 mbar_arrive(bar(L::kBarSchedFull + buf));
                 break;
             }
@@ -298,164 +314,264 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int hq = bh % p.Hq;
             const int qb0 = 2 * pr;
             const bool has1 = qb0 + 1 < p.QB;
-            const bool ragged_kv = (p.N & 127) != 0;
-            int T = 0, n0 = 0, n1 = 0;
-            if (!p.has_block_mask) {
-                // every tile of both rows; the tile crossing N is partial
-                for (int c = 0; c < p.KB; c += 32) {
-                    const int kb = c + lane;
-                    if (kb < p.KB) {
-                        const bool part = ragged_kv && kb == p.KB - 1;
-                        uint32_t tags = kTagIn0 | (part ? kTagPart0 : 0u);
-                        if (has1) tags |= kTagIn1 | (part ? kTagPart1 : 0u);
-                        entries[kb] = static_cast<uint32_t>(kb) | (tags << 16);
+            // the unit's first buffer
+            if (!mbar_wait(bar(L::kBarSchedEmpty + (iter & 1)), ((static_cast<uint32_t>(iter) >> 1) & 1u) ^ 1u,
+                           abort_flag))
+                break;
+            // Each row's document interval [first, last] of kv positions with the
+            // row's document id (kv ids are non-decreasing), into the unit's first
+            // buffer sb0. Rows in a run usually share one id, so each distinct id
+            // is searched once, with a 33-way warp search over the kv ids.
+            auto doc_intervals = [&](uint8_t* sb0) {
+                if (dnf.has_doc && p.has_block_mask) {
+                    const int db = dnf.doc_batch > 1 ? b : 0;
+                    const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
+                    const int32_t* kd_row = dnf.kv_doc + static_cast<int64_t>(db) * p.N;
+                    int32_t* dlo = reinterpret_cast<int32_t*>(sb0 + L::kSchedDocLo);
+                    int32_t* dhi = reinterpret_cast<int32_t*>(sb0 + L::kSchedDocHi);
+#pragma unroll 1
+                    for (int r0 = 0; r0 < 256; r0 += 32) {
+                        const int64_t q = static_cast<int64_t>(qb0) * 128 + r0 + lane;
+                        const bool valid = q < p.M;
+                        const int32_t d = valid ? __ldg(qd_row + q) : 0;
+                        int lo = 0, hi = -1;
+                        bool pending = valid;
+                        unsigned todo;
+                        while ((todo = __ballot_sync(0xFFFFFFFFu, pending)) != 0u) {
+                            const int32_t x = __shfl_sync(0xFFFFFFFFu, d, __ffs(todo) - 1);
+                            const int first = warp_lower_bound(kd_row, p.N, x, lane);
+                            const int past = warp_lower_bound(kd_row, p.N, static_cast<int64_t>(x) + 1, lane);
+                            if (pending && d == x) {
+                                lo = first;
+                                hi = past - 1;
+                                pending = false;
+                            }
+                        }
+                        dlo[r0 + lane] = lo;
+                        dhi[r0 + lane] = hi;
                     }
                 }
-                T = p.KB;
-                n0 = p.KB;
-                n1 = has1 ? p.KB : 0;
-            } else {
+            };
+            if constexpr (LONG) doc_intervals(sched_base(iter & 1));
+            // the two rows' partial and full lists (block mask only): list l is
+            // list_at(l), l = 0 partial row0, 1 full row0, 2 partial row1, 3 full row1
+            int cnt[4] = {0, 0, 0, 0};
+            int64_t row0 = 0;
+            auto list_at = [&](int l) -> const int32_t* {
+                return ((l & 1) ? p.full_idx : p.kv_idx) + (row0 + (l >> 1)) * p.KB;
+            };
+            if (p.has_block_mask) {
                 const int bb = p.Bm > 1 ? b : 0;
                 const int hh = p.Hm > 1 ? hq : 0;
-                const int64_t row0 = (static_cast<int64_t>(bb) * p.Hm + hh) * p.QB + qb0;
-                int cnt[4] = {0, 0, 0, 0};
-                const int32_t* lists[4] = {p.kv_idx + row0 * p.KB, p.full_idx + row0 * p.KB,
-                                           p.kv_idx + (row0 + 1) * p.KB, p.full_idx + (row0 + 1) * p.KB};
-                {
-                    int v = 0;
-                    if (lane == 0) v = __ldg(p.kv_num + row0);
-                    if (lane == 1) v = __ldg(p.full_num + row0);
-                    if (has1 && lane == 2) v = __ldg(p.kv_num + row0 + 1);
-                    if (has1 && lane == 3) v = __ldg(p.full_num + row0 + 1);
-                    bool bad = v < 0 || v > p.KB;
-                    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
-                    v = bad ? 0 : v;
+                row0 = (static_cast<int64_t>(bb) * p.Hm + hh) * p.QB + qb0;
+                int v = 0;
+                if (lane == 0) v = __ldg(p.kv_num + row0);
+                if (lane == 1) v = __ldg(p.full_num + row0);
+                if (has1 && lane == 2) v = __ldg(p.kv_num + row0 + 1);
+                if (has1 && lane == 3) v = __ldg(p.full_num + row0 + 1);
+                bool bad = v < 0 || v > p.KB;
+                if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
+                v = bad ? 0 : v;
 #pragma unroll
-                    for (int l = 0; l < 4; ++l) cnt[l] = __shfl_sync(0xFFFFFFFFu, v, l);
-                }
+                for (int l = 0; l < 4; ++l) cnt[l] = __shfl_sync(0xFFFFFFFFu, v, l);
+            }
+            // Marks bit l of flags[kb - base] for each block kb of list l in
+            // [base, base + span).
+            auto mark = [&](int base, int span) {
                 bool bad = false;
 #pragma unroll
                 for (int l = 0; l < 4; ++l) {
+                    const int32_t* list = list_at(l);
                     for (int j = lane; j < cnt[l]; j += 32) {
-                        const int kb = __ldg(lists[l] + j);
-                        if (kb >= 0 && kb < p.KB) {
-                            flags[kb] |= static_cast<uint8_t>(1u << l);
-                        } else {
+                        const int kb = __ldg(list + j);
+                        if (kb < 0 || kb >= p.KB) {
                             bad = true;
+                        } else if (kb >= base && kb - base < span) {
+                            flags[kb - base] |= static_cast<uint8_t>(1u << l);
                         }
                     }
                     __syncwarp();
                 }
                 if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
-                const uint32_t below = (1u << lane) - 1u;
-                for (int c = 0; c < p.KB; c += 32) {
-                    const int kb = c + lane;
-                    uint32_t f = 0;
-                    if (kb < p.KB) {
-                        f = flags[kb];
-                        flags[kb] = 0;
-                    }
-                    // list bits: 0 partial row0, 1 full row0, 2 partial row1, 3 full row1.
-                    // A block listed as both partial and full is treated as partial.
-                    uint32_t tags = 0;
-                    if (f & 3u) tags |= kTagIn0 | ((f & 1u) ? kTagPart0 : 0u);
-                    if (f & 12u) tags |= kTagIn1 | ((f & 4u) ? kTagPart1 : 0u);
-                    if (ragged_kv && kb == p.KB - 1 && tags) {
-                        if (tags & kTagIn0) tags |= kTagPart0;
-                        if (tags & kTagIn1) tags |= kTagPart1;
-                    }
-                    const unsigned bal = __ballot_sync(0xFFFFFFFFu, tags != 0);
-                    if (tags) entries[T + __popc(bal & below)] = static_cast<uint32_t>(kb) | (tags << 16);
-                    T += __popc(bal);
-                    n0 += __popc(__ballot_sync(0xFFFFFFFFu, (tags & kTagIn0) != 0));
-                    n1 += __popc(__ballot_sync(0xFFFFFFFFu, (tags & kTagIn1) != 0));
-                }
-            }
-            if (p.num_splits > 1) {
-                // keep this unit's slice [lo, hi) of the stream, moved to the front
-                // (a chunk is read before it is written, and never overlaps a later
-                // chunk's source)
-                const int lo = static_cast<int>((static_cast<int64_t>(T) * split) / p.num_splits);
-                const int hi = static_cast<int>((static_cast<int64_t>(T) * (split + 1)) / p.num_splits);
-                n0 = 0;
-                n1 = 0;
-                for (int c = 0; c < hi - lo; c += 32) {
-                    const bool in = c + lane < hi - lo;
-                    const uint32_t e = in ? entries[lo + c + lane] : 0u;
-                    __syncwarp();
-                    if (in) entries[c + lane] = e;
-                    __syncwarp();
-                    const uint32_t tags = sched_entry_tags(e);
-                    n0 += __popc(__ballot_sync(0xFFFFFFFFu, in && (tags & kTagIn0)));
-                    n1 += __popc(__ballot_sync(0xFFFFFFFFu, in && (tags & kTagIn1)));
-                }
-                T = hi - lo;
-            }
-            if (dnf.has_doc && p.has_block_mask) {
-                // Each row's document interval [first, last] of kv positions with
-                // the row's document id (kv ids are non-decreasing). Rows in a run
-                // usually share one id, so each distinct id is searched once, with
-                // a 33-way warp search over the kv ids.
-                const int db = dnf.doc_batch > 1 ? b : 0;
-                const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
-                const int32_t* kd_row = dnf.kv_doc + static_cast<int64_t>(db) * p.N;
-                int32_t* dlo = reinterpret_cast<int32_t*>(sb + L::kSchedDocLo);
-                int32_t* dhi = reinterpret_cast<int32_t*>(sb + L::kSchedDocHi);
-#pragma unroll 1
-                for (int r0 = 0; r0 < 256; r0 += 32) {
-                    const int64_t q = static_cast<int64_t>(qb0) * 128 + r0 + lane;
-                    const bool valid = q < p.M;
-                    const int32_t d = valid ? __ldg(qd_row + q) : 0;
-                    int lo = 0, hi = -1;
-                    bool pending = valid;
-                    unsigned todo;
-                    while ((todo = __ballot_sync(0xFFFFFFFFu, pending)) != 0u) {
-                        const int32_t x = __shfl_sync(0xFFFFFFFFu, d, __ffs(todo) - 1);
-                        const int first = warp_lower_bound(kd_row, p.N, x, lane);
-                        const int past = warp_lower_bound(kd_row, p.N, static_cast<int64_t>(x) + 1, lane);
-                        if (pending && d == x) {
-                            lo = first;
-                            hi = past - 1;
-                            pending = false;
+            };
+            // The unit's windows: kMaxKB blocks each from its first listed block.
+            int klo = 0, nwin = 1;
+            if (LONG && p.KB > kMaxKB) {
+                int khi = p.KB - 1;
+                if (p.has_block_mask) {
+                    int mn = 0x7FFFFFFF, mx = -1;
+#pragma unroll
+                    for (int l = 0; l < 4; ++l) {
+                        const int32_t* list = list_at(l);
+                        for (int j = lane; j < cnt[l]; j += 32) {
+                            const int kb = __ldg(list + j);
+                            if (kb >= 0 && kb < p.KB) {
+                                mn = min(mn, kb);
+                                mx = max(mx, kb);
+                            }
                         }
                     }
-                    dlo[r0 + lane] = lo;
-                    dhi[r0 + lane] = hi;
+                    mn = __reduce_min_sync(0xFFFFFFFFu, mn);
+                    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+                    klo = mx >= 0 ? mn : 0;
+                    khi = mx;
                 }
+                nwin = khi >= klo ? (khi - klo) / kMaxKB + 1 : 1;
             }
-            if (lane == 0) {
-                hdr->T = T;
-                hdr->b = b;
-                hdr->hq = hq;
-                hdr->qb0 = qb0;
-                hdr->split = split;
-                hdr->n0 = n0;
-                hdr->n1 = n1;
-                float slope = 0.f;
-                if (SCORE == kScoreAlibi || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap)
-                    slope = p.slopes ? __ldg(p.slopes + hq)
-                                     : exp2f(-8.0f * static_cast<float>(p.alibi_h0 + hq + 1) /
-                                             static_cast<float>(p.alibi_heads));
-                hdr->slope = slope;
-                // Pull this unit's Q tiles into L2 now; they are loaded into shared
-                // memory only when the unit before has finished with its own.
-                const int zq = b * p.Hq + hq;
-                for (int qq = 0; qq < 2; ++qq) {
-                    if ((qq == 0 ? n0 : n1) == 0) continue;
+            // Split-KV over several windows: the slice [g_lo, g_hi) of the
+            // unit's stream needs the stream's length first.
+            int g_lo = 0, g_hi = 0x7FFFFFFF;
+            if (LONG && p.num_splits > 1 && nwin > 1) {
+                int total = p.KB;
+                if (p.has_block_mask) {
+                    total = 0;
+                    for (int w = 0; w < nwin; ++w) {
+                        const int base = klo + w * kMaxKB;
+                        const int span = min(kMaxKB, p.KB - base);
+                        mark(base, span);
+                        for (int c = 0; c < span; c += 32) {
+                            uint32_t f = 0;
+                            if (c + lane < span) {
+                                f = flags[c + lane];
+                                flags[c + lane] = 0;
+                            }
+                            total += __popc(__ballot_sync(0xFFFFFFFFu, f != 0));
+                        }
+                        __syncwarp();
+                    }
+                }
+                g_lo = static_cast<int>((static_cast<int64_t>(total) * split) / p.num_splits);
+                g_hi = static_cast<int>((static_cast<int64_t>(total) * (split + 1)) / p.num_splits);
+            }
+            int g = 0;  // stream entries before this window
+            bool ok = true;
+            for (int w = 0; w < nwin; ++w, ++iter) {
+                const int buf = iter & 1;
+                const uint32_t use = static_cast<uint32_t>(iter >> 1);
+                if (w > 0 && !mbar_wait(bar(L::kBarSchedEmpty + buf), (use & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sb = sched_base(buf);
+                SchedHeader* hdr = reinterpret_cast<SchedHeader*>(sb + L::kSchedHeader);
+                uint32_t* entries = reinterpret_cast<uint32_t*>(sb + L::kSchedEntries);
+                const int base = klo + w * kMaxKB;
+                const int span = min(kMaxKB, p.KB - base);
+                if (p.has_block_mask) mark(base, span);
+                // the union of both rows' blocks in the window, ascending, with
+                // tags; a block listed as both partial and full is partial, and
+                // the tile crossing N is partial
+                int T = 0, n0 = 0, n1 = 0;
+                for (int c = 0; c < span; c += 32) {
+                    const int kr = c + lane;
+                    uint32_t tags = 0;
+                    if (kr < span) {
+                        if (p.has_block_mask) {
+                            const uint32_t f = flags[kr];
+                            flags[kr] = 0;
+                            if (f & 3u) tags |= kTagIn0 | ((f & 1u) ? kTagPart0 : 0u);
+                            if (f & 12u) tags |= kTagIn1 | ((f & 4u) ? kTagPart1 : 0u);
+                        } else {
+                            tags = kTagIn0 | (has1 ? kTagIn1 : 0u);
+                        }
+                        if (ragged_kv && base + kr == p.KB - 1) {
+                            if (tags & kTagIn0) tags |= kTagPart0;
+                            if (tags & kTagIn1) tags |= kTagPart1;
+                        }
+                    }
+                    const unsigned bal = __ballot_sync(0xFFFFFFFFu, tags != 0);
+                    if constexpr (LONG) {
+                        // keep the stream entries g.. of the split's slice [g_lo, g_hi)
+                        const int gi = g + __popc(bal & below);
+                        const bool keep = tags != 0 && gi >= g_lo && gi < g_hi;
+                        const unsigned kbal = __ballot_sync(0xFFFFFFFFu, keep);
+                        if (keep) entries[T + __popc(kbal & below)] = static_cast<uint32_t>(kr) | (tags << 16);
+                        T += __popc(kbal);
+                        g += __popc(bal);
+                        n0 += __popc(__ballot_sync(0xFFFFFFFFu, keep && (tags & kTagIn0)));
+                        n1 += __popc(__ballot_sync(0xFFFFFFFFu, keep && (tags & kTagIn1)));
+                    } else {
+                        if (tags) entries[T + __popc(bal & below)] = static_cast<uint32_t>(kr) | (tags << 16);
+                        T += __popc(bal);
+                        n0 += __popc(__ballot_sync(0xFFFFFFFFu, (tags & kTagIn0) != 0));
+                        n1 += __popc(__ballot_sync(0xFFFFFFFFu, (tags & kTagIn1) != 0));
+                    }
+                }
+                if (p.num_splits > 1 && nwin == 1) {
+                    // keep this unit's slice [lo, hi) of the stream, moved to the front
+                    // (a chunk is read before it is written, and never overlaps a later
+                    // chunk's source)
+                    const int lo = static_cast<int>((static_cast<int64_t>(T) * split) / p.num_splits);
+                    const int hi = static_cast<int>((static_cast<int64_t>(T) * (split + 1)) / p.num_splits);
+                    n0 = 0;
+                    n1 = 0;
+                    for (int c = 0; c < hi - lo; c += 32) {
+                        const bool in = c + lane < hi - lo;
+                        const uint32_t e = in ? entries[lo + c + lane] : 0u;
+                        __syncwarp();
+                        if (in) entries[c + lane] = e;
+                        __syncwarp();
+                        const uint32_t tags = sched_entry_tags(e);
+                        n0 += __popc(__ballot_sync(0xFFFFFFFFu, in && (tags & kTagIn0)));
+                        n1 += __popc(__ballot_sync(0xFFFFFFFFu, in && (tags & kTagIn1)));
+                    }
+                    T = hi - lo;
+                }
+                if constexpr (!LONG) doc_intervals(sb);
+                if (lane == 0) {
+                    hdr->T = T;
+                    hdr->b = b;
+                    hdr->hq = hq;
+                    hdr->qb0 = qb0;
+                    hdr->split = split;
+                    hdr->n0 = n0;
+                    hdr->n1 = n1;
+                    hdr->kb_base = base;
+                    hdr->seg = (w == 0 ? kSegFirst : 0) | (w == nwin - 1 ? kSegLast : 0) | (nwin > 1 ? kSegMany : 0);
+                    float slope = 0.f;
+                    if (SCORE == kScoreAlibi || SCORE == kScoreSoftcapAlibi || SCORE == kScoreAlibiSoftcap)
+                        slope = p.slopes ? __ldg(p.slopes + hq)
+                                         : exp2f(-8.0f * static_cast<float>(p.alibi_h0 + hq + 1) /
+                                                 static_cast<float>(p.alibi_heads));
+                    hdr->slope = slope;
+                    if (w == 0) {
+                        // Pull this unit's Q tiles into L2 now; they are loaded into
+                        // shared memory only when the unit before has finished with
+                        // its own.
+                        const int zq = b * p.Hq + hq;
+                        for (int qq = 0; qq < 2; ++qq) {
+                            if ((qq == 0 ? n0 : n1) == 0) continue;
 #pragma unroll
-                    for (int h = 0; h < D / 64; ++h) tma_prefetch_3d(&tm_q, h * 64, (qb0 + qq) * 128, zq);
+                            for (int h = 0; h < D / 64; ++h) tma_prefetch_3d(&tm_q, h * 64, (qb0 + qq) * 128, zq);
+                        }
+                    }
                 }
+                __syncwarp();
+                mbar_arrive(bar(L::kBarSchedFull + buf));
             }
-            __syncwarp();
-            mbar_arrive(bar(L::kBarSchedFull + buf));
+            if (!ok) break;
         }
     } else if (warp == kWarpLoad) {
         // ================================================= TMA producer warp
         uint32_t kv_pos = 0;  // ring positions used so far
         uint32_t q_uses[2] = {0, 0};
+        bool q_loaded[2] = {false, false};  // a unit of several segments: its Q tile i is loaded
         const uint32_t tile_bytes = L::kTileBytes;
         const uint64_t pol_kv = l2_policy_evict_last();
         const uint64_t pol_q = l2_policy_evict_first();
+        // Q tile i of q-block qb of head zq, once the unit before is done with the slot
+        auto load_q = [&](int i, int qb, int zq) -> bool {
+            if (q_uses[i] > 0 && !mbar_wait(bar(L::kBarQEmpty + i), (q_uses[i] - 1) & 1u, abort_flag)) return false;
+            ++q_uses[i];
+            if (lane == 0) {
+                const uint32_t qb_bar = bar(L::kBarQFull + i);
+                mbar_arrive_expect_tx(qb_bar, tile_bytes);
+                const uint32_t dst = sbase + (i == 0 ? L::kQ0 : L::kQ1);
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h) tma_load_3d_hint(dst + h * 16384, &tm_q, h * 64, qb * 128, zq, qb_bar, pol_q);
+            }
+            return true;
+        };
         for (int iter = 0;; ++iter) {
             const int buf = iter & 1;
             if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) break;
@@ -467,26 +583,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int zq = hdr.b * p.Hq + hdr.hq;
             const int zkv = hdr.b * p.Hkv + hkv;
             bool ok = true;
-            for (int i = 0; i < 2 && ok; ++i) {
-                const int ni = i == 0 ? hdr.n0 : hdr.n1;
-                if (ni == 0) continue;
-                if (q_uses[i] > 0) {
-                    ok = mbar_wait(bar(L::kBarQEmpty + i), (q_uses[i] - 1) & 1u, abort_flag);
-                    if (!ok) break;
-                }
-                ++q_uses[i];
-                if (lane == 0) {
-                    const uint32_t qb_bar = bar(L::kBarQFull + i);
-                    mbar_arrive_expect_tx(qb_bar, tile_bytes);
-                    const uint32_t dst = sbase + (i == 0 ? L::kQ0 : L::kQ1);
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h)
-                        tma_load_3d_hint(dst + h * 16384, &tm_q, h * 64, (hdr.qb0 + i) * 128, zq, qb_bar, pol_q);
-                }
+            // A unit of one segment knows which Q tiles it needs up front; a unit
+            // of several loads each Q tile before its first K tile.
+            const bool many = LONG && (hdr.seg & kSegMany) != 0;
+            if (LONG && (hdr.seg & kSegFirst)) {
+                q_loaded[0] = false;
+                q_loaded[1] = false;
+            }
+            if (!many) {
+                for (int i = 0; i < 2 && ok; ++i)
+                    if ((i == 0 ? hdr.n0 : hdr.n1) > 0) ok = load_q(i, hdr.qb0 + i, zq);
             }
             if (!ok) break;
             for (int n = 0; n < hdr.T && ok; ++n) {
-                const int kb = static_cast<int>(sched_entry_kb(entries[n]));
+                const uint32_t e = entries[n];
+                if (many) {
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        if (ok && ((sched_entry_tags(e) >> i) & 1u) && !q_loaded[i]) {
+                            ok = load_q(i, hdr.qb0 + i, zq);
+                            q_loaded[i] = true;
+                        }
+                    }
+                    if (!ok) break;
+                }
+                const int kb = (LONG ? hdr.kb_base : 0) + static_cast<int>(sched_entry_kb(e));
 #pragma unroll
                 for (int kv = 0; kv < 2; ++kv) {  // 0 = K, 1 = V
                     const uint32_t s = kv_pos % kRing;
@@ -609,6 +730,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (has_cur) ++e;
             return true;
         };
+        // A unit's state carries over its segments: s_done (this q-block's S
+        // products so far) and started (an entry has started). In a unit of
+        // several segments the q-block's tile count is not known ahead, so its
+        // Q slot and O are released at the unit's end instead of at its last
+        // tile.
+        int s_done = 0;
+        bool started = false;
         for (int iter = 0; ok; ++iter) {
             const int buf = iter & 1;
             if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) break;
@@ -617,14 +745,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (hdr.T < 0) break;
             const uint32_t* entries = reinterpret_cast<const uint32_t*>(sb + L::kSchedEntries);
             const int ni = i == 0 ? hdr.n0 : hdr.n1;
-            int s_done = 0;
+            const bool many = LONG && (hdr.seg & kSegMany) != 0;
+            if (!LONG || (hdr.seg & kSegFirst)) {
+                s_done = 0;
+                started = false;
+            }
             for (int n = 0; n < hdr.T && ok; ++n) {
                 const bool cur_in = (sched_entry_tags(entries[n]) >> i) & 1u;
                 const bool cur_first = cur_in && s_done == 0;
                 if (cur_in) ++s_done;
-                ok = step(n > 0, true, cur_in, cur_first, cur_in && s_done == ni);
+                ok = step(LONG ? started : n > 0, true, cur_in, cur_first, !many && cur_in && s_done == ni);
+                started = true;
             }
-            if (ok && hdr.T > 0) ok = step(true, false, false, false, false);  // finish the unit's last entry
+            if (ok && (LONG ? (hdr.seg & kSegLast) != 0 : hdr.T > 0)) {
+                if (!LONG || started) ok = step(true, false, false, false, false);  // finish the unit's last entry
+                if (ok && many && s_done > 0) {
+                    if (elect_one()) {
+                        mma_commit(bar(L::kBarQEmpty + i));
+                        mma_commit(bar(L::kBarOFull + i));
+                    }
+                    __syncwarp();
+                }
+            }
             if (!ok) break;
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
@@ -645,13 +787,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t s_waits = 0, o_waits = 0;
         bool ok = true;
         for (int iter = 0; ok; ++iter) {
-            const int buf = iter & 1;
+            int buf = iter & 1;
             if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) break;
             const uint8_t* sb = sched_base(buf);
-            const SchedHeader hdr = *reinterpret_cast<const SchedHeader*>(sb + L::kSchedHeader);
+            SchedHeader hdr = *reinterpret_cast<const SchedHeader*>(sb + L::kSchedHeader);
             if (hdr.T < 0) break;
-            const uint32_t* entries = reinterpret_cast<const uint32_t*>(sb + L::kSchedEntries);
-            const int ni = i == 0 ? hdr.n0 : hdr.n1;
+            const int ni = i == 0 ? hdr.n0 : hdr.n1;  // this q-block's tiles (one-segment units)
             const int qb = hdr.qb0 + i;
             const int q = qb * 128 + r;
             const bool row_valid = qb < p.QB && q < p.M;
@@ -682,178 +823,195 @@ __global__ void __launch_bounds__(kThreads, 1)
             float m_ref = -INFINITY;
             float l_sum = 0.f;
             int processed = 0;
-            for (int n = 0; n < hdr.T && ok; ++n) {
-                const uint32_t e = entries[n];
-                const uint32_t tags = sched_entry_tags(e);
-                if (!((tags >> i) & 1u)) continue;  // not this q-block's tile
-                const int kb = static_cast<int>(sched_entry_kb(e));
-                const bool partial = (tags >> (2 + i)) & 1u;
-                if (!mbar_wait(bar(L::kBarSFull + i), s_waits & 1u, abort_flag)) {
+            // The unit's segments, in order: the row state above carries over;
+            // every buffer but the last is released as soon as its entries are
+            // done.
+            for (;;) {
+                const uint32_t* entries = reinterpret_cast<const uint32_t*>(sb + L::kSchedEntries);
+                for (int n = 0; n < hdr.T && ok; ++n) {
+                    const uint32_t e = entries[n];
+                    const uint32_t tags = sched_entry_tags(e);
+                    if (!((tags >> i) & 1u)) continue;  // not this q-block's tile
+                    const int kb = (LONG ? hdr.kb_base : 0) + static_cast<int>(sched_entry_kb(e));
+                    const bool partial = (tags >> (2 + i)) & 1u;
+                    if (!mbar_wait(bar(L::kBarSFull + i), s_waits & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    ++s_waits;
+                    __syncwarp();  // tcgen05.ld/st are warp-collective: reconverge after the waits
+                    tc_fence_after();
+                    float x[128];
+                    {
+                        uint32_t* xr = reinterpret_cast<uint32_t*>(x);
+                        tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(xr + 0));
+                        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32));
+                        tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(xr + 64));
+                        tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(xr + 96));
+                        tc_wait_ld();
+                    }
+                    // score_mod on every visited tile. Other modes move to base-2
+                    // units here; the plain mode keeps raw scores and folds
+                    // scale * log2(e) into the exponent's FFMA below.
+                    // Column pairs go through the packed f32x2 FMA pipe (the same
+                    // roundings as one column at a time).
+                    if constexpr (SCORE != kScoreNone) {
+                        const float tile_bias = sl2 * static_cast<float>(kb * 128 - q);
+                        const float tile_pos = static_cast<float>(kb * 128 - q);  // exact below 2^24
+                        const float u_mul = p.scale * p.inv_cap;
+                        const float capl2 = p.cap * kLog2e;
+#pragma unroll
+                        for (int j = 0; j < 128; j += 2) {
+                            const float j0 = static_cast<float>(j), j1 = static_cast<float>(j + 1);
+                            if constexpr (SCORE == kScoreSoftcap) {
+                                float u0, u1;
+                                mul2(u0, u1, x[j], x[j + 1], u_mul, u_mul);
+                                mul2(x[j], x[j + 1], capl2, capl2, tanh_approx(u0), tanh_approx(u1));
+                            } else if constexpr (SCORE == kScoreAlibi) {
+                                float c0, c1;
+                                fma2(c0, c1, sl2, sl2, j0, j1, tile_bias, tile_bias);
+                                fma2(x[j], x[j + 1], x[j], x[j + 1], p.scale_log2, p.scale_log2, c0, c1);
+                            } else if constexpr (SCORE == kScoreSoftcapAlibi) {
+                                float u0, u1, c0, c1;
+                                mul2(u0, u1, x[j], x[j + 1], u_mul, u_mul);
+                                fma2(c0, c1, sl2, sl2, j0, j1, tile_bias, tile_bias);
+                                fma2(x[j], x[j + 1], capl2, capl2, tanh_approx(u0), tanh_approx(u1), c0, c1);
+                            } else {  // ALiBi, then the soft-cap
+                                float r0, r1, b0, b1, t0, t1;
+                                add2(r0, r1, tile_pos, tile_pos, j0, j1);       // kv - q, exact
+                                mul2(b0, b1, hdr.slope, hdr.slope, r0, r1);
+                                fma2(t0, t1, x[j], x[j + 1], p.scale, p.scale, b0, b1);
+                                mul2(t0, t1, t0, t1, p.inv_cap, p.inv_cap);
+                                mul2(x[j], x[j + 1], capl2, capl2, tanh_approx(t0), tanh_approx(t1));
+                            }
+                        }
+                    }
+                    // mask_mod on partial tiles only
+                    if (partial) {
+                        const int64_t c0 = static_cast<int64_t>(kb) * 128;
+                        const int64_t c1 = (c0 + 127 < p.N - 1) ? c0 + 127 : p.N - 1;
+                        const int64_t ds = row_ds, de = row_de;
+                        uint32_t w[4] = {0u, 0u, 0u, 0u};
+                        if (fast_mask) {
+                            const int tc0 = static_cast<int>(c0), tc1 = static_cast<int>(c1);
+#pragma unroll
+                            for (int t = 0; t < kRowTerms; ++t) {
+                                if (t >= dnf.n_terms) break;  // uniform: the mask's own term count
+                                int lo = iv_lo[t], hi = iv_hi[t];
+                                lo = (lo > tc0 ? lo : tc0) - tc0;
+                                hi = (hi < tc1 ? hi : tc1) - tc0;
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) w[k] |= range_bits32(lo - 32 * k, hi - 32 * k);
+                            }
+                        } else if (p.has_block_mask) {
+                            for (int t = 0; t < dnf.n_terms; ++t) {
+                                int64_t lo, hi;
+                                term_interval(dnf, t, q, c0, c1, ds, de, lo, hi);
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) w[k] |= range_bits(lo, hi, c0 + 32 * k);
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) w[k] = range_bits(c0, c1, c0 + 32 * k);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 128; ++j)
+                            if (!((w[j >> 5] >> (j & 31)) & 1u)) x[j] = -INFINITY;
+                    }
+                    // row max: eight independent chains of three-input max
+                    float mx[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        mx[k] = x[k];
+#pragma unroll
+                        for (int j = 8; j + 16 <= 128; j += 16) mx[k] = fmax3(mx[k], x[j + k], x[j + 8 + k]);
+                        mx[k] = fmaxf(mx[k], x[120 + k]);
+                    }
+                    constexpr bool kRaw = SCORE == kScoreNone;
+                    const float cmul = kRaw ? p.scale_log2 : 1.f;  // scale > 0, so max commutes with it
+                    float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+                    if constexpr (kRaw) mt *= cmul;
+                    // lazy reference update
+                    bool need_rescale = false;
+                    float alpha = 1.f;
+                    if (mt > m_ref + kRescaleThreshold) {  // false while mt is -inf
+                        if (m_ref != -INFINITY) {
+                            alpha = ex2_approx(m_ref - mt);
+                            need_rescale = processed > 0;
+                        }
+                        l_sum *= alpha;
+                        m_ref = mt;
+                    }
+                    const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                    // P = 2^(x * cmul - m). The first kEmuCols columns of every
+                    // 32-column chunk use the FMA-pipe exp2, the rest MUFU ex2.
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) {
+                            const int j = 32 * c + 2 * jj;
+                            float a0, a1, p0, p1;
+                            fma2(a0, a1, x[j], x[j + 1], cmul, cmul, neg_m, neg_m);
+                            if (2 * jj < kEmuCols<D>) {
+                                exp2_poly2(p0, p1, a0, a1);
+                            } else {
+                                p0 = ex2_approx(a0);
+                                p1 = ex2_approx(a1);
+                            }
+                            if constexpr (!kTcRowSum<D>)
+                                add2(acc[2 * (jj & 3)], acc[2 * (jj & 3) + 1], acc[2 * (jj & 3)], acc[2 * (jj & 3) + 1],
+                                     p0, p1);
+                            pk[jj] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st16(t_s + 16 * c, pk);
+                    }
+                    // a row whose every element in this tile is masked adds nothing
+                    // (the FMA-pipe exp2 returns 2^-125 rather than 0 for -inf). With the
+                    // tensor core's row sum such a row adds 2^-125 per column against its
+                    // reference, which stays negligible; a row that never has an allowed
+                    // key keeps m_ref = -inf and the epilogue treats it as empty.
+                    if (!kTcRowSum<D> && mt != -INFINITY)
+                        l_sum += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+                    // O rescale after P is out of registers (lower register peak); with
+                    // the tensor core's row sum, l (column D) is rescaled with O
+                    if (__any_sync(0xFFFFFFFFu, need_rescale)) {
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(t_o + 32 * c, o);
+                            tc_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                            tmem_st32(t_o + 32 * c, o);
+                        }
+                        if constexpr (kTcRowSum<D>) {
+                            uint32_t o[16];
+                            tmem_ld16(t_o + D, o);
+                            tc_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                            tmem_st16(t_o + D, o);
+                        }
+                    }
+                    tc_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(L::kBarPFull + i));
+                    ++processed;
+                }
+                if (!ok || !LONG || (hdr.seg & kSegLast)) break;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::kBarSchedEmpty + buf));
+                ++iter;
+                buf = iter & 1;
+                if (!mbar_wait(bar(L::kBarSchedFull + buf), static_cast<uint32_t>(iter >> 1) & 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
-                ++s_waits;
-                __syncwarp();  // tcgen05.ld/st are warp-collective: reconverge after the waits
-                tc_fence_after();
-                float x[128];
-                {
-                    uint32_t* xr = reinterpret_cast<uint32_t*>(x);
-                    tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(xr + 0));
-                    tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32));
-                    tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(xr + 64));
-                    tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(xr + 96));
-                    tc_wait_ld();
-                }
-                // score_mod on every visited tile. Other modes move to base-2
-                // units here; the plain mode keeps raw scores and folds
-                // scale * log2(e) into the exponent's FFMA below.
-                // Column pairs go through the packed f32x2 FMA pipe (the same
-                // roundings as one column at a time).
-                if constexpr (SCORE != kScoreNone) {
-                    const float tile_bias = sl2 * static_cast<float>(kb * 128 - q);
-                    const float tile_pos = static_cast<float>(kb * 128 - q);  // exact below 2^24
-                    const float u_mul = p.scale * p.inv_cap;
-                    const float capl2 = p.cap * kLog2e;
-#pragma unroll
-                    for (int j = 0; j < 128; j += 2) {
-                        const float j0 = static_cast<float>(j), j1 = static_cast<float>(j + 1);
-                        if constexpr (SCORE == kScoreSoftcap) {
-                            float u0, u1;
-                            mul2(u0, u1, x[j], x[j + 1], u_mul, u_mul);
-                            mul2(x[j], x[j + 1], capl2, capl2, tanh_approx(u0), tanh_approx(u1));
-                        } else if constexpr (SCORE == kScoreAlibi) {
-                            float c0, c1;
-                            fma2(c0, c1, sl2, sl2, j0, j1, tile_bias, tile_bias);
-                            fma2(x[j], x[j + 1], x[j], x[j + 1], p.scale_log2, p.scale_log2, c0, c1);
-                        } else if constexpr (SCORE == kScoreSoftcapAlibi) {
-                            float u0, u1, c0, c1;
-                            mul2(u0, u1, x[j], x[j + 1], u_mul, u_mul);
-                            fma2(c0, c1, sl2, sl2, j0, j1, tile_bias, tile_bias);
-                            fma2(x[j], x[j + 1], capl2, capl2, tanh_approx(u0), tanh_approx(u1), c0, c1);
-                        } else {  // ALiBi, then the soft-cap
-                            float r0, r1, b0, b1, t0, t1;
-                            add2(r0, r1, tile_pos, tile_pos, j0, j1);       // kv - q, exact
-                            mul2(b0, b1, hdr.slope, hdr.slope, r0, r1);
-                            fma2(t0, t1, x[j], x[j + 1], p.scale, p.scale, b0, b1);
-                            mul2(t0, t1, t0, t1, p.inv_cap, p.inv_cap);
-                            mul2(x[j], x[j + 1], capl2, capl2, tanh_approx(t0), tanh_approx(t1));
-                        }
-                    }
-                }
-                // mask_mod on partial tiles only
-                if (partial) {
-                    const int64_t c0 = static_cast<int64_t>(kb) * 128;
-                    const int64_t c1 = (c0 + 127 < p.N - 1) ? c0 + 127 : p.N - 1;
-                    const int64_t ds = row_ds, de = row_de;
-                    uint32_t w[4] = {0u, 0u, 0u, 0u};
-                    if (fast_mask) {
-                        const int tc0 = static_cast<int>(c0), tc1 = static_cast<int>(c1);
-#pragma unroll
-                        for (int t = 0; t < kRowTerms; ++t) {
-                            if (t >= dnf.n_terms) break;  // uniform: the mask's own term count
-                            int lo = iv_lo[t], hi = iv_hi[t];
-                            lo = (lo > tc0 ? lo : tc0) - tc0;
-                            hi = (hi < tc1 ? hi : tc1) - tc0;
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) w[k] |= range_bits32(lo - 32 * k, hi - 32 * k);
-                        }
-                    } else if (p.has_block_mask) {
-                        for (int t = 0; t < dnf.n_terms; ++t) {
-                            int64_t lo, hi;
-                            term_interval(dnf, t, q, c0, c1, ds, de, lo, hi);
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) w[k] |= range_bits(lo, hi, c0 + 32 * k);
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) w[k] = range_bits(c0, c1, c0 + 32 * k);
-                    }
-#pragma unroll
-                    for (int j = 0; j < 128; ++j)
-                        if (!((w[j >> 5] >> (j & 31)) & 1u)) x[j] = -INFINITY;
-                }
-                // row max: eight independent chains of three-input max
-                float mx[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    mx[k] = x[k];
-#pragma unroll
-                    for (int j = 8; j + 16 <= 128; j += 16) mx[k] = fmax3(mx[k], x[j + k], x[j + 8 + k]);
-                    mx[k] = fmaxf(mx[k], x[120 + k]);
-                }
-                constexpr bool kRaw = SCORE == kScoreNone;
-                const float cmul = kRaw ? p.scale_log2 : 1.f;  // scale > 0, so max commutes with it
-                float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-                if constexpr (kRaw) mt *= cmul;
-                // lazy reference update
-                bool need_rescale = false;
-                float alpha = 1.f;
-                if (mt > m_ref + kRescaleThreshold) {  // false while mt is -inf
-                    if (m_ref != -INFINITY) {
-                        alpha = ex2_approx(m_ref - mt);
-                        need_rescale = processed > 0;
-                    }
-                    l_sum *= alpha;
-                    m_ref = mt;
-                }
-                const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-                // P = 2^(x * cmul - m). The first kEmuCols columns of every
-                // 32-column chunk use the FMA-pipe exp2, the rest MUFU ex2.
-                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int j = 32 * c + 2 * jj;
-                        float a0, a1, p0, p1;
-                        fma2(a0, a1, x[j], x[j + 1], cmul, cmul, neg_m, neg_m);
-                        if (2 * jj < kEmuCols<D>) {
-                            exp2_poly2(p0, p1, a0, a1);
-                        } else {
-                            p0 = ex2_approx(a0);
-                            p1 = ex2_approx(a1);
-                        }
-                        if constexpr (!kTcRowSum<D>)
-                            add2(acc[2 * (jj & 3)], acc[2 * (jj & 3) + 1], acc[2 * (jj & 3)], acc[2 * (jj & 3) + 1],
-                                 p0, p1);
-                        pk[jj] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(t_s + 16 * c, pk);
-                }
-                // a row whose every element in this tile is masked adds nothing
-                // (the FMA-pipe exp2 returns 2^-125 rather than 0 for -inf). With the
-                // tensor core's row sum such a row adds 2^-125 per column against its
-                // reference, which stays negligible; a row that never has an allowed
-                // key keeps m_ref = -inf and the epilogue treats it as empty.
-                if (!kTcRowSum<D> && mt != -INFINITY)
-                    l_sum += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-                // O rescale after P is out of registers (lower register peak); with
-                // the tensor core's row sum, l (column D) is rescaled with O
-                if (__any_sync(0xFFFFFFFFu, need_rescale)) {
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(t_o + 32 * c, o);
-                        tc_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                        tmem_st32(t_o + 32 * c, o);
-                    }
-                    if constexpr (kTcRowSum<D>) {
-                        uint32_t o[16];
-                        tmem_ld16(t_o + D, o);
-                        tc_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                        tmem_st16(t_o + D, o);
-                    }
-                }
-                tc_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(L::kBarPFull + i));
-                ++processed;
+                sb = sched_base(buf);
+                hdr = *reinterpret_cast<const SchedHeader*>(sb + L::kSchedHeader);
             }
             if (!ok) break;
             // epilogue: out = O / l, lse = ln2 * (m + log2 l)
@@ -863,7 +1021,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // read again after the O-full wait below; this read only fixes
                 // the row's empty case early for the lse)
                 l_sum = 0.f;
-                if (ni > 0) {
+                if ((LONG ? processed : ni) > 0) {
                     if (!mbar_wait(bar(L::kBarOFull + i), o_waits & 1u, abort_flag)) break;
                     __syncwarp();
                     tc_fence_after();
@@ -882,7 +1040,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int64_t wrow = (static_cast<int64_t>(hdr.split) * p.B * p.Hq +
                                       static_cast<int64_t>(hdr.b) * p.Hq + hdr.hq) * p.M + q;
                 float4* dst = reinterpret_cast<float4*>(p.ws_o + wrow * D);
-                if (ni > 0) {
+                if ((LONG ? processed : ni) > 0) {
                     if (!mbar_wait(bar(L::kBarOFull + i), o_waits & 1u, abort_flag)) break;
                     ++o_waits;
                     __syncwarp();
@@ -905,7 +1063,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int v = 0; v < D / 4; ++v) dst[v] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
                 if (row_valid) p.ws_lse[wrow] = row_lse;
-            } else if (ni > 0) {
+            } else if ((LONG ? processed : ni) > 0) {
                 if (!mbar_wait(bar(L::kBarOFull + i), o_waits & 1u, abort_flag)) break;
                 ++o_waits;
                 __syncwarp();

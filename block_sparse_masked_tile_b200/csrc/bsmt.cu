@@ -154,7 +154,7 @@ bsmt_status build_dnf(const bsmt_mask_spec* spec, int64_t B, bsmt::MaskDnf* out)
 // ------------------------------------------------------------- device info
 std::mutex g_mu;
 int g_sm_count[64] = {0};
-bool g_attr_set[64][16] = {{false}};
+bool g_attr_set[64][32] = {{false}};
 
 bsmt_status sm_count(int* dev_out, int* n_out) {
     int dev = 0;
@@ -323,15 +323,15 @@ bsmt_status parse_score(const bsmt_score_spec* score, int64_t Hq, ScoreArgs* out
     return BSMT_OK;
 }
 
-template <int D, int SCORE>
-bsmt_status launch_attn(int dev, int nsm, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const CUtensorMap& to, const bsmt::AttnParams& p, const bsmt::MaskDnf& dnf,
-                        cudaStream_t stream) {
-    auto kern = bsmt::attn_fwd_kernel<D, SCORE>;
+template <int D, int SCORE, bool LONG>
+bsmt_status launch_attn_kind(int dev, int nsm, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& to, const bsmt::AttnParams& p, const bsmt::MaskDnf& dnf,
+                             cudaStream_t stream) {
+    auto kern = bsmt::attn_fwd_kernel<D, SCORE, LONG>;
     const int smem = bsmt::SmemLayout<D>::kAlloc;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        const int slot = (D == 128 ? 8 : 0) + SCORE;
+        const int slot = (LONG ? 16 : 0) + (D == 128 ? 8 : 0) + SCORE;
         if (!g_attr_set[dev][slot]) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -343,6 +343,15 @@ bsmt_status launch_attn(int dev, int nsm, const CUtensorMap& tq, const CUtensorM
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
     return BSMT_OK;
+}
+
+// Rows of more than kMaxKB kv blocks take the kernel's windowed variant.
+template <int D, int SCORE>
+bsmt_status launch_attn(int dev, int nsm, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const CUtensorMap& to, const bsmt::AttnParams& p, const bsmt::MaskDnf& dnf,
+                        cudaStream_t stream) {
+    if (p.KB > bsmt::kMaxKB) return launch_attn_kind<D, SCORE, true>(dev, nsm, tq, tk, tv, to, p, dnf, stream);
+    return launch_attn_kind<D, SCORE, false>(dev, nsm, tq, tk, tv, to, p, dnf, stream);
 }
 
 template <int D>
@@ -476,8 +485,6 @@ bsmt_status attention(const void* q, const void* k, const void* v, int64_t B, in
     if (M > kMaxLen || N > kMaxLen) return fail(BSMT_ERR_UNSUPPORTED, "sequence length above %lld", static_cast<long long>(kMaxLen));
     if (B * Hq > 0x7FFFFFFF || B * Hkv > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "B*H above 2^31");
     const int64_t QB = (M + 127) / 128, KB = (N + 127) / 128;
-    if (KB > bsmt::kMaxKB)
-        return fail(BSMT_ERR_UNSUPPORTED, "KV_LEN=%lld: at most %d kv blocks per row", static_cast<long long>(N), bsmt::kMaxKB);
     // a tensor with no elements may be passed as NULL (its pointer is never used)
     const bool q_has = B * Hq * M > 0, kv_has = B * Hkv * N > 0;
     if ((q_has && (!q || !out || !lse)) || (kv_has && (!k || !v)))

@@ -254,6 +254,8 @@ bsmt_status bsmt_block_mask_to_dense(const bsmt_block_mask* kv, int32_t* dense, 
  * A block listed in both lists of a row is treated as PARTIAL; the order of
  * a list does not matter. A count outside [0, KB] or an index outside
  * [0, KB) is skipped and reported as BSMT_ERR_DEVICE_BOUNDS.
+ * N is not limited beyond the int32 positions (< 2^31 - 256): a row's kv
+ * blocks are visited in windows of 1024 blocks, in order.
  */
 bsmt_status bsmt_flex_attention_fwd(const void* q, const void* k, const void* v,
                                     int64_t B, int64_t Hq, int64_t Hkv, int64_t M, int64_t N,

@@ -148,7 +148,7 @@ def test_flex_attention_argument_errors():
     assert attn(out=FAKE + 4) == INVALID
     assert attn(lse=FAKE + 2) == INVALID
     assert attn(scale=float("inf")) == INVALID
-    assert attn(N=1024 * 128 + 1) == UNSUPPORTED
+    assert attn(N=(1 << 31) - 255) == UNSUPPORTED  # kv positions must fit int32 with a tile to spare
 
 
 def test_flex_attention_score_errors():
@@ -237,7 +237,7 @@ def test_host_entry_argument_errors():
     assert host_call(ws_bytes=1000) == INVALID                # too small
     assert host_call(spec=spec_of([(C, 0), (AND, 2)])) == INVALID
     assert host_call(spec=spec_of([(DOC, 0)])) == INVALID    # document without ids
-    assert host_call(N=1025 * 128) == UNSUPPORTED            # more kv blocks than a row supports
+    assert host_call(N=(1 << 31) - 255) == UNSUPPORTED       # kv positions beyond int32
     sc = _ScoreSpec()
     sc.num_ops = 1
     sc.ops[0].kind = bsmt.SCORE_SOFTCAP
