@@ -107,8 +107,12 @@ constexpr int kBwdEmuCols = 8;
 
 // A scheduled unit in shared memory (two buffers, filled by the scheduler warp).
 struct BwdUnit {
-    int32_t T;  // entries; -1 ends the work
+    int32_t T;  // entries of this buffer; -1 ends the work
     int32_t b, hq, hkv, blk;
+    // LONG kernels: the unit's entries and the first of this buffer's. A unit
+    // of more than kBwdMaxEntries entries goes out in several buffers
+    // (segments), every one full but the last.
+    int32_t total, off;
 };
 
 template <int D>
@@ -343,7 +347,10 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* out,
     }
 }
 
-template <int D, int SCORE, bool KVSIDE>
+// LONG: lists longer than kBwdMaxEntries blocks, or units of more entries
+// (GQA group x list length), handed out in segments. Without it every unit
+// fits one buffer and the segment logic folds away.
+template <int D, int SCORE, bool KVSIDE, bool LONG>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -407,7 +414,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // A block in both lists counts as partial; with a ragged KV_LEN the
         // last kv block is partial (dq).
         uint8_t* flags = smem + L::kFlags;
-        for (int j = lane; j < p.list_len; j += 32) flags[j] = 0;
+        for (int j = lane; j < (LONG ? kBwdMaxEntries : p.list_len); j += 32) flags[j] = 0;
         __syncwarp();
         const int heads = KVSIDE ? p.group : 1;
         const bool ragged_last = !KVSIDE && (p.N & 127) != 0;
@@ -442,76 +449,208 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 hq = bh - b * p.Hq;
                 hkv = hq / p.group;
             }
-            uint32_t* entries = list_of(buf);
-            int T = 0;
-            bool bad = false;
-            for (int g = 0; g < heads; ++g) {
-                if (!p.has_block_mask) {
+            if constexpr (!LONG) {
+                uint32_t* entries = list_of(buf);
+                int T = 0;
+                bool bad = false;
+                for (int g = 0; g < heads; ++g) {
+                    if (!p.has_block_mask) {
+                        for (int c = 0; c < p.list_len; c += 32) {
+                            const int j = c + lane;
+                            if (j < p.list_len) {
+                                const bool part = ragged_last && j == p.list_len - 1;
+                                entries[T + j] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(g) << 16) |
+                                                 (part ? kBwdPartial : 0u);
+                            }
+                        }
+                        T += p.list_len;
+                        continue;
+                    }
+                    const int hl = KVSIDE ? hq + g : hq;
+                    const int bb = p.Bm > 1 ? b : 0;
+                    const int hh = p.Hm > 1 ? hl : 0;
+                    const int64_t row = (static_cast<int64_t>(bb) * p.Hm + hh) * p.list_rows + blk;
+                    int v = 0;
+                    if (lane == 0) v = __ldg(p.num + row);
+                    if (lane == 1) v = __ldg(p.full_num + row);
+                    if (v < 0 || v > p.list_len) {
+                        bad = true;
+                        v = 0;
+                    }
+                    const int cnt0 = __shfl_sync(0xFFFFFFFFu, v, 0);
+                    const int cnt1 = __shfl_sync(0xFFFFFFFFu, v, 1);
+                    const int32_t* l0 = p.idx + row * p.list_len;
+                    const int32_t* l1 = p.full_idx + row * p.list_len;
+                    for (int j = lane; j < cnt0; j += 32) {
+                        const int x = __ldg(l0 + j);
+                        if (x >= 0 && x < p.list_len) flags[x] |= 1u;
+                        else bad = true;
+                    }
+                    __syncwarp();
+                    for (int j = lane; j < cnt1; j += 32) {
+                        const int x = __ldg(l1 + j);
+                        if (x >= 0 && x < p.list_len) flags[x] |= 2u;
+                        else bad = true;
+                    }
+                    __syncwarp();
                     for (int c = 0; c < p.list_len; c += 32) {
                         const int j = c + lane;
+                        uint32_t f = 0;
                         if (j < p.list_len) {
-                            const bool part = ragged_last && j == p.list_len - 1;
-                            entries[T + j] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(g) << 16) |
-                                             (part ? kBwdPartial : 0u);
+                            f = flags[j];
+                            flags[j] = 0;
                         }
+                        const bool part = (f & 1u) || (f != 0u && ragged_last && j == p.list_len - 1);
+                        const unsigned bal = __ballot_sync(0xFFFFFFFFu, f != 0u);
+                        if (f)
+                            entries[T + __popc(bal & below)] = static_cast<uint32_t>(j) |
+                                                               (static_cast<uint32_t>(g) << 16) |
+                                                               (part ? kBwdPartial : 0u);
+                        T += __popc(bal);
                     }
-                    T += p.list_len;
-                    continue;
+                    __syncwarp();
                 }
-                const int hl = KVSIDE ? hq + g : hq;
-                const int bb = p.Bm > 1 ? b : 0;
-                const int hh = p.Hm > 1 ? hl : 0;
-                const int64_t row = (static_cast<int64_t>(bb) * p.Hm + hh) * p.list_rows + blk;
-                int v = 0;
-                if (lane == 0) v = __ldg(p.num + row);
-                if (lane == 1) v = __ldg(p.full_num + row);
-                if (v < 0 || v > p.list_len) {
+                if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
+                if (lane == 0) {
+                    hdr->T = T;
+                    hdr->b = b;
+                    hdr->hq = hq;
+                    hdr->hkv = hkv;
+                    hdr->blk = blk;
+                }
+                __syncwarp();
+                mbar_arrive(bar(L::kBarListFull + buf));
+            } else {
+                // Windows of kBwdMaxEntries list positions for the flags; the
+                // unit's entries are counted first, so that a full buffer goes
+                // out marked as continued exactly when entries remain.
+                constexpr int kCap = kBwdMaxEntries;
+                bool bad = false;
+                auto counts = [&](int g, int& cnt0, int& cnt1, const int32_t*& l0, const int32_t*& l1) {
+                    const int hl = KVSIDE ? hq + g : hq;
+                    const int bb = p.Bm > 1 ? b : 0;
+                    const int hh = p.Hm > 1 ? hl : 0;
+                    const int64_t row = (static_cast<int64_t>(bb) * p.Hm + hh) * p.list_rows + blk;
+                    int v = 0;
+                    if (lane == 0) v = __ldg(p.num + row);
+                    if (lane == 1) v = __ldg(p.full_num + row);
+                    if (v < 0 || v > p.list_len) {
+                        bad = true;
+                        v = 0;
+                    }
+                    cnt0 = __shfl_sync(0xFFFFFFFFu, v, 0);
+                    cnt1 = __shfl_sync(0xFFFFFFFFu, v, 1);
+                    l0 = p.idx + row * p.list_len;
+                    l1 = p.full_idx + row * p.list_len;
+                };
+                // bit 1: partial list, bit 2: full list, for positions [w0, w0 + span)
+                auto mark = [&](int cnt0, int cnt1, const int32_t* l0, const int32_t* l1, int w0, int span) {
+                    for (int j = lane; j < cnt0; j += 32) {
+                        const int x = __ldg(l0 + j);
+                        if (x < 0 || x >= p.list_len) bad = true;
+                        else if (x >= w0 && x - w0 < span) flags[x - w0] |= 1u;
+                    }
+                    __syncwarp();
+                    for (int j = lane; j < cnt1; j += 32) {
+                        const int x = __ldg(l1 + j);
+                        if (x < 0 || x >= p.list_len) bad = true;
+                        else if (x >= w0 && x - w0 < span) flags[x - w0] |= 2u;
+                    }
+                    __syncwarp();
+                };
+                int total = 0;
+                for (int g = 0; g < heads; ++g) {
+                    if (!p.has_block_mask) {
+                        total += p.list_len;
+                        continue;
+                    }
+                    int cnt0, cnt1;
+                    const int32_t *l0, *l1;
+                    counts(g, cnt0, cnt1, l0, l1);
+                    for (int w0 = 0; w0 < p.list_len; w0 += kCap) {
+                        const int span = min(kCap, p.list_len - w0);
+                        mark(cnt0, cnt1, l0, l1, w0, span);
+                        for (int c = 0; c < span; c += 32) {
+                            uint32_t f = 0;
+                            if (c + lane < span) {
+                                f = flags[c + lane];
+                                flags[c + lane] = 0;
+                            }
+                            total += __popc(__ballot_sync(0xFFFFFFFFu, f != 0u));
+                        }
+                        __syncwarp();
+                    }
+                }
+                int cur = buf, T = 0, off = 0;
+                uint32_t* ents = list_of(cur);
+                auto publish = [&](int t) {
+                    BwdUnit* hh = hdr_of(cur);
+                    if (lane == 0) {
+                        hh->T = t;
+                        hh->b = b;
+                        hh->hq = hq;
+                        hh->hkv = hkv;
+                        hh->blk = blk;
+                        hh->total = total;
+                        hh->off = off;
+                    }
+                    __syncwarp();
+                    mbar_arrive(bar(L::kBarListFull + cur));
+                };
+                bool ok = true;
+                for (int g = 0; g < heads && ok; ++g) {
+                    int cnt0 = 0, cnt1 = 0;
+                    const int32_t *l0 = nullptr, *l1 = nullptr;
+                    if (p.has_block_mask) counts(g, cnt0, cnt1, l0, l1);
+                    for (int w0 = 0; w0 < p.list_len && ok; w0 += kCap) {
+                        const int span = min(kCap, p.list_len - w0);
+                        if (p.has_block_mask) mark(cnt0, cnt1, l0, l1, w0, span);
+                        for (int c = 0; c < span; c += 32) {
+                            const int j = w0 + c + lane;
+                            uint32_t f = 0;
+                            if (c + lane < span) {
+                                if (p.has_block_mask) {
+                                    f = flags[c + lane];
+                                    flags[c + lane] = 0;
+                                } else {
+                                    f = 2u;  // every block, as full
+                                }
+                            }
+                            const bool part = (f & 1u) || (f != 0u && ragged_last && j == p.list_len - 1);
+                            const uint32_t ent = static_cast<uint32_t>(j) | (static_cast<uint32_t>(g) << 16) |
+                                                 (part ? kBwdPartial : 0u);
+                            const unsigned bal = __ballot_sync(0xFFFFFFFFu, f != 0u);
+                            const int pos = T + __popc(bal & below);
+                            if (f != 0u && pos < kCap) ents[pos] = ent;
+                            T += __popc(bal);
+                            if (T >= kCap && off + kCap < total) {
+                                // a full buffer with entries left: it goes out, and the
+                                // chunk's remaining entries open the next one
+                                publish(kCap);
+                                ++it;
+                                cur = it & 1;
+                                if (!mbar_wait(bar(L::kBarListEmpty + cur), static_cast<uint32_t>((it >> 1) & 1) ^ 1u,
+                                               abort_flag)) {
+                                    ok = false;
+                                    break;
+                                }
+                                ents = list_of(cur);
+                                off += kCap;
+                                if (f != 0u && pos >= kCap) ents[pos - kCap] = ent;
+                                T -= kCap;
+                            }
+                        }
+                        __syncwarp();
+                    }
+                }
+                if (!ok) break;
+                if (T > kCap) {  // (the two passes read the same lists, so this does not happen)
                     bad = true;
-                    v = 0;
+                    T = kCap;
                 }
-                const int cnt0 = __shfl_sync(0xFFFFFFFFu, v, 0);
-                const int cnt1 = __shfl_sync(0xFFFFFFFFu, v, 1);
-                const int32_t* l0 = p.idx + row * p.list_len;
-                const int32_t* l1 = p.full_idx + row * p.list_len;
-                for (int j = lane; j < cnt0; j += 32) {
-                    const int x = __ldg(l0 + j);
-                    if (x >= 0 && x < p.list_len) flags[x] |= 1u;
-                    else bad = true;
-                }
-                __syncwarp();
-                for (int j = lane; j < cnt1; j += 32) {
-                    const int x = __ldg(l1 + j);
-                    if (x >= 0 && x < p.list_len) flags[x] |= 2u;
-                    else bad = true;
-                }
-                __syncwarp();
-                for (int c = 0; c < p.list_len; c += 32) {
-                    const int j = c + lane;
-                    uint32_t f = 0;
-                    if (j < p.list_len) {
-                        f = flags[j];
-                        flags[j] = 0;
-                    }
-                    const bool part = (f & 1u) || (f != 0u && ragged_last && j == p.list_len - 1);
-                    const unsigned bal = __ballot_sync(0xFFFFFFFFu, f != 0u);
-                    if (f)
-                        entries[T + __popc(bal & below)] = static_cast<uint32_t>(j) |
-                                                           (static_cast<uint32_t>(g) << 16) |
-                                                           (part ? kBwdPartial : 0u);
-                    T += __popc(bal);
-                }
-                __syncwarp();
+                if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
+                publish(T);
             }
-            if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) record_status(BSMT_ERR_DEVICE_BOUNDS);
-            if (lane == 0) {
-                hdr->T = T;
-                hdr->b = b;
-                hdr->hq = hq;
-                hdr->hkv = hkv;
-                hdr->blk = blk;
-            }
-            __syncwarp();
-            mbar_arrive(bar(L::kBarListFull + buf));
         }
     } else if (warp == kBwdWarpLoad) {
         // ================================================= TMA producer warp
@@ -525,13 +664,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint32_t* entries = list_of(buf);
             bool ok = true;
             if (hdr.T > 0) {
-                // K, V (dk/dv) or Q, dO (dq) of the unit, once the last unit's S and dP are issued
-                if (fixed_uses > 0 &&
+                // K, V (dk/dv) or Q, dO (dq) of the unit (with its first segment),
+                // once the last unit's S and dP are issued
+                if ((!LONG || hdr.off == 0) && fixed_uses > 0 &&
                     !mbar_wait(bar(L::kBarFixedEmpty), (fixed_uses - 1) & 1u, abort_flag))
                     break;
-                ++fixed_uses;
                 const int zf = KVSIDE ? hdr.b * p.Hkv + hdr.hkv : hdr.b * p.Hq + hdr.hq;
-                if (lane == 0) {
+                if (!LONG || hdr.off == 0) ++fixed_uses;
+                if ((!LONG || hdr.off == 0) && lane == 0) {
                     const uint32_t fb = bar(L::kBarFixedFull);
                     mbar_arrive_expect_tx(fb, 2 * tile);
 #pragma unroll
@@ -622,64 +762,73 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const BwdUnit hdr = *hdr_of(buf);
             if (hdr.T < 0) break;
             const int T = hdr.T;
+            // a segment's entries are entries off .. off + T - 1 of the unit's total
+            const int total = LONG ? hdr.total : T;
+            const int off = LONG ? hdr.off : 0;
             if (T > 0) {
-                // the unit's fixed tiles; S(first) overwrites S once the last P phase has read it
-                if (!(ok = wait_phase(L::kBarFixedFull, units))) break;
-                if (pend_p && !(ok = wait_phase(L::kBarPFull, ge - 1))) break;
-                if (!(ok = wait_tiles(ge))) break;
-                issue_s(ge);
-                issue_dp(ge);
-                if (T == 1 && elect_one()) mma_commit(bar(L::kBarFixedEmpty));
-                __syncwarp();
+                if (off == 0) {
+                    // the unit's fixed tiles; S(first) overwrites S once the last P phase has read it
+                    if (!(ok = wait_phase(L::kBarFixedFull, units))) break;
+                    if (pend_p && !(ok = wait_phase(L::kBarPFull, ge - 1))) break;
+                    if (!(ok = wait_tiles(ge))) break;
+                    issue_s(ge);
+                    issue_dp(ge);
+                    if (total == 1 && elect_one()) mma_commit(bar(L::kBarFixedEmpty));
+                    __syncwarp();
+                }
                 for (int n = 0; n < T && ok; ++n) {
                     const uint32_t g = ge + n;
                     const uint32_t t0 = t0_of(g);
+                    const int nu = off + n;  // entry of the unit
+                    const bool more = nu + 1 < total;
                     // The first accumulating product of a unit overwrites the
                     // accumulators: the previous unit's epilogue must have read them.
-                    const bool acc_wait = n == 0 && units > 0;
+                    const bool acc_wait = nu == 0 && units > 0;
                     if constexpr (KVSIDE) {
                         // dV(g) += P(g)^T dO(g), S(g+1), dK(g) += dS(g)^T Q(g), dP(g+1)
                         if (!(ok = wait_phase(L::kBarPFull, g))) break;
                         if (acc_wait && !(ok = wait_phase(L::kBarAccEmpty, units - 1))) break;
-                        if (elect_one()) issue_acc(tm_a0, tm_s, t0 + L::kTile, n == 0);
+                        if (elect_one()) issue_acc(tm_a0, tm_s, t0 + L::kTile, nu == 0);
                         __syncwarp();
-                        if (n + 1 < T) {
+                        if (more) {
                             if (!(ok = wait_tiles(g + 1))) break;
                             issue_s(g + 1);
                         }
                         if (!(ok = wait_phase(L::kBarDsFull, g))) break;
                         if (elect_one()) {
-                            issue_acc(tm_a1, tm_dp, t0, n == 0);
+                            issue_acc(tm_a1, tm_dp, t0, nu == 0);
                             mma_commit(bar(L::kBarTEmpty + (g & 1u)));
                         }
                         __syncwarp();
                     } else {
                         // S(g+1) once the P phase of g has read S(g), dQ(g) += dS(g) K(g), dP(g+1)
-                        if (n + 1 < T) {
+                        if (more) {
                             if (!(ok = wait_phase(L::kBarPFull, g) && wait_tiles(g + 1))) break;
                             issue_s(g + 1);
                         }
                         if (!(ok = wait_phase(L::kBarDsFull, g))) break;
                         if (acc_wait && !(ok = wait_phase(L::kBarAccEmpty, units - 1))) break;
                         if (elect_one()) {
-                            issue_acc(tm_a0, tm_dp, t0, n == 0);
+                            issue_acc(tm_a0, tm_dp, t0, nu == 0);
                             mma_commit(bar(L::kBarTEmpty + (g & 1u)));
                         }
                         __syncwarp();
                     }
-                    if (n + 1 < T) {
+                    if (more) {
                         issue_dp(g + 1);
                         // the unit's last S and dP are issued: its fixed tiles may be replaced
-                        if (n + 2 == T && elect_one()) mma_commit(bar(L::kBarFixedEmpty));
+                        if (nu + 2 == total && elect_one()) mma_commit(bar(L::kBarFixedEmpty));
                         __syncwarp();
                     }
                 }
                 if (!ok) break;
-                if (elect_one()) mma_commit(bar(L::kBarAccFull));
-                __syncwarp();
-                pend_p = !KVSIDE;  // the dq side does not wait for its last P phase
                 ge += T;
-                ++units;
+                if (off + T == total) {  // the unit's last segment
+                    if (elect_one()) mma_commit(bar(L::kBarAccFull));
+                    __syncwarp();
+                    pend_p = !KVSIDE;  // the dq side does not wait for its last P phase
+                    ++units;
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::kBarListEmpty + buf));
@@ -704,12 +853,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t ge = 0, units = 0;
         bool ok = true;
         for (int it = 0; ok; ++it) {
-            const int buf = it & 1;
+            int buf = it & 1;
             if (!mbar_wait(bar(L::kBarListFull + buf), static_cast<uint32_t>((it >> 1) & 1), abort_flag)) break;
-            const BwdUnit hdr = *hdr_of(buf);
+            BwdUnit hdr = *hdr_of(buf);
             if (hdr.T < 0) break;
-            const uint32_t* entries = list_of(buf);
-            const int T = hdr.T;
+            const int total = LONG ? hdr.total : hdr.T;  // the unit's entries
             const int b = hdr.b, hq = hdr.hq, hkv = hdr.hkv;
             const int db = db_of ? b : 0;
             const int64_t row_idx = static_cast<int64_t>(hdr.blk) * 128 + r;  // this thread's kv (dk/dv) or q (dq)
@@ -726,7 +874,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     my_doc = __ldg(dnf.kv_doc + static_cast<int64_t>(db) * p.N + row_idx);
                     my_doc_ok = true;
                 }
-            } else if (T > 0) {
+            } else if (total > 0) {
                 const float2 ldr = p.ld[static_cast<int64_t>(b * p.Hq + hq) * p.QB * 128 + row_idx];
                 nl_row = make_float2(ldr.x, ldr.x);
                 nd_row = make_float2(ldr.y, ldr.y);
@@ -755,136 +903,153 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     }
                 }
             }
-            for (int n = 0; n < T && ok; ++n) {
-                const uint32_t g_ent = ge + n;
-                const uint32_t ent = entries[n];
-                const int eb = static_cast<int>(ent & 0xFFFFu);
-                const int g = static_cast<int>((ent >> 16) & 0xFFu);
-                const bool partial = (ent & kBwdPartial) != 0u;
-                const int64_t c0 = static_cast<int64_t>(eb) * 128 + 64 * h;  // first column (q or kv) of this warpgroup
-                // mask words over the warpgroup's 64 columns (bit j: column c0 + j allowed)
-                uint32_t w0 = 0xFFFFFFFFu, w1 = 0xFFFFFFFFu;
-                if (partial) {
-                    w0 = 0u;
-                    w1 = 0u;
-                    if constexpr (KVSIDE) {
-                        uint32_t d0 = 0xFFFFFFFFu, d1 = 0xFFFFFFFFu;
-                        if (dnf.term_has_doc) {
-                            d0 = 0u;
-                            d1 = 0u;
-                            if (my_doc_ok) {
-                                const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
+            // The unit's segments, in order (one but for LONG units of many entries);
+            // each buffer but the unit's last is released once its entries are done.
+            for (;;) {
+                const uint32_t* entries = list_of(buf);
+                const int T = hdr.T;
+                for (int n = 0; n < T && ok; ++n) {
+                    const uint32_t g_ent = ge + n;
+                    const uint32_t ent = entries[n];
+                    const int eb = static_cast<int>(ent & 0xFFFFu);
+                    const int g = static_cast<int>((ent >> 16) & 0xFFu);
+                    const bool partial = (ent & kBwdPartial) != 0u;
+                    const int64_t c0 = static_cast<int64_t>(eb) * 128 + 64 * h;  // first column (q or kv) of this warpgroup
+                    // mask words over the warpgroup's 64 columns (bit j: column c0 + j allowed)
+                    uint32_t w0 = 0xFFFFFFFFu, w1 = 0xFFFFFFFFu;
+                    if (partial) {
+                        w0 = 0u;
+                        w1 = 0u;
+                        if constexpr (KVSIDE) {
+                            uint32_t d0 = 0xFFFFFFFFu, d1 = 0xFFFFFFFFu;
+                            if (dnf.term_has_doc) {
+                                d0 = 0u;
+                                d1 = 0u;
+                                if (my_doc_ok) {
+                                    const int32_t* qd_row = dnf.q_doc + static_cast<int64_t>(db) * p.M;
 #pragma unroll 8
-                                for (int j = 0; j < 64; ++j) {
-                                    const int64_t q = c0 + j;
-                                    const bool m = q < p.M && __ldg(qd_row + q) == my_doc;
-                                    if (j < 32) d0 |= (m ? 1u : 0u) << j;
-                                    else d1 |= (m ? 1u : 0u) << (j - 32);
+                                    for (int j = 0; j < 64; ++j) {
+                                        const int64_t q = c0 + j;
+                                        const bool m = q < p.M && __ldg(qd_row + q) == my_doc;
+                                        if (j < 32) d0 |= (m ? 1u : 0u) << j;
+                                        else d1 |= (m ? 1u : 0u) << (j - 32);
+                                    }
                                 }
                             }
-                        }
-                        if (row_idx < p.N) {
-                            for (int t = 0; t < dnf.n_terms; ++t) {
-                                int64_t lo, hi;
-                                term_q_interval(dnf, t, row_idx, p.M, lo, hi);
-                                uint32_t a0 = range_bits(lo, hi, c0);
-                                uint32_t a1 = range_bits(lo, hi, c0 + 32);
-                                if ((dnf.term_has_doc >> t) & 1u) {
-                                    a0 &= d0;
-                                    a1 &= d1;
+                            if (row_idx < p.N) {
+                                for (int t = 0; t < dnf.n_terms; ++t) {
+                                    int64_t lo, hi;
+                                    term_q_interval(dnf, t, row_idx, p.M, lo, hi);
+                                    uint32_t a0 = range_bits(lo, hi, c0);
+                                    uint32_t a1 = range_bits(lo, hi, c0 + 32);
+                                    if ((dnf.term_has_doc >> t) & 1u) {
+                                        a0 &= d0;
+                                        a1 &= d1;
+                                    }
+                                    w0 |= a0;
+                                    w1 |= a1;
                                 }
-                                w0 |= a0;
-                                w1 |= a1;
-                            }
-                        }
-                    } else {
-                        const int64_t c1 = (c0 + 63 < p.N - 1) ? c0 + 63 : p.N - 1;
-                        if (masked_path) {
-                            for (int t = 0; t < dnf.n_terms; ++t) {
-                                int64_t lo, hi;
-                                term_interval(dnf, t, row_idx, c0, c1, row_ds, row_de, lo, hi);
-                                w0 |= range_bits(lo, hi, c0);
-                                w1 |= range_bits(lo, hi, c0 + 32);
                             }
                         } else {
-                            w0 = range_bits(c0, c1, c0);
-                            w1 = range_bits(c0, c1, c0 + 32);
+                            const int64_t c1 = (c0 + 63 < p.N - 1) ? c0 + 63 : p.N - 1;
+                            if (masked_path) {
+                                for (int t = 0; t < dnf.n_terms; ++t) {
+                                    int64_t lo, hi;
+                                    term_interval(dnf, t, row_idx, c0, c1, row_ds, row_de, lo, hi);
+                                    w0 |= range_bits(lo, hi, c0);
+                                    w1 |= range_bits(lo, hi, c0 + 32);
+                                }
+                            } else {
+                                w0 = range_bits(c0, c1, c0);
+                                w1 = range_bits(c0, c1, c0 + 32);
+                            }
                         }
                     }
+                    float slope = slope_unit;
+                    if constexpr (KVSIDE && kAlibi)
+                        slope = p.slopes ? __ldg(p.slopes + hq + g)
+                                         : exp2f(-8.0f * static_cast<float>(p.alibi_h0 + hq + g + 1) /
+                                                 static_cast<float>(p.alibi_heads));
+                    // kv - q at the warpgroup's column 0; it moves by -1 (dk/dv) or +1 (dq) per column
+                    const float dkv0 = KVSIDE ? static_cast<float>(row_idx - c0) : static_cast<float>(c0 - row_idx);
+                    constexpr float kStep = KVSIDE ? -1.f : 1.f;
+                    BwdCols hb;
+                    if constexpr (SCORE == kScoreAlibiSoftcap) {
+                        hb.bias0 = slope * dkv0;
+                        hb.bstep = slope * kStep;
+                    } else {
+                        hb.bias0 = slope * kLog2e * dkv0;
+                        hb.bstep = slope * kLog2e * kStep;
+                    }
+                    const float4* ld4 = reinterpret_cast<const float4*>(ld_smem + 128 * (g_ent & 1u) + 64 * h);
+                    float pg[64];  // P * dz/ds of this thread's 64 columns, from the P phase to the dS phase
+                    // ---- P phase: S -> P (bf16 into TMEM for dV on the dk/dv side)
+                    if (!mbar_wait(bar(L::kBarSFull), g_ent & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    __syncwarp();  // tcgen05.ld/st are warp-collective: reconverge after the wait
+                    tc_fence_after();
+                    {
+                        // the second 32 columns load while the first are computed
+                        float x[64];
+                        tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(x));
+                        tc_wait_ld();
+                        tmem_ld32(t_s + 32u, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {
+                            if (c == 1) tc_wait_ld();
+                            uint32_t pk[16];
+                            if (partial)
+                                bwd_p_chunk<SCORE, KVSIDE, true>(p, x, ld4, nl_row, hb, 32 * c, c == 0 ? w0 : w1, pg, pk);
+                            else
+                                bwd_p_chunk<SCORE, KVSIDE, false>(p, x, ld4, nl_row, hb, 32 * c, 0u, pg, pk);
+                            if constexpr (KVSIDE) tmem_st16(t_s + 16u * c, pk);
+                        }
+                    }
+                    if constexpr (KVSIDE) tc_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(L::kBarPFull));
+                    // ---- dS phase: dP -> dS (bf16 into TMEM for dK or dQ)
+                    if (!mbar_wait(bar(L::kBarDpFull), g_ent & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    __syncwarp();
+                    tc_fence_after();
+                    {
+                        float dp[64];
+                        tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dp));
+                        tc_wait_ld();
+                        tmem_ld32(t_dp + 32u, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {
+                            if (c == 1) tc_wait_ld();
+                            uint32_t dk[16];
+                            bwd_ds_chunk<KVSIDE>(dp, ld4, nd_row, pg, 32 * c, dk);
+                            tmem_st16(t_dp + 16u * c, dk);
+                        }
+                    }
+                    tc_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(L::kBarDsFull));
                 }
-                float slope = slope_unit;
-                if constexpr (KVSIDE && kAlibi)
-                    slope = p.slopes ? __ldg(p.slopes + hq + g)
-                                     : exp2f(-8.0f * static_cast<float>(p.alibi_h0 + hq + g + 1) /
-                                             static_cast<float>(p.alibi_heads));
-                // kv - q at the warpgroup's column 0; it moves by -1 (dk/dv) or +1 (dq) per column
-                const float dkv0 = KVSIDE ? static_cast<float>(row_idx - c0) : static_cast<float>(c0 - row_idx);
-                constexpr float kStep = KVSIDE ? -1.f : 1.f;
-                BwdCols hb;
-                if constexpr (SCORE == kScoreAlibiSoftcap) {
-                    hb.bias0 = slope * dkv0;
-                    hb.bstep = slope * kStep;
-                } else {
-                    hb.bias0 = slope * kLog2e * dkv0;
-                    hb.bstep = slope * kLog2e * kStep;
-                }
-                const float4* ld4 = reinterpret_cast<const float4*>(ld_smem + 128 * (g_ent & 1u) + 64 * h);
-                float pg[64];  // P * dz/ds of this thread's 64 columns, from the P phase to the dS phase
-                // ---- P phase: S -> P (bf16 into TMEM for dV on the dk/dv side)
-                if (!mbar_wait(bar(L::kBarSFull), g_ent & 1u, abort_flag)) {
+                if (!ok) break;
+                ge += T;
+                if (!LONG || hdr.off + T == total) break;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(L::kBarListEmpty + buf));
+                ++it;
+                buf = it & 1;
+                if (!mbar_wait(bar(L::kBarListFull + buf), static_cast<uint32_t>((it >> 1) & 1), abort_flag)) {
                     ok = false;
                     break;
                 }
-                __syncwarp();  // tcgen05.ld/st are warp-collective: reconverge after the wait
-                tc_fence_after();
-                {
-                    // the second 32 columns load while the first are computed
-                    float x[64];
-                    tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(x));
-                    tc_wait_ld();
-                    tmem_ld32(t_s + 32u, *reinterpret_cast<uint32_t(*)[32]>(x + 32));
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        if (c == 1) tc_wait_ld();
-                        uint32_t pk[16];
-                        if (partial)
-                            bwd_p_chunk<SCORE, KVSIDE, true>(p, x, ld4, nl_row, hb, 32 * c, c == 0 ? w0 : w1, pg, pk);
-                        else
-                            bwd_p_chunk<SCORE, KVSIDE, false>(p, x, ld4, nl_row, hb, 32 * c, 0u, pg, pk);
-                        if constexpr (KVSIDE) tmem_st16(t_s + 16u * c, pk);
-                    }
-                }
-                if constexpr (KVSIDE) tc_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(L::kBarPFull));
-                // ---- dS phase: dP -> dS (bf16 into TMEM for dK or dQ)
-                if (!mbar_wait(bar(L::kBarDpFull), g_ent & 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                __syncwarp();
-                tc_fence_after();
-                {
-                    float dp[64];
-                    tmem_ld32(t_dp, *reinterpret_cast<uint32_t(*)[32]>(dp));
-                    tc_wait_ld();
-                    tmem_ld32(t_dp + 32u, *reinterpret_cast<uint32_t(*)[32]>(dp + 32));
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        if (c == 1) tc_wait_ld();
-                        uint32_t dk[16];
-                        bwd_ds_chunk<KVSIDE>(dp, ld4, nd_row, pg, 32 * c, dk);
-                        tmem_st16(t_dp + 16u * c, dk);
-                    }
-                }
-                tc_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(L::kBarDsFull));
+                hdr = *hdr_of(buf);
             }
             if (!ok) break;
-            ge += T;
             // -------------------------------------------------- epilogue
             // dk/dv: warpgroup 0 writes dV, warpgroup 1 writes dK (times scale).
             // dq: warpgroup h writes columns [h D/2, (h+1) D/2) of dQ (times
@@ -900,7 +1065,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             else
                 dst = p.g0 + static_cast<int64_t>(b * p.Hq + hq) * p.q_sbh + row_idx * p.q_ss + h * (D / 2);
             uint4* d4 = reinterpret_cast<uint4*>(dst);
-            if (T > 0) {
+            if (total > 0) {
                 if (!(ok = mbar_wait(bar(L::kBarAccFull), units & 1u, abort_flag))) break;
                 ++units;
                 __syncwarp();

@@ -826,7 +826,7 @@ extern "C" bsmt_status bsmt_flex_attention_fwd_packed(const void* q, const void*
 
 // ------------------------------------------------------------------ backward
 namespace {
-bool g_bwd_attr_set[64][20] = {{false}};
+bool g_bwd_attr_set[64][40] = {{false}};
 
 __global__ void zero_kernel(uint4* p, int64_t n) {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -842,14 +842,15 @@ bsmt_status zero_bf16(void* p, int64_t elems, int nsm, cudaStream_t s) {
     return BSMT_OK;
 }
 
-template <int D, int SCORE, bool KVSIDE>
-bsmt_status launch_bwd(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const bsmt::BwdParams& p, const bsmt::MaskDnf& dnf, cudaStream_t s) {
-    auto kern = bsmt::attn_bwd_kernel<D, SCORE, KVSIDE>;
+template <int D, int SCORE, bool KVSIDE, bool LONG>
+bsmt_status launch_bwd_kind(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const bsmt::BwdParams& p, const bsmt::MaskDnf& dnf,
+                            cudaStream_t s) {
+    auto kern = bsmt::attn_bwd_kernel<D, SCORE, KVSIDE, LONG>;
     const int smem = bsmt::BwdSmem<D>::kAlloc;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        const int slot = (D == 128 ? 10 : 0) + 2 * SCORE + (KVSIDE ? 1 : 0);
+        const int slot = (LONG ? 20 : 0) + (D == 128 ? 10 : 0) + 2 * SCORE + (KVSIDE ? 1 : 0);
         if (!g_bwd_attr_set[dev][slot]) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -864,6 +865,17 @@ bsmt_status launch_bwd(int dev, const CUtensorMap& tq, const CUtensorMap& tk, co
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(BSMT_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
     return BSMT_OK;
+}
+
+// Units of more entries than one buffer holds (list length x heads), or lists
+// longer than the flag window, take the kernel's segmented variant.
+template <int D, int SCORE, bool KVSIDE>
+bsmt_status launch_bwd(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const bsmt::BwdParams& p, const bsmt::MaskDnf& dnf, cudaStream_t s) {
+    const int64_t per_unit = static_cast<int64_t>(p.list_len) * (KVSIDE ? p.group : 1);
+    if (per_unit > bsmt::kBwdMaxEntries)
+        return launch_bwd_kind<D, SCORE, KVSIDE, true>(dev, tq, tk, tv, tdo, p, dnf, s);
+    return launch_bwd_kind<D, SCORE, KVSIDE, false>(dev, tq, tk, tv, tdo, p, dnf, s);
 }
 
 template <int D, bool KVSIDE>
@@ -917,12 +929,12 @@ bsmt_status backward(const void* q, const void* k, const void* v, const void* ou
     if (B * Hq > 0x7FFFFFFF || B * Hkv > 0x7FFFFFFF) return fail(BSMT_ERR_UNSUPPORTED, "B*H above 2^31");
     const int64_t QB = (M + 127) / 128, KB = (N + 127) / 128;
     const int64_t group = Hq / Hkv;
-    if (KB > bsmt::kBwdMaxEntries)
-        return fail(BSMT_ERR_UNSUPPORTED, "KV_LEN=%lld: at most %d kv blocks per row", static_cast<long long>(N),
-                    bsmt::kBwdMaxEntries);
-    if (group * QB > bsmt::kBwdMaxEntries || group > 255)
-        return fail(BSMT_ERR_UNSUPPORTED, "Q_LEN=%lld with %lld query heads per kv head: at most %d q-blocks x heads",
-                    static_cast<long long>(M), static_cast<long long>(group), bsmt::kBwdMaxEntries);
+    // entries hold a block number in 16 bits and a head of the GQA group in 8
+    if (KB > 65536 || QB > 65536)
+        return fail(BSMT_ERR_UNSUPPORTED, "Q_LEN=%lld, KV_LEN=%lld: at most 65536 blocks of 128 per sequence",
+                    static_cast<long long>(M), static_cast<long long>(N));
+    if (group > 255)
+        return fail(BSMT_ERR_UNSUPPORTED, "%lld query heads per kv head: at most 255", static_cast<long long>(group));
     const bool q_has = B * Hq * M > 0, kv_has = B * Hkv * N > 0;
     if ((q_has && (!q || !out || !dout || !lse || !dq)) || (kv_has && (!k || !v || !dk || !dv)))
         return fail(BSMT_ERR_INVALID_ARGUMENT, "q, k, v, out, dout, lse, dq, dk and dv must be non-NULL when they hold elements");

@@ -445,8 +445,8 @@ bsmt_status bsmt_flex_attention_bwd_workspace_bytes(int64_t B, int64_t Hq, int64
  *   workspace  caller-owned device memory, 256-byte aligned, at least
  *           bsmt_flex_attention_bwd_workspace_bytes bytes; written and read
  *           back by the call, reusable once the stream has passed it
- * Limits: ceil(N/128) <= 2048 and (Hq/Hkv) * ceil(M/128) <= 2048, else
- * BSMT_ERR_UNSUPPORTED. Calls that share a workspace must not overlap in
+ * Limits: ceil(M/128) and ceil(N/128) at most 65536, Hq/Hkv at most 255,
+ * else BSMT_ERR_UNSUPPORTED. Calls that share a workspace must not overlap in
  * time (it holds the kernels' work counters). Bad list entries are skipped and reported as
  * BSMT_ERR_DEVICE_BOUNDS. Stream-ordered on `stream`. */
 bsmt_status bsmt_flex_attention_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,

@@ -382,8 +382,9 @@ def test_backward_argument_errors():
     assert bwd(ptr=FAKE + 8) == INVALID                      # misaligned tensors
     assert bwd(lse=FAKE + 2) == INVALID
     assert bwd(scale=float("nan")) == INVALID
-    assert bwd(N=2049 * 128) == UNSUPPORTED                  # more than 2048 kv blocks per dq row
-    assert bwd(Hq=8, Hkv=1, gqa=1, M=257 * 128) == UNSUPPORTED  # 8 heads x 257 q-blocks > 2048 entries
+    assert bwd(N=65537 * 128) == UNSUPPORTED                 # block numbers beyond 16 bits
+    assert bwd(M=65537 * 128) == UNSUPPORTED
+    assert bwd(Hq=256, Hkv=1, gqa=1) == UNSUPPORTED         # a GQA group beyond 255 heads
     # a block mask without its q-side lists
     c = _BlockMask()
     c.kv_num_blocks = c.kv_indices = c.full_kv_num_blocks = c.full_kv_indices = FAKE

@@ -276,12 +276,12 @@ def test_autograd_through_flex_attention():
         bsmt.flex_attention(qg, kg, vg, block_mask=bm, enable_gqa=True, num_splits=2)
 
 
-def test_maximum_length_forward_and_backward():
-    """The longest sequences the library takes: KV_LEN = 1024 kv blocks (the
-    forward's limit) with GQA 2:1, so a dk/dv unit walks 2 heads x 1024
-    q-blocks = 2048 entries (the backward's limit). Sampled query rows are
-    compared for out, lse and dq; dk/dv rows for keys near the end, which
-    few queries reach under the causal mask."""
+def test_one_buffer_boundary_forward_and_backward():
+    """KV_LEN = 1024 kv blocks (the forward's one window) with GQA 2:1, so a
+    dk/dv unit walks 2 heads x 1024 q-blocks = 2048 entries, exactly one
+    buffer of the backward's scheduler. Sampled query rows are compared for
+    out, lse and dq; dk/dv rows for keys near the end, which few queries
+    reach under the causal mask."""
     from oracle import attention as oa
     from tests.gpu_helpers import assert_attention_close
     L, D = 1024 * 128, 64
