@@ -40,7 +40,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libbsmt.so")
 
 # ------------------------------------------------------------------ C ABI
-MAX_NODES = 32
+MAX_NODES = 64
 MAX_SCORE_OPS = 2
 (MASK_NOOP, MASK_CAUSAL, MASK_WINDOW, MASK_PREFIX_LM, MASK_SINK, MASK_DOCUMENT, MASK_AND, MASK_OR) = range(8)
 SCORE_NONE, SCORE_SOFTCAP, SCORE_ALIBI = 0, 1, 2

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -49,9 +50,78 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 constexpr int64_t kMaxLen = (int64_t(1) << 31) - 256;
 
 // ------------------------------------------------------------------ DNF
-struct Dnf {
-    std::vector<std::vector<bsmt::DnfLeaf>> terms;
+// One AND-term of the mask program in canonical form. Leaves of one kind in
+// a term collapse to the strictest: CAUSAL and DOCUMENT are idempotent, and
+// for the others the smaller argument allows a subset of rows' keys
+// (WINDOW(W): kv >= q - W + 1; PREFIX_LM(P): kv <= max(P - 1, q); SINK(S):
+// kv <= S - 1). So a term is at most one leaf of each kind, and the empty
+// term is NOOP.
+struct Term {
+    bool causal = false, doc = false, has_w = false, has_p = false, has_s = false;
+    int32_t w = 0, pf = 0, s = 0;
+    bool operator==(const Term& o) const {
+        return causal == o.causal && doc == o.doc && has_w == o.has_w && has_p == o.has_p && has_s == o.has_s &&
+               (!has_w || w == o.w) && (!has_p || pf == o.pf) && (!has_s || s == o.s);
+    }
 };
+
+Term leaf_term(int32_t kind, int32_t arg) {
+    Term t;
+    switch (kind) {
+        case BSMT_MASK_CAUSAL: t.causal = true; break;
+        case BSMT_MASK_DOCUMENT: t.doc = true; break;
+        case BSMT_MASK_WINDOW: t.has_w = true; t.w = arg; break;
+        case BSMT_MASK_PREFIX_LM: t.has_p = true; t.pf = arg; break;
+        case BSMT_MASK_SINK: t.has_s = true; t.s = arg; break;
+        default: break;  // NOOP
+    }
+    return t;
+}
+
+// a AND b
+Term term_and(const Term& a, const Term& b) {
+    Term t = a;
+    t.causal = a.causal || b.causal;
+    t.doc = a.doc || b.doc;
+    if (b.has_w) t.w = a.has_w ? std::min(a.w, b.w) : b.w;
+    if (b.has_p) t.pf = a.has_p ? std::min(a.pf, b.pf) : b.pf;
+    if (b.has_s) t.s = a.has_s ? std::min(a.s, b.s) : b.s;
+    t.has_w = a.has_w || b.has_w;
+    t.has_p = a.has_p || b.has_p;
+    t.has_s = a.has_s || b.has_s;
+    return t;
+}
+
+// Every key `inner` allows, `outer` allows too: each of outer's leaves has a
+// leaf of the same kind in inner that is at least as strict.
+bool term_within(const Term& inner, const Term& outer) {
+    if (outer.causal && !inner.causal) return false;
+    if (outer.doc && !inner.doc) return false;
+    if (outer.has_w && !(inner.has_w && inner.w <= outer.w)) return false;
+    if (outer.has_p && !(inner.has_p && inner.pf <= outer.pf)) return false;
+    if (outer.has_s && !(inner.has_s && inner.s <= outer.s)) return false;
+    return true;
+}
+
+// The same union of terms without repeats and without terms that another
+// term contains.
+void simplify(std::vector<Term>& terms) {
+    std::vector<Term> uniq;
+    for (const Term& t : terms)
+        if (std::find(uniq.begin(), uniq.end(), t) == uniq.end()) uniq.push_back(t);
+    std::vector<Term> out;
+    for (size_t i = 0; i < uniq.size(); ++i) {
+        bool inside = false;
+        for (size_t j = 0; j < uniq.size() && !inside; ++j) inside = j != i && term_within(uniq[i], uniq[j]);
+        if (!inside) out.push_back(uniq[i]);
+    }
+    terms = std::move(out);
+}
+
+// Terms held while the program is evaluated; only the final count must fit
+// kMaxTerms, since later ANDs and ORs can merge terms again.
+constexpr size_t kMaxWorkTerms = 1024;
+static_assert(5 * bsmt::kMaxTerms <= bsmt::kMaxLeaves, "a canonical term has at most one leaf of each of 5 kinds");
 
 bsmt_status build_dnf(const bsmt_mask_spec* spec, int64_t B, bsmt::MaskDnf* out) {
     std::memset(out, 0, sizeof(*out));
@@ -64,56 +134,45 @@ bsmt_status build_dnf(const bsmt_mask_spec* spec, int64_t B, bsmt::MaskDnf* out)
     if (spec->num_nodes < 1 || spec->num_nodes > BSMT_MAX_MASK_NODES)
         return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: num_nodes=%d outside [1, %d]", spec->num_nodes,
                     BSMT_MAX_MASK_NODES);
-    std::vector<Dnf> stack;
+    std::vector<std::vector<Term>> stack;
     bool has_doc = false;
-    auto too_big = [](const Dnf& d) {
-        size_t leaves = 0;
-        for (auto& t : d.terms) leaves += t.size();
-        return d.terms.size() > size_t(bsmt::kMaxTerms) || leaves > size_t(bsmt::kMaxLeaves);
-    };
     for (int i = 0; i < spec->num_nodes; ++i) {
         const bsmt_mask_node nd = spec->nodes[i];
         switch (nd.kind) {
             case BSMT_MASK_NOOP:
-                stack.push_back(Dnf{{{}}});
-                break;
             case BSMT_MASK_CAUSAL:
             case BSMT_MASK_WINDOW:
             case BSMT_MASK_PREFIX_LM:
             case BSMT_MASK_SINK:
             case BSMT_MASK_DOCUMENT:
                 if (nd.kind == BSMT_MASK_DOCUMENT) has_doc = true;
-                stack.push_back(Dnf{{{bsmt::DnfLeaf{nd.kind, nd.arg}}}});
+                stack.push_back({leaf_term(nd.kind, nd.arg)});
                 break;
             case BSMT_MASK_AND:
             case BSMT_MASK_OR: {
                 if (nd.arg < 1 || size_t(nd.arg) > stack.size())
                     return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: node %d (%s) takes %d operands, %zu available", i,
                                 nd.kind == BSMT_MASK_AND ? "AND" : "OR", nd.arg, stack.size());
-                std::vector<Dnf> ops(stack.end() - nd.arg, stack.end());
+                std::vector<std::vector<Term>> ops(stack.end() - nd.arg, stack.end());
                 stack.resize(stack.size() - nd.arg);
-                Dnf res;
+                std::vector<Term> res;
                 if (nd.kind == BSMT_MASK_OR) {
-                    for (auto& d : ops)
-                        for (auto& t : d.terms) res.terms.push_back(t);
+                    for (auto& d : ops) res.insert(res.end(), d.begin(), d.end());
+                    simplify(res);
                 } else {
-                    res.terms = {{}};
+                    res = {Term{}};
                     for (auto& d : ops) {
-                        Dnf nxt;
-                        for (auto& a : res.terms)
-                            for (auto& b : d.terms) {
-                                auto t = a;
-                                t.insert(t.end(), b.begin(), b.end());
-                                nxt.terms.push_back(std::move(t));
-                            }
+                        std::vector<Term> nxt;
+                        for (auto& a : res)
+                            for (auto& b : d) nxt.push_back(term_and(a, b));
+                        simplify(nxt);
                         res = std::move(nxt);
-                        if (too_big(res)) break;
+                        if (res.size() > kMaxWorkTerms) break;
                     }
                 }
-                if (too_big(res))
-                    return fail(BSMT_ERR_UNSUPPORTED,
-                                "mask spec: more than %d alternatives or %d leaves after distributing AND over OR",
-                                bsmt::kMaxTerms, bsmt::kMaxLeaves);
+                if (res.size() > kMaxWorkTerms)
+                    return fail(BSMT_ERR_UNSUPPORTED, "mask spec: more than %zu alternatives while distributing AND over OR",
+                                kMaxWorkTerms);
                 stack.push_back(std::move(res));
                 break;
             }
@@ -123,6 +182,10 @@ bsmt_status build_dnf(const bsmt_mask_spec* spec, int64_t B, bsmt::MaskDnf* out)
     }
     if (stack.size() != 1)
         return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: program leaves %zu values (expected 1)", stack.size());
+    const std::vector<Term>& terms = stack[0];
+    if (terms.size() > size_t(bsmt::kMaxTerms))
+        return fail(BSMT_ERR_UNSUPPORTED, "mask spec: %zu alternatives after distributing AND over OR (at most %d)",
+                    terms.size(), bsmt::kMaxTerms);
     if (has_doc) {
         if (spec->q_doc_ids == nullptr || spec->kv_doc_ids == nullptr)
             return fail(BSMT_ERR_INVALID_ARGUMENT, "mask spec: DOCUMENT needs q_doc_ids and kv_doc_ids");
@@ -132,19 +195,23 @@ bsmt_status build_dnf(const bsmt_mask_spec* spec, int64_t B, bsmt::MaskDnf* out)
             return fail(BSMT_ERR_SHAPE_MISMATCH, "mask spec: doc_batch=%d must be 1 or B=%lld", spec->doc_batch,
                         static_cast<long long>(B));
     }
-    const Dnf& d = stack[0];
-    out->n_terms = static_cast<int32_t>(d.terms.size());
+    out->n_terms = static_cast<int32_t>(terms.size());
     int pos = 0;
-    for (size_t t = 0; t < d.terms.size(); ++t) {
+    for (size_t t = 0; t < terms.size(); ++t) {
+        const Term& tm = terms[t];
         out->term_begin[t] = pos;
-        for (auto& lf : d.terms[t]) {
-            if (lf.kind == BSMT_MASK_NOOP) continue;
-            if (lf.kind == BSMT_MASK_DOCUMENT) out->term_has_doc |= 1u << t;
-            out->leaves[pos++] = lf;
+        if (tm.causal) out->leaves[pos++] = bsmt::DnfLeaf{BSMT_MASK_CAUSAL, 0};
+        if (tm.has_w) out->leaves[pos++] = bsmt::DnfLeaf{BSMT_MASK_WINDOW, tm.w};
+        if (tm.has_p) out->leaves[pos++] = bsmt::DnfLeaf{BSMT_MASK_PREFIX_LM, tm.pf};
+        if (tm.has_s) out->leaves[pos++] = bsmt::DnfLeaf{BSMT_MASK_SINK, tm.s};
+        if (tm.doc) {
+            out->leaves[pos++] = bsmt::DnfLeaf{BSMT_MASK_DOCUMENT, 0};
+            out->term_has_doc |= 1u << t;
         }
     }
-    out->term_begin[d.terms.size()] = pos;
-    out->has_doc = has_doc ? 1 : 0;
+    out->term_begin[terms.size()] = pos;
+    // a program whose DOCUMENT leaves all fell inside other terms needs no ids
+    out->has_doc = out->term_has_doc != 0u ? 1 : 0;
     out->q_doc = spec->q_doc_ids;
     out->kv_doc = spec->kv_doc_ids;
     out->doc_batch = spec->doc_batch < 1 ? 1 : spec->doc_batch;
@@ -372,7 +439,7 @@ bsmt_status launch_attn_score(int score, int dev, int nsm, const CUtensorMap& tq
 
 extern "C" {
 
-int32_t bsmt_version(void) { return (2 << 16) | 0; }
+int32_t bsmt_version(void) { return (2 << 16) | 1; }
 
 const char* bsmt_last_error(void) { return g_last_error.c_str(); }
 

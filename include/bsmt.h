@@ -82,12 +82,20 @@ typedef enum bsmt_status {
  * packed documents: each document's keys are contiguous. q_doc_ids may be
  * in any order. bsmt_create_block_mask checks the kv order on the device.
  *
- * Limits: at most BSMT_MAX_MASK_NODES nodes. After AND is distributed over
- * OR, the program must have at most BSMT_MAX_MASK_TERMS alternatives and at
- * most BSMT_MAX_MASK_LEAVES leaf occurrences in total. A larger program
- * returns BSMT_ERR_UNSUPPORTED.
+ * The library distributes AND over OR and simplifies as it goes: within an
+ * alternative (an AND of leaves), leaves of one kind collapse to the
+ * strictest (one CAUSAL, one DOCUMENT, the smallest W, P and S), repeated
+ * alternatives merge, and an alternative that another one contains is
+ * dropped (each of the other's leaves has one of the same kind in it, at
+ * least as strict). The result is the same predicate.
+ *
+ * Limits: at most BSMT_MAX_MASK_NODES nodes, and at most
+ * BSMT_MAX_MASK_TERMS alternatives after the simplification (1024 while
+ * the program is evaluated); each alternative then has at most 5 leaves,
+ * within BSMT_MAX_MASK_LEAVES. A larger program returns
+ * BSMT_ERR_UNSUPPORTED.
  */
-#define BSMT_MAX_MASK_NODES 32
+#define BSMT_MAX_MASK_NODES 64
 #define BSMT_MAX_MASK_TERMS 16
 #define BSMT_MAX_MASK_LEAVES 128
 

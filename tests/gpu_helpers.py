@@ -1,4 +1,6 @@
 """Shared helpers for the GPU parity tests (CUDA path vs the fp64 oracle)."""
+import ctypes
+
 import numpy as np
 import torch
 
@@ -56,23 +58,18 @@ def assert_attention_close(out, lse, ref_out, ref_lse, what=""):
     return float(err.max(initial=0.0)), float(lerr.max(initial=0.0))
 
 
-def dnf_size(tree):
-    """(alternatives, leaf occurrences) after distributing AND over OR."""
-    kind = tree[0]
-    if kind in ("and", "or"):
-        parts = [dnf_size(c) for c in tree[1:]]
-        if kind == "or":
-            return sum(t for t, _ in parts), sum(lv for _, lv in parts)
-        terms, leaves = 1, 0
-        for t, lv in parts:
-            leaves = leaves * t + lv * terms
-            terms *= t
-        return terms, leaves
-    return 1, 1
-
-
 def within_dnf_limits(tree) -> bool:
+    """Whether the library takes this mask program: its node count and its
+    alternatives after the library's own simplification fit the limits. A
+    host-only check (a block mask with no rows launches nothing)."""
     if tree is None:
         return True
-    t, lv = dnf_size(tree)
-    return t <= 16 and lv <= 128
+    mm = bsmt.mask_from_tree(tree)
+    if len(mm.nodes) > bsmt.MAX_NODES:
+        return False
+    spec, keep = mm._spec(torch.device("cpu"), 1)
+    out = bsmt._BlockMask()
+    st = bsmt._lib.bsmt_create_block_mask(ctypes.byref(spec), max(1, spec.doc_batch), 1, 0, 0, 128, 128,
+                                          ctypes.byref(out), None)
+    del keep
+    return st == 0

@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version():
-    assert _lib.bsmt_version() == (2 << 16)
+    assert _lib.bsmt_version() == (2 << 16) | 1
 
 
 def shape(*args):
@@ -105,16 +105,28 @@ def test_create_block_mask_malformed(nodes, code):
     assert _lib.bsmt_last_error()
 
 
-def test_create_block_mask_too_many_terms():
-    # AND of 5 binary ORs expands to 32 alternatives (> 16)
+def test_create_block_mask_alternatives_after_simplification():
+    # AND of 5 binary ORs of CAUSAL and SINK(2) expands to 32 alternatives,
+    # which collapse to {CAUSAL} and {SINK(2)}: one leaf of a kind per
+    # alternative, and CAUSAL AND SINK lies inside both
     nodes = []
     for _ in range(5):
         nodes += [(C, 0), (S, 2), (OR, 2)]
     nodes.append((AND, 5))
     st, _ = build(spec_of(nodes), M=0, N=10)
-    assert st == UNSUPPORTED
-    # 16 alternatives are still accepted
-    st, _ = build(spec_of(nodes[:-1 - 3] + [(AND, 4)]), M=0, N=10)
+    assert st == OK, _lib.bsmt_last_error()
+    # an OR of 17 alternatives WINDOW(w) AND SINK(s) with w rising and s
+    # falling: none contains another, so 17 remain (> 16)
+    nodes = [n for i in range(17) for n in [(W, 10 + i), (S, 100 - i), (AND, 2)]] + [(OR, 17)]
+    assert len(nodes) == 52
+    st, _ = build(spec_of(nodes), M=0, N=10)
+    assert st == UNSUPPORTED and "17 alternatives" in _lib.bsmt_last_error().decode()
+    # 16 of them are accepted; a repeat of one adds nothing
+    nodes = [n for i in range(16) for n in [(W, 10 + i), (S, 100 - i), (AND, 2)]]
+    st, _ = build(spec_of(nodes + [(W, 10), (S, 100), (AND, 2), (OR, 17)]), M=0, N=10)
+    assert st == OK, _lib.bsmt_last_error()
+    # ... and one with a stricter window and sink than another lies inside it
+    st, _ = build(spec_of(nodes + [(W, 9), (S, 99), (AND, 2), (OR, 17)]), M=0, N=10)
     assert st == OK, _lib.bsmt_last_error()
 
 

@@ -71,6 +71,27 @@ def test_random_masks_and_shapes(seed):
     run_case(seed, B, Hq, Hkv, M, N, D, tree, mods)
 
 
+@pytest.mark.parametrize("seed", range(8))
+def test_deep_masks(seed):
+    # four-level programs, simplified by the library before the kernels see
+    # them (more than 4 alternatives take the kernel's general mask path)
+    rng = np.random.default_rng(900 + seed)
+    D = int(rng.choice([64, 128]))
+    Hkv = int(rng.integers(1, 3))
+    Hq = Hkv * int(rng.choice([1, 2]))
+    M = int(rng.integers(100, 700))
+    N = int(rng.integers(100, 700))
+    tree = workloads.random_mask_tree(rng, 1, M, N, depth=4)
+    mods = [(), (("softcap", 20.0),), (("alibi", None),)][int(rng.integers(3))]
+    run_case(seed, 1, Hq, Hkv, M, N, D, tree, mods)
+
+
+def test_and_of_five_ors():
+    # 32 alternatives before the library's simplification
+    from tests.test_gpu_block_mask import _and_of_ors
+    run_case(77, 1, 4, 2, 1000, 1000, 128, _and_of_ors(1000), (("alibi", None),))
+
+
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("S", [1, 4, 31, 32, 33])
 def test_sink_tiles(D, S):

@@ -124,6 +124,16 @@ def test_random_masks_and_shapes(seed):
     run_case(seed, B, Hq, Hkv, M, N, D, tree, mods)
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_deep_masks(seed):
+    # four-level programs after the library's simplification, on both walks
+    rng = np.random.default_rng(950 + seed)
+    M = int(rng.integers(100, 600))
+    N = int(rng.integers(100, 600))
+    tree = workloads.random_mask_tree(rng, 1, M, N, depth=4)
+    run_case(970 + seed, 1, 2, 1, M, N, 64, tree, ())
+
+
 def test_broadcast_block_mask():
     run_case(21, 2, 4, 2, 512, 512, 128, ("and", ("causal",), ("window", 200)), (), mask_B=1, mask_H=1)
 

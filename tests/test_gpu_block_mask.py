@@ -44,6 +44,48 @@ def test_random_specs_bit_exact(seed):
     assert_block_mask_equal(block_mask_numpy(bm), want)
 
 
+@pytest.mark.parametrize("seed", range(12))
+def test_deep_specs_bit_exact(seed):
+    # programs four and five levels deep: most expand to more than 16
+    # alternatives before the library's simplification (one leaf of a kind
+    # per alternative, repeats and contained alternatives dropped), and the
+    # simplified program must give the same tiles as the oracle's direct
+    # evaluation of the tree
+    rng = np.random.default_rng(700 + seed)
+    B = int(rng.integers(1, 3))
+    H = int(rng.integers(1, 3))
+    M = int(rng.integers(1, 900))
+    N = int(rng.integers(1, 900))
+    while True:  # a program of 12 to 64 nodes
+        tree = workloads.random_mask_tree(rng, B, M, N, depth=4 + seed % 2)
+        if 12 <= len(bsmt.mask_from_tree(tree).nodes) <= bsmt.MAX_NODES:
+            break
+    if not within_dnf_limits(tree):
+        with pytest.raises(bsmt.BsmtError, match="UNSUPPORTED"):
+            gpu_block_mask(tree, B, H, M, N)
+        return
+    bm = gpu_block_mask(tree, B, H, M, N)
+    want = obm.create_block_mask(tree, B, H, M, N)
+    assert_block_mask_equal(block_mask_numpy(bm), want)
+
+
+def _and_of_ors(L):
+    ids = np.repeat(np.arange(4, dtype=np.int32), [L // 4, L // 4, L // 4, L - 3 * (L // 4)])[None]
+    return ("and", ("or", ("causal",), ("sink", 64)), ("or", ("window", 300), ("prefix_lm", 200)),
+            ("or", ("causal",), ("window", 500)), ("or", ("sink", 32), ("document", ids, ids)),
+            ("or", ("causal",), ("prefix_lm", 100)))
+
+
+def test_and_of_five_ors_bit_exact():
+    # 2^5 = 32 alternatives when AND is distributed over OR, fewer once
+    # simplified; the tiles must equal the oracle's direct evaluation
+    L = 1000
+    tree = _and_of_ors(L)
+    assert within_dnf_limits(tree)
+    bm = gpu_block_mask(tree, 1, 2, L, L)
+    assert_block_mask_equal(block_mask_numpy(bm), obm.create_block_mask(tree, 1, 2, L, L))
+
+
 def test_broadcast_none_b_h():
     tree = ("and", ("causal",), ("window", 300))
     bm = gpu_block_mask(tree, None, None, 1000, 1000)
