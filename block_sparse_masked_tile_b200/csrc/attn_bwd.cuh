@@ -245,40 +245,25 @@ __device__ __forceinline__ void bwd_ds_chunk(const float* dp, const float4* ld4,
     }
 }
 
-// The q interval [lo, hi] one non-document leaf allows for a fixed key kv
-// (the leaves of mask_dnf.cuh read along the other axis):
+// The q interval [lo, hi] of term t for a fixed key kv, within [0, M - 1]
+// (document leaves excluded): each leaf of mask_dnf.cuh read along the other
+// axis,
 //   CAUSAL kv <= q             -> q >= kv
 //   WINDOW q - kv < W          -> q <= kv + W - 1
 //   PREFIX_LM kv < P or q >= kv -> every q when kv < P, else q >= kv
 //   SINK kv < S                -> every q when kv < S, else none
-__device__ __forceinline__ void leaf_clamp_q(int32_t kind, int32_t arg, int64_t kv, int64_t& lo, int64_t& hi) {
-    switch (kind) {
-        case BSMT_MASK_CAUSAL:
-            lo = lo > kv ? lo : kv;
-            break;
-        case BSMT_MASK_WINDOW: {
-            const int64_t h = kv + static_cast<int64_t>(arg) - 1;
-            hi = hi < h ? hi : h;
-            break;
-        }
-        case BSMT_MASK_PREFIX_LM:
-            if (kv >= static_cast<int64_t>(arg)) lo = lo > kv ? lo : kv;
-            break;
-        case BSMT_MASK_SINK:
-            if (kv >= static_cast<int64_t>(arg)) hi = -1;
-            break;
-        default:  // NOOP; DOCUMENT is applied by the caller
-            break;
-    }
-}
-
-// q interval of term t for key kv, within [0, M-1] (document leaves excluded).
 __device__ __forceinline__ void term_q_interval(const MaskDnf& m, int t, int64_t kv, int64_t M, int64_t& lo,
                                                 int64_t& hi) {
+    const DnfTerm& tm = m.terms[t];
     lo = 0;
     hi = M - 1;
-    for (int i = m.term_begin[t]; i < m.term_begin[t + 1]; ++i)
-        if (m.leaves[i].kind != BSMT_MASK_DOCUMENT) leaf_clamp_q(m.leaves[i].kind, m.leaves[i].arg, kv, lo, hi);
+    if (tm.flags & kTermCausal) lo = lo > kv ? lo : kv;
+    if (tm.flags & kTermWindow) {
+        const int64_t h = kv + static_cast<int64_t>(tm.w) - 1;
+        hi = hi < h ? hi : h;
+    }
+    if ((tm.flags & kTermPrefix) && kv >= static_cast<int64_t>(tm.pf)) lo = lo > kv ? lo : kv;
+    if ((tm.flags & kTermSink) && kv >= static_cast<int64_t>(tm.s)) hi = -1;
 }
 
 // (-lse2, -delta) per padded query row: lse2 = lse * log2(e) (+inf where lse

@@ -121,14 +121,12 @@ void simplify(std::vector<Term>& terms) {
 // Terms held while the program is evaluated; only the final count must fit
 // kMaxTerms, since later ANDs and ORs can merge terms again.
 constexpr size_t kMaxWorkTerms = 1024;
-static_assert(5 * bsmt::kMaxTerms <= bsmt::kMaxLeaves, "a canonical term has at most one leaf of each of 5 kinds");
+static_assert(5 * BSMT_MAX_MASK_TERMS <= BSMT_MAX_MASK_LEAVES, "a canonical term has at most one leaf of each of 5 kinds");
 
 bsmt_status build_dnf(const bsmt_mask_spec* spec, int64_t B, bsmt::MaskDnf* out) {
     std::memset(out, 0, sizeof(*out));
-    if (spec == nullptr) {  // NOOP
+    if (spec == nullptr) {  // NOOP: one term without leaves
         out->n_terms = 1;
-        out->term_begin[0] = 0;
-        out->term_begin[1] = 0;
         return BSMT_OK;
     }
     if (spec->num_nodes < 1 || spec->num_nodes > BSMT_MAX_MASK_NODES)
@@ -196,20 +194,17 @@ bsmt_status build_dnf(const bsmt_mask_spec* spec, int64_t B, bsmt::MaskDnf* out)
                         static_cast<long long>(B));
     }
     out->n_terms = static_cast<int32_t>(terms.size());
-    int pos = 0;
     for (size_t t = 0; t < terms.size(); ++t) {
         const Term& tm = terms[t];
-        out->term_begin[t] = pos;
-        if (tm.causal) out->leaves[pos++] = bsmt::DnfLeaf{BSMT_MASK_CAUSAL, 0};
-        if (tm.has_w) out->leaves[pos++] = bsmt::DnfLeaf{BSMT_MASK_WINDOW, tm.w};
-        if (tm.has_p) out->leaves[pos++] = bsmt::DnfLeaf{BSMT_MASK_PREFIX_LM, tm.pf};
-        if (tm.has_s) out->leaves[pos++] = bsmt::DnfLeaf{BSMT_MASK_SINK, tm.s};
-        if (tm.doc) {
-            out->leaves[pos++] = bsmt::DnfLeaf{BSMT_MASK_DOCUMENT, 0};
-            out->term_has_doc |= 1u << t;
-        }
+        bsmt::DnfTerm& d = out->terms[t];
+        d.flags = (tm.causal ? bsmt::kTermCausal : 0u) | (tm.has_w ? bsmt::kTermWindow : 0u) |
+                  (tm.has_p ? bsmt::kTermPrefix : 0u) | (tm.has_s ? bsmt::kTermSink : 0u) |
+                  (tm.doc ? bsmt::kTermDoc : 0u);
+        d.w = tm.w;
+        d.pf = tm.pf;
+        d.s = tm.s;
+        if (tm.doc) out->term_has_doc |= 1u << t;
     }
-    out->term_begin[terms.size()] = pos;
     // a program whose DOCUMENT leaves all fell inside other terms needs no ids
     out->has_doc = out->term_has_doc != 0u ? 1 : 0;
     out->q_doc = spec->q_doc_ids;

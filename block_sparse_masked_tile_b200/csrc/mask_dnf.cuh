@@ -24,67 +24,52 @@
 namespace bsmt {
 
 constexpr int kMaxTerms = BSMT_MAX_MASK_TERMS;
-constexpr int kMaxLeaves = BSMT_MAX_MASK_LEAVES;
 
-struct DnfLeaf {
-    int32_t kind;
-    int32_t arg;
+// One AND-term in canonical form: at most one leaf of each kind (the host
+// keeps the strictest), so a term is a set of flags and three arguments.
+constexpr uint32_t kTermCausal = 1u, kTermWindow = 2u, kTermPrefix = 4u, kTermSink = 8u, kTermDoc = 16u;
+
+struct DnfTerm {
+    uint32_t flags;    // kTerm* bits; 0 is NOOP
+    int32_t w, pf, s;  // the WINDOW W, PREFIX_LM P and SINK S of the term, when flagged
 };
 
 struct MaskDnf {
-    int32_t n_terms;                    // 0 means "nothing allowed"
-    int32_t term_begin[kMaxTerms + 1];  // leaves of term t: [term_begin[t], term_begin[t+1])
-    uint32_t term_has_doc;              // bit t: term t contains a DOCUMENT leaf
-    DnfLeaf leaves[kMaxLeaves];
+    int32_t n_terms;        // 0 means "nothing allowed"
+    uint32_t term_has_doc;  // bit t: term t has a DOCUMENT leaf
+    DnfTerm terms[kMaxTerms];
     const int32_t* q_doc;
     const int32_t* kv_doc;
     int32_t doc_batch;
     int32_t has_doc;
 };
 
-// Clamp [lo, hi] by one non-document leaf for query row q (64-bit so that
-// extreme W / P / S values cannot overflow).
-__host__ __device__ __forceinline__ void leaf_clamp(int32_t kind, int32_t arg, int64_t q, int64_t& lo,
-                                                    int64_t& hi) {
-    switch (kind) {
-        case BSMT_MASK_CAUSAL:
-            hi = hi < q ? hi : q;
-            break;
-        case BSMT_MASK_WINDOW: {
-            const int64_t l = q - static_cast<int64_t>(arg) + 1;
-            lo = lo > l ? lo : l;
-            break;
-        }
-        case BSMT_MASK_PREFIX_LM: {
-            const int64_t pm1 = static_cast<int64_t>(arg) - 1;
-            const int64_t h = pm1 > q ? pm1 : q;
-            hi = hi < h ? hi : h;
-            break;
-        }
-        case BSMT_MASK_SINK: {
-            const int64_t h = static_cast<int64_t>(arg) - 1;
-            hi = hi < h ? hi : h;
-            break;
-        }
-        default:  // NOOP; DOCUMENT is applied by the caller
-            break;
-    }
-}
-
 // Interval allowed by term t for row q, clamped to [lo0, hi0], using the
-// row's document interval [ds, de] when the term has a DOCUMENT leaf.
+// row's document interval [ds, de] when the term has a DOCUMENT leaf
+// (64-bit, so that extreme W / P / S values cannot overflow). The term's
+// fields are read together, with no dependence between them.
 __device__ __forceinline__ void term_interval(const MaskDnf& m, int t, int64_t q, int64_t lo0, int64_t hi0,
                                               int64_t ds, int64_t de, int64_t& lo, int64_t& hi) {
+    const DnfTerm tm = m.terms[t];
     lo = lo0;
     hi = hi0;
-    for (int i = m.term_begin[t]; i < m.term_begin[t + 1]; ++i) {
-        const int32_t kind = m.leaves[i].kind;
-        if (kind == BSMT_MASK_DOCUMENT) {
-            lo = lo > ds ? lo : ds;
-            hi = hi < de ? hi : de;
-        } else {
-            leaf_clamp(kind, m.leaves[i].arg, q, lo, hi);
-        }
+    if (tm.flags & kTermCausal) hi = hi < q ? hi : q;
+    if (tm.flags & kTermWindow) {
+        const int64_t l = q - static_cast<int64_t>(tm.w) + 1;
+        lo = lo > l ? lo : l;
+    }
+    if (tm.flags & kTermPrefix) {
+        const int64_t pm1 = static_cast<int64_t>(tm.pf) - 1;
+        const int64_t h = pm1 > q ? pm1 : q;
+        hi = hi < h ? hi : h;
+    }
+    if (tm.flags & kTermSink) {
+        const int64_t h = static_cast<int64_t>(tm.s) - 1;
+        hi = hi < h ? hi : h;
+    }
+    if (tm.flags & kTermDoc) {
+        lo = lo > ds ? lo : ds;
+        hi = hi < de ? hi : de;
     }
 }
 
