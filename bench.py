@@ -119,31 +119,49 @@ def reduce_over_ranks(dist, device, times_ms, units):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    """nvidia-smi clock / throttle sampling around the timed region.
+
+    Samples arrive every 20 ms; each is stamped with the host's monotonic
+    clock when it is read. ``mark_start`` / ``mark_end`` bracket the timed
+    region, and ``summary`` keeps the samples read inside it (plus one
+    interval after its end, the sample that covers its last stretch). A
+    region shorter than the interval may hold none: then the summary uses
+    every sample of the sampler's life and says so (``in_window`` false)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 20
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.lines: list[str] = []
+        self.lines: list[tuple[float, str]] = []
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.INTERVAL_MS)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
-            time.sleep(0.3)
+            deadline = time.monotonic() + 3.0
+            while not self.lines and time.monotonic() < deadline:  # the sampler is running
+                time.sleep(0.005)
         except FileNotFoundError:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
+        time.sleep(2 * self.INTERVAL_MS / 1000)  # let the sample that covers the region's end arrive
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -154,9 +172,13 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        in_window = [ln for t, ln in self.lines
+                     if self.t0 is not None and self.t1 is not None and
+                     self.t0 <= t <= self.t1 + self.INTERVAL_MS / 1000]
+        chosen = in_window if in_window else [ln for _, ln in self.lines]
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in chosen:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -168,9 +190,12 @@ class ClockSampler:
             for name, val in zip(names, parts[5:9]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
+        window_ms = None if self.t0 is None or self.t1 is None else round((self.t1 - self.t0) * 1e3, 1)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0, "in_window": False,
+                    "window_ms": window_ms, "interval_ms": self.INTERVAL_MS}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "in_window": bool(in_window), "window_ms": window_ms, "interval_ms": self.INTERVAL_MS}
 
 
 def _time_launches(fn, reps: int = 20) -> float:
@@ -570,11 +595,13 @@ def main():
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
+        clk.mark_start()
         start.record(stream)
         for i in range(args.steps):
             step(ev[i])
         end.record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark_end()
     if dist:
         dist.barrier()
     bsmt.check_device_status(dev)

@@ -55,3 +55,24 @@ def test_cpu_baseline_counts_kept_tiles_and_times_the_block_mask():
     cls = obm.tile_classes(data["mask"], 0, w.M, w.N)
     r2 = bench.cpu_baseline(w, data, cls=cls)
     assert "3 kept tiles" in r2["sample"] and "block_mask" not in r2
+
+
+def test_clock_sampler_keeps_the_timed_window():
+    """The summary keeps the samples read inside the timed region (and one
+    interval after it); with none there it falls back to all samples and
+    says so."""
+    s = bench.ClockSampler(0)
+    row = "0, {mhz}, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, {cap}"
+    s.lines = [(1.000, row.format(mhz=1000, cap="Not Active")),   # before the region
+               (2.005, row.format(mhz=1965, cap="Active")),       # inside
+               (2.030, row.format(mhz=1950, cap="Not Active")),   # inside
+               (2.070, row.format(mhz=1900, cap="Not Active")),   # within one interval after the end
+               (3.000, row.format(mhz=500, cap="Not Active"))]    # after
+    s.t0, s.t1 = 2.0, 2.05
+    c = s.summary()
+    assert c["in_window"] and c["samples"] == 3 and c["sm_mhz"] == 1950.0
+    assert c["reasons"] == ["sw_power_cap"] and c["sm_max_mhz"] == 1965.0
+    assert c["window_ms"] == 50.0
+    s.t0, s.t1 = 2.5, 2.51  # no sample inside: every sample is used
+    c = s.summary()
+    assert not c["in_window"] and c["samples"] == 5
