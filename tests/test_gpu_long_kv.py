@@ -139,3 +139,39 @@ def test_static_scratch_long_kv_matches_workspace_form():
         assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])
     # the workspace does not grow with N
     assert bsmt.splitkv_workspace_bytes(1, 2, 300, 128, 2) == (2 * 600 * 128 * 4 + 255) // 256 * 256 + 2 * 600 * 4
+
+
+def test_host_entry_long_rows():
+    # the host-buffer entry over rows of more than one window: its pieces run
+    # the same kernels, so the bits equal the device path's
+    q, k, v = workloads.random_inputs(86, 1, 4, 2, 300, 140000, 64)
+    tree = ("or", ("sink", 4), ("window", 3000))
+    mm = bsmt.mask_from_tree(tree, device="cuda")
+    out_h, lse_h = bsmt.flex_attention_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), mask_mod=mm,
+                                            enable_gqa=True, chunks=2)
+    bm = bsmt.create_block_mask(mm, 1, 4, 300, 140000)
+    out_d, lse_d = bsmt.flex_attention(q.cuda(), k.cuda(), v.cuda(), block_mask=bm, enable_gqa=True)
+    bsmt.check_device_status()
+    assert torch.equal(out_h, out_d.cpu()) and torch.equal(lse_h, lse_d.cpu())
+    _compare_all(_oracle_all(q, k, v, tree, ()), out_d, lse_d, "host entry, long rows")
+
+
+def test_varlen_pack_longer_than_one_window():
+    # 150 packed sequences, 160k tokens in all: the pack's kv blocks exceed
+    # one window, each unit's listed blocks lie within its own sequences
+    rng = np.random.default_rng(87)
+    lens = rng.integers(300, 1900, size=150)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total = int(cu[-1])
+    assert total > WINDOW
+    g = torch.Generator().manual_seed(88)
+    q, k, v = (torch.randn((total, h, 64), generator=g).to(torch.bfloat16) for h in (4, 2, 2))
+    cuq = torch.from_numpy(cu).cuda()
+    out, lse = bsmt.flex_attention_varlen(q.cuda(), k.cuda(), v.cuda(), cuq, cuq, causal=True, enable_gqa=True)
+    bsmt.check_device_status()
+    ro, rl = oa.flex_attention_varlen(q, k, v, cu, cu, True, (), None, True)
+    # out [total, Hq, D] and lse [Hq, total]; every causal row sees its own key
+    assert np.abs(out.float().cpu().numpy() - ro).max() <= OUT_TOL
+    got_l = lse.cpu().numpy()
+    assert np.all(np.isfinite(rl)) and np.all(np.isfinite(got_l))
+    assert np.abs(got_l - rl).max() <= LSE_TOL
