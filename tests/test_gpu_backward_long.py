@@ -67,3 +67,17 @@ def test_autograd_long_rows():
     ref = ob.flex_attention_backward(q, k, v, dout, None, (), None, True)
     got = [t.grad.float().cpu().numpy().astype(np.float64) for t in (qd, kd, vd)]
     assert_grads_close(got, ref, "autograd long rows")
+
+
+def test_dkdv_units_over_two_buffers_two_batch_rows_broadcast_mask():
+    # B = 2 with a block mask built once for B = H = 1 (broadcast), GQA 8:1
+    # over 260 q-blocks and 333 keys: kv-block 0 (the sink keys for most
+    # queries, the window for the first ones) is listed for every q-block,
+    # 2080 entries in two buffers; the others for the first q-blocks only
+    tree = ("and", ("causal",), ("or", ("sink", 16), ("window", 1000)))
+    M, N = 260 * 128, 333
+    q, k, v = workloads.random_inputs(98, 2, 8, 1, M, N, 64)
+    dout = workloads.grad_output(99, 2, 8, M, 64)
+    got = gpu_backward(q, k, v, dout, tree, (), None, True, True, mask_B=1, mask_H=1)
+    ref = ob.flex_attention_backward(q, k, v, dout, tree, (), None, True)
+    assert_grads_close(got, ref, "two batch rows, broadcast mask")

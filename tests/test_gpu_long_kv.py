@@ -175,3 +175,18 @@ def test_varlen_pack_longer_than_one_window():
     got_l = lse.cpu().numpy()
     assert np.all(np.isfinite(rl)) and np.all(np.isfinite(got_l))
     assert np.abs(got_l - rl).max() <= LSE_TOL
+
+
+def test_two_batch_rows_documents_per_row():
+    # B = 2 with different document ids per batch row (doc_batch = 2) and GQA;
+    # row 1's first document spans the window edge, row 0's does not
+    N = 136000
+    lens0 = [60000, 76000]
+    lens1 = [120000, 16000]
+    ids = np.stack([np.repeat(np.arange(2), lens0), np.repeat(np.arange(2), lens1)]).astype(np.int32)
+    tree = ("and", ("document", ids, ids), ("causal",))
+    q, k, v = workloads.random_inputs(89, 2, 2, 1, N, N, 64)
+    rows = list(range(WINDOW - 64, WINDOW + 64)) + list(range(119900, 120100)) + list(range(135900, 136000))
+    for splits in (1, 3):
+        out, lse = _gpu(q, k, v, tree, (), splits)
+        _compare_rows(q, k, v, tree, (), out, lse, rows, f"two batch rows, splits={splits}")
