@@ -281,6 +281,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         int iter = 0;
         const uint32_t below = (1u << lane) - 1u;
         const bool ragged_kv = (p.N & 127) != 0;
+        // the document searched last (batch row of the ids, id, kv interval):
+        // consecutive rows, and the rows of consecutive units, mostly share it
+        // (kept by the kernel for rows of at most kMaxKB kv blocks, whose
+        // scheduler has the registers for it)
+        int32_t cache_db = -1, cache_id = 0, cache_lo = 0, cache_hi = -1;
         // Units go out in a serpentine order: round k gives CTA c unit
         // k * G + c for even k and k * G + (G - 1 - c) for odd k (G CTAs). The
         // order runs longest first, so alternating the direction evens out
@@ -321,7 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Each row's document interval [first, last] of kv positions with the
             // row's document id (kv ids are non-decreasing), into the unit's first
             // buffer sb0. Rows in a run usually share one id, so each distinct id
-            // is searched once, with a 33-way warp search over the kv ids.
+            // is searched once, with a 33-way warp search over the kv ids, and the
+            // last search serves the rows that follow with the same id.
             auto doc_intervals = [&](uint8_t* sb0) {
                 if (dnf.has_doc && p.has_block_mask) {
                     const int db = dnf.doc_batch > 1 ? b : 0;
@@ -336,6 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int32_t d = valid ? __ldg(qd_row + q) : 0;
                         int lo = 0, hi = -1;
                         bool pending = valid;
+                        if (!LONG && pending && db == cache_db && d == cache_id) {
+                            lo = cache_lo;
+                            hi = cache_hi;
+                            pending = false;
+                        }
                         unsigned todo;
                         while ((todo = __ballot_sync(0xFFFFFFFFu, pending)) != 0u) {
                             const int32_t x = __shfl_sync(0xFFFFFFFFu, d, __ffs(todo) - 1);
@@ -345,6 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 lo = first;
                                 hi = past - 1;
                                 pending = false;
+                            }
+                            if constexpr (!LONG) {  // (x and the results are the same in every lane)
+                                cache_db = db;
+                                cache_id = x;
+                                cache_lo = first;
+                                cache_hi = past - 1;
                             }
                         }
                         dlo[r0 + lane] = lo;
