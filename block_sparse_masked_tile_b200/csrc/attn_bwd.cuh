@@ -837,6 +837,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float2* ld_smem = reinterpret_cast<const float2*>(smem + L::kLd);
         uint32_t ge = 0, units = 0;
         bool ok = true;
+        // dq: the document this warp searched last (batch row of the ids, id,
+        // kv span), which a later unit's rows often share
+        int32_t cache_db = -1, cache_id = 0;
+        int64_t cache_lo = 0, cache_hi = -1;
         for (int it = 0; ok; ++it) {
             int buf = it & 1;
             if (!mbar_wait(bar(L::kBarListFull + buf), static_cast<uint32_t>((it >> 1) & 1), abort_flag)) break;
@@ -875,6 +879,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const bool valid = row_idx < p.M;
                     const int32_t d = valid ? __ldg(qd_row + row_idx) : 0;
                     bool pending = valid;
+                    if (!LONG && pending && db == cache_db && d == cache_id) {
+                        row_ds = cache_lo;
+                        row_de = cache_hi;
+                        pending = false;
+                    }
                     unsigned todo;
                     while ((todo = __ballot_sync(0xFFFFFFFFu, pending)) != 0u) {
                         const int32_t x = __shfl_sync(0xFFFFFFFFu, d, __ffs(todo) - 1);
@@ -884,6 +893,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             row_ds = first;
                             row_de = past - 1;
                             pending = false;
+                        }
+                        if constexpr (!LONG) {  // (x and the results are the same in every lane)
+                            cache_db = db;
+                            cache_id = x;
+                            cache_lo = first;
+                            cache_hi = past - 1;
                         }
                     }
                 }
